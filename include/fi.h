@@ -1,0 +1,168 @@
+/*
+ * fi.h -- exact online causal long convolution for stacks of long-convolution
+ * (LCSM, Hyena-style) mixer layers, with the relaxed block schedule of
+ * "Flash Inference: Near Linear Time Inference for Long Convolution Sequence
+ * Models and Beyond" (Oncescu, Purandare, Idreos, Kakade; arXiv 2410.12982),
+ * built for NVIDIA B200 (sm_100a).
+ *
+ * What is computed (summary page, "Definizione del Compito" and "Architettura
+ * del Modello"): for layers l = 1..M, channels d, sequences b and positions t,
+ *
+ *     y^l_t[b][d] = sum_{s <= t} h^l[d][t-s] * a^{l-1}_s[b][d]      (the mixer)
+ *     a^l_t       = R(tanh(y^l_t))                                 (the block)
+ *     a^0_t       = x_t                                            (the tokens)
+ *
+ * with R the identity (FI_F32) or round-to-nearest-even to bfloat16 (FI_BF16).
+ * Each position is computed once every earlier position is known ("online"):
+ * at step i the library adds the contribution of inputs [i-U, i) to outputs
+ * [i, i+U), U = largest power of two dividing i (Algorithm 1 / 2 on the page),
+ * for all layers at once (Algorithm 3), then finishes position i with the
+ * h[0] term ("red cell") and the block, layer after layer.
+ *
+ * Conventions shared by every call:
+ *   - All pointers named in a call are DEVICE pointers unless the name ends in
+ *     "_host". Token-shaped buffers are row-major [B][D] (or [n][B][D]).
+ *   - fp32 buffers are 4-byte aligned, bf16 buffers 2-byte aligned.
+ *   - Every call is asynchronous on the context's CUDA stream (the stream given
+ *     to fi_init or fi_set_stream); buffers passed in must stay valid until the
+ *     stream reaches that point. Only fi_init, fi_destroy, the *_host call and
+ *     fi_profile_read synchronise.
+ *   - Errors are returned as fi_status; no exception crosses this boundary.
+ *     fi_last_error() gives a message for the last failing call on this thread.
+ *     After FI_E_CUDA the context should be destroyed.
+ *   - A context is not thread-safe; use one per host thread.
+ */
+#ifndef FI_H
+#define FI_H
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define FI_API __attribute__((visibility("default")))
+#else
+#define FI_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FI_OK = 0,
+  FI_E_INVALID = 1,     /* bad argument: null pointer, size out of range, L not a power of two */
+  FI_E_OOM = 2,         /* a device or pinned-host allocation failed */
+  FI_E_CUDA = 3,        /* a CUDA runtime call or kernel launch failed */
+  FI_E_STATE = 4,       /* not allowed in the current state (e.g. stepping past max_len) */
+  FI_E_TIMEOUT = 5,     /* reserved: a bounded device-side wait gave up */
+  FI_E_UNSUPPORTED = 6  /* valid request outside what this build implements */
+} fi_status;
+
+typedef enum { FI_F32 = 0, FI_BF16 = 1 } fi_dtype;
+
+typedef struct {
+  int32_t layers;    /* M >= 1 */
+  int32_t channels;  /* D >= 1 */
+  int32_t max_len;   /* L, a power of two, 2 <= L <= 2^17 */
+  int32_t batch;     /* B >= 1 (independent sequences sharing the filters) */
+  int32_t dtype;     /* fi_dtype of filters and tokens; accumulation is always fp32 */
+  int32_t chunk;     /* 0 = automatic; else block sides below this run on chip (power of two, 2..64) */
+  int32_t fft_from;  /* 0 = automatic; else the smallest block side computed by FFT (power of two >= 64) */
+  int32_t reserved[5]; /* must be 0 */
+} fi_config;
+
+typedef struct fi_ctx fi_ctx;
+
+/* Create a context.
+ * h: filters, device, [M][D][L] of cfg->dtype (h^l[d][t] at ((l*D)+d)*L+t).
+ *    The library copies them (widened to fp32) and precomputes, for every block
+ *    side U >= fft_from, the spectrum of h[0..2U) (page: "Precomputazione FFT"),
+ *    so the caller may free h once fi_init returns.
+ * stream: a cudaStream_t (NULL = legacy default stream).
+ * Allocates the state (fp32, (M+1)*B*D*L values), filters and spectra on the
+ * current device. On error *out is NULL and nothing is leaked.
+ * Errors: FI_E_INVALID (null, sizes, reserved != 0), FI_E_UNSUPPORTED (sizes this
+ * build cannot schedule), FI_E_OOM, FI_E_CUDA. */
+FI_API fi_status fi_init(fi_ctx** out, const fi_config* cfg, const void* h, void* stream);
+
+/* One position (Algorithm 2, one iteration): with t = current position,
+ * add the step-t block (U = lowbit(t)) into every layer's accumulators, then run
+ * the red cell and block through the M layers.
+ * x_t: device [B][D] of cfg->dtype, the token at position t.
+ * y_t: device [B][D] fp32, receives y^M_t (last layer's mixer output, before tanh).
+ * Errors: FI_E_INVALID (null), FI_E_STATE (position == max_len). */
+FI_API fi_status fi_step(fi_ctx* ctx, const void* x_t, float* y_t);
+
+/* Closed-loop generation of n positions from the current position p on device:
+ * x_p = x0, and for t >= p: x_{t+1} = R(tanh(y^M_t) + eps_scale * eps[t-p]).
+ * x0:    device [B][D] of cfg->dtype.
+ * eps:   device [n][B][D] fp32 sampler noise.
+ * y_out: device [n][B][D] fp32, receives y^M_t for t = p..p+n-1.
+ * rec:   NULL, or device [M][n][B][D] fp32 that receives y^l_t for every layer
+ *        (test and inspection hook; costs one extra write per layer and position).
+ * Leaves the context at position p+n with the same state fi_step would leave.
+ * Errors: FI_E_INVALID (null, n < 0), FI_E_STATE (p + n > max_len). */
+FI_API fi_status fi_generate(fi_ctx* ctx, int32_t n, const void* x0, const float* eps,
+                      float eps_scale, float* y_out, float* rec);
+
+/* fi_generate with HOST buffers: copies x0_host and eps_host to the device,
+ * generates, copies y^M back to y_out_host, and returns when the copy is done.
+ * Host buffers may be pageable or pinned (pinned is faster). Staging device
+ * buffers are allocated on first use and kept by the context. */
+FI_API fi_status fi_generate_host(fi_ctx* ctx, int32_t n, const void* x0_host, const float* eps_host,
+                           float eps_scale, float* y_out_host);
+
+/* The same closed-loop generation by the Lazy method of the page ("Tre Strategie
+ * di Calcolo": every y^l_t summed in full when needed, O(L^2) in total), with
+ * all layers' sums for a position in one launch (the page's parallel Lazy).
+ * Arguments and state effects as fi_generate (rec not offered). This is the
+ * quadratic baseline the relaxed schedule is measured against. */
+FI_API fi_status fi_generate_lazy(fi_ctx* ctx, int32_t n, const void* x0, const float* eps,
+                           float eps_scale, float* y_out);
+
+/* Rewind to position 0. O(1): no memory is cleared, because every accumulator
+ * is first written (not added to) by the block that first reaches it. */
+FI_API fi_status fi_reset(fi_ctx* ctx);
+
+/* Current position (number of positions already produced). */
+FI_API fi_status fi_position(const fi_ctx* ctx, int32_t* pos);
+
+/* Copy the recorded activations a^layer_t for t < position into dst,
+ * device [position][B][D] fp32; layer in [0, M-1] (layer 0 = the tokens). */
+FI_API fi_status fi_read_activations(fi_ctx* ctx, int32_t layer, float* dst);
+
+/* Change the stream later calls run on. */
+FI_API fi_status fi_set_stream(fi_ctx* ctx, void* stream);
+
+/* The block side at or above which the context uses FFT blocks, and the
+ * on-chip block bound it chose (after automatic selection). */
+FI_API fi_status fi_get_plan(const fi_ctx* ctx, int32_t* chunk, int32_t* fft_from);
+
+/* Kernel timing. With profiling on, every kernel launch of fi_generate is
+ * bracketed by CUDA events on the context's stream; fi_profile_read
+ * synchronises and returns, per kernel class, the launch count and the summed
+ * device time in milliseconds since the last read. Classes: 0 = on-chip chunk
+ * (small blocks + red cells), 1 = direct blocks from HBM, 2 = FFT blocks,
+ * 3 = per-position red cells (fi_step / lazy), 4 = lazy sums. */
+#define FI_NUM_KERNEL_CLASSES 5
+FI_API fi_status fi_profile(fi_ctx* ctx, int32_t enable);
+FI_API fi_status fi_profile_read(fi_ctx* ctx, int32_t counts[FI_NUM_KERNEL_CLASSES],
+                          double ms[FI_NUM_KERNEL_CLASSES]);
+
+/* Release everything the context owns (synchronises its stream first). NULL is allowed. */
+FI_API fi_status fi_destroy(fi_ctx* ctx);
+
+FI_API const char* fi_status_str(fi_status s);
+FI_API const char* fi_last_error(void);
+
+/* Test hook: run the library's device FFT (the one its FFT blocks use) on
+ * `count` complex sequences of length 2^log2n (6 <= log2n <= 14), interleaved
+ * (re, im) fp32, device buffers in[count][2^log2n][2] -> out (may alias in).
+ * Forward is exp(-2 pi i k n / N), inverse exp(+...), both unnormalised.
+ * Synchronous. */
+FI_API fi_status fi_debug_fft(int32_t log2n, int32_t count, const float* in, float* out,
+                       int32_t inverse, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* FI_H */

@@ -1,0 +1,170 @@
+// Complex FFT of N = 2^k points held in shared memory, used by the FFT blocks
+// (Lemma 1 of the Flash Inference summary page: tau by FFT) and by the filter
+// spectrum precompute ("Precomputazione FFT").
+//
+// Formulation: Stockham autosort, decimation in time (Govindaraju et al.,
+// "High Performance Discrete Fourier Transforms on Graphics Processors", SC'08):
+// in pass s with radix R and Ns = product of the earlier radices, element j of
+// N/R reads R values at stride N/R, multiplies value r by W_{Ns*R}^{r*(j mod Ns)},
+// runs an R-point DFT in registers and writes value r to
+// (j div Ns)*Ns*R + (j mod Ns) + r*Ns. The output is in natural order.
+//
+// T threads cooperate on one transform, each holding P = N/T points; the radix
+// is min(16, P) (the last pass takes what is left). Each pass loads all of a
+// thread's points, synchronises, then stores, so one buffer suffices. Shared
+// memory indices are padded by one slot per 16 (idx + idx/16) so the stride-16
+// stores of the first pass do not collide in the same bank.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include <utility>
+
+#include "fi_internal.cuh"
+
+namespace fi {
+
+__host__ __device__ constexpr int fft_pad(int i) { return i + (i >> 4); }
+__host__ __device__ constexpr int fft_smem_elems(int n) { return n + (n >> 4); }
+__host__ __device__ constexpr int clog2(int v) { return v <= 1 ? 0 : 1 + clog2(v >> 1); }
+__host__ __device__ constexpr int cmin(int a, int b) { return a < b ? a : b; }
+
+__device__ __forceinline__ float2 cadd(float2 a, float2 b) { return make_float2(a.x + b.x, a.y + b.y); }
+__device__ __forceinline__ float2 csub(float2 a, float2 b) { return make_float2(a.x - b.x, a.y - b.y); }
+__device__ __forceinline__ float2 cconj(float2 a) { return make_float2(a.x, -a.y); }
+__device__ __forceinline__ float2 cscale(float2 a, float s) { return make_float2(a.x * s, a.y * s); }
+__device__ __forceinline__ float2 cmul(float2 a, float2 b) {
+  return make_float2(fmaf(a.x, b.x, -a.y * b.y), fmaf(a.x, b.y, a.y * b.x));
+}
+// multiply by i and by -i
+__device__ __forceinline__ float2 cmul_i(float2 a) { return make_float2(-a.y, a.x); }
+__device__ __forceinline__ float2 cmul_mi(float2 a) { return make_float2(a.y, -a.x); }
+
+// cos and sin of 2*pi*m/16, m in [0, 16) (exact decimal expansions of the constants).
+__device__ __forceinline__ float cos16(int m) {
+  constexpr float c1 = 0.92387953251128675613f, s1 = 0.38268343236508977173f, r2 = 0.70710678118654752440f;
+  switch (m & 15) {
+    case 0: return 1.f;   case 1: return c1;  case 2: return r2;  case 3: return s1;
+    case 4: return 0.f;   case 5: return -s1; case 6: return -r2; case 7: return -c1;
+    case 8: return -1.f;  case 9: return -c1; case 10: return -r2; case 11: return -s1;
+    case 12: return 0.f;  case 13: return s1; case 14: return r2;  default: return c1;
+  }
+}
+__device__ __forceinline__ float sin16(int m) { return cos16(m - 4); }  // sin x = cos(x - pi/2)
+
+// v * W_16^m where W_16 = exp(-2 pi i / 16) (forward) or its conjugate (inverse).
+// m is a compile-time constant after unrolling, so the branches fold away.
+template <bool INV>
+__device__ __forceinline__ float2 mul_w16(float2 v, int m) {
+  m &= 15;
+  if (m == 0) return v;
+  if (m == 8) return make_float2(-v.x, -v.y);
+  if (m == 4) return INV ? cmul_i(v) : cmul_mi(v);
+  if (m == 12) return INV ? cmul_mi(v) : cmul_i(v);
+  const float c = cos16(m);
+  const float s = INV ? sin16(m) : -sin16(m);
+  return cmul(v, make_float2(c, s));
+}
+
+__host__ __device__ constexpr int bitrev(int x, int bits) {
+  return bits == 0 ? 0 : ((x & 1) << (bits - 1)) | bitrev(x >> 1, bits - 1);
+}
+template <int K, int BITS>
+constexpr int kBitrev = bitrev(K, BITS);
+
+// v[k] = t[bitrev(k)] with every index a template constant.
+template <int BITS, int... K>
+__device__ __forceinline__ void bitrev_copy(float2* v, const float2* t, std::integer_sequence<int, K...>) {
+  ((v[K] = t[kBitrev<K, BITS>]), ...);
+}
+
+// One decimation-in-frequency stage of butterflies with half-span SPAN, then the
+// next stage (template recursion keeps every index a compile-time constant).
+template <int R, int SPAN, bool INV>
+__device__ __forceinline__ void dif_stage(float2* v) {
+#pragma unroll
+  for (int g0 = 0; g0 < R; g0 += 2 * SPAN) {
+#pragma unroll
+    for (int j = 0; j < SPAN; ++j) {
+      const float2 a = v[g0 + j], b = v[g0 + j + SPAN];
+      v[g0 + j] = cadd(a, b);
+      v[g0 + j + SPAN] = mul_w16<INV>(csub(a, b), j * (16 / (2 * SPAN)));
+    }
+  }
+  if constexpr (SPAN > 1) dif_stage<R, SPAN / 2, INV>(v);
+}
+
+// R-point DFT of v[0..R) in registers (R = 2, 4, 8 or 16): decimation in
+// frequency, then a fixed permutation undoes the bit reversal.
+template <int R, bool INV>
+__device__ __forceinline__ void dft_reg(float2* v) {
+  constexpr int B = clog2(R);
+  dif_stage<R, R / 2, INV>(v);
+  float2 t[R];
+#pragma unroll
+  for (int k = 0; k < R; ++k) t[k] = v[k];
+  bitrev_copy<B>(v, t, std::make_integer_sequence<int, R>{});
+}
+
+struct SyncWarp { __device__ __forceinline__ void operator()() const { __syncwarp(); } };
+struct SyncBlock { __device__ __forceinline__ void operator()() const { __syncthreads(); } };
+
+template <int N, int T, bool INV, int DONE, class Sync>
+struct FftPass {
+  static constexpr int LOGN = clog2(N);
+  static constexpr int P = N / T;
+  static constexpr int RB = cmin(cmin(4, clog2(P)), LOGN - DONE);
+  static constexpr int R = 1 << RB;
+  static constexpr int Ns = 1 << DONE;
+
+  __device__ __forceinline__ static void run(float2* sm, int tid, const float2* __restrict__ tw, Sync sync) {
+    float2 v[P];
+#pragma unroll
+    for (int k = 0; k < P / R; ++k) {
+      const int j = tid + k * T;
+#pragma unroll
+      for (int r = 0; r < R; ++r) v[k * R + r] = sm[fft_pad(j + r * (N / R))];
+    }
+#pragma unroll
+    for (int k = 0; k < P / R; ++k) {
+      const int j = tid + k * T;
+      if (Ns > 1) {
+        const int kk = j & (Ns - 1);
+        constexpr int stride = kTwiddleN / (Ns * R);
+#pragma unroll
+        for (int r = 1; r < R; ++r) {
+          float2 w = __ldg(tw + r * kk * stride);
+          if (INV) w.y = -w.y;
+          v[k * R + r] = cmul(v[k * R + r], w);
+        }
+      }
+      dft_reg<R, INV>(v + k * R);
+    }
+    sync();
+#pragma unroll
+    for (int k = 0; k < P / R; ++k) {
+      const int j = tid + k * T;
+      const int kk = j & (Ns - 1);
+      const int e = (j - kk) * R + kk;
+#pragma unroll
+      for (int r = 0; r < R; ++r) sm[fft_pad(e + r * Ns)] = v[k * R + r];
+    }
+    sync();
+    if constexpr (DONE + RB < LOGN) FftPass<N, T, INV, DONE + RB, Sync>::run(sm, tid, tw, sync);
+  }
+};
+
+// In-place transform of sm[fft_pad(0..N)) by the T threads with tid in [0, T).
+// Callers synchronise before (data written) and may read results right after.
+template <int N, int T, bool INV, class Sync>
+__device__ __forceinline__ void fft_smem(float2* sm, int tid, const float2* __restrict__ tw, Sync sync) {
+  static_assert((N & (N - 1)) == 0 && N >= 2 * T && T >= 32, "bad FFT shape");
+  FftPass<N, T, INV, 0, Sync>::run(sm, tid, tw, sync);
+}
+
+// Threads per transform for N points: one warp up to 512 points, else 16 points per thread.
+__host__ __device__ constexpr int fft_threads(int n) { return n <= 512 ? 32 : n / 16; }
+// Transforms per CTA: several warps for the warp-sized transforms.
+__host__ __device__ constexpr int fft_per_cta(int n) { return n <= 512 ? 4 : 1; }
+
+}  // namespace fi

@@ -1,0 +1,435 @@
+// C-ABI of the library (declared in include/fi.h): argument checks, device
+// memory, and the host side of the relaxed schedule (which block runs at
+// which step, and on which kernel).
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <string>
+#include <vector>
+
+#include "fi_internal.cuh"
+
+using namespace fi;
+
+namespace {
+
+thread_local std::string g_last_error;
+
+fi_status fail(fi_status s, const std::string& msg) {
+  g_last_error = msg;
+  return s;
+}
+
+fi_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(FI_E_CUDA, std::string(what) + ": " + cudaGetErrorString(e));
+}
+
+#define FI_CUDA(call, what)                         \
+  do {                                              \
+    cudaError_t e_ = (call);                        \
+    if (e_ != cudaSuccess) return cuda_fail(e_, what); \
+  } while (0)
+
+struct EventPair {
+  cudaEvent_t a, b;
+  int cls;
+};
+
+}  // namespace
+
+struct fi_ctx {
+  Dims g{};
+  fi_config cfg{};
+  cudaStream_t st = nullptr;
+  int device = 0, num_sms = 0;
+  size_t max_smem = 0;
+  int pos = 0;
+  int lazy_mode = 0;  // 1 after fi_generate_lazy until fi_reset
+  int chunk = 0, fft_from = 0, q_lo = 0, q_hi = -1;
+  int chunk_G = 0;
+  float* state = nullptr;
+  float* taps = nullptr;
+  float2* spectra = nullptr;
+  float2* twiddle = nullptr;
+  size_t spec_off[32] = {};
+  // staging for fi_generate_host
+  void* d_x0 = nullptr;
+  float* d_eps = nullptr;
+  float* d_y = nullptr;
+  size_t stage_n = 0;
+  // profiling
+  int prof = 0;
+  std::vector<EventPair> ev_live, ev_free;
+};
+
+namespace {
+
+bool pow2(int64_t v) { return v > 0 && (v & (v - 1)) == 0; }
+
+void free_ctx(fi_ctx* c) {
+  if (!c) return;
+  cudaFree(c->state);
+  cudaFree(c->taps);
+  cudaFree(c->spectra);
+  cudaFree(c->twiddle);
+  cudaFree(c->d_x0);
+  cudaFree(c->d_eps);
+  cudaFree(c->d_y);
+  for (auto& e : c->ev_live) { cudaEventDestroy(e.a); cudaEventDestroy(e.b); }
+  for (auto& e : c->ev_free) { cudaEventDestroy(e.a); cudaEventDestroy(e.b); }
+  delete c;
+}
+
+fi_status dev_alloc(void** p, size_t bytes, const char* what) {
+  cudaError_t e = cudaMalloc(p, bytes);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    *p = nullptr;
+    return fail(FI_E_OOM, std::string("cudaMalloc failed for ") + what + " (" + std::to_string(bytes) + " bytes): " +
+                              cudaGetErrorString(e));
+  }
+  return FI_OK;
+}
+
+// Kernel launch wrapped in profiling events when enabled.
+template <class F>
+fi_status timed(fi_ctx* c, int cls, F&& launch, const char* what) {
+  EventPair ep{};
+  if (c->prof) {
+    if (!c->ev_free.empty()) {
+      ep = c->ev_free.back();
+      c->ev_free.pop_back();
+    } else {
+      FI_CUDA(cudaEventCreate(&ep.a), "cudaEventCreate");
+      FI_CUDA(cudaEventCreate(&ep.b), "cudaEventCreate");
+    }
+    ep.cls = cls;
+    FI_CUDA(cudaEventRecord(ep.a, c->st), "cudaEventRecord");
+  }
+  cudaError_t e = launch();
+  if (e != cudaSuccess) return cuda_fail(e, what);
+  if (c->prof) {
+    FI_CUDA(cudaEventRecord(ep.b, c->st), "cudaEventRecord");
+    c->ev_live.push_back(ep);
+  }
+  return FI_OK;
+}
+
+// The block of step i (side U = lowbit(i)), read from and written to HBM.
+fi_status run_block(fi_ctx* c, int i) {
+  const int U = i & -i;
+  const int q = ilog2((uint32_t)U);
+  if (q >= c->q_lo && q <= c->q_hi) {
+    return timed(c, KC_FFT, [&] { return launch_tile_fft(c->g, c->state, c->spectra + c->spec_off[q], c->twiddle, i, c->st); },
+                 "FFT block launch");
+  }
+  return timed(c, KC_DIRECT, [&] { return launch_tile_direct(c->g, c->state, c->taps, i, c->st); },
+               "direct block launch");
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* fi_status_str(fi_status s) {
+  switch (s) {
+    case FI_OK: return "ok";
+    case FI_E_INVALID: return "invalid argument";
+    case FI_E_OOM: return "out of device memory";
+    case FI_E_CUDA: return "CUDA error";
+    case FI_E_STATE: return "invalid state";
+    case FI_E_TIMEOUT: return "device wait timed out";
+    case FI_E_UNSUPPORTED: return "unsupported";
+  }
+  return "unknown status";
+}
+
+const char* fi_last_error(void) { return g_last_error.c_str(); }
+
+fi_status fi_init(fi_ctx** out, const fi_config* cfg, const void* h, void* stream) {
+  if (!out) return fail(FI_E_INVALID, "out is NULL");
+  *out = nullptr;
+  if (!cfg || !h) return fail(FI_E_INVALID, "cfg or h is NULL");
+  for (int k = 0; k < 5; ++k)
+    if (cfg->reserved[k] != 0) return fail(FI_E_INVALID, "reserved fields must be 0");
+  if (cfg->layers < 1 || cfg->channels < 1 || cfg->batch < 1) return fail(FI_E_INVALID, "layers, channels, batch must be >= 1");
+  if (!pow2(cfg->max_len) || cfg->max_len < 2 || cfg->max_len > (1 << 17))
+    return fail(FI_E_INVALID, "max_len must be a power of two in [2, 2^17]");
+  if (cfg->dtype != FI_F32 && cfg->dtype != FI_BF16) return fail(FI_E_INVALID, "dtype must be FI_F32 or FI_BF16");
+  if (cfg->chunk != 0 && (!pow2(cfg->chunk) || cfg->chunk < 2 || cfg->chunk > 64))
+    return fail(FI_E_INVALID, "chunk must be 0 or a power of two in [2, 64]");
+  if (cfg->fft_from != 0 && (!pow2(cfg->fft_from) || cfg->fft_from < (1 << kMinFftLog2)))
+    return fail(FI_E_INVALID, "fft_from must be 0 or a power of two >= 64");
+  const int64_t S = (int64_t)cfg->batch * cfg->channels;
+  if (S > (1 << 24) || (int64_t)cfg->layers * cfg->channels > (1 << 24) || cfg->layers > 4096)
+    return fail(FI_E_UNSUPPORTED, "too many streams or layers");
+
+  fi_ctx* c = new (std::nothrow) fi_ctx();
+  if (!c) return fail(FI_E_OOM, "host allocation failed");
+  c->cfg = *cfg;
+  c->st = reinterpret_cast<cudaStream_t>(stream);
+  Dims& g = c->g;
+  g.M = cfg->layers;
+  g.D = cfg->channels;
+  g.L = cfg->max_len;
+  g.B = cfg->batch;
+  g.S = (int)S;
+  g.P = ilog2((uint32_t)g.L);
+  g.bf16 = cfg->dtype == FI_BF16;
+
+  auto bail = [&](fi_status s) { free_ctx(c); return s; };
+  cudaError_t e;
+  if ((e = cudaGetDevice(&c->device)) != cudaSuccess) return bail(cuda_fail(e, "cudaGetDevice"));
+  int v = 0;
+  if ((e = cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, c->device)) != cudaSuccess)
+    return bail(cuda_fail(e, "cudaDeviceGetAttribute"));
+  c->num_sms = v;
+  if ((e = cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerBlockOptin, c->device)) != cudaSuccess)
+    return bail(cuda_fail(e, "cudaDeviceGetAttribute"));
+  c->max_smem = (size_t)v;
+
+  // Plan: blocks below `chunk` on chip, FFT from `fft_from` up to the largest
+  // transform one CTA holds, direct blocks from HBM in between and above.
+  c->chunk = cfg->chunk ? cfg->chunk : 32;
+  if (c->chunk > g.L) c->chunk = g.L;
+  c->fft_from = cfg->fft_from ? cfg->fft_from : 128;
+  c->q_lo = ilog2((uint32_t)c->fft_from);
+  c->q_hi = g.P - 1 < kMaxFftLog2 ? g.P - 1 : kMaxFftLog2;
+  if (c->q_lo < kMinFftLog2) c->q_lo = kMinFftLog2;
+  c->chunk_G = chunk_streams_per_cta(g, c->chunk, c->num_sms, c->max_smem);
+  if (c->chunk_G == 0) return bail(fail(FI_E_UNSUPPORTED, "too many layers for the on-chip chunk window"));
+  if ((e = configure_chunk(chunk_smem_bytes(g, c->chunk, c->chunk_G))) != cudaSuccess)
+    return bail(cuda_fail(e, "configure chunk kernel"));
+
+  fi_status s;
+  const size_t state_n = (size_t)(g.M + 1) * g.S * g.L;
+  if ((s = dev_alloc((void**)&c->state, state_n * sizeof(float), "state")) != FI_OK) return bail(s);
+  const size_t taps_n = (size_t)g.M * g.D * g.L;
+  if ((s = dev_alloc((void**)&c->taps, taps_n * sizeof(float), "filters")) != FI_OK) return bail(s);
+  size_t spec_n = 0;
+  for (int q = c->q_lo; q <= c->q_hi; ++q) {
+    c->spec_off[q] = spec_n;
+    spec_n += (size_t)g.M * g.D * ((size_t(1) << q) + 1);
+  }
+  if (spec_n && (s = dev_alloc((void**)&c->spectra, spec_n * sizeof(float2), "spectra")) != FI_OK) return bail(s);
+  if ((s = dev_alloc((void**)&c->twiddle, (size_t)kTwiddleN * sizeof(float2), "twiddles")) != FI_OK) return bail(s);
+
+  std::vector<float2> tw(kTwiddleN);
+  for (int m = 0; m < kTwiddleN; ++m) {
+    const double ang = 2.0 * M_PI * (double)m / (double)kTwiddleN;
+    tw[m] = make_float2((float)std::cos(ang), (float)(-std::sin(ang)));
+  }
+  if ((e = cudaMemcpyAsync(c->twiddle, tw.data(), tw.size() * sizeof(float2), cudaMemcpyHostToDevice, c->st)) != cudaSuccess)
+    return bail(cuda_fail(e, "twiddle upload"));
+  if ((e = launch_widen_filters(h, g.bf16, taps_n, c->taps, c->st)) != cudaSuccess) return bail(cuda_fail(e, "filter copy"));
+  for (int q = c->q_lo; q <= c->q_hi; ++q)
+    if ((e = launch_spectra(g, c->taps, c->spectra + c->spec_off[q], c->twiddle, q, c->st)) != cudaSuccess)
+      return bail(cuda_fail(e, "spectra precompute"));
+  if ((e = cudaStreamSynchronize(c->st)) != cudaSuccess) return bail(cuda_fail(e, "fi_init synchronize"));
+  *out = c;
+  return FI_OK;
+}
+
+fi_status fi_destroy(fi_ctx* c) {
+  if (!c) return FI_OK;
+  cudaStreamSynchronize(c->st);
+  free_ctx(c);
+  return FI_OK;
+}
+
+fi_status fi_reset(fi_ctx* c) {
+  if (!c) return fail(FI_E_INVALID, "ctx is NULL");
+  c->pos = 0;
+  c->lazy_mode = 0;
+  return FI_OK;
+}
+
+fi_status fi_position(const fi_ctx* c, int32_t* pos) {
+  if (!c || !pos) return fail(FI_E_INVALID, "NULL argument");
+  *pos = c->pos;
+  return FI_OK;
+}
+
+fi_status fi_set_stream(fi_ctx* c, void* stream) {
+  if (!c) return fail(FI_E_INVALID, "ctx is NULL");
+  c->st = reinterpret_cast<cudaStream_t>(stream);
+  return FI_OK;
+}
+
+fi_status fi_get_plan(const fi_ctx* c, int32_t* chunk, int32_t* fft_from) {
+  if (!c) return fail(FI_E_INVALID, "ctx is NULL");
+  if (chunk) *chunk = c->chunk;
+  if (fft_from) *fft_from = c->q_lo <= c->q_hi ? (1 << c->q_lo) : 0;
+  return FI_OK;
+}
+
+fi_status fi_step(fi_ctx* c, const void* x_t, float* y_t) {
+  if (!c || !x_t || !y_t) return fail(FI_E_INVALID, "NULL argument");
+  if (c->pos >= c->g.L) return fail(FI_E_STATE, "position == max_len");
+  if (c->lazy_mode) return fail(FI_E_STATE, "context holds a lazy generation; call fi_reset");
+  fi_status s;
+  if (c->pos >= 1 && (s = run_block(c, c->pos)) != FI_OK) return s;
+  const int t = c->pos;
+  if ((s = timed(c, KC_TOKEN, [&] { return launch_token(c->g, c->state, c->taps, t, x_t, nullptr, 0.f, y_t, c->st); },
+                 "red-cell launch")) != FI_OK)
+    return s;
+  c->pos++;
+  return FI_OK;
+}
+
+fi_status fi_generate(fi_ctx* c, int32_t n, const void* x0, const float* eps, float eps_scale, float* y_out,
+                      float* rec) {
+  if (!c) return fail(FI_E_INVALID, "ctx is NULL");
+  if (n < 0) return fail(FI_E_INVALID, "n < 0");
+  if (n == 0) return FI_OK;
+  if (!x0 || !eps || !y_out) return fail(FI_E_INVALID, "NULL buffer");
+  if ((int64_t)c->pos + n > c->g.L) return fail(FI_E_STATE, "position + n > max_len");
+  if (c->lazy_mode) return fail(FI_E_STATE, "context holds a lazy generation; call fi_reset");
+  const int CH = c->chunk;
+  const int base = c->pos, end = c->pos + n;
+  int p = base;
+  fi_status s;
+  while (p < end) {
+    const int cst = (p / CH) * CH;
+    const int p1 = (cst + CH < end) ? cst + CH : end;
+    int last_done = p - 1;
+    if (p == cst && cst > 0) {
+      if ((s = run_block(c, cst)) != FI_OK) return s;
+      last_done = cst;
+    }
+    ChunkArgs a{};
+    a.state = c->state;
+    a.taps = c->taps;
+    a.x0 = (p == base) ? x0 : nullptr;
+    a.eps = eps;
+    a.eps_scale = eps_scale;
+    a.y_out = y_out;
+    a.rec = rec;
+    a.n_gen = n;
+    a.gen_base = base;
+    a.c = cst;
+    a.chunk = CH;
+    a.p0 = p;
+    a.p1 = p1;
+    a.last_done = last_done;
+    if ((s = timed(c, KC_CHUNK, [&] { return launch_chunk(c->g, a, c->chunk_G, c->st); }, "chunk launch")) != FI_OK)
+      return s;
+    p = p1;
+  }
+  c->pos = end;
+  return FI_OK;
+}
+
+fi_status fi_generate_host(fi_ctx* c, int32_t n, const void* x0_host, const float* eps_host, float eps_scale,
+                           float* y_out_host) {
+  if (!c) return fail(FI_E_INVALID, "ctx is NULL");
+  if (n < 0) return fail(FI_E_INVALID, "n < 0");
+  if (n == 0) return FI_OK;
+  if (!x0_host || !eps_host || !y_out_host) return fail(FI_E_INVALID, "NULL buffer");
+  if ((int64_t)c->pos + n > c->g.L) return fail(FI_E_STATE, "position + n > max_len");
+  const size_t row = (size_t)c->g.S;
+  const size_t esz = c->g.bf16 ? 2 : 4;
+  if ((size_t)n > c->stage_n) {
+    cudaFree(c->d_x0);
+    cudaFree(c->d_eps);
+    cudaFree(c->d_y);
+    c->d_x0 = nullptr;
+    c->d_eps = c->d_y = nullptr;
+    c->stage_n = 0;
+    fi_status s;
+    if ((s = dev_alloc(&c->d_x0, row * 4, "staging x0")) != FI_OK) return s;
+    if ((s = dev_alloc((void**)&c->d_eps, row * n * sizeof(float), "staging eps")) != FI_OK) return s;
+    if ((s = dev_alloc((void**)&c->d_y, row * n * sizeof(float), "staging y")) != FI_OK) return s;
+    c->stage_n = (size_t)n;
+  }
+  FI_CUDA(cudaMemcpyAsync(c->d_x0, x0_host, row * esz, cudaMemcpyHostToDevice, c->st), "x0 upload");
+  FI_CUDA(cudaMemcpyAsync(c->d_eps, eps_host, row * n * sizeof(float), cudaMemcpyHostToDevice, c->st), "eps upload");
+  fi_status s = fi_generate(c, n, c->d_x0, c->d_eps, eps_scale, c->d_y, nullptr);
+  if (s != FI_OK) return s;
+  FI_CUDA(cudaMemcpyAsync(y_out_host, c->d_y, row * n * sizeof(float), cudaMemcpyDeviceToHost, c->st), "y download");
+  FI_CUDA(cudaStreamSynchronize(c->st), "fi_generate_host synchronize");
+  return FI_OK;
+}
+
+fi_status fi_generate_lazy(fi_ctx* c, int32_t n, const void* x0, const float* eps, float eps_scale, float* y_out) {
+  if (!c) return fail(FI_E_INVALID, "ctx is NULL");
+  if (n < 0) return fail(FI_E_INVALID, "n < 0");
+  if (n == 0) return FI_OK;
+  if (!x0 || !eps || !y_out) return fail(FI_E_INVALID, "NULL buffer");
+  if ((int64_t)c->pos + n > c->g.L) return fail(FI_E_STATE, "position + n > max_len");
+  if (c->pos > 0 && !c->lazy_mode) return fail(FI_E_STATE, "context holds a relaxed generation; call fi_reset");
+  c->lazy_mode = 1;
+  const size_t row = (size_t)c->g.S;
+  const int base = c->pos;
+  fi_status s;
+  for (int t = base; t < base + n; ++t) {
+    if ((s = timed(c, KC_LAZY, [&] { return launch_lazy_sums(c->g, c->state, c->taps, t, c->st); }, "lazy launch")) !=
+        FI_OK)
+      return s;
+    const void* xt = (t == base) ? x0 : nullptr;
+    const float* et = eps + (size_t)(t - base) * row;
+    float* yt = y_out + (size_t)(t - base) * row;
+    if ((s = timed(c, KC_TOKEN, [&] { return launch_token(c->g, c->state, c->taps, t, xt, et, eps_scale, yt, c->st); },
+                   "red-cell launch")) != FI_OK)
+      return s;
+  }
+  c->pos = base + n;
+  return FI_OK;
+}
+
+fi_status fi_read_activations(fi_ctx* c, int32_t layer, float* dst) {
+  if (!c || !dst) return fail(FI_E_INVALID, "NULL argument");
+  if (layer < 0 || layer >= c->g.M) return fail(FI_E_INVALID, "layer must be in [0, M-1]");
+  FI_CUDA(launch_read_layer(c->g, c->state, layer, c->pos, dst, c->st), "read activations");
+  return FI_OK;
+}
+
+fi_status fi_profile(fi_ctx* c, int32_t enable) {
+  if (!c) return fail(FI_E_INVALID, "ctx is NULL");
+  c->prof = enable ? 1 : 0;
+  return FI_OK;
+}
+
+fi_status fi_profile_read(fi_ctx* c, int32_t counts[FI_NUM_KERNEL_CLASSES], double ms[FI_NUM_KERNEL_CLASSES]) {
+  if (!c || !counts || !ms) return fail(FI_E_INVALID, "NULL argument");
+  FI_CUDA(cudaStreamSynchronize(c->st), "profile synchronize");
+  for (int k = 0; k < FI_NUM_KERNEL_CLASSES; ++k) {
+    counts[k] = 0;
+    ms[k] = 0.0;
+  }
+  for (auto& e : c->ev_live) {
+    float t = 0.f;
+    FI_CUDA(cudaEventElapsedTime(&t, e.a, e.b), "cudaEventElapsedTime");
+    counts[e.cls] += 1;
+    ms[e.cls] += t;
+    c->ev_free.push_back(e);
+  }
+  c->ev_live.clear();
+  return FI_OK;
+}
+
+fi_status fi_debug_fft(int32_t log2n, int32_t count, const float* in, float* out, int32_t inverse, void* stream) {
+  if (!in || !out || count < 0) return fail(FI_E_INVALID, "bad argument");
+  if (log2n < kMinFftLog2 || log2n > kMaxFftLog2) return fail(FI_E_INVALID, "log2n must be in [6, 14]");
+  if (count == 0) return FI_OK;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  std::vector<float2> tw(kTwiddleN);
+  for (int m = 0; m < kTwiddleN; ++m) {
+    const double ang = 2.0 * M_PI * (double)m / (double)kTwiddleN;
+    tw[m] = make_float2((float)std::cos(ang), (float)(-std::sin(ang)));
+  }
+  float2* dtw = nullptr;
+  fi_status s = dev_alloc((void**)&dtw, tw.size() * sizeof(float2), "twiddles");
+  if (s != FI_OK) return s;
+  cudaError_t e = cudaMemcpyAsync(dtw, tw.data(), tw.size() * sizeof(float2), cudaMemcpyHostToDevice, st);
+  if (e == cudaSuccess)
+    e = launch_debug_fft(log2n, count, reinterpret_cast<const float2*>(in), reinterpret_cast<float2*>(out), inverse,
+                         dtw, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  cudaFree(dtw);
+  if (e != cudaSuccess) return cuda_fail(e, "debug FFT");
+  return FI_OK;
+}
+
+}  // extern "C"

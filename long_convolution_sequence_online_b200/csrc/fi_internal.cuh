@@ -1,0 +1,108 @@
+// Internal declarations shared by the C-ABI layer and the kernels.
+//
+// Device memory layout (all fp32):
+//   state   [M+1][S][L]   slot array per layer l = 0..M, S = B*D streams with
+//                          stream index s = d*B + b (a channel's sequences are
+//                          adjacent). For a position t below the current one,
+//                          slot (l, s, t) holds the activation a^l_t; at or
+//                          above it, slot (l, s, t) holds layer l's accumulator
+//                          (page, "Ottimizzazione della Memoria": b^l_i is kept
+//                          in a^l_i's place). l = 0 holds the tokens.
+//   taps    [M][D][L]     filters widened to fp32 (bf16 values are exact in fp32).
+//   spectra per level q with U = 2^q >= fft_from: [M][D][U+1] complex, the
+//                          real-input DFT of h[0..2U) divided by 2U.
+//   twiddle [2^15]         exp(-2 pi i m / 2^15), computed in double on the host.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "../../include/fi.h"
+
+namespace fi {
+
+constexpr int kTwiddleLog2 = 15;              // table covers real FFTs of length <= 2^15
+constexpr int kTwiddleN = 1 << kTwiddleLog2;
+constexpr int kMaxFftLog2 = 14;               // complex FFT points held in one CTA's shared memory
+constexpr int kMinFftLog2 = 6;
+
+enum KernelClass { KC_CHUNK = 0, KC_DIRECT = 1, KC_FFT = 2, KC_TOKEN = 3, KC_LAZY = 4 };
+
+struct Dims {
+  int M, D, L, B, S;   // layers, channels, max length, batch, streams
+  int P;               // log2 L
+  int bf16;            // tokens and filters are bf16
+};
+
+__host__ __device__ inline size_t slot_index(const Dims& g, int l, int s, int t) {
+  return ((size_t)l * g.S + s) * (size_t)g.L + t;
+}
+
+__device__ __forceinline__ float round_act(float v, int bf16) {
+  return bf16 ? __bfloat162float(__float2bfloat16_rn(v)) : v;
+}
+
+__device__ __forceinline__ float load_token(const void* p, size_t i, int bf16) {
+  return bf16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(p)[i])
+              : reinterpret_cast<const float*>(p)[i];
+}
+
+inline int ilog2(uint32_t v) { int r = 0; while ((1u << (r + 1)) <= v && r < 31) ++r; return r; }
+inline bool is_pow2(int64_t v) { return v > 0 && (v & (v - 1)) == 0; }
+inline int lowbit(int i) { return i & -i; }
+inline int highbit(int i) { int r = 1; while ((int64_t)r * 2 <= i) r *= 2; return r; }
+
+// ---------------------------------------------------------------- launchers (kernels/*.cu)
+// All return cudaSuccess or the launch error.
+
+// Red cells + blocks of one position for all streams (fi_step, lazy).
+cudaError_t launch_token(const Dims& g, float* state, const float* taps, int t, const void* x_t,
+                         const float* eps_t, float eps_scale, float* y_t, cudaStream_t st);
+
+// Direct block of step i (side U = lowbit(i)) from HBM for all layers and streams;
+// overwrite = the block is the first to reach its targets (i a power of two).
+cudaError_t launch_tile_direct(const Dims& g, float* state, const float* taps, int i,
+                               cudaStream_t st);
+
+// FFT block of step i (side U = lowbit(i), 2^kMinFftLog2 <= U <= 2^kMaxFftLog2).
+cudaError_t launch_tile_fft(const Dims& g, float* state, const float2* spectrum_q,
+                            const float2* twiddle, int i, cudaStream_t st);
+
+// Spectra of one level q for all (layer, channel).
+cudaError_t launch_spectra(const Dims& g, const float* taps, float2* spectrum_q,
+                           const float2* twiddle, int q, cudaStream_t st);
+
+// The chunk kernel: positions [p0, p1) inside the aligned chunk [c, c+chunk),
+// small blocks (side < chunk) on chip, red cells, blocks and the sampler.
+struct ChunkArgs {
+  float* state;
+  const float* taps;
+  const void* x0;        // token at p0 when first_call (dtype of the context), else NULL
+  const float* eps;      // [n][B][D] relative to gen_base
+  float eps_scale;
+  float* y_out;          // [n][B][D] relative to gen_base
+  float* rec;            // NULL or [M][n][B][D]
+  int n_gen;             // n of the generate call (rec stride)
+  int gen_base;          // first position of the generate call
+  int c, chunk, p0, p1;  // chunk start, chunk length, positions to produce
+  int last_done;         // last step whose blocks have reached HBM before this launch
+};
+cudaError_t launch_chunk(const Dims& g, const ChunkArgs& a, int streams_per_cta, cudaStream_t st);
+cudaError_t configure_chunk(size_t smem);   // allow `smem` bytes of dynamic shared memory
+int chunk_streams_per_cta(const Dims& g, int chunk, int num_sms, size_t max_smem);
+size_t chunk_smem_bytes(const Dims& g, int chunk, int streams_per_cta);
+
+// Lazy sums of position t for all layers: slot(l, s, t) = sum_{s' < t} h^l[t-s'] a^{l-1}_{s'}.
+cudaError_t launch_lazy_sums(const Dims& g, float* state, const float* taps, int t, cudaStream_t st);
+
+// Debug: batch of complex FFTs with the tile FFT code.
+cudaError_t launch_debug_fft(int log2n, int count, const float2* in, float2* out, int inverse,
+                             const float2* twiddle, cudaStream_t st);
+
+// Conversions for fi_init / fi_read_activations.
+cudaError_t launch_widen_filters(const void* h, int bf16, size_t n, float* out, cudaStream_t st);
+cudaError_t launch_read_layer(const Dims& g, const float* state, int layer, int pos, float* dst,
+                              cudaStream_t st);
+
+}  // namespace fi

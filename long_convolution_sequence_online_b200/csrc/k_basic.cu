@@ -1,0 +1,170 @@
+// Per-position red cells, direct blocks read from HBM, the Lazy method's sums
+// and the layout conversions.
+#include "fi_internal.cuh"
+
+namespace fi {
+
+// ---------------------------------------------------------------------------
+// Red cells and blocks of position t for every stream (Algorithm 2's per-layer
+// loop: b^l_t += a^{l-1}_t h^l_0, a^l_t = R(tanh(b^l_t))). One thread carries one
+// stream through all M layers, since each layer needs the previous one's output.
+// x_t: token buffer [B][D] of the context dtype, or NULL to take the token
+// already in slot (0, s, t). eps_t: NULL, or [B][D] noise for the sampler
+// x_{t+1} = R(tanh(y^M_t) + eps_scale * eps_t), written to slot (0, s, t+1).
+// ---------------------------------------------------------------------------
+__global__ void k_token(Dims g, float* __restrict__ state, const float* __restrict__ taps, int t,
+                        const void* __restrict__ x_t, const float* __restrict__ eps_t, float eps_scale,
+                        float* __restrict__ y_t) {
+  const int s = blockIdx.x * blockDim.x + threadIdx.x;
+  if (s >= g.S) return;
+  const int d = s / g.B, b = s - d * g.B;
+  const size_t io = (size_t)b * g.D + d;
+  float a;
+  if (x_t) {
+    a = round_act(load_token(x_t, io, g.bf16), g.bf16);
+    state[slot_index(g, 0, s, t)] = a;
+  } else {
+    a = state[slot_index(g, 0, s, t)];
+  }
+  float y = 0.f;
+  for (int l = 1; l <= g.M; ++l) {
+    const size_t si = slot_index(g, l, s, t);
+    const float acc = (t == 0) ? 0.f : state[si];
+    const float h0 = taps[((size_t)(l - 1) * g.D + d) * g.L];
+    y = fmaf(h0, a, acc);
+    if (l < g.M) {
+      a = round_act(tanhf(y), g.bf16);
+      state[si] = a;
+    }
+  }
+  y_t[io] = y;
+  if (eps_t && t + 1 < g.L) state[slot_index(g, 0, s, t + 1)] = round_act(tanhf(y) + eps_scale * eps_t[io], g.bf16);
+}
+
+cudaError_t launch_token(const Dims& g, float* state, const float* taps, int t, const void* x_t,
+                         const float* eps_t, float eps_scale, float* y_t, cudaStream_t st) {
+  const int threads = 128;
+  k_token<<<(g.S + threads - 1) / threads, threads, 0, st>>>(g, state, taps, t, x_t, eps_t, eps_scale, y_t);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Direct block of step i, side U = lowbit(i) (the gray block of Algorithm 1 by
+// its definition, tau(a, [i-U, i-1], h, [i, i+U-1])): for every layer l and
+// stream s, slot(l, s, i+u') (+)= sum_{u<U} h^l[U+u'-u] * a^{l-1}[i-U+u].
+// One CTA per (layer, channel, sequence); the 2U-1 taps and U sources are
+// staged in shared memory. The block at a power-of-two step is the first to
+// reach its targets and stores instead of adding.
+// ---------------------------------------------------------------------------
+__global__ void k_tile_direct(Dims g, float* __restrict__ state, const float* __restrict__ taps, int i, int U,
+                              int overwrite) {
+  extern __shared__ float dsm[];
+  float* hs = dsm;          // taps h[0..2U)
+  float* xs = dsm + 2 * U;  // sources a[i-U..i)
+  const long cta = blockIdx.x;          // ((l-1)*D + d)*B + b
+  const int b = (int)(cta % g.B);
+  const long ld = cta / g.B;
+  const int d = (int)(ld % g.D);
+  const int l = (int)(ld / g.D) + 1;
+  const int s = d * g.B + b;
+  const float* hp = taps + ((size_t)(l - 1) * g.D + d) * g.L;
+  const float* xp = state + slot_index(g, l - 1, s, i - U);
+  for (int j = threadIdx.x; j < 2 * U; j += blockDim.x) hs[j] = hp[j];
+  for (int j = threadIdx.x; j < U; j += blockDim.x) xs[j] = xp[j];
+  __syncthreads();
+  float* dp = state + slot_index(g, l, s, i);
+  for (int up = threadIdx.x; up < U; up += blockDim.x) {
+    float sum = 0.f;
+    for (int u = 0; u < U; ++u) sum = fmaf(hs[U + up - u], xs[u], sum);
+    dp[up] = overwrite ? sum : dp[up] + sum;
+  }
+}
+
+cudaError_t launch_tile_direct(const Dims& g, float* state, const float* taps, int i, cudaStream_t st) {
+  const int U = i & -i;
+  const size_t smem = (size_t)3 * U * sizeof(float);
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(k_tile_direct, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  const long blocks = (long)g.M * g.D * g.B;
+  const int threads = U >= 256 ? 256 : (U < 32 ? 32 : U);
+  k_tile_direct<<<(unsigned)blocks, threads, smem, st>>>(g, state, taps, i, U, is_pow2(i) ? 1 : 0);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// The Lazy method's sum for position t (summary page, "Tre Strategie di
+// Calcolo", Metodo Lazy), all layers in one launch: slot(l, s, t) =
+// sum_{s' < t} h^l[t-s'] a^{l-1}[s']. One warp per (layer, channel, group of up
+// to 4 sequences), so each tap is read once per group.
+// ---------------------------------------------------------------------------
+__global__ void k_lazy(Dims g, float* __restrict__ state, const float* __restrict__ taps, int t) {
+  const long warp = ((long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  const int nbg = (g.B + 3) / 4;
+  if (warp >= (long)g.M * g.D * nbg) return;
+  const int bg = (int)(warp % nbg);
+  const long ld = warp / nbg;
+  const int d = (int)(ld % g.D);
+  const int l = (int)(ld / g.D) + 1;
+  const int b0 = bg * 4, nb = min(4, g.B - b0);
+  const float* hp = taps + ((size_t)(l - 1) * g.D + d) * g.L;
+  const float* xp[4];
+  for (int j = 0; j < 4; ++j) xp[j] = state + slot_index(g, l - 1, d * g.B + b0 + min(j, nb - 1), 0);
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int sp = lane; sp < t; sp += 32) {
+    const float h = hp[t - sp];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[j] = fmaf(h, xp[j][sp], acc[j]);
+  }
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+    for (int o = 16; o > 0; o >>= 1) acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], o);
+  if (lane < nb) {
+    float v = acc[0];
+#pragma unroll
+    for (int j = 1; j < 4; ++j) v = (lane == j) ? acc[j] : v;
+    state[slot_index(g, l, d * g.B + b0 + lane, t)] = v;
+  }
+}
+
+cudaError_t launch_lazy_sums(const Dims& g, float* state, const float* taps, int t, cudaStream_t st) {
+  const long warps = (long)g.M * g.D * ((g.B + 3) / 4);
+  const int threads = 256;
+  const long blocks = (warps * 32 + threads - 1) / threads;
+  k_lazy<<<(unsigned)blocks, threads, 0, st>>>(g, state, taps, t);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Layout conversions.
+// ---------------------------------------------------------------------------
+__global__ void k_widen(const void* __restrict__ h, int bf16, size_t n, float* __restrict__ out) {
+  for (size_t k = (size_t)blockIdx.x * blockDim.x + threadIdx.x; k < n; k += (size_t)gridDim.x * blockDim.x)
+    out[k] = load_token(h, k, bf16);
+}
+
+cudaError_t launch_widen_filters(const void* h, int bf16, size_t n, float* out, cudaStream_t st) {
+  k_widen<<<148 * 8, 256, 0, st>>>(h, bf16, n, out);
+  return cudaGetLastError();
+}
+
+// dst[t][b][d] = slot(layer, d*B+b, t) for t < pos.
+__global__ void k_read_layer(Dims g, const float* __restrict__ state, int layer, int pos, float* __restrict__ dst) {
+  const size_t total = (size_t)pos * g.S;
+  for (size_t k = (size_t)blockIdx.x * blockDim.x + threadIdx.x; k < total; k += (size_t)gridDim.x * blockDim.x) {
+    const int t = (int)(k / g.S);
+    const int r = (int)(k - (size_t)t * g.S);  // r = b*D + d
+    const int b = r / g.D, d = r - b * g.D;
+    dst[k] = state[slot_index(g, layer, d * g.B + b, t)];
+  }
+}
+
+cudaError_t launch_read_layer(const Dims& g, const float* state, int layer, int pos, float* dst, cudaStream_t st) {
+  if (pos == 0) return cudaSuccess;
+  k_read_layer<<<148 * 8, 256, 0, st>>>(g, state, layer, pos, dst);
+  return cudaGetLastError();
+}
+
+}  // namespace fi

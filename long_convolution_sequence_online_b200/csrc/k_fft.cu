@@ -1,0 +1,233 @@
+// FFT blocks (Lemma 1 and the circular-convolution trick of the Flash Inference
+// summary page, "Punti di Innovazione Tecnica" 3) and the filter spectra
+// ("Precomputazione FFT").
+//
+// A block of side U at step i adds sum_{s in [i-U, i)} h[t-s] a[s] to every
+// target t in [i, i+U). With xx = [a[i-U..i) || 0_U] and hh = h[0..2U), the
+// length-2U circular convolution xx (*) hh equals that sum at indices [U, 2U),
+// so one real FFT of length 2U, a product with the precomputed spectrum of
+// h[0..2U) and one inverse real FFT give the block.
+//
+// Real FFTs of length 2N (N = U) run as complex FFTs of N points on
+// z[m] = x[2m] + i x[2m+1], followed by the usual split:
+//   E[k] = (Z[k] + conj Z[N-k]) / 2,  O[k] = -i (Z[k] - conj Z[N-k]) / 2,
+//   X[k] = E[k] + W_{2N}^k O[k],      X[N-k] = conj(E[k] - W_{2N}^k O[k]).
+// The inverse packs Y = X * H back into N points,
+//   Z'[k] = (Y[k] + conj Y[N-k]) + i (Y[k] - conj Y[N-k]) conj(W_{2N}^k),
+// whose inverse complex FFT carries 2N * (y[2m] + i y[2m+1]); the 1/(2N) is
+// folded into the stored spectrum. Zero padding means z[m] = 0 for m >= N/2,
+// and only y[N..2N) (m >= N/2) is kept.
+#include "fi_internal.cuh"
+#include "fft.cuh"
+
+namespace fi {
+
+// Spectrum split + product + inverse pack, in place on sm (N complex points).
+// H: N+1 spectrum values. Threads [0, T) of the transform.
+template <int N, int T>
+__device__ __forceinline__ void spectral_product(float2* sm, int tid, const float2* __restrict__ H,
+                                                 const float2* __restrict__ tw) {
+  constexpr int twstep = kTwiddleN / (2 * N);
+  for (int k = tid; k <= N / 2; k += T) {
+    const int kk = (N - k) & (N - 1);
+    const float2 zk = sm[fft_pad(k)], zn = sm[fft_pad(kk)];
+    const float2 E = make_float2(0.5f * (zk.x + zn.x), 0.5f * (zk.y - zn.y));
+    const float2 O = make_float2(0.5f * (zk.y + zn.y), -0.5f * (zk.x - zn.x));
+    const float2 W = __ldg(tw + k * twstep);
+    const float2 WO = cmul(W, O);
+    const float2 Xk = cadd(E, WO);
+    const float2 Xn = cconj(csub(E, WO));
+    const float2 Yk = cmul(Xk, __ldg(H + k));
+    const float2 Yn = cmul(Xn, __ldg(H + (N - k)));
+    const float2 A = cadd(Yk, cconj(Yn));
+    const float2 Bv = cmul(csub(Yk, cconj(Yn)), cconj(W));
+    sm[fft_pad(k)] = make_float2(A.x - Bv.y, A.y + Bv.x);
+    if (k != 0 && k != N / 2) sm[fft_pad(N - k)] = make_float2(A.x + Bv.y, -A.y + Bv.x);
+  }
+}
+
+// One FFT block for every (layer, stream): item = (l-1)*S + s.
+template <int N>
+__global__ void __launch_bounds__(fft_threads(N) * fft_per_cta(N))
+k_tile_fft(Dims g, float* __restrict__ state, const float2* __restrict__ spec,
+           const float2* __restrict__ tw, int i, int overwrite) {
+  constexpr int T = fft_threads(N), F = fft_per_cta(N);
+  extern __shared__ float2 fsm[];
+  const int sub = threadIdx.x / T, tid = threadIdx.x - sub * T;
+  float2* sm = fsm + sub * fft_smem_elems(N);
+  const long item = (long)blockIdx.x * F + sub;
+  const long items = (long)g.M * g.S;
+  const bool active = item < items;
+  const int l = active ? (int)(item / g.S) + 1 : 1;
+  const int s = active ? (int)(item % g.S) : 0;
+  const int d = s / g.B;
+  const float2* src = reinterpret_cast<const float2*>(state + slot_index(g, l - 1, s, i - N));
+  float2* dst = reinterpret_cast<float2*>(state + slot_index(g, l, s, i));
+  const float2* H = spec + ((size_t)(l - 1) * g.D + d) * (N + 1);
+
+  for (int m = tid; m < N; m += T) sm[fft_pad(m)] = (active && m < N / 2) ? src[m] : make_float2(0.f, 0.f);
+  if (T == 32) __syncwarp(); else __syncthreads();
+  if constexpr (T == 32) {
+    fft_smem<N, T, false>(sm, tid, tw, SyncWarp());
+    spectral_product<N, T>(sm, tid, H, tw);
+    __syncwarp();
+    fft_smem<N, T, true>(sm, tid, tw, SyncWarp());
+  } else {
+    fft_smem<N, T, false>(sm, tid, tw, SyncBlock());
+    spectral_product<N, T>(sm, tid, H, tw);
+    __syncthreads();
+    fft_smem<N, T, true>(sm, tid, tw, SyncBlock());
+  }
+  if (!active) return;
+  for (int j = tid; j < N / 2; j += T) {
+    const float2 v = sm[fft_pad(N / 2 + j)];
+    if (overwrite) {
+      dst[j] = v;
+    } else {
+      const float2 o = dst[j];
+      dst[j] = make_float2(o.x + v.x, o.y + v.y);
+    }
+  }
+}
+
+// Spectrum of h[0..2N) / (2N) for one (layer, channel): item = l*D + d.
+template <int N>
+__global__ void __launch_bounds__(fft_threads(N) * fft_per_cta(N))
+k_spectra(Dims g, const float* __restrict__ taps, float2* __restrict__ spec, const float2* __restrict__ tw) {
+  constexpr int T = fft_threads(N), F = fft_per_cta(N);
+  constexpr int twstep = kTwiddleN / (2 * N);
+  extern __shared__ float2 fsm[];
+  const int sub = threadIdx.x / T, tid = threadIdx.x - sub * T;
+  float2* sm = fsm + sub * fft_smem_elems(N);
+  const long item = (long)blockIdx.x * F + sub;
+  const bool active = item < (long)g.M * g.D;
+  const float2* src = reinterpret_cast<const float2*>(taps + (size_t)(active ? item : 0) * g.L);
+  for (int m = tid; m < N; m += T) sm[fft_pad(m)] = active ? src[m] : make_float2(0.f, 0.f);
+  if constexpr (T == 32) {
+    __syncwarp();
+    fft_smem<N, T, false>(sm, tid, tw, SyncWarp());
+  } else {
+    __syncthreads();
+    fft_smem<N, T, false>(sm, tid, tw, SyncBlock());
+  }
+  if (!active) return;
+  float2* H = spec + (size_t)item * (N + 1);
+  const float scale = 1.0f / (2.0f * N);
+  for (int k = tid; k <= N / 2; k += T) {
+    const int kk = (N - k) & (N - 1);
+    const float2 zk = sm[fft_pad(k)], zn = sm[fft_pad(kk)];
+    const float2 E = make_float2(0.5f * (zk.x + zn.x), 0.5f * (zk.y - zn.y));
+    const float2 O = make_float2(0.5f * (zk.y + zn.y), -0.5f * (zk.x - zn.x));
+    const float2 WO = cmul(__ldg(tw + k * twstep), O);
+    H[k] = cscale(cadd(E, WO), scale);
+    if (k != N / 2) H[N - k] = cscale(cconj(csub(E, WO)), scale);
+  }
+}
+
+template <int N>
+__global__ void __launch_bounds__(fft_threads(N) * fft_per_cta(N))
+k_debug_fft(int count, const float2* __restrict__ in, float2* __restrict__ out, int inverse,
+            const float2* __restrict__ tw) {
+  constexpr int T = fft_threads(N), F = fft_per_cta(N);
+  extern __shared__ float2 fsm[];
+  const int sub = threadIdx.x / T, tid = threadIdx.x - sub * T;
+  float2* sm = fsm + sub * fft_smem_elems(N);
+  const long item = (long)blockIdx.x * F + sub;
+  const bool active = item < count;
+  for (int m = tid; m < N; m += T) sm[fft_pad(m)] = active ? in[item * N + m] : make_float2(0.f, 0.f);
+  if constexpr (T == 32) {
+    __syncwarp();
+    if (inverse) fft_smem<N, T, true>(sm, tid, tw, SyncWarp());
+    else fft_smem<N, T, false>(sm, tid, tw, SyncWarp());
+  } else {
+    __syncthreads();
+    if (inverse) fft_smem<N, T, true>(sm, tid, tw, SyncBlock());
+    else fft_smem<N, T, false>(sm, tid, tw, SyncBlock());
+  }
+  if (!active) return;
+  for (int m = tid; m < N; m += T) out[item * N + m] = sm[fft_pad(m)];
+}
+
+// ------------------------------------------------------------------ dispatch
+template <int N>
+static size_t fft_smem_bytes() { return (size_t)fft_per_cta(N) * fft_smem_elems(N) * sizeof(float2); }
+
+template <class K>
+static cudaError_t prepare(K kernel, size_t smem) {
+  if (smem > 48 * 1024) return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  return cudaSuccess;
+}
+
+template <int N>
+static cudaError_t tile_fft_n(const Dims& g, float* state, const float2* spec, const float2* tw, int i,
+                              cudaStream_t st) {
+  const size_t smem = fft_smem_bytes<N>();
+  cudaError_t e = prepare(k_tile_fft<N>, smem);
+  if (e != cudaSuccess) return e;
+  const long items = (long)g.M * g.S;
+  const long blocks = (items + fft_per_cta(N) - 1) / fft_per_cta(N);
+  const int overwrite = is_pow2(i) ? 1 : 0;
+  k_tile_fft<N><<<(unsigned)blocks, fft_threads(N) * fft_per_cta(N), smem, st>>>(g, state, spec, tw, i, overwrite);
+  return cudaGetLastError();
+}
+
+template <int N>
+static cudaError_t spectra_n(const Dims& g, const float* taps, float2* spec, const float2* tw, cudaStream_t st) {
+  const size_t smem = fft_smem_bytes<N>();
+  cudaError_t e = prepare(k_spectra<N>, smem);
+  if (e != cudaSuccess) return e;
+  const long items = (long)g.M * g.D;
+  const long blocks = (items + fft_per_cta(N) - 1) / fft_per_cta(N);
+  k_spectra<N><<<(unsigned)blocks, fft_threads(N) * fft_per_cta(N), smem, st>>>(g, taps, spec, tw);
+  return cudaGetLastError();
+}
+
+template <int N>
+static cudaError_t debug_fft_n(int count, const float2* in, float2* out, int inverse, const float2* tw,
+                               cudaStream_t st) {
+  const size_t smem = fft_smem_bytes<N>();
+  cudaError_t e = prepare(k_debug_fft<N>, smem);
+  if (e != cudaSuccess) return e;
+  const long blocks = ((long)count + fft_per_cta(N) - 1) / fft_per_cta(N);
+  k_debug_fft<N><<<(unsigned)blocks, fft_threads(N) * fft_per_cta(N), smem, st>>>(count, in, out, inverse, tw);
+  return cudaGetLastError();
+}
+
+#define FI_FFT_SWITCH(q, CALL)            \
+  switch (q) {                            \
+    case 6: return CALL(64);              \
+    case 7: return CALL(128);             \
+    case 8: return CALL(256);             \
+    case 9: return CALL(512);             \
+    case 10: return CALL(1024);           \
+    case 11: return CALL(2048);           \
+    case 12: return CALL(4096);           \
+    case 13: return CALL(8192);           \
+    case 14: return CALL(16384);          \
+    default: return cudaErrorInvalidValue; \
+  }
+
+cudaError_t launch_tile_fft(const Dims& g, float* state, const float2* spectrum_q, const float2* twiddle, int i,
+                            cudaStream_t st) {
+  const int U = i & -i;
+  const int q = ilog2((uint32_t)U);
+#define CALL(n) tile_fft_n<n>(g, state, spectrum_q, twiddle, i, st)
+  FI_FFT_SWITCH(q, CALL)
+#undef CALL
+}
+
+cudaError_t launch_spectra(const Dims& g, const float* taps, float2* spectrum_q, const float2* twiddle, int q,
+                           cudaStream_t st) {
+#define CALL(n) spectra_n<n>(g, taps, spectrum_q, twiddle, st)
+  FI_FFT_SWITCH(q, CALL)
+#undef CALL
+}
+
+cudaError_t launch_debug_fft(int log2n, int count, const float2* in, float2* out, int inverse,
+                             const float2* twiddle, cudaStream_t st) {
+#define CALL(n) debug_fft_n<n>(count, in, out, inverse, twiddle, st)
+  FI_FFT_SWITCH(log2n, CALL)
+#undef CALL
+}
+
+}  // namespace fi

@@ -1,0 +1,98 @@
+"""The C-ABI library loads on a machine without a GPU, exports every symbol that
+include/fi.h declares, and rejects bad arguments before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fi.h")
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"FI_API\s+[\w\s\*]+?\b(fi_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_symbols()
+    for must in ("fi_init", "fi_step", "fi_generate", "fi_reset", "fi_destroy"):
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol():
+    from long_convolution_sequence_online_b200 import fi
+    lib = ctypes.CDLL(fi.LIB_PATH)
+    missing = [n for n in declared_symbols() if not hasattr(lib, n)]
+    assert not missing, missing
+    assert sorted(fi.EXPORTED) == declared_symbols()
+
+
+def test_status_strings():
+    from long_convolution_sequence_online_b200 import fi
+    assert fi.status_str(0) == "ok"
+    assert fi.status_str(fi.FI_E_STATE) == "invalid state"
+    assert fi.status_str(99) == "unknown status"
+
+
+def _init(cfg, h=ctypes.c_void_p(16)):
+    from long_convolution_sequence_online_b200 import fi
+    out = ctypes.c_void_p(1)
+    s = fi.lib.fi_init(ctypes.byref(out), ctypes.byref(cfg), h, None)
+    return s, out
+
+
+@pytest.mark.parametrize("fields,why", [
+    (dict(layers=0, channels=4, max_len=64, batch=1), "layers"),
+    (dict(layers=1, channels=0, max_len=64, batch=1), "channels"),
+    (dict(layers=1, channels=4, max_len=48, batch=1), "power of two"),
+    (dict(layers=1, channels=4, max_len=1, batch=1), "power of two"),
+    (dict(layers=1, channels=4, max_len=1 << 18, batch=1), "power of two"),
+    (dict(layers=1, channels=4, max_len=64, batch=0), "batch"),
+    (dict(layers=1, channels=4, max_len=64, batch=1, dtype=7), "dtype"),
+    (dict(layers=1, channels=4, max_len=64, batch=1, chunk=3), "chunk"),
+    (dict(layers=1, channels=4, max_len=64, batch=1, chunk=128), "chunk"),
+    (dict(layers=1, channels=4, max_len=64, batch=1, fft_from=32), "fft_from"),
+])
+def test_init_rejects_bad_config_without_gpu(fields, why):
+    from long_convolution_sequence_online_b200 import fi
+    cfg = fi.Config(**fields)
+    s, out = _init(cfg)
+    assert s == fi.FI_E_INVALID
+    assert out.value is None
+    assert why in fi.lib.fi_last_error().decode()
+
+
+def test_init_rejects_reserved_and_nulls():
+    from long_convolution_sequence_online_b200 import fi
+    cfg = fi.Config(1, 4, 64, 1)
+    cfg.reserved[2] = 1
+    assert _init(cfg)[0] == fi.FI_E_INVALID
+    cfg = fi.Config(1, 4, 64, 1)
+    assert _init(cfg, h=None)[0] == fi.FI_E_INVALID
+    assert fi.lib.fi_init(None, ctypes.byref(cfg), ctypes.c_void_p(16), None) == fi.FI_E_INVALID
+
+
+def test_calls_on_null_context_are_rejected():
+    from long_convolution_sequence_online_b200 import fi
+    L = fi.lib
+    assert L.fi_destroy(None) == fi.FI_OK
+    assert L.fi_reset(None) == fi.FI_E_INVALID
+    assert L.fi_step(None, None, None) == fi.FI_E_INVALID
+    assert L.fi_generate(None, 4, None, None, 0.1, None, None) == fi.FI_E_INVALID
+    assert L.fi_generate_lazy(None, 4, None, None, 0.1, None) == fi.FI_E_INVALID
+    assert L.fi_generate_host(None, 4, None, None, 0.1, None) == fi.FI_E_INVALID
+    p = ctypes.c_int32()
+    assert L.fi_position(None, ctypes.byref(p)) == fi.FI_E_INVALID
+    assert L.fi_read_activations(None, 0, None) == fi.FI_E_INVALID
+    assert L.fi_profile(None, 1) == fi.FI_E_INVALID
+    assert L.fi_debug_fft(5, 1, ctypes.c_void_p(16), ctypes.c_void_p(16), 0, None) == fi.FI_E_INVALID
+    assert L.fi_debug_fft(15, 1, ctypes.c_void_p(16), ctypes.c_void_p(16), 0, None) == fi.FI_E_INVALID
+
+
+def test_python_binding_refuses_cpu_tensors():
+    torch = pytest.importorskip("torch")
+    from long_convolution_sequence_online_b200 import fi
+    with pytest.raises(ValueError):
+        fi._ptr(torch.zeros(4))
