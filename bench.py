@@ -1,0 +1,524 @@
+"""Benchmark: mixer tokens/s of exact online long convolution on B200.
+
+One step = one closed-loop generation of the whole sequence (fi_reset, then
+fi_generate over L positions) for the 18-layer x 864-channel, L = 32768, B = 4
+fp32 workload; tokens per step = B * L. Inputs (filters, first token, noise)
+are resident in HBM before timing; the state the step streams through (8.6 GB)
+is far larger than L2, so no flush is needed between steps.
+
+Also reported: the dominant kernel's roofline (from CUDA events recorded around
+every launch during the timed steps), the whole-run roofline of the schedule's
+algorithmic bytes and flops, end-to-end throughput through fi_generate_host
+(host buffers, copies inside the timed region), the quadratic Lazy baseline on
+the GPU (extrapolated from a measured prefix), and the float64 oracle on the
+host cores (a bounded sample, extrapolated).
+
+python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--workload NAME]
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import multiprocessing as mp
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "mixer tokens/s at 18x864, L=32K on 1 B200"
+UNIT = "tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+NOMINAL_HBM_GBS = 8000.0            # the HBM figure the roofline target is quoted against
+FP32_LANES_PER_SM = 128
+NUM_SMS = 148
+L2_BYTES = 126 * 1024 * 1024
+
+
+# ----------------------------------------------------------------------------- cost model
+def schedule_levels(L: int):
+    """(U, count): blocks of side U = 2^q occur 2^(P-1-q) times per layer and stream."""
+    P = int(math.log2(L))
+    return [(1 << q, 1 << (P - 1 - q)) for q in range(P)]
+
+
+def fft_flops(U: int) -> float:
+    """Model flops of one FFT block per stream: two real FFTs of length 2U plus the product."""
+    return 2 * 2.5 * (2 * U) * math.log2(2 * U) + 7 * U
+
+
+def cost_model(w: synth.Workload, chunk: int, fft_from: int, fft_max: int = 1 << 14):
+    """Algorithmic bytes and flops of one full generation, split by kernel class.
+
+    Bytes (compulsory HBM traffic of the schedule): per block of side U and (layer,
+    channel) the taps (2U-1)*s_h (direct) or the spectrum (U+1)*8 (FFT); per (layer,
+    sequence, channel) the U sources (s_x each) and the accumulator read-modify-write
+    (2U*4); per position and (layer, sequence, channel) the accumulator row (4) and
+    the activation write (s_x); per position and (sequence, channel) token, noise and
+    output (s_x + 4 + 4). Flops: direct block 2U^2, FFT block fft_flops(U), red cell 3.
+    """
+    M, D, L, B = w.layers, w.channels, w.length, w.batch
+    s = 2 if w.dtype == "bf16" else 4
+    out = {k: {"bytes": 0.0, "flops": 0.0, "blocks": 0} for k in ("chunk", "direct", "fft")}
+    for U, n in schedule_levels(L):
+        if U < chunk:
+            cls = "chunk"
+        elif fft_from <= U <= fft_max:
+            cls = "fft"
+        else:
+            cls = "direct"
+        per_ld = (U + 1) * 8 if cls == "fft" else (2 * U - 1) * s
+        per_lbd = U * s + 2 * U * 4
+        out[cls]["bytes"] += n * (M * D * per_ld + M * B * D * per_lbd)
+        out[cls]["flops"] += n * M * B * D * (fft_flops(U) if cls == "fft" else 2.0 * U * U)
+        out[cls]["blocks"] += n
+    out["chunk"]["bytes"] += L * (M * B * D * (4 + s) + B * D * (s + 8))
+    out["chunk"]["flops"] += L * M * B * D * 3.0
+    tot = {"bytes": sum(v["bytes"] for v in out.values()), "flops": sum(v["flops"] for v in out.values())}
+    return out, tot
+
+
+def survey_closed_form_bytes(w: synth.Workload) -> float:
+    """The schedule's block bytes in closed form, M*D*(L/2)*log2(L)*(8 + B(s_x+8))."""
+    s = 2 if w.dtype == "bf16" else 4
+    return w.layers * w.channels * (w.length / 2) * math.log2(w.length) * (8 + w.batch * (s + 8))
+
+
+def lazy_bytes(w: synth.Workload) -> float:
+    """HBM bytes of the Lazy method: every position re-reads its whole history and taps."""
+    s = 2 if w.dtype == "bf16" else 4
+    pairs = w.length * (w.length - 1) / 2
+    return pairs * w.layers * w.channels * (w.batch * s + s)
+
+
+# ----------------------------------------------------------------------------- peaks and clocks
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "sm_max_mhz": float(p.get("sm_max_mhz", 1965.0)), "source": "measured"}
+    except Exception:
+        return dict(FALLBACK_PEAKS, sm_max_mhz=1965.0, source="fallback")
+
+
+def fp32_peak_tflops(mhz: float) -> float:
+    return NUM_SMS * FP32_LANES_PER_SM * 2 * mhz * 1e6 / 1e12
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms while running."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            import tempfile
+            fd, self.path = tempfile.mkstemp(prefix="clocks", suffix=".csv")
+            os.close(fd)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.fh, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.fh.close()
+
+    def summary(self):
+        if self.proc is None or not self.path:
+            return None
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append((float(parts[1]), float(parts[2]), float(parts[3]), parts[5:9]))
+                except ValueError:
+                    continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [r[0] for r in rows]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[k] for r in rows for k, v in enumerate(r[3]) if v.lower() == "active"})
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": max(r[1] for r in rows),
+                "power_w_max": max(r[2] for r in rows), "samples": len(rows), "reasons": reasons}
+
+
+# ----------------------------------------------------------------------------- distributed plumbing
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", str(rank)))
+    return world, rank, local
+
+
+def dist_init(world: int, backend: str):
+    if world <= 1:
+        return False
+    import torch.distributed as dist
+    os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+    dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return True
+
+
+def rank_seed(seed: int, rank: int) -> int:
+    """Each rank draws an independent batch of the same workload (weak scaling)."""
+    return seed + 1000003 * rank
+
+
+def reduce_max(value: float, device=None) -> float:
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(device=None):
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        if device is not None:
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+# ----------------------------------------------------------------------------- oracle on the host
+def _oracle_job(args):
+    """Run the float64 oracle on a stream subset for the first n positions (test infra)."""
+    name, seed, streams, n = args
+    import oracle
+    w = synth.WORKLOADS[name]
+    lam = synth.decay_rates(w, seed)
+    chans = sorted({d for (_, d) in streams})
+    h = np.empty((w.layers, len(streams), w.length))
+    for l in range(w.layers):
+        hl = synth.filter_layer(w, seed, l, lam, np.array(chans))
+        for j, (_, d) in enumerate(streams):
+            hl64 = hl[chans.index(d)].astype(np.float64)
+            h[l, j] = oracle.bf16_round(hl64) if w.dtype == "bf16" else hl64
+    x0 = synth.first_token(w, seed)
+    eps = synth.noise(w, seed, n)
+    x0s = np.array([x0[b, d] for (b, d) in streams], dtype=np.float64)
+    epss = np.stack([eps[:, b, d] for (b, d) in streams], axis=1)
+    t0 = time.perf_counter()
+    oracle.online_lcsm(h, x0s, epss, 0.1, w.dtype == "bf16", n=n)
+    return time.perf_counter() - t0
+
+
+def oracle_baseline(w: synth.Workload, seed: int, n_pos: int, streams_per_core: int, cores: int | None = None):
+    """Time the oracle on `cores` processes x streams_per_core streams x n_pos positions,
+    then extrapolate to the whole workload by its O(L^2) cost (work ~ streams * n^2)."""
+    cores = cores or os.cpu_count() or 1
+    rng = np.random.default_rng(seed + 17)
+    jobs = []
+    for c in range(cores):
+        st = [(int(rng.integers(w.batch)), int(rng.integers(w.channels))) for _ in range(streams_per_core)]
+        jobs.append((w.name, seed, st, n_pos))
+    ctx = mp.get_context("spawn")
+    t0 = time.perf_counter()
+    with ctx.Pool(cores) as pool:
+        per = pool.map(_oracle_job, jobs)
+    wall = time.perf_counter() - t0
+    compute = max(per)
+    sample_streams = cores * streams_per_core
+    work_sample = sample_streams * n_pos * (n_pos + 1) / 2
+    work_full = w.streams * w.length * (w.length + 1) / 2
+    t_full = compute * work_full / work_sample
+    return {
+        "value": w.batch * w.length / t_full,
+        "unit": UNIT,
+        "cores": cores,
+        "kind": "oracle",
+        "sample": (f"float64 oracle, all {w.layers} layers, {sample_streams} (sequence, channel) streams x first "
+                   f"{n_pos} positions ({cores} spawned processes, {compute:.1f} s compute, {wall:.1f} s wall); "
+                   f"extrapolated by streams x n^2 to {w.streams} streams x {w.length} positions"),
+        "extrapolated": True,
+        "seconds_sample": compute,
+    }
+
+
+# ----------------------------------------------------------------------------- GPU arm
+def source_sha(paths):
+    h = hashlib.sha256()
+    for p in paths:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+KERNEL_SOURCES = {
+    "chunk": ["long_convolution_sequence_online_b200/csrc/k_chunk.cu"],
+    "fft": ["long_convolution_sequence_online_b200/csrc/k_fft.cu", "long_convolution_sequence_online_b200/csrc/fft.cuh"],
+    "direct": ["long_convolution_sequence_online_b200/csrc/k_basic.cu"],
+}
+
+
+def ncu_traffic(cls: str, workload: str):
+    """Per-launch DRAM bytes of a kernel class from the committed ncu summary, if still current."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+        e = rec[cls]
+        if e.get("source_sha") != source_sha(KERNEL_SOURCES[cls]) or e.get("workload") != workload:
+            return None
+        return float(e["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+def gpu_arm(args, world, rank, local):
+    import torch
+    from long_convolution_sequence_online_b200 import fi
+
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    w = synth.WORKLOADS[args.workload]
+    seed = rank_seed(args.seed, rank)
+    h = synth.filters(w, seed)
+    x0 = synth.first_token(w, seed)
+    eps = synth.noise(w, seed)
+    td = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    h_d = torch.from_numpy(h).to(device).to(td)
+    x0_d = torch.from_numpy(x0).to(device).to(td).contiguous()
+    eps_d = torch.from_numpy(eps).to(device)
+    y_d = torch.empty((w.length, w.batch, w.channels), dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream(device)
+    t_init = time.perf_counter()
+    ctx = fi.Context(h_d, w.batch, w.dtype, chunk=args.chunk, fft_from=args.fft_from, stream=stream)
+    t_init = time.perf_counter() - t_init
+    del h_d
+    chunk, fft_from = ctx.plan()
+
+    def step():
+        ctx.reset()
+        ctx.generate(w.length, x0_d, eps_d, y_d, 0.1)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(device)
+
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    ctx.profile(True)
+    ctx.profile_read()
+    with ClockSampler(local) as clocks:
+        barrier(device)
+        torch.cuda.synchronize(device)
+        for k in range(args.steps):
+            ev[k][0].record(stream)
+            step()
+            ev[k][1].record(stream)
+        torch.cuda.synchronize(device)
+        barrier(device)
+    prof = ctx.profile_read()
+    ctx.profile(False)
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    total_ms = reduce_max(float(sum(step_ms)), device)
+    ms_per_step = total_ms / args.steps
+    tokens_per_step = w.batch * w.length
+    value = world * tokens_per_step * args.steps / (total_ms / 1e3)
+
+    # --- end to end: host buffers through the C-ABI call, copies inside the timed region
+    x0_h = torch.from_numpy(x0.astype(np.float32) if w.dtype == "f32" else x0).to(td).pin_memory()
+    eps_h = torch.from_numpy(eps).pin_memory()
+    y_h = torch.empty((w.length, w.batch, w.channels), dtype=torch.float32).pin_memory()
+
+    def e2e_step():
+        ctx.reset()
+        ctx.generate_host_ptr(w.length, x0_h.data_ptr(), eps_h.data_ptr(), y_h.data_ptr(), 0.1)
+
+    e2e = None
+    if args.e2e_steps > 0:
+        e2e_step()
+        barrier(device)
+        t0 = time.perf_counter()
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        e2e_s = reduce_max(time.perf_counter() - t0, device)
+        e2e = {"value": world * tokens_per_step * args.e2e_steps / e2e_s, "unit": UNIT,
+               "h2d_bytes_per_step": int(x0_h.numel() * x0_h.element_size() + eps_h.numel() * 4),
+               "d2h_bytes_per_step": int(y_h.numel() * 4),
+               "timing": "host wall clock around fi_generate_host (synchronous), max over ranks"}
+
+    # --- roofline: dominant kernel class during the timed steps
+    peaks = measured_peaks()
+    clk = clocks.summary()
+    model, tot = cost_model(w, chunk, fft_from)
+    classes = {}
+    for cls in ("chunk", "direct", "fft"):
+        n, ms = prof[cls]
+        if n == 0:
+            continue
+        secs = ms / 1e3
+        byt = model[cls]["bytes"] * args.steps
+        flo = model[cls]["flops"] * args.steps
+        classes[cls] = {"launches": n, "ms": ms, "avg_launch_us": 1e3 * ms / n, "bytes": byt, "flops": flo,
+                        "gbs": byt / secs / 1e9, "tflops": flo / secs / 1e12}
+    dom = max(classes, key=lambda k: classes[k]["ms"])
+    d = classes[dom]
+    mhz = peaks["sm_max_mhz"]
+    fp32_peak = fp32_peak_tflops(mhz)
+    t_mem = d["bytes"] / (peaks["hbm_gbs"] * 1e9)
+    t_alu = d["flops"] / (fp32_peak * 1e12)
+    per_launch_bytes = d["bytes"] / d["launches"]
+    traffic = ncu_traffic(dom, w.name)
+    if t_mem >= t_alu:
+        roof = {"bound": "hbm", "achieved": d["gbs"], "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": d["gbs"] / peaks["hbm_gbs"]}
+    else:
+        roof = {"bound": "alu", "achieved": d["tflops"], "peak": fp32_peak, "unit": "TFLOP/s",
+                "frac": d["tflops"] / fp32_peak}
+    roof.update({"traffic": traffic, "kernel": dom, "peak_source": peaks["source"],
+                 "algorithmic_bytes_per_launch": per_launch_bytes, "avg_launch_us": d["avg_launch_us"],
+                 "launches": d["launches"]})
+    # whole-run roofline of the schedule (bytes at HBM bandwidth vs flops at the FP32 peak)
+    run_s = ms_per_step / 1e3
+    t_roof_meas = max(tot["bytes"] / (peaks["hbm_gbs"] * 1e9), tot["flops"] / (fp32_peak * 1e12))
+    t_roof_nom = max(tot["bytes"] / (NOMINAL_HBM_GBS * 1e9), tot["flops"] / (fp32_peak * 1e12))
+    step_roof = {"algorithmic_bytes": tot["bytes"], "algorithmic_flops": tot["flops"],
+                 "roofline_ms_measured_hbm": 1e3 * t_roof_meas, "frac_of_measured": t_roof_meas / run_s,
+                 "roofline_ms_8tbs": 1e3 * t_roof_nom, "frac_of_8tbs": t_roof_nom / run_s,
+                 "achieved_gbs": tot["bytes"] / run_s / 1e9, "fp32_peak_tflops": fp32_peak}
+
+    # --- quadratic Lazy baseline on the GPU: measured on two prefixes, extrapolated a*n + b*n^2/2
+    lazy = None
+    if args.lazy_prefix > 0 and rank == 0:
+        n1, n2 = args.lazy_prefix // 4, args.lazy_prefix
+        times = []
+        for n in (n1, n2):
+            ctx.reset()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            ctx.generate_lazy(n, x0_d, eps_d, y_d, 0.1)
+            e1.record(stream)
+            torch.cuda.synchronize(device)
+            times.append(e0.elapsed_time(e1) / 1e3)
+        A = np.array([[n1, n1 * n1 / 2], [n2, n2 * n2 / 2]])
+        a_, b_ = np.linalg.solve(A, np.array(times))
+        Lf = w.length
+        t_lazy = a_ * Lf + b_ * Lf * Lf / 2
+        lazy = {"seconds_extrapolated": t_lazy, "measured_prefixes": [n1, n2], "measured_s": times,
+                "speedup": t_lazy / run_s, "tokens_s": tokens_per_step / t_lazy,
+                "lazy_bytes": lazy_bytes(w), "achieved_gbs": lazy_bytes(w) / t_lazy / 1e9}
+        ctx.reset()
+    ctx.close()
+
+    launches_per_step = sum(prof[k][0] for k in prof) / args.steps
+    res = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32" if w.dtype == "f32" else "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "layers": w.layers, "channels": w.channels, "seq_len": w.length,
+                   "batch": w.batch, "global_batch": w.batch * world, "tokens_per_step": tokens_per_step,
+                   "parallelism": f"dp{world}" if world > 1 else "single",
+                   "plan": {"chunk": chunk, "fft_from": fft_from, "fft_max": 1 << 14},
+                   "l2": "inputs larger than L2 (state 8.6 GB streamed every step)",
+                   "step": "fi_reset + fi_generate over all L positions, closed loop",
+                   "init_s": t_init},
+        "roofline": roof,
+        "step_roofline": step_roof,
+        "kernels": classes,
+        "e2e": e2e,
+        "gpu_launches": int(round(launches_per_step * args.steps)),
+        "clocks": clk,
+        "speedup_vs_lazy": lazy,
+        "step_ms": step_ms,
+    }
+    return res
+
+
+# ----------------------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--workload", default=synth.HEADLINE, choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--chunk", type=int, default=0)
+    ap.add_argument("--fft-from", dest="fft_from", type=int, default=0)
+    ap.add_argument("--e2e-steps", dest="e2e_steps", type=int, default=3)
+    ap.add_argument("--lazy-prefix", dest="lazy_prefix", type=int, default=4096)
+    ap.add_argument("--oracle-positions", dest="oracle_positions", type=int, default=6144)
+    ap.add_argument("--oracle-streams", dest="oracle_streams", type=int, default=4)
+    ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
+    args = ap.parse_args()
+
+    world, rank, local = dist_env()
+    w = synth.WORKLOADS[args.workload]
+
+    if args.impl == "reference":
+        # The reference arm is the float64 oracle on the host cores (rank 0 only).
+        if rank != 0:
+            return
+        per = []
+        for k in range(args.warmup + args.steps):
+            r = oracle_baseline(w, args.seed + k, max(256, args.oracle_positions // 3), args.oracle_streams)
+            if k >= args.warmup:
+                per.append(r)
+        value = float(np.mean([r["value"] for r in per]))
+        t_step = w.batch * w.length / value
+        cpu = {k: per[-1][k] for k in ("unit", "cores", "kind", "sample")}
+        cpu["value"] = value
+        print(json.dumps({
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1e3 * t_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": w.name, "layers": w.layers, "channels": w.channels, "seq_len": w.length,
+                       "batch": w.batch, "step": "one bounded oracle sample per step, extrapolated"},
+            "cpu_baseline": cpu,
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        }))
+        return
+
+    dist_on = dist_init(world, "nccl")
+    try:
+        res = gpu_arm(args, world, rank, local)
+    finally:
+        if dist_on:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+    if rank == 0:
+        if args.cpu_baseline and world == 1:
+            res["cpu_baseline"] = oracle_baseline(w, args.seed, args.oracle_positions, args.oracle_streams)
+        else:
+            res["cpu_baseline"] = None
+        print(json.dumps(res))
+
+
+if __name__ == "__main__":
+    main()

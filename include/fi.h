@@ -25,8 +25,8 @@
  *   - fp32 buffers are 4-byte aligned, bf16 buffers 2-byte aligned.
  *   - Every call is asynchronous on the context's CUDA stream (the stream given
  *     to fi_init or fi_set_stream); buffers passed in must stay valid until the
- *     stream reaches that point. Only fi_init, fi_destroy, the *_host call and
- *     fi_profile_read synchronise.
+ *     stream reaches that point. Only fi_init, fi_destroy, fi_sync, the *_host
+ *     call and fi_profile_read synchronise.
  *   - Errors are returned as fi_status; no exception crosses this boundary.
  *     fi_last_error() gives a message for the last failing call on this thread.
  *     After FI_E_CUDA the context should be destroyed.
@@ -118,6 +118,12 @@ FI_API fi_status fi_generate_host(fi_ctx* ctx, int32_t n, const void* x0_host, c
  * quadratic baseline the relaxed schedule is measured against. */
 FI_API fi_status fi_generate_lazy(fi_ctx* ctx, int32_t n, const void* x0, const float* eps,
                            float eps_scale, float* y_out);
+
+/* Wait until every call issued on the context's stream has finished. Returns
+ * FI_E_TIMEOUT if a bounded device-side wait inside a kernel gave up since the
+ * last check (the results of those calls are then invalid; the flag is cleared).
+ * The kernels' internal waits are all bounded, so no call can hang the GPU. */
+FI_API fi_status fi_sync(fi_ctx* ctx);
 
 /* Rewind to position 0. O(1): no memory is cleared, because every accumulator
  * is first written (not added to) by the block that first reaches it. */

@@ -109,62 +109,139 @@ __device__ __forceinline__ void dft_reg(float2* v) {
 struct SyncWarp { __device__ __forceinline__ void operator()() const { __syncwarp(); } };
 struct SyncBlock { __device__ __forceinline__ void operator()() const { __syncthreads(); } };
 
-template <int N, int T, bool INV, int DONE, class Sync>
-struct FftPass {
+// v[r] *= w^r for r = 1..R-1 (w = W_{Ns R}^{kk}, forward sign; conjugated for the
+// inverse). w, w^4 and w^8 come from the table; the other powers are products of
+// at most three table values, so each carries a few roundings at most.
+template <int R, bool INV>
+__device__ __forceinline__ void apply_twiddles(float2* v, const float2* __restrict__ tw, int base) {
+  auto ld = [&](int r) {
+    float2 w = __ldg(tw + r * base);
+    if (INV) w.y = -w.y;
+    return w;
+  };
+  const float2 w1 = ld(1);
+  v[1] = cmul(v[1], w1);
+  if constexpr (R == 2) return;
+  const float2 w2 = cmul(w1, w1);
+  const float2 w3 = cmul(w2, w1);
+  v[2] = cmul(v[2], w2);
+  v[3] = cmul(v[3], w3);
+  if constexpr (R == 4) return;
+  const float2 w4 = ld(4);
+  v[4] = cmul(v[4], w4);
+  v[5] = cmul(v[5], cmul(w4, w1));
+  v[6] = cmul(v[6], cmul(w4, w2));
+  v[7] = cmul(v[7], cmul(w4, w3));
+  if constexpr (R == 8) return;
+  const float2 w8 = ld(8);
+  const float2 w12 = cmul(w8, w4);
+  v[8] = cmul(v[8], w8);
+  v[9] = cmul(v[9], cmul(w8, w1));
+  v[10] = cmul(v[10], cmul(w8, w2));
+  v[11] = cmul(v[11], cmul(w8, w3));
+  v[12] = cmul(v[12], w12);
+  v[13] = cmul(v[13], cmul(w12, w1));
+  v[14] = cmul(v[14], cmul(w12, w2));
+  v[15] = cmul(v[15], cmul(w12, w3));
+}
+
+// Shape of the transform: T threads, P = N/T points each, passes of radix
+// min(16, P) until the last pass takes what is left.
+template <int N, int T>
+struct FftShape {
   static constexpr int LOGN = clog2(N);
   static constexpr int P = N / T;
-  static constexpr int RB = cmin(cmin(4, clog2(P)), LOGN - DONE);
-  static constexpr int R = 1 << RB;
-  static constexpr int Ns = 1 << DONE;
+  static constexpr int RBMAX = cmin(4, clog2(P));
+  static constexpr int rb(int done) { return cmin(RBMAX, LOGN - done); }
+  static constexpr bool last(int done) { return done + rb(done) >= LOGN; }
+};
 
-  __device__ __forceinline__ static void run(float2* sm, int tid, const float2* __restrict__ tw, Sync sync) {
-    float2 v[P];
+// Twiddles and R-point DFTs of one pass on the P points a thread holds
+// (butterfly k in v[k*R .. k*R+R), butterfly index j = tid + k*T).
+template <int N, int T, bool INV, int DONE>
+__device__ __forceinline__ void pass_compute(float2* v, int tid, const float2* __restrict__ tw) {
+  using S = FftShape<N, T>;
+  constexpr int R = 1 << S::rb(DONE);
+  constexpr int Ns = 1 << DONE;
 #pragma unroll
-    for (int k = 0; k < P / R; ++k) {
-      const int j = tid + k * T;
-#pragma unroll
-      for (int r = 0; r < R; ++r) v[k * R + r] = sm[fft_pad(j + r * (N / R))];
-    }
-#pragma unroll
-    for (int k = 0; k < P / R; ++k) {
-      const int j = tid + k * T;
-      if (Ns > 1) {
-        const int kk = j & (Ns - 1);
-        constexpr int stride = kTwiddleN / (Ns * R);
-#pragma unroll
-        for (int r = 1; r < R; ++r) {
-          float2 w = __ldg(tw + r * kk * stride);
-          if (INV) w.y = -w.y;
-          v[k * R + r] = cmul(v[k * R + r], w);
-        }
-      }
-      dft_reg<R, INV>(v + k * R);
-    }
-    sync();
-#pragma unroll
-    for (int k = 0; k < P / R; ++k) {
+  for (int k = 0; k < S::P / R; ++k) {
+    if constexpr (Ns > 1) {
       const int j = tid + k * T;
       const int kk = j & (Ns - 1);
-      const int e = (j - kk) * R + kk;
-#pragma unroll
-      for (int r = 0; r < R; ++r) sm[fft_pad(e + r * Ns)] = v[k * R + r];
+      apply_twiddles<R, INV>(v + k * R, tw, kk * (kTwiddleN / (Ns * R)));
     }
-    sync();
-    if constexpr (DONE + RB < LOGN) FftPass<N, T, INV, DONE + RB, Sync>::run(sm, tid, tw, sync);
+    dft_reg<R, INV>(v + k * R);
   }
-};
+}
+
+// Stockham load of one pass: value r of butterfly j sits at j + r*N/R.
+template <int N, int T, int DONE>
+__device__ __forceinline__ void pass_load(const float2* sm, float2* v, int tid) {
+  using S = FftShape<N, T>;
+  constexpr int R = 1 << S::rb(DONE);
+#pragma unroll
+  for (int k = 0; k < S::P / R; ++k) {
+#pragma unroll
+    for (int r = 0; r < R; ++r) v[k * R + r] = sm[fft_pad(tid + k * T + r * (N / R))];
+  }
+}
+
+// Stockham store of one pass: output r of butterfly j goes to (j - kk)*R + kk + r*Ns.
+template <int N, int T, int DONE>
+__device__ __forceinline__ void pass_store(float2* sm, const float2* v, int tid) {
+  using S = FftShape<N, T>;
+  constexpr int R = 1 << S::rb(DONE);
+  constexpr int Ns = 1 << DONE;
+#pragma unroll
+  for (int k = 0; k < S::P / R; ++k) {
+    const int j = tid + k * T;
+    const int kk = j & (Ns - 1);
+    const int e = (j - kk) * R + kk;
+#pragma unroll
+    for (int r = 0; r < R; ++r) sm[fft_pad(e + r * Ns)] = v[k * R + r];
+  }
+}
+
+// Passes DONE.. that go shared memory -> shared memory, stopping before the
+// last pass when STOP_BEFORE_LAST (the caller finishes it with its own store).
+template <int N, int T, bool INV, int DONE, bool STOP_BEFORE_LAST, class Sync>
+__device__ __forceinline__ void smem_passes(float2* sm, int tid, const float2* __restrict__ tw, Sync sync) {
+  using S = FftShape<N, T>;
+  if constexpr (DONE < S::LOGN) {
+    if constexpr (!(STOP_BEFORE_LAST && S::last(DONE))) {
+      float2 v[S::P];
+      pass_load<N, T, DONE>(sm, v, tid);
+      pass_compute<N, T, INV, DONE>(v, tid, tw);
+      sync();
+      pass_store<N, T, DONE>(sm, v, tid);
+      sync();
+      smem_passes<N, T, INV, DONE + S::rb(DONE), STOP_BEFORE_LAST>(sm, tid, tw, sync);
+    }
+  }
+}
+
+// Start of the last pass.
+template <int N, int T, int DONE = 0>
+constexpr int last_pass_done() {
+  using S = FftShape<N, T>;
+  if constexpr (S::last(DONE)) return DONE;
+  else return last_pass_done<N, T, DONE + S::rb(DONE)>();
+}
 
 // In-place transform of sm[fft_pad(0..N)) by the T threads with tid in [0, T).
 // Callers synchronise before (data written) and may read results right after.
 template <int N, int T, bool INV, class Sync>
 __device__ __forceinline__ void fft_smem(float2* sm, int tid, const float2* __restrict__ tw, Sync sync) {
-  static_assert((N & (N - 1)) == 0 && N >= 2 * T && T >= 32, "bad FFT shape");
-  FftPass<N, T, INV, 0, Sync>::run(sm, tid, tw, sync);
+  static_assert((N & (N - 1)) == 0 && N >= 2 * T, "bad FFT shape");
+  smem_passes<N, T, INV, 0, false>(sm, tid, tw, sync);
 }
 
-// Threads per transform for N points: one warp up to 512 points, else 16 points per thread.
-__host__ __device__ constexpr int fft_threads(int n) { return n <= 512 ? 32 : n / 16; }
-// Transforms per CTA: several warps for the warp-sized transforms.
-__host__ __device__ constexpr int fft_per_cta(int n) { return n <= 512 ? 4 : 1; }
+// Threads per transform: 16 points per thread (32 for the largest transform, to
+// stay within 512 threads and 128 registers each).
+__host__ __device__ constexpr int fft_threads(int n) { return n >= 16384 ? n / 32 : n / 16; }
+// Threads per CTA: whole warps; small transforms share a warp.
+__host__ __device__ constexpr int fft_cta_threads(int n) { return fft_threads(n) >= 128 ? fft_threads(n) : 128; }
+// Transforms per CTA.
+__host__ __device__ constexpr int fft_per_cta(int n) { return fft_cta_threads(n) / fft_threads(n); }
 
 }  // namespace fi

@@ -52,6 +52,7 @@ struct fi_ctx {
   float* taps = nullptr;
   float2* spectra = nullptr;
   float2* twiddle = nullptr;
+  int* err = nullptr;      // device flag: a bounded wait in a kernel gave up
   size_t spec_off[32] = {};
   // staging for fi_generate_host
   void* d_x0 = nullptr;
@@ -73,6 +74,7 @@ void free_ctx(fi_ctx* c) {
   cudaFree(c->taps);
   cudaFree(c->spectra);
   cudaFree(c->twiddle);
+  cudaFree(c->err);
   cudaFree(c->d_x0);
   cudaFree(c->d_eps);
   cudaFree(c->d_y);
@@ -126,6 +128,18 @@ fi_status run_block(fi_ctx* c, int i) {
   }
   return timed(c, KC_DIRECT, [&] { return launch_tile_direct(c->g, c->state, c->taps, i, c->st); },
                "direct block launch");
+}
+
+// Synchronise the context's stream and report a device-side wait that gave up.
+fi_status sync_and_check(fi_ctx* c) {
+  FI_CUDA(cudaStreamSynchronize(c->st), "synchronize");
+  int flag = 0;
+  FI_CUDA(cudaMemcpy(&flag, c->err, sizeof(int), cudaMemcpyDeviceToHost), "read error flag");
+  if (flag) {
+    FI_CUDA(cudaMemset(c->err, 0, sizeof(int)), "clear error flag");
+    return fail(FI_E_TIMEOUT, "a bounded device-side wait gave up; results of the last calls are invalid");
+  }
+  return FI_OK;
 }
 
 }  // namespace
@@ -191,9 +205,11 @@ fi_status fi_init(fi_ctx** out, const fi_config* cfg, const void* h, void* strea
 
   // Plan: blocks below `chunk` on chip, FFT from `fft_from` up to the largest
   // transform one CTA holds, direct blocks from HBM in between and above.
-  c->chunk = cfg->chunk ? cfg->chunk : 32;
+  c->chunk = cfg->chunk ? cfg->chunk : 64;
   if (c->chunk > g.L) c->chunk = g.L;
-  c->fft_from = cfg->fft_from ? cfg->fft_from : 128;
+  // FFT blocks pay off once a launch has enough (layer, stream) rows to fill the
+  // GPU; tiny stacks keep direct blocks up to side 512.
+  c->fft_from = cfg->fft_from ? cfg->fft_from : ((int64_t)g.M * g.S >= 2048 ? 64 : 1024);
   c->q_lo = ilog2((uint32_t)c->fft_from);
   c->q_hi = g.P - 1 < kMaxFftLog2 ? g.P - 1 : kMaxFftLog2;
   if (c->q_lo < kMinFftLog2) c->q_lo = kMinFftLog2;
@@ -214,6 +230,8 @@ fi_status fi_init(fi_ctx** out, const fi_config* cfg, const void* h, void* strea
   }
   if (spec_n && (s = dev_alloc((void**)&c->spectra, spec_n * sizeof(float2), "spectra")) != FI_OK) return bail(s);
   if ((s = dev_alloc((void**)&c->twiddle, (size_t)kTwiddleN * sizeof(float2), "twiddles")) != FI_OK) return bail(s);
+  if ((s = dev_alloc((void**)&c->err, sizeof(int), "error flag")) != FI_OK) return bail(s);
+  if ((e = cudaMemsetAsync(c->err, 0, sizeof(int), c->st)) != cudaSuccess) return bail(cuda_fail(e, "error flag"));
 
   std::vector<float2> tw(kTwiddleN);
   for (int m = 0; m < kTwiddleN; ++m) {
@@ -313,6 +331,7 @@ fi_status fi_generate(fi_ctx* c, int32_t n, const void* x0, const float* eps, fl
     a.p0 = p;
     a.p1 = p1;
     a.last_done = last_done;
+    a.err = c->err;
     if ((s = timed(c, KC_CHUNK, [&] { return launch_chunk(c->g, a, c->chunk_G, c->st); }, "chunk launch")) != FI_OK)
       return s;
     p = p1;
@@ -348,8 +367,12 @@ fi_status fi_generate_host(fi_ctx* c, int32_t n, const void* x0_host, const floa
   fi_status s = fi_generate(c, n, c->d_x0, c->d_eps, eps_scale, c->d_y, nullptr);
   if (s != FI_OK) return s;
   FI_CUDA(cudaMemcpyAsync(y_out_host, c->d_y, row * n * sizeof(float), cudaMemcpyDeviceToHost, c->st), "y download");
-  FI_CUDA(cudaStreamSynchronize(c->st), "fi_generate_host synchronize");
-  return FI_OK;
+  return sync_and_check(c);
+}
+
+fi_status fi_sync(fi_ctx* c) {
+  if (!c) return fail(FI_E_INVALID, "ctx is NULL");
+  return sync_and_check(c);
 }
 
 fi_status fi_generate_lazy(fi_ctx* c, int32_t n, const void* x0, const float* eps, float eps_scale, float* y_out) {

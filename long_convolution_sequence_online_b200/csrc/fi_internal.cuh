@@ -87,6 +87,7 @@ struct ChunkArgs {
   int gen_base;          // first position of the generate call
   int c, chunk, p0, p1;  // chunk start, chunk length, positions to produce
   int last_done;         // last step whose blocks have reached HBM before this launch
+  int* err;              // device flag set to 1 when a bounded wait gives up
 };
 cudaError_t launch_chunk(const Dims& g, const ChunkArgs& a, int streams_per_cta, cudaStream_t st);
 cudaError_t configure_chunk(size_t smem);   // allow `smem` bytes of dynamic shared memory

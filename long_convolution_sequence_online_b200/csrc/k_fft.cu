@@ -46,9 +46,61 @@ __device__ __forceinline__ void spectral_product(float2* sm, int tid, const floa
   }
 }
 
+template <int N, class Sync>
+__device__ __forceinline__ void tile_fft_body(float2* sm, int tid, bool active, const float2* __restrict__ src,
+                                              float2* __restrict__ dst, const float2* __restrict__ H,
+                                              const float2* __restrict__ tw, int overwrite, Sync sync) {
+  constexpr int T = fft_threads(N);
+  using S = FftShape<N, T>;
+  // Forward pass 0 straight from HBM: z[m] = (x[2m], x[2m+1]) for m < N/2, zero above.
+  {
+    constexpr int R = 1 << S::rb(0);
+    float2 v[S::P];
+#pragma unroll
+    for (int k = 0; k < S::P / R; ++k) {
+      const int j = tid + k * T;
+#pragma unroll
+      for (int r = 0; r < R; ++r)
+        v[k * R + r] = (active && r < R / 2) ? src[j + r * (N / R)] : make_float2(0.f, 0.f);
+    }
+    pass_compute<N, T, false, 0>(v, tid, tw);
+    pass_store<N, T, 0>(sm, v, tid);
+    sync();
+  }
+  smem_passes<N, T, false, S::rb(0), false>(sm, tid, tw, sync);
+  spectral_product<N, T>(sm, tid, H, tw);
+  sync();
+  smem_passes<N, T, true, 0, true>(sm, tid, tw, sync);
+  // Last inverse pass straight to HBM: only outputs m >= N/2 (r >= R/2) are kept.
+  {
+    constexpr int DL = last_pass_done<N, T>();
+    constexpr int R = 1 << S::rb(DL);
+    float2 v[S::P];
+    pass_load<N, T, DL>(sm, v, tid);
+    pass_compute<N, T, true, DL>(v, tid, tw);
+    if (active) {
+#pragma unroll
+      for (int k = 0; k < S::P / R; ++k) {
+        const int j = tid + k * T;
+#pragma unroll
+        for (int r = R / 2; r < R; ++r) {
+          const int m = j + r * (N / R) - N / 2;
+          const float2 o = v[k * R + r];
+          if (overwrite) {
+            dst[m] = o;
+          } else {
+            const float2 p = dst[m];
+            dst[m] = make_float2(p.x + o.x, p.y + o.y);
+          }
+        }
+      }
+    }
+  }
+}
+
 // One FFT block for every (layer, stream): item = (l-1)*S + s.
 template <int N>
-__global__ void __launch_bounds__(fft_threads(N) * fft_per_cta(N))
+__global__ void __launch_bounds__(fft_cta_threads(N))
 k_tile_fft(Dims g, float* __restrict__ state, const float2* __restrict__ spec,
            const float2* __restrict__ tw, int i, int overwrite) {
   constexpr int T = fft_threads(N), F = fft_per_cta(N);
@@ -64,35 +116,13 @@ k_tile_fft(Dims g, float* __restrict__ state, const float2* __restrict__ spec,
   const float2* src = reinterpret_cast<const float2*>(state + slot_index(g, l - 1, s, i - N));
   float2* dst = reinterpret_cast<float2*>(state + slot_index(g, l, s, i));
   const float2* H = spec + ((size_t)(l - 1) * g.D + d) * (N + 1);
-
-  for (int m = tid; m < N; m += T) sm[fft_pad(m)] = (active && m < N / 2) ? src[m] : make_float2(0.f, 0.f);
-  if (T == 32) __syncwarp(); else __syncthreads();
-  if constexpr (T == 32) {
-    fft_smem<N, T, false>(sm, tid, tw, SyncWarp());
-    spectral_product<N, T>(sm, tid, H, tw);
-    __syncwarp();
-    fft_smem<N, T, true>(sm, tid, tw, SyncWarp());
-  } else {
-    fft_smem<N, T, false>(sm, tid, tw, SyncBlock());
-    spectral_product<N, T>(sm, tid, H, tw);
-    __syncthreads();
-    fft_smem<N, T, true>(sm, tid, tw, SyncBlock());
-  }
-  if (!active) return;
-  for (int j = tid; j < N / 2; j += T) {
-    const float2 v = sm[fft_pad(N / 2 + j)];
-    if (overwrite) {
-      dst[j] = v;
-    } else {
-      const float2 o = dst[j];
-      dst[j] = make_float2(o.x + v.x, o.y + v.y);
-    }
-  }
+  if constexpr (T <= 32) tile_fft_body<N>(sm, tid, active, src, dst, H, tw, overwrite, SyncWarp());
+  else tile_fft_body<N>(sm, tid, active, src, dst, H, tw, overwrite, SyncBlock());
 }
 
 // Spectrum of h[0..2N) / (2N) for one (layer, channel): item = l*D + d.
 template <int N>
-__global__ void __launch_bounds__(fft_threads(N) * fft_per_cta(N))
+__global__ void __launch_bounds__(fft_cta_threads(N))
 k_spectra(Dims g, const float* __restrict__ taps, float2* __restrict__ spec, const float2* __restrict__ tw) {
   constexpr int T = fft_threads(N), F = fft_per_cta(N);
   constexpr int twstep = kTwiddleN / (2 * N);
@@ -103,7 +133,7 @@ k_spectra(Dims g, const float* __restrict__ taps, float2* __restrict__ spec, con
   const bool active = item < (long)g.M * g.D;
   const float2* src = reinterpret_cast<const float2*>(taps + (size_t)(active ? item : 0) * g.L);
   for (int m = tid; m < N; m += T) sm[fft_pad(m)] = active ? src[m] : make_float2(0.f, 0.f);
-  if constexpr (T == 32) {
+  if constexpr (T <= 32) {
     __syncwarp();
     fft_smem<N, T, false>(sm, tid, tw, SyncWarp());
   } else {
@@ -125,7 +155,7 @@ k_spectra(Dims g, const float* __restrict__ taps, float2* __restrict__ spec, con
 }
 
 template <int N>
-__global__ void __launch_bounds__(fft_threads(N) * fft_per_cta(N))
+__global__ void __launch_bounds__(fft_cta_threads(N))
 k_debug_fft(int count, const float2* __restrict__ in, float2* __restrict__ out, int inverse,
             const float2* __restrict__ tw) {
   constexpr int T = fft_threads(N), F = fft_per_cta(N);
@@ -135,7 +165,7 @@ k_debug_fft(int count, const float2* __restrict__ in, float2* __restrict__ out, 
   const long item = (long)blockIdx.x * F + sub;
   const bool active = item < count;
   for (int m = tid; m < N; m += T) sm[fft_pad(m)] = active ? in[item * N + m] : make_float2(0.f, 0.f);
-  if constexpr (T == 32) {
+  if constexpr (T <= 32) {
     __syncwarp();
     if (inverse) fft_smem<N, T, true>(sm, tid, tw, SyncWarp());
     else fft_smem<N, T, false>(sm, tid, tw, SyncWarp());
@@ -167,7 +197,7 @@ static cudaError_t tile_fft_n(const Dims& g, float* state, const float2* spec, c
   const long items = (long)g.M * g.S;
   const long blocks = (items + fft_per_cta(N) - 1) / fft_per_cta(N);
   const int overwrite = is_pow2(i) ? 1 : 0;
-  k_tile_fft<N><<<(unsigned)blocks, fft_threads(N) * fft_per_cta(N), smem, st>>>(g, state, spec, tw, i, overwrite);
+  k_tile_fft<N><<<(unsigned)blocks, fft_cta_threads(N), smem, st>>>(g, state, spec, tw, i, overwrite);
   return cudaGetLastError();
 }
 
@@ -178,7 +208,7 @@ static cudaError_t spectra_n(const Dims& g, const float* taps, float2* spec, con
   if (e != cudaSuccess) return e;
   const long items = (long)g.M * g.D;
   const long blocks = (items + fft_per_cta(N) - 1) / fft_per_cta(N);
-  k_spectra<N><<<(unsigned)blocks, fft_threads(N) * fft_per_cta(N), smem, st>>>(g, taps, spec, tw);
+  k_spectra<N><<<(unsigned)blocks, fft_cta_threads(N), smem, st>>>(g, taps, spec, tw);
   return cudaGetLastError();
 }
 
@@ -189,7 +219,7 @@ static cudaError_t debug_fft_n(int count, const float2* in, float2* out, int inv
   cudaError_t e = prepare(k_debug_fft<N>, smem);
   if (e != cudaSuccess) return e;
   const long blocks = ((long)count + fft_per_cta(N) - 1) / fft_per_cta(N);
-  k_debug_fft<N><<<(unsigned)blocks, fft_threads(N) * fft_per_cta(N), smem, st>>>(count, in, out, inverse, tw);
+  k_debug_fft<N><<<(unsigned)blocks, fft_cta_threads(N), smem, st>>>(count, in, out, inverse, tw);
   return cudaGetLastError();
 }
 

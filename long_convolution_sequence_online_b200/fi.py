@@ -19,7 +19,7 @@ FI_F32, FI_BF16 = 0, 1
 NUM_KERNEL_CLASSES = 5
 KERNEL_CLASSES = ("chunk", "direct", "fft", "token", "lazy")
 
-EXPORTED = ("fi_init", "fi_step", "fi_generate", "fi_generate_host", "fi_generate_lazy", "fi_reset",
+EXPORTED = ("fi_init", "fi_step", "fi_generate", "fi_generate_host", "fi_generate_lazy", "fi_sync", "fi_reset",
             "fi_position", "fi_read_activations", "fi_set_stream", "fi_get_plan", "fi_profile",
             "fi_profile_read", "fi_destroy", "fi_status_str", "fi_last_error", "fi_debug_fft")
 
@@ -49,6 +49,7 @@ def _load():
         "fi_generate_host": [vp, i32, vp, vp, f32, vp],
         "fi_generate_lazy": [vp, i32, vp, vp, f32, vp],
         "fi_reset": [vp],
+        "fi_sync": [vp],
         "fi_position": [vp, ctypes.POINTER(i32)],
         "fi_read_activations": [vp, i32, vp],
         "fi_set_stream": [vp, vp],
@@ -154,6 +155,9 @@ class Context:
 
     def generate_lazy(self, n: int, x0, eps, y_out, eps_scale: float = 0.1):
         _check(lib.fi_generate_lazy(self._h, n, _ptr(x0), _ptr(eps), eps_scale, _ptr(y_out)), "fi_generate_lazy")
+
+    def sync(self):
+        _check(lib.fi_sync(self._h), "fi_sync")
 
     def reset(self):
         _check(lib.fi_reset(self._h), "fi_reset")

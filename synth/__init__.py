@@ -66,6 +66,12 @@ for _b in (8, 32, 64):
     WORKLOADS[f"sweep-8x2048-L16K-bf16-B{_b}"] = dataclasses.replace(
         _w, batch=_b, name=f"sweep-8x2048-L16K-bf16-B{_b}")
 
+# Reduced-footprint shapes of the headline stack for profiler captures (about 1 GB
+# on the device): the full layer/channel/batch shape at L = 2048, and a 64-channel
+# slice at the full length L = 32768 (which reaches the largest FFT blocks).
+WORKLOADS["hyena-18x864-L2K-B4"] = Workload("hyena-18x864-L2K-B4", 18, 864, 2048, 4, "f32", 1e-3, 1e-1)
+WORKLOADS["hyena-18x64-L32K-B4"] = Workload("hyena-18x64-L32K-B4", 18, 64, 32768, 4, "f32", 1e-3, 1e-1)
+
 HEADLINE = "hyena-18x864-L32K-B4"
 
 
