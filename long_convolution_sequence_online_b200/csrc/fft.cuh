@@ -10,7 +10,7 @@
 // (j div Ns)*Ns*R + (j mod Ns) + r*Ns. The output is in natural order.
 //
 // T threads cooperate on one transform, each holding P = N/T points; the radix
-// is min(16, P) (the last pass takes what is left). Each pass loads all of a
+// is min(32, P) (the last pass takes what is left). Each pass loads all of a
 // thread's points, synchronises, then stores, so one buffer suffices. Shared
 // memory indices are padded by one slot per 16 (idx + idx/16) so the stride-16
 // stores of the first pass do not collide in the same bank.
@@ -40,29 +40,34 @@ __device__ __forceinline__ float2 cmul(float2 a, float2 b) {
 __device__ __forceinline__ float2 cmul_i(float2 a) { return make_float2(-a.y, a.x); }
 __device__ __forceinline__ float2 cmul_mi(float2 a) { return make_float2(a.y, -a.x); }
 
-// cos and sin of 2*pi*m/16, m in [0, 16) (exact decimal expansions of the constants).
-__device__ __forceinline__ float cos16(int m) {
-  constexpr float c1 = 0.92387953251128675613f, s1 = 0.38268343236508977173f, r2 = 0.70710678118654752440f;
-  switch (m & 15) {
-    case 0: return 1.f;   case 1: return c1;  case 2: return r2;  case 3: return s1;
-    case 4: return 0.f;   case 5: return -s1; case 6: return -r2; case 7: return -c1;
-    case 8: return -1.f;  case 9: return -c1; case 10: return -r2; case 11: return -s1;
-    case 12: return 0.f;  case 13: return s1; case 14: return r2;  default: return c1;
-  }
+// cos of 2*pi*m/32 for m in [0, 32), by quadrant symmetry from the first
+// quadrant's values (decimal expansions of the constants).
+__host__ __device__ constexpr float cos32(int m) {
+  constexpr float q[9] = {1.0f,
+                          0.98078528040323044913f,   // cos(pi/16)
+                          0.92387953251128675613f,   // cos(pi/8)
+                          0.83146961230254523708f,   // cos(3pi/16)
+                          0.70710678118654752440f,   // cos(pi/4)
+                          0.55557023301960222474f,   // cos(5pi/16)
+                          0.38268343236508977173f,   // cos(3pi/8)
+                          0.19509032201612826785f,   // cos(7pi/16)
+                          0.0f};
+  m &= 31;
+  return m <= 8 ? q[m] : m <= 16 ? -q[16 - m] : m <= 24 ? -q[m - 16] : q[32 - m];
 }
-__device__ __forceinline__ float sin16(int m) { return cos16(m - 4); }  // sin x = cos(x - pi/2)
+__host__ __device__ constexpr float sin32(int m) { return cos32(m - 8); }  // sin x = cos(x - pi/2)
 
-// v * W_16^m where W_16 = exp(-2 pi i / 16) (forward) or its conjugate (inverse).
+// v * W_32^m where W_32 = exp(-2 pi i / 32) (forward) or its conjugate (inverse).
 // m is a compile-time constant after unrolling, so the branches fold away.
 template <bool INV>
-__device__ __forceinline__ float2 mul_w16(float2 v, int m) {
-  m &= 15;
+__device__ __forceinline__ float2 mul_w32(float2 v, int m) {
+  m &= 31;
   if (m == 0) return v;
-  if (m == 8) return make_float2(-v.x, -v.y);
-  if (m == 4) return INV ? cmul_i(v) : cmul_mi(v);
-  if (m == 12) return INV ? cmul_mi(v) : cmul_i(v);
-  const float c = cos16(m);
-  const float s = INV ? sin16(m) : -sin16(m);
+  if (m == 16) return make_float2(-v.x, -v.y);
+  if (m == 8) return INV ? cmul_i(v) : cmul_mi(v);
+  if (m == 24) return INV ? cmul_mi(v) : cmul_i(v);
+  const float c = cos32(m);
+  const float s = INV ? sin32(m) : -sin32(m);
   return cmul(v, make_float2(c, s));
 }
 
@@ -88,13 +93,13 @@ __device__ __forceinline__ void dif_stage(float2* v) {
     for (int j = 0; j < SPAN; ++j) {
       const float2 a = v[g0 + j], b = v[g0 + j + SPAN];
       v[g0 + j] = cadd(a, b);
-      v[g0 + j + SPAN] = mul_w16<INV>(csub(a, b), j * (16 / (2 * SPAN)));
+      v[g0 + j + SPAN] = mul_w32<INV>(csub(a, b), j * (32 / (2 * SPAN)));
     }
   }
   if constexpr (SPAN > 1) dif_stage<R, SPAN / 2, INV>(v);
 }
 
-// R-point DFT of v[0..R) in registers (R = 2, 4, 8 or 16): decimation in
+// R-point DFT of v[0..R) in registers (R = 2, 4, 8, 16 or 32): decimation in
 // frequency, then a fixed permutation undoes the bit reversal.
 template <int R, bool INV>
 __device__ __forceinline__ void dft_reg(float2* v) {
@@ -110,8 +115,8 @@ struct SyncWarp { __device__ __forceinline__ void operator()() const { __syncwar
 struct SyncBlock { __device__ __forceinline__ void operator()() const { __syncthreads(); } };
 
 // v[r] *= w^r for r = 1..R-1 (w = W_{Ns R}^{kk}, forward sign; conjugated for the
-// inverse). w, w^4 and w^8 come from the table; the other powers are products of
-// at most three table values, so each carries a few roundings at most.
+// inverse). w, w^4, w^8 (and w^16) come from the table; the other powers are
+// products of at most four table values, so each carries a few roundings at most.
 template <int R, bool INV>
 __device__ __forceinline__ void apply_twiddles(float2* v, const float2* __restrict__ tw, int base) {
   auto ld = [&](int r) {
@@ -143,15 +148,26 @@ __device__ __forceinline__ void apply_twiddles(float2* v, const float2* __restri
   v[13] = cmul(v[13], cmul(w12, w1));
   v[14] = cmul(v[14], cmul(w12, w2));
   v[15] = cmul(v[15], cmul(w12, w3));
+  if constexpr (R == 16) return;
+  const float2 w16 = ld(16);
+  const float2 w20 = cmul(w16, w4), w24 = cmul(w16, w8), w28 = cmul(w24, w4);
+  const float2 wb[4] = {w16, w20, w24, w28};
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    v[16 + 4 * q] = cmul(v[16 + 4 * q], wb[q]);
+    v[17 + 4 * q] = cmul(v[17 + 4 * q], cmul(wb[q], w1));
+    v[18 + 4 * q] = cmul(v[18 + 4 * q], cmul(wb[q], w2));
+    v[19 + 4 * q] = cmul(v[19 + 4 * q], cmul(wb[q], w3));
+  }
 }
 
 // Shape of the transform: T threads, P = N/T points each, passes of radix
-// min(16, P) until the last pass takes what is left.
+// min(32, P) until the last pass takes what is left.
 template <int N, int T>
 struct FftShape {
   static constexpr int LOGN = clog2(N);
   static constexpr int P = N / T;
-  static constexpr int RBMAX = cmin(4, clog2(P));
+  static constexpr int RBMAX = cmin(5, clog2(P));
   static constexpr int rb(int done) { return cmin(RBMAX, LOGN - done); }
   static constexpr bool last(int done) { return done + rb(done) >= LOGN; }
 };
@@ -236,9 +252,9 @@ __device__ __forceinline__ void fft_smem(float2* sm, int tid, const float2* __re
   smem_passes<N, T, INV, 0, false>(sm, tid, tw, sync);
 }
 
-// Threads per transform: 16 points per thread (32 for the largest transform, to
-// stay within 512 threads and 128 registers each).
-__host__ __device__ constexpr int fft_threads(int n) { return n >= 16384 ? n / 32 : n / 16; }
+// Threads per transform: 32 points per thread from 512 points up (radix-32
+// passes: two passes up to 1024 points, three up to 32768), 16 below.
+__host__ __device__ constexpr int fft_threads(int n) { return n >= 512 ? n / 32 : n / 16; }
 // Threads per CTA: whole warps; small transforms share a warp.
 __host__ __device__ constexpr int fft_cta_threads(int n) { return fft_threads(n) >= 128 ? fft_threads(n) : 128; }
 // Transforms per CTA.

@@ -106,19 +106,20 @@ __device__ __forceinline__ void gray_block(int U, const float* src, float* dst, 
 }
 
 // tanh for the block and the sampler, without branches (every lane of the chain
-// warp takes the same path).
-// fp32 activations: t0 = the hardware tanh approximation (relative error about
-// 1e-5) and e = 2^(2 y log2 e) = e^(2y) are computed side by side; one Newton
-// step on t (e + 1) = e - 1, using 1/(e+1) = (1 - t)/2, gives
-//     t1 = t0 - (t0 (e + 1) - (e - 1)) (1 - t0) / 2,
-// whose error is quadratic in t0's; what remains is the rounding of e and of
-// e - 1 near y = 0, below 2e-7 in absolute terms. The exponent is capped at
-// 2^126 so that e stays finite (tanh is then exactly +-1 in fp32).
-// bf16 activations: the approximation alone (its error is far below bfloat16's
-// 2^-9), since the result is rounded to bf16 right after.
+// warp takes the same path). fp32 activations: for |y| >= 1/8,
+// 1 - 2 / (1 + 2^(2 |y| log2 e)) with the hardware exp2 and reciprocal; below
+// 1/8 the odd Taylor series to y^9 (truncation < 1e-11 there); absolute error
+// within 1.5e-7 everywhere, about the rounding of an fp32 value near 1.
+// bf16 activations: the hardware tanh approximation (relative error about 1e-5,
+// far below bfloat16's 2^-9), since the result is rounded to bf16 right after.
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float rcp_approx(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
 __device__ __forceinline__ float tanh_approx(float x) {
@@ -133,11 +134,14 @@ __device__ __forceinline__ float round_to(float v) {
 }
 template <bool BF16>
 __device__ __forceinline__ float block_tanh(float y) {
-  const float t0 = tanh_approx(y);
-  if constexpr (BF16) return t0;
-  const float e = ex2_approx(fminf(y * 2.88539008177792681f, 126.0f));
-  const float r = fmaf(t0, e + 1.0f, 1.0f - e);
-  return fmaf(-r, fmaf(-0.5f, t0, 0.5f), t0);
+  if constexpr (BF16) return tanh_approx(y);
+  const float ax = fabsf(y);
+  const float e = ex2_approx(ax * 2.88539008177792681f);   // e^(2|y|); +inf for large |y| gives 1
+  const float big = fmaf(-2.0f, rcp_approx(1.0f + e), 1.0f);
+  const float x2 = y * y;
+  const float p = fmaf(fmaf(fmaf(fmaf(62.0f / 2835.0f, x2, -17.0f / 315.0f), x2, 2.0f / 15.0f), x2, -1.0f / 3.0f),
+                       x2 * ax, ax);
+  return copysignf(ax < 0.125f ? p : big, y);
 }
 
 // Hardware barriers in shared memory (mbarrier): arrive has release semantics
@@ -210,29 +214,39 @@ __global__ void __launch_bounds__(kChunkMaxThreads) k_chunk(Dims g, ChunkArgs a,
 
   // Prologue: every load is an asynchronous 4-byte copy into shared memory
   // (zero-filled where the slot holds nothing yet), so the loads of a thread
-  // overlap instead of waiting one by one on HBM latency.
-  for (int k = tid; k < M * Gd * CH; k += nt) {
-    const int j = k % CH, rest = k / CH, dl = rest % Gd, l = rest / Gd;
-    cp_async4(tp + (l * GdMax + dl) * TPS + j, a.taps + ((size_t)l * g.D + d_lo + dl) * g.L + j, true);
+  // overlap instead of waiting one by one on HBM latency. Rows are spread over
+  // warps and positions over lanes, so index arithmetic is per row.
+  const int wid = tid >> 5, lid = tid & 31, nw = nt >> 5;
+  for (int row = wid; row < M * Gd; row += nw) {
+    const int l = row / Gd, dl = row - l * Gd;
+    const float* src = a.taps + ((size_t)l * g.D + d_lo + dl) * g.L;
+    float* dst = tp + (l * GdMax + dl) * TPS;
+    for (int j = lid; j < CH; j += 32) cp_async4(dst + j, src + j, true);
   }
   // Slots already in HBM: tokens and activations below p0; the token at p0 when
   // no x0 is given; accumulators that some block has reached (the first block to
   // reach position t runs at step highbit(t)). Everything else starts at 0.
-  for (int k = tid; k < (M + 1) * Gc * CH; k += nt) {
-    const int r = k % CH, rest = k / CH, gg = rest % Gc, l = rest / Gc;
-    const int t = a.c + r;
-    bool valid = false;
-    if (t < g.L) {
-      valid = t < a.p0;
-      if (l == 0) valid = valid || (t == a.p0 && a.x0 == nullptr);
-      else valid = valid || (t >= 1 && highbit_dev(t) <= a.last_done);
+  for (int row = wid; row < (M + 1) * Gc; row += nw) {
+    const int l = row / Gc, gg = row - l * Gc;
+    const float* src = a.state + slot_index(g, l, s0 + gg, 0);
+    float* dst = win + (l * G + gg) * CHP;
+    for (int r = lid; r < CH; r += 32) {
+      const int t = a.c + r;
+      bool valid = false;
+      if (t < g.L) {
+        valid = t < a.p0;
+        if (l == 0) valid = valid || (t == a.p0 && a.x0 == nullptr);
+        else valid = valid || (t >= 1 && highbit_dev(t) <= a.last_done);
+      }
+      cp_async4(dst + r, src + (valid ? t : 0), valid);
     }
-    cp_async4(win + (l * G + gg) * CHP + r, a.state + slot_index(g, l, s0 + gg, valid ? t : 0), valid);
   }
-  for (int k = tid; k < (r1 - r0) * Gc; k += nt) {
-    const int gg = k % Gc, r = r0 + k / Gc;
-    const int s = s0 + gg, d = s / g.B, b = s - d * g.B;
-    cp_async4(ep + r * G + gg, a.eps + (size_t)(a.c + r - a.gen_base) * g.S + (size_t)b * g.D + d, true);
+  for (int r = r0 + wid; r < r1; r += nw) {
+    const float* src = a.eps + (size_t)(a.c + r - a.gen_base) * g.S;
+    for (int gg = lid; gg < Gc; gg += 32) {
+      const int s = s0 + gg, d = s / g.B, b = s - d * g.B;
+      cp_async4(ep + r * G + gg, src + (size_t)b * g.D + d, true);
+    }
   }
   cp_async_wait_all();
   __syncthreads();
@@ -339,19 +353,33 @@ __global__ void __launch_bounds__(kChunkMaxThreads) k_chunk(Dims g, ChunkArgs a,
   __syncthreads();
 
   // Outputs of the positions produced, then the next chunk's first token.
-  for (int k = tid; k < (r1 - r0) * Gc; k += nt) {
-    const int gg = k % Gc, r = r0 + k / Gc;
-    const int s = s0 + gg, d = s / g.B, b = s - d * g.B;
-    a.y_out[(size_t)(a.c + r - a.gen_base) * g.S + (size_t)b * g.D + d] = ys[r * G + gg];
+  const int wid2 = tid >> 5, lid2 = tid & 31, nw2 = nt >> 5;
+  for (int r = r0 + wid2; r < r1; r += nw2) {
+    float* dst = a.y_out + (size_t)(a.c + r - a.gen_base) * g.S;
+    for (int gg = lid2; gg < Gc; gg += 32) {
+      const int s = s0 + gg, d = s / g.B, b = s - d * g.B;
+      dst[(size_t)b * g.D + d] = ys[r * G + gg];
+    }
   }
   if (r1 == CH && a.c + CH < g.L && tid < Gc) a.state[slot_index(g, 0, s0 + tid, a.c + CH)] = win[tid * CHP + CH];
-  // Write back positions [p0, c+CH): new tokens and activations below p1,
-  // accumulators (including the small blocks' partial sums) from p1 on.
-  const int nr = CH - r0;
-  for (int k = tid; k < (M + 1) * Gc * nr; k += nt) {
-    const int r = r0 + k % nr, rest = k / nr, gg = rest % Gc, l = rest / Gc;
-    const int t = a.c + r;
-    if (t < g.L) a.state[slot_index(g, l, s0 + gg, t)] = win[(l * G + gg) * CHP + r];
+  // Write back positions [p0, c+CH) of layers 0..M-1: new tokens and
+  // activations below p1, accumulators (including the small blocks' partial
+  // sums) from p1 on. Layer M's slots below p1 were consumed and nothing reads
+  // them again; its accumulators from p1 on are still needed.
+  for (int row = wid2; row < (M + 1) * Gc; row += nw2) {
+    const int l = row / Gc, gg = row - l * Gc;
+    float* dst = a.state + slot_index(g, l, s0 + gg, a.c);
+    const float* src = win + (l * G + gg) * CHP;
+    const int rb = l == M ? r1 : r0;            // first slot to write
+    const int re = min(CH, g.L - a.c);          // past the last
+    if ((a.c & 3) == 0 && (rb & 3) == 0 && (re & 3) == 0) {
+      for (int q = (rb >> 2) + lid2; q < (re >> 2); q += 32) {
+        const int r = 4 * q;
+        reinterpret_cast<float4*>(dst)[q] = make_float4(src[r], src[r + 1], src[r + 2], src[r + 3]);
+      }
+    } else {
+      for (int r = rb + lid2; r < re; r += 32) dst[r] = src[r];
+    }
   }
 }
 

@@ -28,6 +28,7 @@ template <int N, int T>
 __device__ __forceinline__ void spectral_product(float2* sm, int tid, const float2* __restrict__ H,
                                                  const float2* __restrict__ tw) {
   constexpr int twstep = kTwiddleN / (2 * N);
+#pragma unroll
   for (int k = tid; k <= N / 2; k += T) {
     const int kk = (N - k) & (N - 1);
     const float2 zk = sm[fft_pad(k)], zn = sm[fft_pad(kk)];
@@ -46,12 +47,24 @@ __device__ __forceinline__ void spectral_product(float2* sm, int tid, const floa
   }
 }
 
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+               "l"(src)
+               : "memory");
+}
+
 template <int N, class Sync>
-__device__ __forceinline__ void tile_fft_body(float2* sm, int tid, bool active, const float2* __restrict__ src,
+__device__ __forceinline__ void tile_fft_body(float2* sm, float2* ds, int tid, bool active, const float2* __restrict__ src,
                                               float2* __restrict__ dst, const float2* __restrict__ H,
                                               const float2* __restrict__ tw, int overwrite, Sync sync) {
   constexpr int T = fft_threads(N);
   using S = FftShape<N, T>;
+  // The accumulators this block adds into travel to shared memory while the
+  // transforms run (16-byte asynchronous copies; the target is 16-byte aligned).
+  if (active && !overwrite) {
+    for (int q = tid; q < N / 4; q += T) cp_async16(ds + 2 * q, dst + 2 * q);
+  }
+  asm volatile("cp.async.commit_group;" ::: "memory");
   // Forward pass 0 straight from HBM: z[m] = (x[2m], x[2m+1]) for m < N/2, zero above.
   {
     constexpr int R = 1 << S::rb(0);
@@ -78,6 +91,8 @@ __device__ __forceinline__ void tile_fft_body(float2* sm, int tid, bool active, 
     float2 v[S::P];
     pass_load<N, T, DL>(sm, v, tid);
     pass_compute<N, T, true, DL>(v, tid, tw);
+    asm volatile("cp.async.wait_all;" ::: "memory");
+    sync();
     if (active) {
 #pragma unroll
       for (int k = 0; k < S::P / R; ++k) {
@@ -89,7 +104,7 @@ __device__ __forceinline__ void tile_fft_body(float2* sm, int tid, bool active, 
           if (overwrite) {
             dst[m] = o;
           } else {
-            const float2 p = dst[m];
+            const float2 p = ds[m];
             dst[m] = make_float2(p.x + o.x, p.y + o.y);
           }
         }
@@ -107,6 +122,7 @@ k_tile_fft(Dims g, float* __restrict__ state, const float2* __restrict__ spec,
   extern __shared__ float2 fsm[];
   const int sub = threadIdx.x / T, tid = threadIdx.x - sub * T;
   float2* sm = fsm + sub * fft_smem_elems(N);
+  float2* ds = fsm + F * fft_smem_elems(N) + sub * (N / 2);   // staged accumulators
   const long item = (long)blockIdx.x * F + sub;
   const long items = (long)g.M * g.S;
   const bool active = item < items;
@@ -116,8 +132,8 @@ k_tile_fft(Dims g, float* __restrict__ state, const float2* __restrict__ spec,
   const float2* src = reinterpret_cast<const float2*>(state + slot_index(g, l - 1, s, i - N));
   float2* dst = reinterpret_cast<float2*>(state + slot_index(g, l, s, i));
   const float2* H = spec + ((size_t)(l - 1) * g.D + d) * (N + 1);
-  if constexpr (T <= 32) tile_fft_body<N>(sm, tid, active, src, dst, H, tw, overwrite, SyncWarp());
-  else tile_fft_body<N>(sm, tid, active, src, dst, H, tw, overwrite, SyncBlock());
+  if constexpr (T <= 32) tile_fft_body<N>(sm, ds, tid, active, src, dst, H, tw, overwrite, SyncWarp());
+  else tile_fft_body<N>(sm, ds, tid, active, src, dst, H, tw, overwrite, SyncBlock());
 }
 
 // Spectrum of h[0..2N) / (2N) for one (layer, channel): item = l*D + d.
@@ -191,7 +207,7 @@ static cudaError_t prepare(K kernel, size_t smem) {
 template <int N>
 static cudaError_t tile_fft_n(const Dims& g, float* state, const float2* spec, const float2* tw, int i,
                               cudaStream_t st) {
-  const size_t smem = fft_smem_bytes<N>();
+  const size_t smem = fft_smem_bytes<N>() + (size_t)fft_per_cta(N) * (N / 2) * sizeof(float2);
   cudaError_t e = prepare(k_tile_fft<N>, smem);
   if (e != cudaSuccess) return e;
   const long items = (long)g.M * g.S;
