@@ -160,6 +160,26 @@ FI_API fi_status fi_destroy(fi_ctx* ctx);
 FI_API const char* fi_status_str(fi_status s);
 FI_API const char* fi_last_error(void);
 
+/* One closed-loop generation from position 0 that allocates no device memory.
+ * For callers that cannot call cudaMalloc: code on a thread with a hard latency
+ * budget (an allocation can block in the driver), code inside a host framework
+ * whose device memory belongs to its own allocator, or code running where
+ * allocation is not permitted. The paper has no counterpart to this call.
+ * Computes what fi_init(cfg, h) followed by fi_generate(n, x0, eps, eps_scale,
+ * y_out, NULL) would, with every block of side >= the on-chip chunk summed
+ * directly (no filter spectra). Arguments as for those two calls; cfg->fft_from
+ * is ignored; returns once the generation has finished on `stream`.
+ * Working memory is one file-scope device array of 8 Mi floats (32 MiB) that
+ * every GPU loading the library keeps until the process exits; the call needs
+ * M*D*L + (M+1)*B*D*L + 64 floats of it (rounded up to 64 per part) and
+ * returns FI_E_INVALID, with the sizes in fi_last_error(), when that is more.
+ * All calls share the array and it keeps the last call's contents (each call
+ * rewrites what it reads); calls whose work overlaps on the GPU race on it.
+ * The first call on a device looks up the array's device address.
+ * Errors: FI_E_INVALID (NULL, sizes, L > 2^15), FI_E_CUDA, FI_E_TIMEOUT. */
+FI_API fi_status fi_generate_noalloc(const fi_config* cfg, const void* h, int32_t n, const void* x0,
+                                     const float* eps, float eps_scale, float* y_out, void* stream);
+
 /* Test hook: run the library's device FFT (the one its FFT blocks use) on
  * `count` complex sequences of length 2^log2n (6 <= log2n <= 14), interleaved
  * (re, im) fp32, device buffers in[count][2^log2n][2] -> out (may alias in).

@@ -38,6 +38,8 @@ struct EventPair {
 
 }  // namespace
 
+void fi::set_last_error(const std::string& msg) { g_last_error = msg; }
+
 struct fi_ctx {
   Dims g{};
   fi_config cfg{};

@@ -18,6 +18,8 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include <string>
+
 #include "../../include/fi.h"
 
 namespace fi {
@@ -100,6 +102,9 @@ cudaError_t launch_lazy_sums(const Dims& g, float* state, const float* taps, int
 // Debug: batch of complex FFTs with the tile FFT code.
 cudaError_t launch_debug_fft(int log2n, int count, const float2* in, float2* out, int inverse,
                              const float2* twiddle, cudaStream_t st);
+
+// Message returned by fi_last_error() for the calling thread.
+void set_last_error(const std::string& msg);
 
 // Conversions for fi_init / fi_read_activations.
 cudaError_t launch_widen_filters(const void* h, int bf16, size_t n, float* out, cudaStream_t st);

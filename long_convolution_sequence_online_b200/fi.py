@@ -21,7 +21,8 @@ KERNEL_CLASSES = ("chunk", "direct", "fft", "token", "lazy")
 
 EXPORTED = ("fi_init", "fi_step", "fi_generate", "fi_generate_host", "fi_generate_lazy", "fi_sync", "fi_reset",
             "fi_position", "fi_read_activations", "fi_set_stream", "fi_get_plan", "fi_profile",
-            "fi_profile_read", "fi_destroy", "fi_status_str", "fi_last_error", "fi_debug_fft")
+            "fi_profile_read", "fi_destroy", "fi_status_str", "fi_last_error", "fi_debug_fft",
+            "fi_generate_noalloc")
 
 
 class FiError(RuntimeError):
@@ -58,6 +59,7 @@ def _load():
         "fi_profile_read": [vp, ctypes.POINTER(i32), ctypes.POINTER(ctypes.c_double)],
         "fi_destroy": [vp],
         "fi_debug_fft": [i32, i32, vp, vp, i32, vp],
+        "fi_generate_noalloc": [ctypes.POINTER(Config), vp, i32, vp, vp, f32, vp, vp],
     }
     for name, args in sig.items():
         fn = getattr(lib, name)
@@ -190,6 +192,15 @@ def debug_fft(log2n: int, x, out, inverse: bool = False, stream=None):
     """The library's device FFT on x (complex64 CUDA tensor [count][2^log2n]) into out."""
     count = x.numel() >> log2n
     _check(lib.fi_debug_fft(log2n, count, _ptr(x), _ptr(out), 1 if inverse else 0, _stream(stream)), "fi_debug_fft")
+
+
+def generate_noalloc(h, batch: int, n: int, x0, eps, y_out, dtype: str = "f32", eps_scale: float = 0.1,
+                     chunk: int = 0, stream=None):
+    """fi_generate_noalloc: one generation from position 0 with no device allocation."""
+    M, D, L = (int(v) for v in h.shape)
+    cfg = Config(M, D, L, int(batch), FI_BF16 if dtype == "bf16" else FI_F32, chunk, 0)
+    _check(lib.fi_generate_noalloc(ctypes.byref(cfg), _ptr(h), n, _ptr(x0), _ptr(eps), eps_scale, _ptr(y_out),
+                                   _stream(stream)), "fi_generate_noalloc")
 
 
 def status_str(s: int) -> str:
