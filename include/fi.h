@@ -180,6 +180,12 @@ FI_API const char* fi_last_error(void);
 FI_API fi_status fi_generate_noalloc(const fi_config* cfg, const void* h, int32_t n, const void* x0,
                                      const float* eps, float eps_scale, float* y_out, void* stream);
 
+/* Test hook: the number of barrier checks after which a device-side wait in
+ * later fi_generate calls gives up (negative restores the default, about a
+ * second of waiting). 0 makes every wait that is not already satisfied give up
+ * at once, which exercises the FI_E_TIMEOUT path of fi_sync without any wait. */
+FI_API fi_status fi_debug_set_wait_limit(fi_ctx* ctx, int32_t limit);
+
 /* Test hook: run the library's device FFT (the one its FFT blocks use) on
  * `count` complex sequences of length 2^log2n (6 <= log2n <= 14), interleaved
  * (re, im) fp32, device buffers in[count][2^log2n][2] -> out (may alias in).

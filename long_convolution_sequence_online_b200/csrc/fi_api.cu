@@ -55,7 +55,9 @@ struct fi_ctx {
   float2* spectra = nullptr;
   float2* twiddle = nullptr;
   int* err = nullptr;      // device flag: a bounded wait in a kernel gave up
+  int wait_limit = kDefaultWaitLimit;
   size_t spec_off[32] = {};
+  float2* part_xs = nullptr;       // forward spectra of source sub-blocks (blocks wider than one transform)
   // staging for fi_generate_host
   void* d_x0 = nullptr;
   float* d_eps = nullptr;
@@ -75,6 +77,7 @@ void free_ctx(fi_ctx* c) {
   cudaFree(c->state);
   cudaFree(c->taps);
   cudaFree(c->spectra);
+  cudaFree(c->part_xs);
   cudaFree(c->twiddle);
   cudaFree(c->err);
   cudaFree(c->d_x0);
@@ -124,6 +127,11 @@ fi_status timed(fi_ctx* c, int cls, F&& launch, const char* what) {
 fi_status run_block(fi_ctx* c, int i) {
   const int U = i & -i;
   const int q = ilog2((uint32_t)U);
+  if (q > kMaxFftLog2 && c->q_lo <= kMaxFftLog2) {
+    return timed(c, KC_FFT,
+                 [&] { return launch_part_block(c->g, c->state, c->part_xs, c->spectra + c->spec_off[q], c->twiddle, i, c->st); },
+                 "partitioned FFT block launch");
+  }
   if (q >= c->q_lo && q <= c->q_hi) {
     return timed(c, KC_FFT, [&] { return launch_tile_fft(c->g, c->state, c->spectra + c->spec_off[q], c->twiddle, i, c->st); },
                  "FFT block launch");
@@ -230,8 +238,21 @@ fi_status fi_init(fi_ctx** out, const fi_config* cfg, const void* h, void* strea
     c->spec_off[q] = spec_n;
     spec_n += (size_t)g.M * g.D * ((size_t(1) << q) + 1);
   }
+  // Blocks wider than the largest transform: 2m-1 segment spectra per level.
+  const int q_part_hi = c->q_lo <= kMaxFftLog2 ? g.P - 1 : -1;
+  int m_max = 0;
+  for (int q = kMaxFftLog2 + 1; q <= q_part_hi; ++q) {
+    const int m = 1 << (q - kMaxFftLog2);
+    c->spec_off[q] = spec_n;
+    spec_n += (size_t)g.M * g.D * (2 * m - 1) * ((size_t(1) << kMaxFftLog2) + 1);
+    m_max = m;
+  }
   if (spec_n && (s = dev_alloc((void**)&c->spectra, spec_n * sizeof(float2), "spectra")) != FI_OK) return bail(s);
   if ((s = dev_alloc((void**)&c->twiddle, (size_t)kTwiddleN * sizeof(float2), "twiddles")) != FI_OK) return bail(s);
+  if (m_max > 0 &&
+      (s = dev_alloc((void**)&c->part_xs, (size_t)g.M * g.S * m_max * ((size_t(1) << kMaxFftLog2) + 1) * sizeof(float2),
+                     "wide-block spectra")) != FI_OK)
+    return bail(s);
   if ((s = dev_alloc((void**)&c->err, sizeof(int), "error flag")) != FI_OK) return bail(s);
   if ((e = cudaMemsetAsync(c->err, 0, sizeof(int), c->st)) != cudaSuccess) return bail(cuda_fail(e, "error flag"));
 
@@ -246,6 +267,10 @@ fi_status fi_init(fi_ctx** out, const fi_config* cfg, const void* h, void* strea
   for (int q = c->q_lo; q <= c->q_hi; ++q)
     if ((e = launch_spectra(g, c->taps, c->spectra + c->spec_off[q], c->twiddle, q, c->st)) != cudaSuccess)
       return bail(cuda_fail(e, "spectra precompute"));
+  for (int q = kMaxFftLog2 + 1; q <= q_part_hi; ++q)
+    if ((e = launch_part_spectra(g, c->taps, c->spectra + c->spec_off[q], c->twiddle, 1 << (q - kMaxFftLog2), c->st)) !=
+        cudaSuccess)
+      return bail(cuda_fail(e, "wide-block spectra precompute"));
   if ((e = cudaStreamSynchronize(c->st)) != cudaSuccess) return bail(cuda_fail(e, "fi_init synchronize"));
   *out = c;
   return FI_OK;
@@ -334,6 +359,7 @@ fi_status fi_generate(fi_ctx* c, int32_t n, const void* x0, const float* eps, fl
     a.p1 = p1;
     a.last_done = last_done;
     a.err = c->err;
+    a.wait_limit = c->wait_limit;
     if ((s = timed(c, KC_CHUNK, [&] { return launch_chunk(c->g, a, c->chunk_G, c->st); }, "chunk launch")) != FI_OK)
       return s;
     p = p1;
@@ -431,6 +457,12 @@ fi_status fi_profile_read(fi_ctx* c, int32_t counts[FI_NUM_KERNEL_CLASSES], doub
     c->ev_free.push_back(e);
   }
   c->ev_live.clear();
+  return FI_OK;
+}
+
+fi_status fi_debug_set_wait_limit(fi_ctx* c, int32_t limit) {
+  if (!c) return fail(FI_E_INVALID, "ctx is NULL");
+  c->wait_limit = limit < 0 ? kDefaultWaitLimit : limit;
   return FI_OK;
 }
 

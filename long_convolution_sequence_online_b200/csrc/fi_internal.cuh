@@ -75,6 +75,14 @@ cudaError_t launch_tile_fft(const Dims& g, float* state, const float2* spectrum_
 cudaError_t launch_spectra(const Dims& g, const float* taps, float2* spectrum_q,
                            const float2* twiddle, int q, cudaStream_t st);
 
+// Blocks of side U = m * 2^kMaxFftLog2 (m >= 2): segment spectra of one level,
+// gspec[M][D][2m-1][N+1] (segment e = rFFT_2N(h[eN .. eN+2N)) / 2N), and the
+// block itself (forward transforms into xs[M*S][m][N+1], then inverse ones).
+cudaError_t launch_part_spectra(const Dims& g, const float* taps, float2* gspec, const float2* twiddle, int m,
+                                cudaStream_t st);
+cudaError_t launch_part_block(const Dims& g, float* state, float2* xs, const float2* gspec, const float2* twiddle,
+                              int i, cudaStream_t st);
+
 // The chunk kernel: positions [p0, p1) inside the aligned chunk [c, c+chunk),
 // small blocks (side < chunk) on chip, red cells, blocks and the sampler.
 struct ChunkArgs {
@@ -90,7 +98,12 @@ struct ChunkArgs {
   int c, chunk, p0, p1;  // chunk start, chunk length, positions to produce
   int last_done;         // last step whose blocks have reached HBM before this launch
   int* err;              // device flag set to 1 when a bounded wait gives up
+  int wait_limit;        // barrier checks before a wait gives up
 };
+
+// Default number of barrier checks before a device-side wait gives up (each
+// check lasts at most about a microsecond, so this is far beyond any real wait).
+constexpr int kDefaultWaitLimit = 1 << 20;
 cudaError_t launch_chunk(const Dims& g, const ChunkArgs& a, int streams_per_cta, cudaStream_t st);
 cudaError_t configure_chunk(size_t smem);   // allow `smem` bytes of dynamic shared memory
 int chunk_streams_per_cta(const Dims& g, int chunk, int num_sms, size_t max_smem);

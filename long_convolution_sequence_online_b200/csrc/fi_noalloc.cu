@@ -150,6 +150,7 @@ fi_status fi_generate_noalloc(const fi_config* cfg, const void* h, int32_t n, co
     a.p1 = p1;
     a.last_done = last_done;
     a.err = err;
+    a.wait_limit = kDefaultWaitLimit;
     if ((e = launch_chunk(g, a, G, st)) != cudaSuccess)
       return noalloc_fail(FI_E_CUDA, std::string("chunk launch: ") + cudaGetErrorString(e));
     p = p1;

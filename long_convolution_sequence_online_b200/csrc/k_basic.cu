@@ -80,8 +80,34 @@ __global__ void k_tile_direct(Dims g, float* __restrict__ state, const float* __
   }
 }
 
+// The same block for sides whose taps and sources do not fit in shared memory:
+// taps and sources are read through the cache (every thread of the CTA reads the
+// same source at the same time, and neighbouring threads neighbouring taps).
+__global__ void k_tile_direct_big(Dims g, float* __restrict__ state, const float* __restrict__ taps, int i, int U,
+                                  int overwrite) {
+  const long cta = blockIdx.x;          // ((l-1)*D + d)*B + b
+  const int b = (int)(cta % g.B);
+  const long ld = cta / g.B;
+  const int d = (int)(ld % g.D);
+  const int l = (int)(ld / g.D) + 1;
+  const int s = d * g.B + b;
+  const float* hp = taps + ((size_t)(l - 1) * g.D + d) * g.L;
+  const float* xp = state + slot_index(g, l - 1, s, i - U);
+  float* dp = state + slot_index(g, l, s, i);
+  for (int up = threadIdx.x; up < U; up += blockDim.x) {
+    float sum = 0.f;
+    for (int u = 0; u < U; ++u) sum = fmaf(__ldg(hp + U + up - u), __ldg(xp + u), sum);
+    dp[up] = overwrite ? sum : dp[up] + sum;
+  }
+}
+
 cudaError_t launch_tile_direct(const Dims& g, float* state, const float* taps, int i, cudaStream_t st) {
   const int U = i & -i;
+  const long blocks_big = (long)g.M * g.D * g.B;
+  if (U > 8192) {
+    k_tile_direct_big<<<(unsigned)blocks_big, 256, 0, st>>>(g, state, taps, i, U, is_pow2(i) ? 1 : 0);
+    return cudaGetLastError();
+  }
   const size_t smem = (size_t)3 * U * sizeof(float);
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(k_tile_direct, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

@@ -23,7 +23,6 @@ namespace fi {
 
 constexpr int kChunkMaxThreads = 512;
 constexpr int kChunkMaxStreams = 128;
-constexpr int kSpinLimit = 1 << 20;     // barrier checks before a wait gives up (far beyond any real wait)
 constexpr int kSuspendHintNs = 1000;   // longest a suspended barrier check may last
 
 struct ChunkShape {
@@ -172,10 +171,10 @@ __device__ __forceinline__ bool mbar_try(uint64_t* bar, int parity) {
 }
 // Bounded wait for the phase of `parity` to complete. The chain (critical path)
 // polls; the tile warps let the hardware suspend them between checks. Gives up
-// after kSpinLimit checks, records the failure in *err and returns false, so no
+// after `limit` checks, records the failure in *err and returns false, so no
 // warp can wait forever (each check lasts at most kSuspendHintNs).
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, int parity, int* err, bool poll) {
-  for (int it = 0; it < kSpinLimit; ++it)
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, int parity, int* err, bool poll, int limit) {
+  for (int it = 0; it < limit; ++it)
     if (poll ? mbar_test(bar, parity) : mbar_try(bar, parity)) return true;
   atomicExch(err, 1);
   return false;
@@ -294,7 +293,7 @@ __global__ void __launch_bounds__(kChunkMaxThreads) k_chunk(Dims g, ChunkArgs a,
       float y = 0.f;
       for (int grp = 0; grp < NG; ++grp) {
         const int lg0 = grp * K + 1, lg1 = min(M, (grp + 1) * K);
-        if (!ready && ok) ok = mbar_wait(&tile_done[grp * CW + warp], (r - rs) & 1, err, true);
+        if (!ready && ok) ok = mbar_wait(&tile_done[grp * CW + warp], (r - rs) & 1, err, true, a.wait_limit);
         const int lend = lg1 < M ? lg1 : M - 1;    // layers with a block (tanh) in this group
         float acc = wrow[lg0 * lstride + r];
         float h0 = hrow[(lg0 - 1) * GdMax];
@@ -340,7 +339,7 @@ __global__ void __launch_bounds__(kChunkMaxThreads) k_chunk(Dims g, ChunkArgs a,
       for (int k = tw; k < M * CW; k += ntw) {
         const int l = k / CW + 1, c = k - (l - 1) * CW;
         const int grp = (l - 1) / K;
-        if (r > r0 && ok) ok = mbar_wait(&act_ready[grp * CW + c], (r - 1 - r0) & 1, err, false);
+        if (r > r0 && ok) ok = mbar_wait(&act_ready[grp * CW + c], (r - 1 - r0) & 1, err, false, a.wait_limit);
         const int gg = c * 32 + lane;
         if (gg < Gc) {
           const int dl = (s0 + gg) / g.B - d_lo;

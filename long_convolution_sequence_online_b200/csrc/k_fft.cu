@@ -53,19 +53,25 @@ __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
                : "memory");
 }
 
-template <int N, class Sync>
-__device__ __forceinline__ void tile_fft_body(float2* sm, float2* ds, int tid, bool active, const float2* __restrict__ src,
-                                              float2* __restrict__ dst, const float2* __restrict__ H,
-                                              const float2* __restrict__ tw, int overwrite, Sync sync) {
+// The accumulators a block adds into travel to shared memory while the
+// transforms run (16-byte asynchronous copies; the target is 16-byte aligned).
+template <int N>
+__device__ __forceinline__ void stage_dst(float2* ds, int tid, bool active, const float2* __restrict__ dst,
+                                          int overwrite) {
   constexpr int T = fft_threads(N);
-  using S = FftShape<N, T>;
-  // The accumulators this block adds into travel to shared memory while the
-  // transforms run (16-byte asynchronous copies; the target is 16-byte aligned).
   if (active && !overwrite) {
     for (int q = tid; q < N / 4; q += T) cp_async16(ds + 2 * q, dst + 2 * q);
   }
   asm volatile("cp.async.commit_group;" ::: "memory");
-  // Forward pass 0 straight from HBM: z[m] = (x[2m], x[2m+1]) for m < N/2, zero above.
+}
+
+// Forward transform of z[m] = (x[2m], x[2m+1]) for m < N/2 and zero above,
+// its first pass read straight from HBM; the result is left in sm.
+template <int N, class Sync>
+__device__ __forceinline__ void fwd_from_global(float2* sm, int tid, bool active, const float2* __restrict__ src,
+                                                const float2* __restrict__ tw, Sync sync) {
+  constexpr int T = fft_threads(N);
+  using S = FftShape<N, T>;
   {
     constexpr int R = 1 << S::rb(0);
     float2 v[S::P];
@@ -81,35 +87,148 @@ __device__ __forceinline__ void tile_fft_body(float2* sm, float2* ds, int tid, b
     sync();
   }
   smem_passes<N, T, false, S::rb(0), false>(sm, tid, tw, sync);
-  spectral_product<N, T>(sm, tid, H, tw);
-  sync();
+}
+
+// Inverse transform of the packed spectrum in sm, its last pass written straight
+// to HBM: only outputs m >= N/2 (the block's targets) are kept, added to the
+// staged accumulators (or stored, for the first block to reach them).
+template <int N, class Sync>
+__device__ __forceinline__ void inv_to_global(float2* sm, const float2* ds, int tid, bool active,
+                                              float2* __restrict__ dst, const float2* __restrict__ tw, int overwrite,
+                                              Sync sync) {
+  constexpr int T = fft_threads(N);
+  using S = FftShape<N, T>;
   smem_passes<N, T, true, 0, true>(sm, tid, tw, sync);
-  // Last inverse pass straight to HBM: only outputs m >= N/2 (r >= R/2) are kept.
-  {
-    constexpr int DL = last_pass_done<N, T>();
-    constexpr int R = 1 << S::rb(DL);
-    float2 v[S::P];
-    pass_load<N, T, DL>(sm, v, tid);
-    pass_compute<N, T, true, DL>(v, tid, tw);
-    asm volatile("cp.async.wait_all;" ::: "memory");
-    sync();
-    if (active) {
+  constexpr int DL = last_pass_done<N, T>();
+  constexpr int R = 1 << S::rb(DL);
+  float2 v[S::P];
+  pass_load<N, T, DL>(sm, v, tid);
+  pass_compute<N, T, true, DL>(v, tid, tw);
+  asm volatile("cp.async.wait_all;" ::: "memory");
+  sync();
+  if (active) {
 #pragma unroll
-      for (int k = 0; k < S::P / R; ++k) {
-        const int j = tid + k * T;
+    for (int k = 0; k < S::P / R; ++k) {
+      const int j = tid + k * T;
 #pragma unroll
-        for (int r = R / 2; r < R; ++r) {
-          const int m = j + r * (N / R) - N / 2;
-          const float2 o = v[k * R + r];
-          if (overwrite) {
-            dst[m] = o;
-          } else {
-            const float2 p = ds[m];
-            dst[m] = make_float2(p.x + o.x, p.y + o.y);
-          }
+      for (int r = R / 2; r < R; ++r) {
+        const int m = j + r * (N / R) - N / 2;
+        const float2 o = v[k * R + r];
+        if (overwrite) {
+          dst[m] = o;
+        } else {
+          const float2 p = ds[m];
+          dst[m] = make_float2(p.x + o.x, p.y + o.y);
         }
       }
     }
+  }
+}
+
+template <int N, class Sync>
+__device__ __forceinline__ void tile_fft_body(float2* sm, float2* ds, int tid, bool active, const float2* __restrict__ src,
+                                              float2* __restrict__ dst, const float2* __restrict__ H,
+                                              const float2* __restrict__ tw, int overwrite, Sync sync) {
+  constexpr int T = fft_threads(N);
+  stage_dst<N>(ds, tid, active, dst, overwrite);
+  fwd_from_global<N>(sm, tid, active, src, tw, sync);
+  spectral_product<N, T>(sm, tid, H, tw);
+  sync();
+  inv_to_global<N>(sm, ds, tid, active, dst, tw, overwrite, sync);
+}
+
+// ---------------------------------------------------------------------------
+// Blocks wider than one transform (U = m*N, N the largest transform): split the
+// sources into m sub-blocks S_j of N and the targets into m sub-blocks T_k. The
+// pair (S_j, T_k) is a block of side N whose lags run over
+// h[U + (k-j-1)N + 1 .. U + (k-j+1)N - 1], so with the spectra
+// G_delta = rFFT_2N(h[U + (delta-1)N .. U + (delta+1)N)) / 2N, delta = k-j in
+// [-(m-1), m-1], target T_k receives irFFT_2N(sum_j X_j * G_{k-j})[N..2N), where
+// X_j = rFFT_2N([S_j || 0]). One forward transform per source sub-block goes to
+// a scratch buffer; one inverse transform per target sub-block reads it.
+// ---------------------------------------------------------------------------
+
+// Half spectrum X[0..N] of the real sequence packed in sm, written to out.
+template <int N, int T>
+__device__ __forceinline__ void store_half_spectrum(const float2* sm, int tid, float2* __restrict__ out,
+                                                    const float2* __restrict__ tw) {
+  constexpr int twstep = kTwiddleN / (2 * N);
+  for (int k = tid; k <= N / 2; k += T) {
+    const int kk = (N - k) & (N - 1);
+    const float2 zk = sm[fft_pad(k)], zn = sm[fft_pad(kk)];
+    const float2 E = make_float2(0.5f * (zk.x + zn.x), 0.5f * (zk.y - zn.y));
+    const float2 O = make_float2(0.5f * (zk.y + zn.y), -0.5f * (zk.x - zn.x));
+    const float2 WO = cmul(__ldg(tw + k * twstep), O);
+    out[k] = cadd(E, WO);
+    if (k != N / 2) out[N - k] = cconj(csub(E, WO));
+  }
+}
+
+// item = row * m + j; row = (l-1)*S + s.
+template <int N>
+__global__ void __launch_bounds__(fft_cta_threads(N))
+k_part_fwd(Dims g, const float* __restrict__ state, float2* __restrict__ xs, const float2* __restrict__ tw, int i,
+           int m) {
+  constexpr int T = fft_threads(N), F = fft_per_cta(N);
+  extern __shared__ float2 fsm[];
+  const int sub = threadIdx.x / T, tid = threadIdx.x - sub * T;
+  float2* sm = fsm + sub * fft_smem_elems(N);
+  const long item = (long)blockIdx.x * F + sub;
+  const bool active = item < (long)g.M * g.S * m;
+  const long row = active ? item / m : 0;
+  const int j = active ? (int)(item - row * m) : 0;
+  const int l = (int)(row / g.S) + 1, s = (int)(row % g.S);
+  const int U = m * N;
+  const float2* src = reinterpret_cast<const float2*>(state + slot_index(g, l - 1, s, i - U + j * N));
+  if constexpr (T <= 32) fwd_from_global<N>(sm, tid, active, src, tw, SyncWarp());
+  else fwd_from_global<N>(sm, tid, active, src, tw, SyncBlock());
+  if (active) store_half_spectrum<N, T>(sm, tid, xs + (size_t)item * (N + 1), tw);
+}
+
+// item = row * m + k: target sub-block k of the row.
+template <int N>
+__global__ void __launch_bounds__(fft_cta_threads(N))
+k_part_inv(Dims g, float* __restrict__ state, const float2* __restrict__ xs, const float2* __restrict__ gspec,
+           const float2* __restrict__ tw, int i, int m, int overwrite) {
+  constexpr int T = fft_threads(N), F = fft_per_cta(N);
+  constexpr int twstep = kTwiddleN / (2 * N);
+  extern __shared__ float2 fsm[];
+  const int sub = threadIdx.x / T, tid = threadIdx.x - sub * T;
+  float2* sm = fsm + sub * fft_smem_elems(N);
+  float2* ds = fsm + F * fft_smem_elems(N) + sub * (N / 2);
+  const long item = (long)blockIdx.x * F + sub;
+  const bool active = item < (long)g.M * g.S * m;
+  const long row = active ? item / m : 0;
+  const int k = active ? (int)(item - row * m) : 0;
+  const int l = (int)(row / g.S) + 1, s = (int)(row % g.S), d = s / g.B;
+  float2* dst = reinterpret_cast<float2*>(state + slot_index(g, l, s, i + k * N));
+  // segment spectra of this (layer, channel): [2m-1][N+1], delta = k - j at index delta + m - 1
+  const float2* G = gspec + ((size_t)(l - 1) * g.D + d) * (2 * m - 1) * (N + 1);
+  const float2* X = xs + (size_t)row * m * (N + 1);
+  stage_dst<N>(ds, tid, active, dst, overwrite);
+  for (int f = tid; f <= N / 2; f += T) {
+    const int fn = N - f;
+    float2 yf = make_float2(0.f, 0.f), yn = make_float2(0.f, 0.f);
+    for (int j = 0; j < m; ++j) {
+      const float2* Xj = X + (size_t)j * (N + 1);
+      const float2* Gd = G + (size_t)(k - j + m - 1) * (N + 1);
+      const float2 a = cmul(Xj[f], Gd[f]);
+      const float2 b = cmul(Xj[fn], Gd[fn]);
+      yf = cadd(yf, a);
+      yn = cadd(yn, b);
+    }
+    const float2 W = __ldg(tw + f * twstep);
+    const float2 A = cadd(yf, cconj(yn));
+    const float2 Bv = cmul(csub(yf, cconj(yn)), cconj(W));
+    sm[fft_pad(f & (N - 1))] = make_float2(A.x - Bv.y, A.y + Bv.x);
+    if (f != 0 && f != N / 2) sm[fft_pad(fn)] = make_float2(A.x + Bv.y, -A.y + Bv.x);
+  }
+  if constexpr (T <= 32) {
+    __syncwarp();
+    inv_to_global<N>(sm, ds, tid, active, dst, tw, overwrite, SyncWarp());
+  } else {
+    __syncthreads();
+    inv_to_global<N>(sm, ds, tid, active, dst, tw, overwrite, SyncBlock());
   }
 }
 
@@ -139,15 +258,19 @@ k_tile_fft(Dims g, float* __restrict__ state, const float2* __restrict__ spec,
 // Spectrum of h[0..2N) / (2N) for one (layer, channel): item = l*D + d.
 template <int N>
 __global__ void __launch_bounds__(fft_cta_threads(N))
-k_spectra(Dims g, const float* __restrict__ taps, float2* __restrict__ spec, const float2* __restrict__ tw) {
+k_spectra(Dims g, const float* __restrict__ taps, float2* __restrict__ spec, const float2* __restrict__ tw, int off,
+          int nseg, int seg0) {
   constexpr int T = fft_threads(N), F = fft_per_cta(N);
   constexpr int twstep = kTwiddleN / (2 * N);
   extern __shared__ float2 fsm[];
   const int sub = threadIdx.x / T, tid = threadIdx.x - sub * T;
   float2* sm = fsm + sub * fft_smem_elems(N);
+  // item = (l*D + d)*nseg + segment; segment e reads h[off + (seg0+e)*N .. + 2N)
   const long item = (long)blockIdx.x * F + sub;
-  const bool active = item < (long)g.M * g.D;
-  const float2* src = reinterpret_cast<const float2*>(taps + (size_t)(active ? item : 0) * g.L);
+  const bool active = item < (long)g.M * g.D * nseg;
+  const long ld = active ? item / nseg : 0;
+  const int e = active ? (int)(item - ld * nseg) : 0;
+  const float2* src = reinterpret_cast<const float2*>(taps + (size_t)ld * g.L + off + (size_t)(seg0 + e) * N);
   for (int m = tid; m < N; m += T) sm[fft_pad(m)] = active ? src[m] : make_float2(0.f, 0.f);
   if constexpr (T <= 32) {
     __syncwarp();
@@ -218,13 +341,14 @@ static cudaError_t tile_fft_n(const Dims& g, float* state, const float2* spec, c
 }
 
 template <int N>
-static cudaError_t spectra_n(const Dims& g, const float* taps, float2* spec, const float2* tw, cudaStream_t st) {
+static cudaError_t spectra_n(const Dims& g, const float* taps, float2* spec, const float2* tw, int nseg,
+                             cudaStream_t st) {
   const size_t smem = fft_smem_bytes<N>();
   cudaError_t e = prepare(k_spectra<N>, smem);
   if (e != cudaSuccess) return e;
-  const long items = (long)g.M * g.D;
+  const long items = (long)g.M * g.D * nseg;
   const long blocks = (items + fft_per_cta(N) - 1) / fft_per_cta(N);
-  k_spectra<N><<<(unsigned)blocks, fft_cta_threads(N), smem, st>>>(g, taps, spec, tw);
+  k_spectra<N><<<(unsigned)blocks, fft_cta_threads(N), smem, st>>>(g, taps, spec, tw, 0, nseg, 0);
   return cudaGetLastError();
 }
 
@@ -264,9 +388,32 @@ cudaError_t launch_tile_fft(const Dims& g, float* state, const float2* spectrum_
 
 cudaError_t launch_spectra(const Dims& g, const float* taps, float2* spectrum_q, const float2* twiddle, int q,
                            cudaStream_t st) {
-#define CALL(n) spectra_n<n>(g, taps, spectrum_q, twiddle, st)
+#define CALL(n) spectra_n<n>(g, taps, spectrum_q, twiddle, 1, st)
   FI_FFT_SWITCH(q, CALL)
 #undef CALL
+}
+
+cudaError_t launch_part_spectra(const Dims& g, const float* taps, float2* gspec, const float2* twiddle, int m,
+                                cudaStream_t st) {
+  return spectra_n<1 << kMaxFftLog2>(g, taps, gspec, twiddle, 2 * m - 1, st);
+}
+
+cudaError_t launch_part_block(const Dims& g, float* state, float2* xs, const float2* gspec, const float2* twiddle,
+                              int i, cudaStream_t st) {
+  constexpr int N = 1 << kMaxFftLog2;
+  const int m = (i & -i) / N;
+  const long items = (long)g.M * g.S * m;
+  const long blocks = (items + fft_per_cta(N) - 1) / fft_per_cta(N);
+  size_t smem = fft_smem_bytes<N>();
+  cudaError_t e = prepare(k_part_fwd<N>, smem);
+  if (e != cudaSuccess) return e;
+  k_part_fwd<N><<<(unsigned)blocks, fft_cta_threads(N), smem, st>>>(g, state, xs, twiddle, i, m);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  smem += (size_t)fft_per_cta(N) * (N / 2) * sizeof(float2);
+  if ((e = prepare(k_part_inv<N>, smem)) != cudaSuccess) return e;
+  k_part_inv<N><<<(unsigned)blocks, fft_cta_threads(N), smem, st>>>(g, state, xs, gspec, twiddle, i, m,
+                                                                   is_pow2(i) ? 1 : 0);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_debug_fft(int log2n, int count, const float2* in, float2* out, int inverse,

@@ -22,7 +22,7 @@ KERNEL_CLASSES = ("chunk", "direct", "fft", "token", "lazy")
 EXPORTED = ("fi_init", "fi_step", "fi_generate", "fi_generate_host", "fi_generate_lazy", "fi_sync", "fi_reset",
             "fi_position", "fi_read_activations", "fi_set_stream", "fi_get_plan", "fi_profile",
             "fi_profile_read", "fi_destroy", "fi_status_str", "fi_last_error", "fi_debug_fft",
-            "fi_generate_noalloc")
+            "fi_generate_noalloc", "fi_debug_set_wait_limit")
 
 
 class FiError(RuntimeError):
@@ -60,6 +60,7 @@ def _load():
         "fi_destroy": [vp],
         "fi_debug_fft": [i32, i32, vp, vp, i32, vp],
         "fi_generate_noalloc": [ctypes.POINTER(Config), vp, i32, vp, vp, f32, vp, vp],
+        "fi_debug_set_wait_limit": [vp, i32],
     }
     for name, args in sig.items():
         fn = getattr(lib, name)
@@ -163,6 +164,9 @@ class Context:
 
     def reset(self):
         _check(lib.fi_reset(self._h), "fi_reset")
+
+    def set_wait_limit(self, limit: int):
+        _check(lib.fi_debug_set_wait_limit(self._h, limit), "fi_debug_set_wait_limit")
 
     @property
     def position(self) -> int:

@@ -126,12 +126,21 @@ def first_token(w: Workload, seed: int) -> np.ndarray:
     return _rng(seed, KIND_X0).standard_normal((w.batch, w.channels), dtype=np.float32)
 
 
-def noise(w: Workload, seed: int, n: int | None = None) -> np.ndarray:
-    """Sampler noise eps, float32 [n][B][D] (unscaled N(0,1))."""
+def noise(w: Workload, seed: int, n: int | None = None, threads: int | None = None) -> np.ndarray:
+    """Sampler noise eps, float32 [n][B][D] (unscaled N(0,1)); one stream per sequence."""
     n = w.length if n is None else n
     out = np.empty((n, w.batch, w.channels), dtype=np.float32)
-    for b in range(w.batch):
+
+    def one(b):
         out[:, b, :] = _rng(seed, KIND_EPS, b).standard_normal((n, w.channels), dtype=np.float32)
+
+    threads = threads or min(w.batch, os.cpu_count() or 1, 16)
+    if threads <= 1:
+        for b in range(w.batch):
+            one(b)
+    else:
+        with _cf.ThreadPoolExecutor(threads) as ex:
+            list(ex.map(one, range(w.batch)))
     return out
 
 

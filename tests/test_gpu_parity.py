@@ -234,3 +234,23 @@ def test_state_errors(fi):
     assert e.value.status == fi.FI_E_INVALID
     ctx.generate(0, inp["x0"], inp["eps"], y)   # n = 0 is a no-op
     assert ctx.position == 0
+
+
+def test_bounded_wait_reports_timeout(fi):
+    # With a wait limit of 0 every device-side wait that is not already satisfied
+    # gives up at once: the kernels finish, and fi_sync reports FI_E_TIMEOUT.
+    w = _workload(3, 8, 256, 2)
+    inp = gpu_inputs(w, 2)
+    ctx = fi.Context(inp["h"], w.batch, w.dtype)
+    y = torch.empty((w.length, w.batch, w.channels), dtype=torch.float32, device="cuda")
+    ctx.set_wait_limit(0)
+    ctx.generate(w.length, inp["x0"], inp["eps"], y, 0.1)
+    with pytest.raises(fi.FiError) as e:
+        ctx.sync()
+    assert e.value.status == fi.FI_E_TIMEOUT
+    # the flag was cleared; with the default limit the context works again
+    ctx.set_wait_limit(-1)
+    ctx.reset()
+    ctx.generate(w.length, inp["x0"], inp["eps"], y, 0.1)
+    ctx.sync()
+    assert torch.isfinite(y).all()
