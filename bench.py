@@ -57,7 +57,7 @@ def fft_flops(U: int) -> float:
     return 2 * 2.5 * (2 * U) * math.log2(2 * U) + 7 * U
 
 
-def cost_model(w: synth.Workload, chunk: int, fft_from: int, fft_max: int = 1 << 14):
+def cost_model(w: synth.Workload, chunk: int, fft_from: int, fft_max: int = 1 << 14, tc_max: int = 0):
     """Algorithmic bytes and flops of one full generation, split by kernel class.
 
     Bytes (compulsory HBM traffic of the schedule): per block of side U and (layer,
@@ -66,14 +66,18 @@ def cost_model(w: synth.Workload, chunk: int, fft_from: int, fft_max: int = 1 <<
     (2U*4); per position and (layer, sequence, channel) the accumulator row (4) and
     the activation write (s_x); per position and (sequence, channel) token, noise and
     output (s_x + 4 + 4). Flops: direct block 2U^2, FFT block fft_flops(U), red cell 3.
+    Tensor-core blocks (sides 64..tc_max) count like direct ones: taps, sources,
+    accumulators, 2U^2 flops per row (the Toeplitz product, not the padded MMA work).
     """
     M, D, L, B = w.layers, w.channels, w.length, w.batch
     s = 2 if w.dtype == "bf16" else 4
-    out = {k: {"bytes": 0.0, "flops": 0.0, "blocks": 0} for k in ("chunk", "direct", "fft")}
+    out = {k: {"bytes": 0.0, "flops": 0.0, "blocks": 0} for k in ("chunk", "direct", "fft", "tc")}
     for U, n in schedule_levels(L):
         if U < chunk:
             cls = "chunk"
-        elif fft_from <= U <= fft_max:
+        elif 64 <= U <= tc_max:
+            cls = "tc"
+        elif fft_from and fft_from <= U <= fft_max:
             cls = "fft"
         else:
             cls = "direct"
@@ -283,6 +287,7 @@ KERNEL_SOURCES = {
     "chunk": ["long_convolution_sequence_online_b200/csrc/k_chunk.cu"],
     "fft": ["long_convolution_sequence_online_b200/csrc/k_fft.cu", "long_convolution_sequence_online_b200/csrc/fft.cuh"],
     "direct": ["long_convolution_sequence_online_b200/csrc/k_basic.cu"],
+    "tc": ["long_convolution_sequence_online_b200/csrc/k_tile_tc.cu"],
 }
 
 
@@ -318,10 +323,11 @@ def gpu_arm(args, world, rank, local):
     y_d = torch.empty((w.length, w.batch, w.channels), dtype=torch.float32, device=device)
     stream = torch.cuda.current_stream(device)
     t_init = time.perf_counter()
-    ctx = fi.Context(h_d, w.batch, w.dtype, chunk=args.chunk, fft_from=args.fft_from, stream=stream)
+    ctx = fi.Context(h_d, w.batch, w.dtype, chunk=args.chunk, fft_from=args.fft_from, stream=stream,
+                     tc_max=args.tc_max)
     t_init = time.perf_counter() - t_init
     del h_d
-    chunk, fft_from = ctx.plan()
+    chunk, fft_from, tc_max = ctx.plan()
 
     def step():
         ctx.reset()
@@ -376,9 +382,9 @@ def gpu_arm(args, world, rank, local):
     # --- roofline: dominant kernel class during the timed steps
     peaks = measured_peaks()
     clk = clocks.summary()
-    model, tot = cost_model(w, chunk, fft_from)
+    model, tot = cost_model(w, chunk, fft_from, tc_max=tc_max)
     classes = {}
-    for cls in ("chunk", "direct", "fft"):
+    for cls in ("chunk", "direct", "fft", "tc"):
         n, ms = prof[cls]
         if n == 0:
             continue
@@ -444,7 +450,7 @@ def gpu_arm(args, world, rank, local):
         "config": {"workload": w.name, "layers": w.layers, "channels": w.channels, "seq_len": w.length,
                    "batch": w.batch, "global_batch": w.batch * world, "tokens_per_step": tokens_per_step,
                    "parallelism": f"dp{world}" if world > 1 else "single",
-                   "plan": {"chunk": chunk, "fft_from": fft_from, "fft_max": 1 << 14},
+                   "plan": {"chunk": chunk, "fft_from": fft_from, "fft_max": 1 << 14, "tc_max": tc_max},
                    "l2": "inputs larger than L2 (state 8.6 GB streamed every step)",
                    "step": "fi_reset + fi_generate over all L positions, closed loop",
                    "init_s": t_init},
@@ -471,6 +477,8 @@ def main():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--chunk", type=int, default=0)
     ap.add_argument("--fft-from", dest="fft_from", type=int, default=0)
+    ap.add_argument("--tc-max", dest="tc_max", type=int, default=0,
+                    help="largest block side on the tensor cores (0 = automatic, -1 = none)")
     ap.add_argument("--e2e-steps", dest="e2e_steps", type=int, default=3)
     ap.add_argument("--lazy-prefix", dest="lazy_prefix", type=int, default=4096)
     ap.add_argument("--oracle-positions", dest="oracle_positions", type=int, default=6144)

@@ -67,7 +67,10 @@ typedef struct {
   int32_t dtype;     /* fi_dtype of filters and tokens; accumulation is always fp32 */
   int32_t chunk;     /* 0 = automatic; else block sides below this run on chip (power of two, 2..64) */
   int32_t fft_from;  /* 0 = automatic; else the smallest block side computed by FFT (power of two >= 64) */
-  int32_t reserved[5]; /* must be 0 */
+  int32_t tc_max;    /* 0 = automatic, -1 = never; else block sides 64..tc_max (power of two >= 64) run
+                        on the tensor cores as Toeplitz products (bf16 contexts: exact bf16 products;
+                        fp32 contexts: three bf16 products of split operands), ahead of FFT */
+  int32_t reserved[4]; /* must be 0 */
 } fi_config;
 
 typedef struct fi_ctx fi_ctx;
@@ -139,17 +142,20 @@ FI_API fi_status fi_read_activations(fi_ctx* ctx, int32_t layer, float* dst);
 /* Change the stream later calls run on. */
 FI_API fi_status fi_set_stream(fi_ctx* ctx, void* stream);
 
-/* The block side at or above which the context uses FFT blocks, and the
- * on-chip block bound it chose (after automatic selection). */
-FI_API fi_status fi_get_plan(const fi_ctx* ctx, int32_t* chunk, int32_t* fft_from);
+/* The plan the context chose (after automatic selection): block sides below
+ * *chunk run on chip, sides 64..*tc_max on the tensor cores (0: none), sides
+ * from *fft_from up by FFT (0: none), any other side directly from HBM.
+ * Each pointer may be NULL. */
+FI_API fi_status fi_get_plan(const fi_ctx* ctx, int32_t* chunk, int32_t* fft_from, int32_t* tc_max);
 
 /* Kernel timing. With profiling on, every kernel launch of fi_generate is
  * bracketed by CUDA events on the context's stream; fi_profile_read
  * synchronises and returns, per kernel class, the launch count and the summed
  * device time in milliseconds since the last read. Classes: 0 = on-chip chunk
  * (small blocks + red cells), 1 = direct blocks from HBM, 2 = FFT blocks,
- * 3 = per-position red cells (fi_step / lazy), 4 = lazy sums. */
-#define FI_NUM_KERNEL_CLASSES 5
+ * 3 = per-position red cells (fi_step / lazy), 4 = lazy sums, 5 = tensor-core
+ * blocks. */
+#define FI_NUM_KERNEL_CLASSES 6
 FI_API fi_status fi_profile(fi_ctx* ctx, int32_t enable);
 FI_API fi_status fi_profile_read(fi_ctx* ctx, int32_t counts[FI_NUM_KERNEL_CLASSES],
                           double ms[FI_NUM_KERNEL_CLASSES]);

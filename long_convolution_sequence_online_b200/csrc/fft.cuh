@@ -24,7 +24,12 @@
 
 namespace fi {
 
-__host__ __device__ constexpr int fft_pad(int i) { return i + (i >> 4); }
+// Shared-memory index of point i: one pad slot per 2^PADSHIFT points, with the
+// span chosen so that the strided Stockham stores of a pass hit distinct banks
+// (32 points per thread: one per 32; 16 or fewer: one per 16).
+template <int N, int T>
+__host__ __device__ constexpr int fft_pad(int i) { return i + (i >> ((N / T >= 32) ? 5 : 4)); }
+// Upper bound of the padded length, for any thread count.
 __host__ __device__ constexpr int fft_smem_elems(int n) { return n + (n >> 4); }
 __host__ __device__ constexpr int clog2(int v) { return v <= 1 ? 0 : 1 + clog2(v >> 1); }
 __host__ __device__ constexpr int cmin(int a, int b) { return a < b ? a : b; }
@@ -198,7 +203,7 @@ __device__ __forceinline__ void pass_load(const float2* sm, float2* v, int tid) 
 #pragma unroll
   for (int k = 0; k < S::P / R; ++k) {
 #pragma unroll
-    for (int r = 0; r < R; ++r) v[k * R + r] = sm[fft_pad(tid + k * T + r * (N / R))];
+    for (int r = 0; r < R; ++r) v[k * R + r] = sm[fft_pad<N, T>(tid + k * T + r * (N / R))];
   }
 }
 
@@ -214,7 +219,7 @@ __device__ __forceinline__ void pass_store(float2* sm, const float2* v, int tid)
     const int kk = j & (Ns - 1);
     const int e = (j - kk) * R + kk;
 #pragma unroll
-    for (int r = 0; r < R; ++r) sm[fft_pad(e + r * Ns)] = v[k * R + r];
+    for (int r = 0; r < R; ++r) sm[fft_pad<N, T>(e + r * Ns)] = v[k * R + r];
   }
 }
 
@@ -244,7 +249,7 @@ constexpr int last_pass_done() {
   else return last_pass_done<N, T, DONE + S::rb(DONE)>();
 }
 
-// In-place transform of sm[fft_pad(0..N)) by the T threads with tid in [0, T).
+// In-place transform of sm[fft_pad<N, T>(0..N)) by the T threads with tid in [0, T).
 // Callers synchronise before (data written) and may read results right after.
 template <int N, int T, bool INV, class Sync>
 __device__ __forceinline__ void fft_smem(float2* sm, int tid, const float2* __restrict__ tw, Sync sync) {
@@ -252,9 +257,14 @@ __device__ __forceinline__ void fft_smem(float2* sm, int tid, const float2* __re
   smem_passes<N, T, INV, 0, false>(sm, tid, tw, sync);
 }
 
-// Threads per transform: 32 points per thread from 512 points up (radix-32
-// passes: two passes up to 1024 points, three up to 32768), 16 below.
-__host__ __device__ constexpr int fft_threads(int n) { return n >= 512 ? n / 32 : n / 16; }
+// Threads per transform: 16 or 32 points per thread, whichever measured faster
+// on B200 for the size (an 18 x 3456-row batch at every side): 32 points where
+// radix-32 passes save a pass (512, 1024, 16384) or tie it (4096), 16 elsewhere
+// (half the registers per thread, so twice the resident warps).
+__host__ __device__ constexpr int fft_points_per_thread(int n) {
+  return (n == 512 || n == 1024 || n == 4096 || n == 16384) ? 32 : 16;
+}
+__host__ __device__ constexpr int fft_threads(int n) { return n / fft_points_per_thread(n); }
 // Threads per CTA: whole warps; small transforms share a warp.
 __host__ __device__ constexpr int fft_cta_threads(int n) { return fft_threads(n) >= 128 ? fft_threads(n) : 128; }
 // Transforms per CTA.

@@ -49,6 +49,8 @@ struct fi_ctx {
   int pos = 0;
   int lazy_mode = 0;  // 1 after fi_generate_lazy until fi_reset
   int chunk = 0, fft_from = 0, q_lo = 0, q_hi = -1;
+  int tc_q_hi = -1;                // block sides 2^6 .. 2^tc_q_hi run on the tensor cores
+  TcPlan tc[32] = {};
   int chunk_G = 0;
   float* state = nullptr;
   float* taps = nullptr;
@@ -132,6 +134,11 @@ fi_status run_block(fi_ctx* c, int i) {
                  [&] { return launch_part_block(c->g, c->state, c->part_xs, c->spectra + c->spec_off[q], c->twiddle, i, c->st); },
                  "partitioned FFT block launch");
   }
+  if (q >= kMinFftLog2 && q <= c->tc_q_hi) {
+    return timed(c, KC_TC,
+                 [&] { return launch_tile_tc(c->g, c->state, c->taps, c->tc[q], i, c->err, c->wait_limit, c->st); },
+                 "tensor-core block launch");
+  }
   if (q >= c->q_lo && q <= c->q_hi) {
     return timed(c, KC_FFT, [&] { return launch_tile_fft(c->g, c->state, c->spectra + c->spec_off[q], c->twiddle, i, c->st); },
                  "FFT block launch");
@@ -175,8 +182,10 @@ fi_status fi_init(fi_ctx** out, const fi_config* cfg, const void* h, void* strea
   if (!out) return fail(FI_E_INVALID, "out is NULL");
   *out = nullptr;
   if (!cfg || !h) return fail(FI_E_INVALID, "cfg or h is NULL");
-  for (int k = 0; k < 5; ++k)
+  for (int k = 0; k < 4; ++k)
     if (cfg->reserved[k] != 0) return fail(FI_E_INVALID, "reserved fields must be 0");
+  if (cfg->tc_max != 0 && cfg->tc_max != -1 && (!pow2(cfg->tc_max) || cfg->tc_max < (1 << kMinFftLog2)))
+    return fail(FI_E_INVALID, "tc_max must be 0, -1 or a power of two >= 64");
   if (cfg->layers < 1 || cfg->channels < 1 || cfg->batch < 1) return fail(FI_E_INVALID, "layers, channels, batch must be >= 1");
   if (!pow2(cfg->max_len) || cfg->max_len < 2 || cfg->max_len > (1 << 17))
     return fail(FI_E_INVALID, "max_len must be a power of two in [2, 2^17]");
@@ -223,6 +232,18 @@ fi_status fi_init(fi_ctx** out, const fi_config* cfg, const void* h, void* strea
   c->q_lo = ilog2((uint32_t)c->fft_from);
   c->q_hi = g.P - 1 < kMaxFftLog2 ? g.P - 1 : kMaxFftLog2;
   if (c->q_lo < kMinFftLog2) c->q_lo = kMinFftLog2;
+  // Tensor-core blocks from side 64 up to tc_max (automatic: none yet), ahead
+  // of FFT: the FFT range starts above them.
+  if (cfg->tc_max > 0) {
+    c->tc_q_hi = ilog2((uint32_t)cfg->tc_max);
+    if (c->tc_q_hi > g.P - 1) c->tc_q_hi = g.P - 1;
+    for (int q = kMinFftLog2; q <= c->tc_q_hi; ++q) {
+      if ((e = tc_prepare(g, 1 << q, g.bf16 ? 0 : 1, c->num_sms, &c->tc[q])) != cudaSuccess)
+        return bail(fail(FI_E_UNSUPPORTED, std::string("tensor-core blocks of side ") + std::to_string(1 << q) +
+                                               " cannot be planned for this batch: " + cudaGetErrorString(e)));
+    }
+    if (c->q_lo <= c->tc_q_hi) c->q_lo = c->tc_q_hi + 1;
+  }
   c->chunk_G = chunk_streams_per_cta(g, c->chunk, c->num_sms, c->max_smem);
   if (c->chunk_G == 0) return bail(fail(FI_E_UNSUPPORTED, "too many layers for the on-chip chunk window"));
   if ((e = configure_chunk(chunk_smem_bytes(g, c->chunk, c->chunk_G))) != cudaSuccess)
@@ -302,10 +323,11 @@ fi_status fi_set_stream(fi_ctx* c, void* stream) {
   return FI_OK;
 }
 
-fi_status fi_get_plan(const fi_ctx* c, int32_t* chunk, int32_t* fft_from) {
+fi_status fi_get_plan(const fi_ctx* c, int32_t* chunk, int32_t* fft_from, int32_t* tc_max) {
   if (!c) return fail(FI_E_INVALID, "ctx is NULL");
   if (chunk) *chunk = c->chunk;
   if (fft_from) *fft_from = c->q_lo <= c->q_hi ? (1 << c->q_lo) : 0;
+  if (tc_max) *tc_max = c->tc_q_hi >= kMinFftLog2 ? (1 << c->tc_q_hi) : 0;
   return FI_OK;
 }
 

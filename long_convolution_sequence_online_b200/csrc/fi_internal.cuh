@@ -29,7 +29,7 @@ constexpr int kTwiddleN = 1 << kTwiddleLog2;
 constexpr int kMaxFftLog2 = 14;               // complex FFT points held in one CTA's shared memory
 constexpr int kMinFftLog2 = 6;
 
-enum KernelClass { KC_CHUNK = 0, KC_DIRECT = 1, KC_FFT = 2, KC_TOKEN = 3, KC_LAZY = 4 };
+enum KernelClass { KC_CHUNK = 0, KC_DIRECT = 1, KC_FFT = 2, KC_TOKEN = 3, KC_LAZY = 4, KC_TC = 5 };
 
 struct Dims {
   int M, D, L, B, S;   // layers, channels, max length, batch, streams
@@ -82,6 +82,18 @@ cudaError_t launch_part_spectra(const Dims& g, const float* taps, float2* gspec,
                                 cudaStream_t st);
 cudaError_t launch_part_block(const Dims& g, float* state, float2* xs, const float2* gspec, const float2* twiddle,
                               int i, cudaStream_t st);
+
+// Tensor-core block of side U (k_tile_tc.cu): M-tile rows MT (64 or 128), J
+// target tiles per product, NR operand rows (B*J padded), K steps of 16 over
+// U + (J-1)*MT reversed sources, accumulator columns, split (fp32 contexts:
+// three bf16 products), dynamic shared memory and grid.
+struct TcPlan {
+  int U, MT, J, NR, K, tmem_cols, split, grid;
+  size_t smem;
+};
+cudaError_t tc_prepare(const Dims& g, int U, int split, int num_sms, TcPlan* out);
+cudaError_t launch_tile_tc(const Dims& g, float* state, const float* taps, const TcPlan& p, int i, int* err,
+                           int wait_limit, cudaStream_t st);
 
 // The chunk kernel: positions [p0, p1) inside the aligned chunk [c, c+chunk),
 // small blocks (side < chunk) on chip, red cells, blocks and the sampler.

@@ -58,8 +58,10 @@ extern "C" {
 fi_status fi_generate_noalloc(const fi_config* cfg, const void* h, int32_t n, const void* x0, const float* eps,
                               float eps_scale, float* y_out, void* stream) {
   if (!cfg || !h || !x0 || !eps || !y_out) return noalloc_fail(FI_E_INVALID, "NULL argument");
-  for (int k = 0; k < 5; ++k)
+  for (int k = 0; k < 4; ++k)
     if (cfg->reserved[k] != 0) return noalloc_fail(FI_E_INVALID, "reserved fields must be 0");
+  if (cfg->tc_max != 0 && cfg->tc_max != -1)
+    return noalloc_fail(FI_E_INVALID, "tc_max must be 0 or -1 (this entry point runs direct blocks only)");
   if (cfg->layers < 1 || cfg->channels < 1 || cfg->batch < 1)
     return noalloc_fail(FI_E_INVALID, "layers, channels, batch must be >= 1");
   if (!pow2_i64(cfg->max_len) || cfg->max_len < 2 || cfg->max_len > (1 << 15))

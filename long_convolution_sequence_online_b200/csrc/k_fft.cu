@@ -31,7 +31,7 @@ __device__ __forceinline__ void spectral_product(float2* sm, int tid, const floa
 #pragma unroll
   for (int k = tid; k <= N / 2; k += T) {
     const int kk = (N - k) & (N - 1);
-    const float2 zk = sm[fft_pad(k)], zn = sm[fft_pad(kk)];
+    const float2 zk = sm[fft_pad<N, T>(k)], zn = sm[fft_pad<N, T>(kk)];
     const float2 E = make_float2(0.5f * (zk.x + zn.x), 0.5f * (zk.y - zn.y));
     const float2 O = make_float2(0.5f * (zk.y + zn.y), -0.5f * (zk.x - zn.x));
     const float2 W = __ldg(tw + k * twstep);
@@ -42,8 +42,8 @@ __device__ __forceinline__ void spectral_product(float2* sm, int tid, const floa
     const float2 Yn = cmul(Xn, __ldg(H + (N - k)));
     const float2 A = cadd(Yk, cconj(Yn));
     const float2 Bv = cmul(csub(Yk, cconj(Yn)), cconj(W));
-    sm[fft_pad(k)] = make_float2(A.x - Bv.y, A.y + Bv.x);
-    if (k != 0 && k != N / 2) sm[fft_pad(N - k)] = make_float2(A.x + Bv.y, -A.y + Bv.x);
+    sm[fft_pad<N, T>(k)] = make_float2(A.x - Bv.y, A.y + Bv.x);
+    if (k != 0 && k != N / 2) sm[fft_pad<N, T>(N - k)] = make_float2(A.x + Bv.y, -A.y + Bv.x);
   }
 }
 
@@ -55,10 +55,9 @@ __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
 
 // The accumulators a block adds into travel to shared memory while the
 // transforms run (16-byte asynchronous copies; the target is 16-byte aligned).
-template <int N>
+template <int N, int T>
 __device__ __forceinline__ void stage_dst(float2* ds, int tid, bool active, const float2* __restrict__ dst,
                                           int overwrite) {
-  constexpr int T = fft_threads(N);
   if (active && !overwrite) {
     for (int q = tid; q < N / 4; q += T) cp_async16(ds + 2 * q, dst + 2 * q);
   }
@@ -67,10 +66,9 @@ __device__ __forceinline__ void stage_dst(float2* ds, int tid, bool active, cons
 
 // Forward transform of z[m] = (x[2m], x[2m+1]) for m < N/2 and zero above,
 // its first pass read straight from HBM; the result is left in sm.
-template <int N, class Sync>
+template <int N, int T, class Sync>
 __device__ __forceinline__ void fwd_from_global(float2* sm, int tid, bool active, const float2* __restrict__ src,
                                                 const float2* __restrict__ tw, Sync sync) {
-  constexpr int T = fft_threads(N);
   using S = FftShape<N, T>;
   {
     constexpr int R = 1 << S::rb(0);
@@ -92,11 +90,10 @@ __device__ __forceinline__ void fwd_from_global(float2* sm, int tid, bool active
 // Inverse transform of the packed spectrum in sm, its last pass written straight
 // to HBM: only outputs m >= N/2 (the block's targets) are kept, added to the
 // staged accumulators (or stored, for the first block to reach them).
-template <int N, class Sync>
+template <int N, int T, class Sync>
 __device__ __forceinline__ void inv_to_global(float2* sm, const float2* ds, int tid, bool active,
                                               float2* __restrict__ dst, const float2* __restrict__ tw, int overwrite,
                                               Sync sync) {
-  constexpr int T = fft_threads(N);
   using S = FftShape<N, T>;
   smem_passes<N, T, true, 0, true>(sm, tid, tw, sync);
   constexpr int DL = last_pass_done<N, T>();
@@ -125,16 +122,15 @@ __device__ __forceinline__ void inv_to_global(float2* sm, const float2* ds, int 
   }
 }
 
-template <int N, class Sync>
+template <int N, int T, class Sync>
 __device__ __forceinline__ void tile_fft_body(float2* sm, float2* ds, int tid, bool active, const float2* __restrict__ src,
                                               float2* __restrict__ dst, const float2* __restrict__ H,
                                               const float2* __restrict__ tw, int overwrite, Sync sync) {
-  constexpr int T = fft_threads(N);
-  stage_dst<N>(ds, tid, active, dst, overwrite);
-  fwd_from_global<N>(sm, tid, active, src, tw, sync);
+  stage_dst<N, T>(ds, tid, active, dst, overwrite);
+  fwd_from_global<N, T>(sm, tid, active, src, tw, sync);
   spectral_product<N, T>(sm, tid, H, tw);
   sync();
-  inv_to_global<N>(sm, ds, tid, active, dst, tw, overwrite, sync);
+  inv_to_global<N, T>(sm, ds, tid, active, dst, tw, overwrite, sync);
 }
 
 // ---------------------------------------------------------------------------
@@ -155,7 +151,7 @@ __device__ __forceinline__ void store_half_spectrum(const float2* sm, int tid, f
   constexpr int twstep = kTwiddleN / (2 * N);
   for (int k = tid; k <= N / 2; k += T) {
     const int kk = (N - k) & (N - 1);
-    const float2 zk = sm[fft_pad(k)], zn = sm[fft_pad(kk)];
+    const float2 zk = sm[fft_pad<N, T>(k)], zn = sm[fft_pad<N, T>(kk)];
     const float2 E = make_float2(0.5f * (zk.x + zn.x), 0.5f * (zk.y - zn.y));
     const float2 O = make_float2(0.5f * (zk.y + zn.y), -0.5f * (zk.x - zn.x));
     const float2 WO = cmul(__ldg(tw + k * twstep), O);
@@ -180,8 +176,8 @@ k_part_fwd(Dims g, const float* __restrict__ state, float2* __restrict__ xs, con
   const int l = (int)(row / g.S) + 1, s = (int)(row % g.S);
   const int U = m * N;
   const float2* src = reinterpret_cast<const float2*>(state + slot_index(g, l - 1, s, i - U + j * N));
-  if constexpr (T <= 32) fwd_from_global<N>(sm, tid, active, src, tw, SyncWarp());
-  else fwd_from_global<N>(sm, tid, active, src, tw, SyncBlock());
+  if constexpr (T <= 32) fwd_from_global<N, T>(sm, tid, active, src, tw, SyncWarp());
+  else fwd_from_global<N, T>(sm, tid, active, src, tw, SyncBlock());
   if (active) store_half_spectrum<N, T>(sm, tid, xs + (size_t)item * (N + 1), tw);
 }
 
@@ -205,7 +201,7 @@ k_part_inv(Dims g, float* __restrict__ state, const float2* __restrict__ xs, con
   // segment spectra of this (layer, channel): [2m-1][N+1], delta = k - j at index delta + m - 1
   const float2* G = gspec + ((size_t)(l - 1) * g.D + d) * (2 * m - 1) * (N + 1);
   const float2* X = xs + (size_t)row * m * (N + 1);
-  stage_dst<N>(ds, tid, active, dst, overwrite);
+  stage_dst<N, T>(ds, tid, active, dst, overwrite);
   for (int f = tid; f <= N / 2; f += T) {
     const int fn = N - f;
     float2 yf = make_float2(0.f, 0.f), yn = make_float2(0.f, 0.f);
@@ -220,24 +216,25 @@ k_part_inv(Dims g, float* __restrict__ state, const float2* __restrict__ xs, con
     const float2 W = __ldg(tw + f * twstep);
     const float2 A = cadd(yf, cconj(yn));
     const float2 Bv = cmul(csub(yf, cconj(yn)), cconj(W));
-    sm[fft_pad(f & (N - 1))] = make_float2(A.x - Bv.y, A.y + Bv.x);
-    if (f != 0 && f != N / 2) sm[fft_pad(fn)] = make_float2(A.x + Bv.y, -A.y + Bv.x);
+    sm[fft_pad<N, T>(f & (N - 1))] = make_float2(A.x - Bv.y, A.y + Bv.x);
+    if (f != 0 && f != N / 2) sm[fft_pad<N, T>(fn)] = make_float2(A.x + Bv.y, -A.y + Bv.x);
   }
   if constexpr (T <= 32) {
     __syncwarp();
-    inv_to_global<N>(sm, ds, tid, active, dst, tw, overwrite, SyncWarp());
+    inv_to_global<N, T>(sm, ds, tid, active, dst, tw, overwrite, SyncWarp());
   } else {
     __syncthreads();
-    inv_to_global<N>(sm, ds, tid, active, dst, tw, overwrite, SyncBlock());
+    inv_to_global<N, T>(sm, ds, tid, active, dst, tw, overwrite, SyncBlock());
   }
 }
 
-// One FFT block for every (layer, stream): item = (l-1)*S + s.
-template <int N>
-__global__ void __launch_bounds__(fft_cta_threads(N))
+// One FFT block for every (layer, stream): item = (l-1)*S + s. T threads per
+// transform, F = cta_threads / T transforms per CTA.
+template <int N, int T = fft_threads(N)>
+__global__ void __launch_bounds__(T >= 128 ? T : 128)
 k_tile_fft(Dims g, float* __restrict__ state, const float2* __restrict__ spec,
            const float2* __restrict__ tw, int i, int overwrite) {
-  constexpr int T = fft_threads(N), F = fft_per_cta(N);
+  constexpr int F = T >= 128 ? 1 : 128 / T;
   extern __shared__ float2 fsm[];
   const int sub = threadIdx.x / T, tid = threadIdx.x - sub * T;
   float2* sm = fsm + sub * fft_smem_elems(N);
@@ -251,8 +248,8 @@ k_tile_fft(Dims g, float* __restrict__ state, const float2* __restrict__ spec,
   const float2* src = reinterpret_cast<const float2*>(state + slot_index(g, l - 1, s, i - N));
   float2* dst = reinterpret_cast<float2*>(state + slot_index(g, l, s, i));
   const float2* H = spec + ((size_t)(l - 1) * g.D + d) * (N + 1);
-  if constexpr (T <= 32) tile_fft_body<N>(sm, ds, tid, active, src, dst, H, tw, overwrite, SyncWarp());
-  else tile_fft_body<N>(sm, ds, tid, active, src, dst, H, tw, overwrite, SyncBlock());
+  if constexpr (T <= 32) tile_fft_body<N, T>(sm, ds, tid, active, src, dst, H, tw, overwrite, SyncWarp());
+  else tile_fft_body<N, T>(sm, ds, tid, active, src, dst, H, tw, overwrite, SyncBlock());
 }
 
 // Spectrum of h[0..2N) / (2N) for one (layer, channel): item = l*D + d.
@@ -271,7 +268,7 @@ k_spectra(Dims g, const float* __restrict__ taps, float2* __restrict__ spec, con
   const long ld = active ? item / nseg : 0;
   const int e = active ? (int)(item - ld * nseg) : 0;
   const float2* src = reinterpret_cast<const float2*>(taps + (size_t)ld * g.L + off + (size_t)(seg0 + e) * N);
-  for (int m = tid; m < N; m += T) sm[fft_pad(m)] = active ? src[m] : make_float2(0.f, 0.f);
+  for (int m = tid; m < N; m += T) sm[fft_pad<N, T>(m)] = active ? src[m] : make_float2(0.f, 0.f);
   if constexpr (T <= 32) {
     __syncwarp();
     fft_smem<N, T, false>(sm, tid, tw, SyncWarp());
@@ -284,7 +281,7 @@ k_spectra(Dims g, const float* __restrict__ taps, float2* __restrict__ spec, con
   const float scale = 1.0f / (2.0f * N);
   for (int k = tid; k <= N / 2; k += T) {
     const int kk = (N - k) & (N - 1);
-    const float2 zk = sm[fft_pad(k)], zn = sm[fft_pad(kk)];
+    const float2 zk = sm[fft_pad<N, T>(k)], zn = sm[fft_pad<N, T>(kk)];
     const float2 E = make_float2(0.5f * (zk.x + zn.x), 0.5f * (zk.y - zn.y));
     const float2 O = make_float2(0.5f * (zk.y + zn.y), -0.5f * (zk.x - zn.x));
     const float2 WO = cmul(__ldg(tw + k * twstep), O);
@@ -303,7 +300,7 @@ k_debug_fft(int count, const float2* __restrict__ in, float2* __restrict__ out, 
   float2* sm = fsm + sub * fft_smem_elems(N);
   const long item = (long)blockIdx.x * F + sub;
   const bool active = item < count;
-  for (int m = tid; m < N; m += T) sm[fft_pad(m)] = active ? in[item * N + m] : make_float2(0.f, 0.f);
+  for (int m = tid; m < N; m += T) sm[fft_pad<N, T>(m)] = active ? in[item * N + m] : make_float2(0.f, 0.f);
   if constexpr (T <= 32) {
     __syncwarp();
     if (inverse) fft_smem<N, T, true>(sm, tid, tw, SyncWarp());
@@ -314,7 +311,7 @@ k_debug_fft(int count, const float2* __restrict__ in, float2* __restrict__ out, 
     else fft_smem<N, T, false>(sm, tid, tw, SyncBlock());
   }
   if (!active) return;
-  for (int m = tid; m < N; m += T) out[item * N + m] = sm[fft_pad(m)];
+  for (int m = tid; m < N; m += T) out[item * N + m] = sm[fft_pad<N, T>(m)];
 }
 
 // ------------------------------------------------------------------ dispatch
@@ -327,16 +324,17 @@ static cudaError_t prepare(K kernel, size_t smem) {
   return cudaSuccess;
 }
 
-template <int N>
+template <int N, int T = fft_threads(N)>
 static cudaError_t tile_fft_n(const Dims& g, float* state, const float2* spec, const float2* tw, int i,
                               cudaStream_t st) {
-  const size_t smem = fft_smem_bytes<N>() + (size_t)fft_per_cta(N) * (N / 2) * sizeof(float2);
-  cudaError_t e = prepare(k_tile_fft<N>, smem);
+  constexpr int F = T >= 128 ? 1 : 128 / T;
+  const size_t smem = (size_t)F * (fft_smem_elems(N) + N / 2) * sizeof(float2);
+  cudaError_t e = prepare(k_tile_fft<N, T>, smem);
   if (e != cudaSuccess) return e;
   const long items = (long)g.M * g.S;
-  const long blocks = (items + fft_per_cta(N) - 1) / fft_per_cta(N);
+  const long blocks = (items + F - 1) / F;
   const int overwrite = is_pow2(i) ? 1 : 0;
-  k_tile_fft<N><<<(unsigned)blocks, fft_cta_threads(N), smem, st>>>(g, state, spec, tw, i, overwrite);
+  k_tile_fft<N, T><<<(unsigned)blocks, T * F, smem, st>>>(g, state, spec, tw, i, overwrite);
   return cudaGetLastError();
 }
 

@@ -1,0 +1,341 @@
+// Gray blocks on the 5th-generation tensor cores (tcgen05, accumulators in
+// tensor memory).
+//
+// The block of step i (side U = lowbit(i), the page's tau(a, [i-U, i-1], h,
+// [i, i+U-1]), "Definizione di Aggregazione di Contribuzione") is, for one
+// (layer, channel) and the B sequences that share its filter, a Toeplitz
+// product Y[u'][b] = sum_u h[U + u' - u] X[u][b]. Written with the sources in
+// reverse order, kappa = i - 1 - u, the matrix becomes a Hankel one,
+// A[r][kappa] = h[r + kappa + 1], whose rows are overlapping windows of the
+// filter. The tensor-core operand descriptor can express that directly: a table
+// of 16-byte entries, entry sigma = h[sigma+1 .. sigma+8] in bf16, read as a
+// K-major operand with both the row-group stride and the K-half stride equal to
+// one core matrix (128 bytes, 8 entries). Nothing of the U x U matrix is ever
+// materialised: the table holds 2U entries.
+//
+// Several target tiles share one product: tile j (targets i + j*MT .. + MT) uses
+// the same table when its sources sit kappa = j*MT further along, so the B
+// operand holds, for each tile j of a group and each sequence b, one row with
+// the sources placed at kappa in [j*MT, j*MT + U) and zeros elsewhere. Narrow
+// batches (B = 4) thus still fill N = B*J >= 8 columns of the instruction.
+//
+// Precision: bf16 contexts hold bf16-exact filters and activations, so one
+// bf16 x bf16 -> fp32 product per K step is exact up to fp32 accumulation. fp32
+// contexts split both operands, v = hi + lo with hi = bf16(v) and
+// lo = bf16(v - hi), and add the three products hi*hi + hi*lo + lo*hi (the
+// dropped lo*lo term and the residuals are below 2^-16 relative per product).
+//
+// One CTA of 4 warps per (layer, channel) item at a time: all threads build the
+// table and the B operand in shared memory, one thread issues the MMAs of every
+// group (each group into its own accumulator columns), a commit arrives on an
+// mbarrier, and each warp reads its 32 accumulator lanes and adds them to the
+// targets in HBM. Every wait is bounded.
+#include "fi_internal.cuh"
+
+namespace fi {
+
+namespace {
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// K-major operand without swizzle: start, leading (K-half) and stride
+// (8-row group) byte offsets, all in 16-byte units; version 1 (bits 46-47).
+__device__ __forceinline__ uint64_t smem_desc(uint32_t start, uint32_t lbo, uint32_t sbo) {
+  return (uint64_t)((start >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+         ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46);
+}
+
+// Instruction descriptor, kind::f16: fp32 accumulator, bf16 A and B, both
+// K-major, N >> 3 at bit 17, M >> 4 at bit 24.
+__host__ __device__ constexpr uint32_t tc_idesc(int M, int N) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_bf16(uint32_t dtmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+      ::"r"(dtmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate) : "memory");
+}
+
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+               ::"r"(smem_addr(bar)) : "memory");
+}
+
+__device__ __forceinline__ void fence_before_sync() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void fence_after_sync() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+__device__ __forceinline__ bool bar_try(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok) : "r"(smem_addr(bar)), "r"(parity), "r"(1000u) : "memory");
+  return ok != 0;
+}
+
+__device__ __forceinline__ bool bar_wait(uint64_t* bar, uint32_t parity, int limit) {
+  for (int it = 0; it < limit; ++it)
+    if (bar_try(bar, parity)) return true;
+  return false;
+}
+
+// 16 accumulator columns of this warp's 32 lanes.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int k = 0; k < 16; ++k) v[k] = __uint_as_float(r[k]);
+}
+
+__device__ __forceinline__ uint16_t bf16_bits(float v) {
+  return __bfloat16_as_ushort(__float2bfloat16_rn(v));
+}
+// hi = bf16(v), lo = bf16(v - hi)
+__device__ __forceinline__ void split_bf16(float v, uint16_t& hi, uint16_t& lo) {
+  const __nv_bfloat16 h = __float2bfloat16_rn(v);
+  hi = __bfloat16_as_ushort(h);
+  lo = bf16_bits(v - __bfloat162float(h));
+}
+
+}  // namespace
+
+// Byte offset of element (row n, column k) of a K-major operand with R rows
+// (R a multiple of 8) in core-matrix order: core (n/8, k/8) at
+// ((k/8)*(R/8) + n/8) * 128, rows 16 bytes apart, elements 2 bytes apart.
+__host__ __device__ constexpr uint32_t tc_b_offset(int R, int n, int k) {
+  return (uint32_t)(((k >> 3) * (R >> 3) + (n >> 3)) * 128 + (n & 7) * 16 + (k & 7) * 2);
+}
+
+template <int MT, bool SPLIT>
+__global__ void __launch_bounds__(128) k_tile_tc(Dims g, float* __restrict__ state, const float* __restrict__ taps,
+                                                 TcPlan p, int i, int overwrite, int* err, int wait_limit) {
+  extern __shared__ __align__(1024) unsigned char tsm[];
+  __shared__ uint64_t mma_bar;
+  __shared__ uint32_t tmem_base_s;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int U = p.U, J = p.J, NR = p.NR, K = p.K;
+  const int NT = U / MT, groups = NT / J;
+  const uint32_t idesc = tc_idesc(MT, NR);
+  // shared memory: table hi [2U][16 B], (table lo), X hi [NR rows][K], (X lo)
+  unsigned char* tab_hi = tsm;
+  unsigned char* tab_lo = tsm + (size_t)32 * U;
+  unsigned char* x_hi = tsm + (SPLIT ? 2 : 1) * (size_t)32 * U;
+  unsigned char* x_lo = x_hi + (size_t)NR * K * 2;
+  const size_t xbytes = (size_t)NR * K * 2;
+
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                 ::"r"(smem_addr(&tmem_base_s)), "r"(p.tmem_cols) : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  if (tid == 0) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_addr(&mma_bar)) : "memory");
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  fence_before_sync();
+  __syncthreads();
+  fence_after_sync();
+  const uint32_t tmem = tmem_base_s;
+  bool ok = true;
+  uint32_t phase = 0;
+
+  const long items = (long)g.M * g.D;
+  for (long item = blockIdx.x; item < items && ok; item += gridDim.x) {
+    const int l = (int)(item / g.D) + 1;
+    const int d = (int)(item - (long)(l - 1) * g.D);
+    const float* hp = taps + ((size_t)(l - 1) * g.D + d) * g.L;
+
+    // Table: entry s = h[s+1 .. s+8] (taps beyond 2U-1 are never multiplied by
+    // a nonzero source; they read as the filter's next taps or zero).
+    for (int s = tid; s < 2 * U; s += 128) {
+      uint32_t wh[4], wl[4];
+#pragma unroll
+      for (int e = 0; e < 8; e += 2) {
+        const int k0 = s + 1 + e, k1 = s + 2 + e;
+        const float v0 = k0 < g.L ? __ldg(hp + k0) : 0.f;
+        const float v1 = k1 < g.L ? __ldg(hp + k1) : 0.f;
+        uint16_t h0, l0, h1, l1;
+        if constexpr (SPLIT) {
+          split_bf16(v0, h0, l0);
+          split_bf16(v1, h1, l1);
+        } else {
+          h0 = bf16_bits(v0); h1 = bf16_bits(v1); l0 = l1 = 0;
+        }
+        wh[e / 2] = (uint32_t)h0 | ((uint32_t)h1 << 16);
+        wl[e / 2] = (uint32_t)l0 | ((uint32_t)l1 << 16);
+      }
+      *reinterpret_cast<uint4*>(tab_hi + (size_t)s * 16) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
+      if constexpr (SPLIT) *reinterpret_cast<uint4*>(tab_lo + (size_t)s * 16) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
+    }
+    // B operand: zero, then the sources of each (tile j, sequence b) row.
+    for (size_t q = (size_t)tid * 16; q < xbytes; q += 128 * 16) {
+      *reinterpret_cast<uint4*>(x_hi + q) = make_uint4(0, 0, 0, 0);
+      if constexpr (SPLIT) *reinterpret_cast<uint4*>(x_lo + q) = make_uint4(0, 0, 0, 0);
+    }
+    __syncthreads();
+    {
+      const int quads = U / 4;
+      for (int w = tid; w < g.B * quads; w += 128) {
+        const int b = w / quads, q4 = w - b * quads;
+        const float4 v = *reinterpret_cast<const float4*>(state + slot_index(g, l - 1, d * g.B + b, i - U) + 4 * q4);
+        // kappa = U - 1 - (4 q4 + e) for element e; four consecutive kappa from kb
+        const int kb = U - 4 - 4 * q4;
+        uint16_t hi[4], lo[4];
+        const float vv[4] = {v.w, v.z, v.y, v.x};   // kappa kb, kb+1, kb+2, kb+3
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          if constexpr (SPLIT) split_bf16(vv[e], hi[e], lo[e]);
+          else { hi[e] = bf16_bits(vv[e]); lo[e] = 0; }
+        }
+        const uint2 wh = make_uint2((uint32_t)hi[0] | ((uint32_t)hi[1] << 16), (uint32_t)hi[2] | ((uint32_t)hi[3] << 16));
+        const uint2 wl = make_uint2((uint32_t)lo[0] | ((uint32_t)lo[1] << 16), (uint32_t)lo[2] | ((uint32_t)lo[3] << 16));
+        for (int j = 0; j < J; ++j) {
+          const uint32_t off = tc_b_offset(NR, j * g.B + b, j * MT + kb);
+          *reinterpret_cast<uint2*>(x_hi + off) = wh;
+          if constexpr (SPLIT) *reinterpret_cast<uint2*>(x_lo + off) = wl;
+        }
+      }
+    }
+    fence_proxy_async();   // generic-proxy writes -> visible to the tensor core
+    __syncthreads();
+
+    if (tid == 0) {
+      fence_after_sync();
+      const uint32_t lbo_b = (uint32_t)(NR / 8) * 128;
+      for (int gi = 0; gi < groups; ++gi) {
+        const uint32_t dcol = tmem + (uint32_t)(gi * NR);
+        for (int ks = 0; ks < K / 16; ++ks) {
+          const uint32_t a_off = (uint32_t)(gi * J * MT + 16 * ks) * 16;
+          const uint32_t b_off = (uint32_t)(2 * ks) * lbo_b;
+          const uint64_t ah = smem_desc(smem_addr(tab_hi) + a_off, 128, 128);
+          const uint64_t bh = smem_desc(smem_addr(x_hi) + b_off, lbo_b, 128);
+          mma_bf16(dcol, ah, bh, idesc, ks > 0 ? 1u : 0u);
+          if constexpr (SPLIT) {
+            const uint64_t al = smem_desc(smem_addr(tab_lo) + a_off, 128, 128);
+            const uint64_t bl = smem_desc(smem_addr(x_lo) + b_off, lbo_b, 128);
+            mma_bf16(dcol, ah, bl, idesc, 1u);
+            mma_bf16(dcol, al, bh, idesc, 1u);
+          }
+        }
+      }
+      mma_commit(&mma_bar);
+    }
+    __syncwarp();
+    // Every thread waits (bounded); the CTA leaves together if any gave up.
+    const bool arrived = bar_wait(&mma_bar, phase, wait_limit);
+    if (__syncthreads_or(!arrived)) {
+      if (tid == 0) atomicExch(err, 1);
+      ok = false;
+      break;
+    }
+    phase ^= 1u;
+    fence_after_sync();
+
+    // Epilogue: row r of tile (gi*J + j) is target i + (gi*J + j)*MT + r;
+    // accumulator lane 32*warp + lane holds row 32*warp + lane (MT = 128) or,
+    // for MT = 64, lanes 0-15 of each warp hold rows 16*warp + lane.
+    const int r = MT == 128 ? 32 * warp + lane : 16 * warp + lane;
+    const bool row_ok = MT == 128 || lane < 16;
+    const int cols = groups * NR;
+    for (int c0 = 0; c0 < cols; c0 += 16) {
+      float v[16];
+      tmem_ld16(tmem + ((uint32_t)(32 * warp) << 16) + (uint32_t)c0, v);
+      if (!row_ok) continue;
+#pragma unroll
+      for (int k = 0; k < 16; ++k) {
+        const int c = c0 + k;
+        const int gi = c / NR, n = c - gi * NR;
+        if (c >= cols || n >= J * g.B) continue;
+        const int j = n / g.B, b = n - j * g.B;
+        float* dst = state + slot_index(g, l, d * g.B + b, i + (gi * J + j) * MT + r);
+        *dst = overwrite ? v[k] : *dst + v[k];
+      }
+    }
+    fence_before_sync();
+    __syncthreads();
+  }
+
+  if (!ok) {
+    // The commit did not arrive in time: give the MMAs another bounded wait
+    // before the accumulator columns are released.
+    bar_wait(&mma_bar, phase, wait_limit);
+  }
+  fence_before_sync();
+  __syncthreads();
+  fence_after_sync();
+  if (warp == 0)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(p.tmem_cols) : "memory");
+}
+
+// ------------------------------------------------------------------ host side
+static int pow2_at_least(int v) { int r = 1; while (r < v) r <<= 1; return r; }
+
+template <int MT, bool SPLIT>
+static cudaError_t tc_occupancy(const TcPlan& p, int* per_sm) {
+  auto kern = k_tile_tc<MT, SPLIT>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem);
+  if (e != cudaSuccess) return e;
+  return cudaOccupancyMaxActiveBlocksPerMultiprocessor(per_sm, kern, 128, p.smem);
+}
+
+cudaError_t tc_prepare(const Dims& g, int U, int split, int num_sms, TcPlan* out) {
+  if (U < 64 || (U & (U - 1)) || U > g.L / 2) return cudaErrorInvalidValue;
+  TcPlan p{};
+  p.U = U;
+  p.MT = (U >= 128 && g.B % 16 == 0) ? 128 : 64;
+  const int NT = U / p.MT;
+  // tiles per group: enough that N = B*J reaches 16 columns
+  int J = 1;
+  while (J < NT && g.B * J < 16) J <<= 1;
+  p.J = J;
+  const int mult = p.MT == 128 ? 16 : 8;
+  p.NR = (g.B * J + mult - 1) / mult * mult;
+  if (p.NR > 256) return cudaErrorInvalidValue;
+  p.K = U + (J - 1) * p.MT;
+  const int cols = (NT / J) * p.NR;
+  if (cols > 512) return cudaErrorInvalidValue;
+  p.tmem_cols = pow2_at_least(cols < 32 ? 32 : cols);
+  p.split = split;
+  // Operands, plus slack past the last one: a B-operand read with its two
+  // strides exchanged would stay inside the allocation.
+  p.smem = (size_t)(split ? 2 : 1) * ((size_t)32 * U + (size_t)p.NR * p.K * 2) + (size_t)p.NR * p.NR * 2 + 256;
+  int occ = 0;
+  cudaError_t e = p.MT == 128 ? (split ? tc_occupancy<128, true>(p, &occ) : tc_occupancy<128, false>(p, &occ))
+                              : (split ? tc_occupancy<64, true>(p, &occ) : tc_occupancy<64, false>(p, &occ));
+  if (e != cudaSuccess) return e;
+  // every resident CTA holds its accumulator columns for its whole life
+  const int by_tmem = 512 / p.tmem_cols;
+  const int per_sm = occ < by_tmem ? occ : by_tmem;
+  if (per_sm < 1) return cudaErrorInvalidConfiguration;
+  const long items = (long)g.M * g.D;
+  long grid = (long)num_sms * per_sm;
+  p.grid = (int)(grid > items ? items : grid);
+  *out = p;
+  return cudaSuccess;
+}
+
+cudaError_t launch_tile_tc(const Dims& g, float* state, const float* taps, const TcPlan& p, int i, int* err,
+                           int wait_limit, cudaStream_t st) {
+  if ((i & -i) != p.U || p.grid < 1) return cudaErrorInvalidValue;
+  const int ow = is_pow2(i) ? 1 : 0;
+  if (p.MT == 128) {
+    if (p.split) k_tile_tc<128, true><<<p.grid, 128, p.smem, st>>>(g, state, taps, p, i, ow, err, wait_limit);
+    else k_tile_tc<128, false><<<p.grid, 128, p.smem, st>>>(g, state, taps, p, i, ow, err, wait_limit);
+  } else {
+    if (p.split) k_tile_tc<64, true><<<p.grid, 128, p.smem, st>>>(g, state, taps, p, i, ow, err, wait_limit);
+    else k_tile_tc<64, false><<<p.grid, 128, p.smem, st>>>(g, state, taps, p, i, ow, err, wait_limit);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace fi

@@ -16,8 +16,8 @@ LIB_PATH = os.path.join(_HERE, "libfi.so")
 
 FI_OK, FI_E_INVALID, FI_E_OOM, FI_E_CUDA, FI_E_STATE, FI_E_TIMEOUT, FI_E_UNSUPPORTED = range(7)
 FI_F32, FI_BF16 = 0, 1
-NUM_KERNEL_CLASSES = 5
-KERNEL_CLASSES = ("chunk", "direct", "fft", "token", "lazy")
+NUM_KERNEL_CLASSES = 6
+KERNEL_CLASSES = ("chunk", "direct", "fft", "token", "lazy", "tc")
 
 EXPORTED = ("fi_init", "fi_step", "fi_generate", "fi_generate_host", "fi_generate_lazy", "fi_sync", "fi_reset",
             "fi_position", "fi_read_activations", "fi_set_stream", "fi_get_plan", "fi_profile",
@@ -34,7 +34,7 @@ class FiError(RuntimeError):
 class Config(ctypes.Structure):
     _fields_ = [("layers", ctypes.c_int32), ("channels", ctypes.c_int32), ("max_len", ctypes.c_int32),
                 ("batch", ctypes.c_int32), ("dtype", ctypes.c_int32), ("chunk", ctypes.c_int32),
-                ("fft_from", ctypes.c_int32), ("reserved", ctypes.c_int32 * 5)]
+                ("fft_from", ctypes.c_int32), ("tc_max", ctypes.c_int32), ("reserved", ctypes.c_int32 * 4)]
 
 
 def _load():
@@ -54,7 +54,7 @@ def _load():
         "fi_position": [vp, ctypes.POINTER(i32)],
         "fi_read_activations": [vp, i32, vp],
         "fi_set_stream": [vp, vp],
-        "fi_get_plan": [vp, ctypes.POINTER(i32), ctypes.POINTER(i32)],
+        "fi_get_plan": [vp, ctypes.POINTER(i32), ctypes.POINTER(i32), ctypes.POINTER(i32)],
         "fi_profile": [vp, i32],
         "fi_profile_read": [vp, ctypes.POINTER(i32), ctypes.POINTER(ctypes.c_double)],
         "fi_destroy": [vp],
@@ -102,7 +102,8 @@ def _stream(stream) -> int | None:
 class Context:
     """One fi_ctx: filters, spectra and state of an M-layer online mixer stack."""
 
-    def __init__(self, h, batch: int, dtype: str = "f32", chunk: int = 0, fft_from: int = 0, stream=None):
+    def __init__(self, h, batch: int, dtype: str = "f32", chunk: int = 0, fft_from: int = 0, stream=None,
+                 tc_max: int = 0):
         import torch
         if h.dim() != 3:
             raise ValueError("h must be [M][D][L]")
@@ -113,7 +114,7 @@ class Context:
         self.M, self.D, self.L, self.B = int(M), int(D), int(L), int(batch)
         self.dtype = dtype
         self.torch_dtype = want
-        cfg = Config(self.M, self.D, self.L, self.B, FI_BF16 if dtype == "bf16" else FI_F32, chunk, fft_from)
+        cfg = Config(self.M, self.D, self.L, self.B, FI_BF16 if dtype == "bf16" else FI_F32, chunk, fft_from, tc_max)
         self._cfg = cfg
         self._h = ctypes.c_void_p()
         _check(lib.fi_init(ctypes.byref(self._h), ctypes.byref(cfg), _ptr(h), _stream(stream)), "fi_init")
@@ -178,9 +179,10 @@ class Context:
         _check(lib.fi_read_activations(self._h, layer, _ptr(dst)), "fi_read_activations")
 
     def plan(self):
-        c, f = ctypes.c_int32(), ctypes.c_int32()
-        _check(lib.fi_get_plan(self._h, ctypes.byref(c), ctypes.byref(f)), "fi_get_plan")
-        return c.value, f.value
+        """(chunk, fft_from, tc_max) after automatic selection; 0 = that kind of block is not used."""
+        c, f, t = ctypes.c_int32(), ctypes.c_int32(), ctypes.c_int32()
+        _check(lib.fi_get_plan(self._h, ctypes.byref(c), ctypes.byref(f), ctypes.byref(t)), "fi_get_plan")
+        return c.value, f.value, t.value
 
     def profile(self, enable: bool):
         _check(lib.fi_profile(self._h, 1 if enable else 0), "fi_profile")

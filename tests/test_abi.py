@@ -54,6 +54,9 @@ def _init(cfg, h=ctypes.c_void_p(16)):
     (dict(layers=1, channels=4, max_len=64, batch=1, chunk=3), "chunk"),
     (dict(layers=1, channels=4, max_len=64, batch=1, chunk=128), "chunk"),
     (dict(layers=1, channels=4, max_len=64, batch=1, fft_from=32), "fft_from"),
+    (dict(layers=1, channels=4, max_len=64, batch=1, tc_max=32), "tc_max"),
+    (dict(layers=1, channels=4, max_len=64, batch=1, tc_max=-2), "tc_max"),
+    (dict(layers=1, channels=4, max_len=64, batch=1, tc_max=96), "tc_max"),
 ])
 def test_init_rejects_bad_config_without_gpu(fields, why):
     from long_convolution_sequence_online_b200 import fi
