@@ -88,8 +88,8 @@ cudaError_t launch_part_block(const Dims& g, float* state, float2* xs, const flo
 // U + (J-1)*MT reversed sources, accumulator columns, split (fp32 contexts:
 // three bf16 products), dynamic shared memory and grid.
 struct TcPlan {
-  int U, MT, J, NR, K, tmem_cols, split, grid;
-  size_t smem;
+  int U, MT, J, NR, K, tmem_cols, split, grid, ipc, per_sm;   // ipc: items per pass of a CTA
+  size_t smem, item_bytes;
 };
 cudaError_t tc_prepare(const Dims& g, int U, int split, int num_sms, TcPlan* out);
 cudaError_t launch_tile_tc(const Dims& g, float* state, const float* taps, const TcPlan& p, int i, int* err,

@@ -84,6 +84,17 @@ __device__ __forceinline__ bool bar_wait(uint64_t* bar, uint32_t parity, int lim
   return false;
 }
 
+// 8 accumulator columns of this warp's 32 lanes.
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8]) {
+  uint32_t r[8];
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int k = 0; k < 8; ++k) v[k] = __uint_as_float(r[k]);
+}
+
 // 16 accumulator columns of this warp's 32 lanes.
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
   uint32_t r[16];
@@ -123,15 +134,17 @@ __global__ void __launch_bounds__(128) k_tile_tc(Dims g, float* __restrict__ sta
   __shared__ uint64_t mma_bar;
   __shared__ uint32_t tmem_base_s;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int U = p.U, J = p.J, NR = p.NR, K = p.K;
+  const int U = p.U, J = p.J, NR = p.NR, K = p.K, IPC = p.ipc;
   const int NT = U / MT, groups = NT / J;
+  const int cols = groups * NR;                 // accumulator columns of one item
   const uint32_t idesc = tc_idesc(MT, NR);
-  // shared memory: table hi [2U][16 B], (table lo), X hi [NR rows][K], (X lo)
-  unsigned char* tab_hi = tsm;
-  unsigned char* tab_lo = tsm + (size_t)32 * U;
-  unsigned char* x_hi = tsm + (SPLIT ? 2 : 1) * (size_t)32 * U;
-  unsigned char* x_lo = x_hi + (size_t)NR * K * 2;
   const size_t xbytes = (size_t)NR * K * 2;
+  // Per item k of a pass, at tsm + k * item_bytes: table hi [2U][16 B],
+  // (table lo), X hi [NR rows][K], (X lo).
+  auto tab_hi = [&](int k) { return tsm + (size_t)k * p.item_bytes; };
+  auto tab_lo = [&](int k) { return tsm + (size_t)k * p.item_bytes + (size_t)32 * U; };
+  auto x_hi = [&](int k) { return tsm + (size_t)k * p.item_bytes + (SPLIT ? 2 : 1) * (size_t)32 * U; };
+  auto x_lo = [&](int k) { return x_hi(k) + xbytes; };
 
   if (warp == 0) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
@@ -150,43 +163,48 @@ __global__ void __launch_bounds__(128) k_tile_tc(Dims g, float* __restrict__ sta
   uint32_t phase = 0;
 
   const long items = (long)g.M * g.D;
-  for (long item = blockIdx.x; item < items && ok; item += gridDim.x) {
-    const int l = (int)(item / g.D) + 1;
-    const int d = (int)(item - (long)(l - 1) * g.D);
-    const float* hp = taps + ((size_t)(l - 1) * g.D + d) * g.L;
+  for (long base = (long)blockIdx.x * IPC; base < items && ok; base += (long)gridDim.x * IPC) {
+    const int nk = (int)(items - base < IPC ? items - base : IPC);   // items in this pass
 
-    // Table: entry s = h[s+1 .. s+8] (taps beyond 2U-1 are never multiplied by
-    // a nonzero source; they read as the filter's next taps or zero).
-    for (int s = tid; s < 2 * U; s += 128) {
-      uint32_t wh[4], wl[4];
+    // Tables: entry s = h[s+1 .. s+8] (taps beyond 2U-1 are never multiplied by
+    // a nonzero source; they read as the filter's next taps or zero). And the
+    // B operands zeroed.
+    for (int k = 0; k < nk; ++k) {
+      const float* hp = taps + (size_t)(base + k) * g.L;       // item = (l-1)*D + d
+      for (int s = tid; s < 2 * U; s += 128) {
+        uint32_t wh[4], wl[4];
 #pragma unroll
-      for (int e = 0; e < 8; e += 2) {
-        const int k0 = s + 1 + e, k1 = s + 2 + e;
-        const float v0 = k0 < g.L ? __ldg(hp + k0) : 0.f;
-        const float v1 = k1 < g.L ? __ldg(hp + k1) : 0.f;
-        uint16_t h0, l0, h1, l1;
-        if constexpr (SPLIT) {
-          split_bf16(v0, h0, l0);
-          split_bf16(v1, h1, l1);
-        } else {
-          h0 = bf16_bits(v0); h1 = bf16_bits(v1); l0 = l1 = 0;
+        for (int e = 0; e < 8; e += 2) {
+          const int k0 = s + 1 + e, k1 = s + 2 + e;
+          const float v0 = k0 < g.L ? __ldg(hp + k0) : 0.f;
+          const float v1 = k1 < g.L ? __ldg(hp + k1) : 0.f;
+          uint16_t h0, l0, h1, l1;
+          if constexpr (SPLIT) {
+            split_bf16(v0, h0, l0);
+            split_bf16(v1, h1, l1);
+          } else {
+            h0 = bf16_bits(v0); h1 = bf16_bits(v1); l0 = l1 = 0;
+          }
+          wh[e / 2] = (uint32_t)h0 | ((uint32_t)h1 << 16);
+          wl[e / 2] = (uint32_t)l0 | ((uint32_t)l1 << 16);
         }
-        wh[e / 2] = (uint32_t)h0 | ((uint32_t)h1 << 16);
-        wl[e / 2] = (uint32_t)l0 | ((uint32_t)l1 << 16);
+        *reinterpret_cast<uint4*>(tab_hi(k) + (size_t)s * 16) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
+        if constexpr (SPLIT) *reinterpret_cast<uint4*>(tab_lo(k) + (size_t)s * 16) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
       }
-      *reinterpret_cast<uint4*>(tab_hi + (size_t)s * 16) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
-      if constexpr (SPLIT) *reinterpret_cast<uint4*>(tab_lo + (size_t)s * 16) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
-    }
-    // B operand: zero, then the sources of each (tile j, sequence b) row.
-    for (size_t q = (size_t)tid * 16; q < xbytes; q += 128 * 16) {
-      *reinterpret_cast<uint4*>(x_hi + q) = make_uint4(0, 0, 0, 0);
-      if constexpr (SPLIT) *reinterpret_cast<uint4*>(x_lo + q) = make_uint4(0, 0, 0, 0);
+      for (size_t q = (size_t)tid * 16; q < xbytes; q += 128 * 16) {
+        *reinterpret_cast<uint4*>(x_hi(k) + q) = make_uint4(0, 0, 0, 0);
+        if constexpr (SPLIT) *reinterpret_cast<uint4*>(x_lo(k) + q) = make_uint4(0, 0, 0, 0);
+      }
     }
     __syncthreads();
+    // B operands: the sources of each (tile j, sequence b) row.
     {
       const int quads = U / 4;
-      for (int w = tid; w < g.B * quads; w += 128) {
-        const int b = w / quads, q4 = w - b * quads;
+      for (int w = tid; w < nk * g.B * quads; w += 128) {
+        const int k = w / (g.B * quads), wr = w - k * (g.B * quads);
+        const int b = wr / quads, q4 = wr - b * quads;
+        const long item = base + k;
+        const int l = (int)(item / g.D) + 1, d = (int)(item - (long)(l - 1) * g.D);
         const float4 v = *reinterpret_cast<const float4*>(state + slot_index(g, l - 1, d * g.B + b, i - U) + 4 * q4);
         // kappa = U - 1 - (4 q4 + e) for element e; four consecutive kappa from kb
         const int kb = U - 4 - 4 * q4;
@@ -201,8 +219,8 @@ __global__ void __launch_bounds__(128) k_tile_tc(Dims g, float* __restrict__ sta
         const uint2 wl = make_uint2((uint32_t)lo[0] | ((uint32_t)lo[1] << 16), (uint32_t)lo[2] | ((uint32_t)lo[3] << 16));
         for (int j = 0; j < J; ++j) {
           const uint32_t off = tc_b_offset(NR, j * g.B + b, j * MT + kb);
-          *reinterpret_cast<uint2*>(x_hi + off) = wh;
-          if constexpr (SPLIT) *reinterpret_cast<uint2*>(x_lo + off) = wl;
+          *reinterpret_cast<uint2*>(x_hi(k) + off) = wh;
+          if constexpr (SPLIT) *reinterpret_cast<uint2*>(x_lo(k) + off) = wl;
         }
       }
     }
@@ -212,19 +230,23 @@ __global__ void __launch_bounds__(128) k_tile_tc(Dims g, float* __restrict__ sta
     if (tid == 0) {
       fence_after_sync();
       const uint32_t lbo_b = (uint32_t)(NR / 8) * 128;
-      for (int gi = 0; gi < groups; ++gi) {
-        const uint32_t dcol = tmem + (uint32_t)(gi * NR);
-        for (int ks = 0; ks < K / 16; ++ks) {
-          const uint32_t a_off = (uint32_t)(gi * J * MT + 16 * ks) * 16;
-          const uint32_t b_off = (uint32_t)(2 * ks) * lbo_b;
-          const uint64_t ah = smem_desc(smem_addr(tab_hi) + a_off, 128, 128);
-          const uint64_t bh = smem_desc(smem_addr(x_hi) + b_off, lbo_b, 128);
-          mma_bf16(dcol, ah, bh, idesc, ks > 0 ? 1u : 0u);
-          if constexpr (SPLIT) {
-            const uint64_t al = smem_desc(smem_addr(tab_lo) + a_off, 128, 128);
-            const uint64_t bl = smem_desc(smem_addr(x_lo) + b_off, lbo_b, 128);
-            mma_bf16(dcol, ah, bl, idesc, 1u);
-            mma_bf16(dcol, al, bh, idesc, 1u);
+      for (int k = 0; k < nk; ++k) {
+        const uint32_t th = smem_addr(tab_hi(k)), tl = smem_addr(tab_lo(k));
+        const uint32_t xh = smem_addr(x_hi(k)), xl = smem_addr(x_lo(k));
+        for (int gi = 0; gi < groups; ++gi) {
+          const uint32_t dcol = tmem + (uint32_t)(k * cols + gi * NR);
+          for (int ks = 0; ks < K / 16; ++ks) {
+            const uint32_t a_off = (uint32_t)(gi * J * MT + 16 * ks) * 16;
+            const uint32_t b_off = (uint32_t)(2 * ks) * lbo_b;
+            const uint64_t ah = smem_desc(th + a_off, 128, 128);
+            const uint64_t bh = smem_desc(xh + b_off, lbo_b, 128);
+            mma_bf16(dcol, ah, bh, idesc, ks > 0 ? 1u : 0u);
+            if constexpr (SPLIT) {
+              const uint64_t al = smem_desc(tl + a_off, 128, 128);
+              const uint64_t bl = smem_desc(xl + b_off, lbo_b, 128);
+              mma_bf16(dcol, ah, bl, idesc, 1u);
+              mma_bf16(dcol, al, bh, idesc, 1u);
+            }
           }
         }
       }
@@ -243,22 +265,33 @@ __global__ void __launch_bounds__(128) k_tile_tc(Dims g, float* __restrict__ sta
 
     // Epilogue: row r of tile (gi*J + j) is target i + (gi*J + j)*MT + r;
     // accumulator lane 32*warp + lane holds row 32*warp + lane (MT = 128) or,
-    // for MT = 64, lanes 0-15 of each warp hold rows 16*warp + lane.
+    // for MT = 64, lanes 0-15 of each warp hold rows 16*warp + lane. Eight
+    // columns at a time: all loads of the old values first, then the stores.
     const int r = MT == 128 ? 32 * warp + lane : 16 * warp + lane;
     const bool row_ok = MT == 128 || lane < 16;
-    const int cols = groups * NR;
-    for (int c0 = 0; c0 < cols; c0 += 16) {
-      float v[16];
-      tmem_ld16(tmem + ((uint32_t)(32 * warp) << 16) + (uint32_t)c0, v);
-      if (!row_ok) continue;
+    for (int k = 0; k < nk; ++k) {
+      const long item = base + k;
+      const int l = (int)(item / g.D) + 1, d = (int)(item - (long)(l - 1) * g.D);
+      for (int c0 = 0; c0 < cols; c0 += 8) {
+        float v[8];
+        tmem_ld8(tmem + ((uint32_t)(32 * warp) << 16) + (uint32_t)(k * cols + c0), v);
+        if (!row_ok) continue;
+        float* dst[8];
+        float old[8];
 #pragma unroll
-      for (int k = 0; k < 16; ++k) {
-        const int c = c0 + k;
-        const int gi = c / NR, n = c - gi * NR;
-        if (c >= cols || n >= J * g.B) continue;
-        const int j = n / g.B, b = n - j * g.B;
-        float* dst = state + slot_index(g, l, d * g.B + b, i + (gi * J + j) * MT + r);
-        *dst = overwrite ? v[k] : *dst + v[k];
+        for (int e = 0; e < 8; ++e) {
+          const int c = c0 + e;
+          const int gi = c / NR, n = c - gi * NR;
+          dst[e] = nullptr;
+          if (n < J * g.B) {
+            const int j = n / g.B, b = n - j * g.B;
+            dst[e] = state + slot_index(g, l, d * g.B + b, i + (gi * J + j) * MT + r);
+          }
+          old[e] = (dst[e] && !overwrite) ? *dst[e] : 0.f;
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          if (dst[e]) *dst[e] = old[e] + v[e];
       }
     }
     fence_before_sync();
@@ -280,12 +313,35 @@ __global__ void __launch_bounds__(128) k_tile_tc(Dims g, float* __restrict__ sta
 // ------------------------------------------------------------------ host side
 static int pow2_at_least(int v) { int r = 1; while (r < v) r <<= 1; return r; }
 
+// CTAs of one plan that fit on an SM: threads, registers and shared memory
+// counted from the kernel's attributes (the dynamic shared-memory limit of the
+// instantiation only ever grows, since several block sides share it).
 template <int MT, bool SPLIT>
-static cudaError_t tc_occupancy(const TcPlan& p, int* per_sm) {
+static cudaError_t tc_occupancy(const TcPlan& p, int device, int* per_sm) {
   auto kern = k_tile_tc<MT, SPLIT>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem);
+  cudaFuncAttributes fa{};
+  cudaError_t e = cudaFuncGetAttributes(&fa, kern);
   if (e != cudaSuccess) return e;
-  return cudaOccupancyMaxActiveBlocksPerMultiprocessor(per_sm, kern, 128, p.smem);
+  if ((size_t)fa.maxDynamicSharedSizeBytes < p.smem)
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, (int)cudaSharedmemCarveoutMaxShared);
+  if (e != cudaSuccess) return e;
+  int sm_smem = 0, sm_regs = 0, sm_threads = 0, sm_blocks = 0, reserved = 0;
+  if ((e = cudaDeviceGetAttribute(&sm_smem, cudaDevAttrMaxSharedMemoryPerMultiprocessor, device)) != cudaSuccess ||
+      (e = cudaDeviceGetAttribute(&sm_regs, cudaDevAttrMaxRegistersPerMultiprocessor, device)) != cudaSuccess ||
+      (e = cudaDeviceGetAttribute(&sm_threads, cudaDevAttrMaxThreadsPerMultiProcessor, device)) != cudaSuccess ||
+      (e = cudaDeviceGetAttribute(&sm_blocks, cudaDevAttrMaxBlocksPerMultiprocessor, device)) != cudaSuccess ||
+      (e = cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, device)) != cudaSuccess)
+    return e;
+  const size_t per_cta_smem = p.smem + fa.sharedSizeBytes + (size_t)reserved;
+  const int regs_cta = ((fa.numRegs * 32 + 255) / 256 * 256) * 4;   // 4 warps, 256-register allocation units
+  int n = sm_threads / 128;
+  if (sm_blocks < n) n = sm_blocks;
+  if (regs_cta > 0 && sm_regs / regs_cta < n) n = sm_regs / regs_cta;
+  if ((int)(sm_smem / per_cta_smem) < n) n = (int)(sm_smem / per_cta_smem);
+  *per_sm = n;
+  return cudaSuccess;
 }
 
 cudaError_t tc_prepare(const Dims& g, int U, int split, int num_sms, TcPlan* out) {
@@ -304,22 +360,32 @@ cudaError_t tc_prepare(const Dims& g, int U, int split, int num_sms, TcPlan* out
   p.K = U + (J - 1) * p.MT;
   const int cols = (NT / J) * p.NR;
   if (cols > 512) return cudaErrorInvalidValue;
-  p.tmem_cols = pow2_at_least(cols < 32 ? 32 : cols);
   p.split = split;
+  // One item's operands (128-byte multiple); items per pass: enough that small
+  // items share the smallest accumulator allocation (32 columns), within 64 KB.
+  p.item_bytes = ((size_t)(split ? 2 : 1) * ((size_t)32 * U + (size_t)p.NR * p.K * 2) + 127) / 128 * 128;
+  p.ipc = cols >= 32 ? 1 : 32 / cols;
+  while (p.ipc > 1 && (size_t)p.ipc * p.item_bytes > 64 * 1024) p.ipc >>= 1;
   // Operands, plus slack past the last one: a B-operand read with its two
   // strides exchanged would stay inside the allocation.
-  p.smem = (size_t)(split ? 2 : 1) * ((size_t)32 * U + (size_t)p.NR * p.K * 2) + (size_t)p.NR * p.NR * 2 + 256;
+  p.smem = (size_t)p.ipc * p.item_bytes + (size_t)p.NR * p.NR * 2 + 256;
+  const int cols_all = p.ipc * cols;
+  p.tmem_cols = pow2_at_least(cols_all < 32 ? 32 : cols_all);
   int occ = 0;
-  cudaError_t e = p.MT == 128 ? (split ? tc_occupancy<128, true>(p, &occ) : tc_occupancy<128, false>(p, &occ))
-                              : (split ? tc_occupancy<64, true>(p, &occ) : tc_occupancy<64, false>(p, &occ));
+  int device = 0;
+  cudaError_t e = cudaGetDevice(&device);
+  if (e != cudaSuccess) return e;
+  e = p.MT == 128 ? (split ? tc_occupancy<128, true>(p, device, &occ) : tc_occupancy<128, false>(p, device, &occ))
+                  : (split ? tc_occupancy<64, true>(p, device, &occ) : tc_occupancy<64, false>(p, device, &occ));
   if (e != cudaSuccess) return e;
   // every resident CTA holds its accumulator columns for its whole life
   const int by_tmem = 512 / p.tmem_cols;
   const int per_sm = occ < by_tmem ? occ : by_tmem;
   if (per_sm < 1) return cudaErrorInvalidConfiguration;
-  const long items = (long)g.M * g.D;
+  const long passes = ((long)g.M * g.D + p.ipc - 1) / p.ipc;
   long grid = (long)num_sms * per_sm;
-  p.grid = (int)(grid > items ? items : grid);
+  p.grid = (int)(grid > passes ? passes : grid);
+  p.per_sm = per_sm;
   *out = p;
   return cudaSuccess;
 }
