@@ -71,6 +71,8 @@ for _b in (8, 32, 64):
 # slice at the full length L = 32768 (which reaches the largest FFT blocks).
 WORKLOADS["hyena-18x864-L2K-B4"] = Workload("hyena-18x864-L2K-B4", 18, 864, 2048, 4, "f32", 1e-3, 1e-1)
 WORKLOADS["hyena-18x64-L32K-B4"] = Workload("hyena-18x64-L32K-B4", 18, 64, 32768, 4, "f32", 1e-3, 1e-1)
+# ... and of the batched bf16 stack (8 layers, B = 64): 128 channels at L = 4096.
+WORKLOADS["sweep-8x128-L4K-bf16-B64"] = Workload("sweep-8x128-L4K-bf16-B64", 8, 128, 4096, 64, "bf16", 1e-3, 1e-1)
 
 HEADLINE = "hyena-18x864-L32K-B4"
 
