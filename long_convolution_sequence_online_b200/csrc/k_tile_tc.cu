@@ -127,182 +127,272 @@ __host__ __device__ constexpr uint32_t tc_b_offset(int R, int n, int k) {
   return (uint32_t)(((k >> 3) * (R >> 3) + (n >> 3)) * 128 + (n & 7) * 16 + (k & 7) * 2);
 }
 
+// Warp roles: warps 0-3 build operands, warp 4 issues the MMAs, warps 5-8 drain
+// the accumulators (warp w reads tensor-memory lanes 32*(w % 4) .. +31). Two
+// stages of operands and accumulators let pass p+1 load while pass p multiplies
+// and pass p-1 drains. Per stage s, three mbarriers: full (loaders -> MMA),
+// done (MMA commit -> loaders, which may overwrite the operands, and -> drain),
+// empty (drain -> MMA, which may overwrite the accumulators). Use k of a stage
+// waits on parity k & 1; no barrier runs more than one phase ahead of a waiter.
+constexpr int kTcLoadWarps = 4;
+constexpr int kTcMmaWarp = kTcLoadWarps;
+constexpr int kTcDrainWarp0 = kTcLoadWarps + 1;
+constexpr int kTcThreads = 32 * (kTcLoadWarps + 1 + 4);
+
+__device__ __forceinline__ void bar_arrive(uint64_t* bar) {
+  asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.shared::cta.b64 st, [%0];\n\t}" ::"r"(smem_addr(bar)) : "memory");
+}
+// OR of `v` over the operand-builder warps (named barrier 1), so they leave
+// their loop together.
+__device__ __forceinline__ bool loaders_any(bool v) {
+  uint32_t out;
+  asm volatile("{\n\t.reg .pred q, p;\n\tsetp.ne.u32 q, %1, 0;\n\tbar.red.or.pred p, 1, %2, q;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+               : "=r"(out) : "r"((uint32_t)v), "r"(32 * kTcLoadWarps) : "memory");
+  return out != 0;
+}
+// Bounded wait that also gives up once another role has given up.
+__device__ __forceinline__ bool bar_wait_or_abort(uint64_t* bar, uint32_t parity, int limit, volatile int* abort_flag) {
+  for (int it = 0; it < limit; ++it) {
+    if (bar_try(bar, parity)) return true;
+    if (*abort_flag) return false;
+  }
+  return false;
+}
+
 template <int MT, bool SPLIT>
-__global__ void __launch_bounds__(128) k_tile_tc(Dims g, float* __restrict__ state, const float* __restrict__ taps,
-                                                 TcPlan p, int i, int overwrite, int* err, int wait_limit) {
+__global__ void __launch_bounds__(kTcThreads) k_tile_tc(Dims g, float* __restrict__ state, const float* __restrict__ taps,
+                                                        TcPlan p, int i, int overwrite, int* err, int wait_limit) {
   extern __shared__ __align__(1024) unsigned char tsm[];
-  __shared__ uint64_t mma_bar;
+  __shared__ uint64_t full_bar[2], done_bar[2], empty_bar[2];
   __shared__ uint32_t tmem_base_s;
+  __shared__ int abort_s;
+  __shared__ int col_ofs[512];   // accumulator column -> target offset from the item's row base, or -1
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int U = p.U, J = p.J, NR = p.NR, K = p.K, IPC = p.ipc;
   const int NT = U / MT, groups = NT / J;
   const int cols = groups * NR;                 // accumulator columns of one item
   const uint32_t idesc = tc_idesc(MT, NR);
   const size_t xbytes = (size_t)NR * K * 2;
-  // Per item k of a pass, at tsm + k * item_bytes: table hi [2U][16 B],
-  // (table lo), X hi [NR rows][K], (X lo).
-  auto tab_hi = [&](int k) { return tsm + (size_t)k * p.item_bytes; };
-  auto tab_lo = [&](int k) { return tsm + (size_t)k * p.item_bytes + (size_t)32 * U; };
-  auto x_hi = [&](int k) { return tsm + (size_t)k * p.item_bytes + (SPLIT ? 2 : 1) * (size_t)32 * U; };
-  auto x_lo = [&](int k) { return x_hi(k) + xbytes; };
+  const size_t stage_bytes = (size_t)IPC * p.item_bytes;
+  // Item k of stage s, at tsm + s * stage_bytes + k * item_bytes: table hi
+  // [2U][16 B], (table lo), X hi [NR rows][K], (X lo).
+  auto item_base = [&](int st, int k) { return tsm + (size_t)st * stage_bytes + (size_t)k * p.item_bytes; };
+  auto tab_hi = [&](int st, int k) { return item_base(st, k); };
+  auto tab_lo = [&](int st, int k) { return item_base(st, k) + (size_t)32 * U; };
+  auto x_hi = [&](int st, int k) { return item_base(st, k) + (SPLIT ? 2 : 1) * (size_t)32 * U; };
+  auto x_lo = [&](int st, int k) { return x_hi(st, k) + xbytes; };
 
   if (warp == 0) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
                  ::"r"(smem_addr(&tmem_base_s)), "r"(p.tmem_cols) : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
+  // Column c of an item: group gi = c / NR, operand row n = c % NR = j*B + b;
+  // its target for accumulator row r is slot (l, d*B + b, i + (gi*J + j)*MT + r),
+  // i.e. the item's row base plus b*L + (gi*J + j)*MT.
+  for (int c = tid; c < cols; c += blockDim.x) {
+    const int gi = c / NR, n = c - gi * NR;
+    const int j = n / g.B, b = n - j * g.B;
+    col_ofs[c] = n < J * g.B ? b * g.L + (gi * J + j) * MT : -1;
+  }
   if (tid == 0) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_addr(&mma_bar)) : "memory");
+    for (int st = 0; st < 2; ++st) {
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(&full_bar[st])), "r"(32 * kTcLoadWarps) : "memory");
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_addr(&done_bar[st])) : "memory");
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 128;" ::"r"(smem_addr(&empty_bar[st])) : "memory");
+    }
+    abort_s = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   fence_before_sync();
   __syncthreads();
   fence_after_sync();
   const uint32_t tmem = tmem_base_s;
-  bool ok = true;
-  uint32_t phase = 0;
+  volatile int* abort_flag = &abort_s;
+  auto give_up = [&]() {
+    *abort_flag = 1;
+    atomicExch(err, 1);
+  };
 
   const long items = (long)g.M * g.D;
-  for (long base = (long)blockIdx.x * IPC; base < items && ok; base += (long)gridDim.x * IPC) {
-    const int nk = (int)(items - base < IPC ? items - base : IPC);   // items in this pass
+  const long first = (long)blockIdx.x * IPC, stride = (long)gridDim.x * IPC;
+  const int npass = first < items ? (int)((items - 1 - first) / stride) + 1 : 0;
+  int last_commit = -1;                          // MMA issuer: last pass committed
 
-    // Tables: entry s = h[s+1 .. s+8] (taps beyond 2U-1 are never multiplied by
-    // a nonzero source; they read as the filter's next taps or zero). And the
-    // B operands zeroed.
-    for (int k = 0; k < nk; ++k) {
-      const float* hp = taps + (size_t)(base + k) * g.L;       // item = (l-1)*D + d
-      for (int s = tid; s < 2 * U; s += 128) {
-        uint32_t wh[4], wl[4];
+  if (warp < kTcLoadWarps) {
+    // ------------------------------------------------------------ operand builders
+    const int lt = tid;                          // 0..127
+    for (int ps = 0; ps < npass; ++ps) {
+      const int st = ps & 1;
+      const long base = first + (long)ps * stride;
+      const int nk = (int)(items - base < IPC ? items - base : IPC);
+      const bool free = ps < 2 || bar_wait_or_abort(&done_bar[st], ((ps - 2) >> 1) & 1, wait_limit, abort_flag);
+      if (loaders_any(!free)) {
+        if (lt == 0) give_up();
+        break;
+      }
+      // Tables: entry s = h[s+1 .. s+8] (taps beyond 2U-1 meet only zero
+      // sources), and the B operands zeroed.
+      for (int k = 0; k < nk; ++k) {
+        const float* hp = taps + (size_t)(base + k) * g.L;       // item = (l-1)*D + d
+        // entries 8t .. 8t+7 from taps h[8t .. 8t+15] (four 16-byte loads)
+        for (int t8 = lt; t8 < 2 * U / 8; t8 += 32 * kTcLoadWarps) {
+          float hv[16];
 #pragma unroll
-        for (int e = 0; e < 8; e += 2) {
-          const int k0 = s + 1 + e, k1 = s + 2 + e;
-          const float v0 = k0 < g.L ? __ldg(hp + k0) : 0.f;
-          const float v1 = k1 < g.L ? __ldg(hp + k1) : 0.f;
-          uint16_t h0, l0, h1, l1;
-          if constexpr (SPLIT) {
-            split_bf16(v0, h0, l0);
-            split_bf16(v1, h1, l1);
-          } else {
-            h0 = bf16_bits(v0); h1 = bf16_bits(v1); l0 = l1 = 0;
+          for (int f = 0; f < 4; ++f) {
+            const int o = 8 * t8 + 4 * f;
+            const float4 v = o + 4 <= g.L ? __ldg(reinterpret_cast<const float4*>(hp + o)) : make_float4(0.f, 0.f, 0.f, 0.f);
+            hv[4 * f] = v.x; hv[4 * f + 1] = v.y; hv[4 * f + 2] = v.z; hv[4 * f + 3] = v.w;
           }
-          wh[e / 2] = (uint32_t)h0 | ((uint32_t)h1 << 16);
-          wl[e / 2] = (uint32_t)l0 | ((uint32_t)l1 << 16);
+#pragma unroll
+          for (int m = 0; m < 8; ++m) {
+            uint32_t wh[4], wl[4];
+#pragma unroll
+            for (int e = 0; e < 8; e += 2) {
+              const float v0 = hv[m + 1 + e], v1 = hv[m + 2 + e];
+              uint16_t h0, l0, h1, l1;
+              if constexpr (SPLIT) {
+                split_bf16(v0, h0, l0);
+                split_bf16(v1, h1, l1);
+              } else {
+                h0 = bf16_bits(v0); h1 = bf16_bits(v1); l0 = l1 = 0;
+              }
+              wh[e / 2] = (uint32_t)h0 | ((uint32_t)h1 << 16);
+              wl[e / 2] = (uint32_t)l0 | ((uint32_t)l1 << 16);
+            }
+            const size_t eo = (size_t)(8 * t8 + m) * 16;
+            *reinterpret_cast<uint4*>(tab_hi(st, k) + eo) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
+            if constexpr (SPLIT) *reinterpret_cast<uint4*>(tab_lo(st, k) + eo) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
+          }
         }
-        *reinterpret_cast<uint4*>(tab_hi(k) + (size_t)s * 16) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
-        if constexpr (SPLIT) *reinterpret_cast<uint4*>(tab_lo(k) + (size_t)s * 16) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
+        for (size_t q = (size_t)lt * 16; q < xbytes; q += 128 * 16) {
+          *reinterpret_cast<uint4*>(x_hi(st, k) + q) = make_uint4(0, 0, 0, 0);
+          if constexpr (SPLIT) *reinterpret_cast<uint4*>(x_lo(st, k) + q) = make_uint4(0, 0, 0, 0);
+        }
       }
-      for (size_t q = (size_t)tid * 16; q < xbytes; q += 128 * 16) {
-        *reinterpret_cast<uint4*>(x_hi(k) + q) = make_uint4(0, 0, 0, 0);
-        if constexpr (SPLIT) *reinterpret_cast<uint4*>(x_lo(k) + q) = make_uint4(0, 0, 0, 0);
-      }
-    }
-    __syncthreads();
-    // B operands: the sources of each (tile j, sequence b) row.
-    {
-      const int quads = U / 4;
-      for (int w = tid; w < nk * g.B * quads; w += 128) {
-        const int k = w / (g.B * quads), wr = w - k * (g.B * quads);
-        const int b = wr / quads, q4 = wr - b * quads;
+      asm volatile("bar.sync 1, %0;" ::"r"(32 * kTcLoadWarps) : "memory");
+      // B operands: the sources of each (tile j, sequence b) row. A thread takes
+      // 8 consecutive sources of one sequence (one 32-byte sector) and writes
+      // them as one 16-byte core-matrix row; consecutive threads take
+      // consecutive sequences, so a warp's stores fill whole core matrices.
+      const int oct = U / 8;
+      for (int w = lt; w < nk * g.B * oct; w += 128) {
+        const int k = w / (g.B * oct), wr = w - k * (g.B * oct);
+        const int q8 = wr / g.B, b = wr - q8 * g.B;
         const long item = base + k;
         const int l = (int)(item / g.D) + 1, d = (int)(item - (long)(l - 1) * g.D);
-        const float4 v = *reinterpret_cast<const float4*>(state + slot_index(g, l - 1, d * g.B + b, i - U) + 4 * q4);
-        // kappa = U - 1 - (4 q4 + e) for element e; four consecutive kappa from kb
-        const int kb = U - 4 - 4 * q4;
-        uint16_t hi[4], lo[4];
-        const float vv[4] = {v.w, v.z, v.y, v.x};   // kappa kb, kb+1, kb+2, kb+3
+        const float4* src = reinterpret_cast<const float4*>(state + slot_index(g, l - 1, d * g.B + b, i - U) + 8 * q8);
+        const float4 v0 = src[0], v1 = src[1];
+        // source 8 q8 + e sits at kappa = U - 1 - 8 q8 - e: kappa kb + m holds element 7 - m
+        const int kb = U - 8 - 8 * q8;
+        const float vv[8] = {v1.w, v1.z, v1.y, v1.x, v0.w, v0.z, v0.y, v0.x};
+        uint32_t wh[4], wl[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          if constexpr (SPLIT) split_bf16(vv[e], hi[e], lo[e]);
-          else { hi[e] = bf16_bits(vv[e]); lo[e] = 0; }
+        for (int m = 0; m < 8; m += 2) {
+          uint16_t h0, l0, h1, l1;
+          if constexpr (SPLIT) {
+            split_bf16(vv[m], h0, l0);
+            split_bf16(vv[m + 1], h1, l1);
+          } else {
+            h0 = bf16_bits(vv[m]); h1 = bf16_bits(vv[m + 1]); l0 = l1 = 0;
+          }
+          wh[m / 2] = (uint32_t)h0 | ((uint32_t)h1 << 16);
+          wl[m / 2] = (uint32_t)l0 | ((uint32_t)l1 << 16);
         }
-        const uint2 wh = make_uint2((uint32_t)hi[0] | ((uint32_t)hi[1] << 16), (uint32_t)hi[2] | ((uint32_t)hi[3] << 16));
-        const uint2 wl = make_uint2((uint32_t)lo[0] | ((uint32_t)lo[1] << 16), (uint32_t)lo[2] | ((uint32_t)lo[3] << 16));
         for (int j = 0; j < J; ++j) {
           const uint32_t off = tc_b_offset(NR, j * g.B + b, j * MT + kb);
-          *reinterpret_cast<uint2*>(x_hi(k) + off) = wh;
-          if constexpr (SPLIT) *reinterpret_cast<uint2*>(x_lo(k) + off) = wl;
+          *reinterpret_cast<uint4*>(x_hi(st, k) + off) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
+          if constexpr (SPLIT) *reinterpret_cast<uint4*>(x_lo(st, k) + off) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
         }
       }
+      fence_proxy_async();   // generic-proxy writes -> visible to the tensor core
+      bar_arrive(&full_bar[st]);
     }
-    fence_proxy_async();   // generic-proxy writes -> visible to the tensor core
-    __syncthreads();
-
-    if (tid == 0) {
-      fence_after_sync();
+  } else if (warp == kTcMmaWarp) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
       const uint32_t lbo_b = (uint32_t)(NR / 8) * 128;
-      for (int k = 0; k < nk; ++k) {
-        const uint32_t th = smem_addr(tab_hi(k)), tl = smem_addr(tab_lo(k));
-        const uint32_t xh = smem_addr(x_hi(k)), xl = smem_addr(x_lo(k));
-        for (int gi = 0; gi < groups; ++gi) {
-          const uint32_t dcol = tmem + (uint32_t)(k * cols + gi * NR);
-          for (int ks = 0; ks < K / 16; ++ks) {
-            const uint32_t a_off = (uint32_t)(gi * J * MT + 16 * ks) * 16;
-            const uint32_t b_off = (uint32_t)(2 * ks) * lbo_b;
-            const uint64_t ah = smem_desc(th + a_off, 128, 128);
-            const uint64_t bh = smem_desc(xh + b_off, lbo_b, 128);
-            mma_bf16(dcol, ah, bh, idesc, ks > 0 ? 1u : 0u);
-            if constexpr (SPLIT) {
-              const uint64_t al = smem_desc(tl + a_off, 128, 128);
-              const uint64_t bl = smem_desc(xl + b_off, lbo_b, 128);
-              mma_bf16(dcol, ah, bl, idesc, 1u);
-              mma_bf16(dcol, al, bh, idesc, 1u);
+      for (int ps = 0; ps < npass; ++ps) {
+        const int st = ps & 1;
+        const long base = first + (long)ps * stride;
+        const int nk = (int)(items - base < IPC ? items - base : IPC);
+        if (!bar_wait_or_abort(&full_bar[st], (ps >> 1) & 1, wait_limit, abort_flag) ||
+            (ps >= 2 && !bar_wait_or_abort(&empty_bar[st], ((ps - 2) >> 1) & 1, wait_limit, abort_flag))) {
+          give_up();
+          break;
+        }
+        fence_after_sync();
+        for (int k = 0; k < nk; ++k) {
+          const uint32_t th = smem_addr(tab_hi(st, k)), tl = smem_addr(tab_lo(st, k));
+          const uint32_t xh = smem_addr(x_hi(st, k)), xl = smem_addr(x_lo(st, k));
+          for (int gi = 0; gi < groups; ++gi) {
+            const uint32_t dcol = tmem + (uint32_t)((st * IPC + k) * cols + gi * NR);
+            for (int ks = 0; ks < K / 16; ++ks) {
+              const uint32_t a_off = (uint32_t)(gi * J * MT + 16 * ks) * 16;
+              const uint32_t b_off = (uint32_t)(2 * ks) * lbo_b;
+              const uint64_t ah = smem_desc(th + a_off, 128, 128);
+              const uint64_t bh = smem_desc(xh + b_off, lbo_b, 128);
+              mma_bf16(dcol, ah, bh, idesc, ks > 0 ? 1u : 0u);
+              if constexpr (SPLIT) {
+                const uint64_t al = smem_desc(tl + a_off, 128, 128);
+                const uint64_t bl = smem_desc(xl + b_off, lbo_b, 128);
+                mma_bf16(dcol, ah, bl, idesc, 1u);
+                mma_bf16(dcol, al, bh, idesc, 1u);
+              }
             }
           }
         }
+        mma_commit(&done_bar[st]);
+        last_commit = ps;
       }
-      mma_commit(&mma_bar);
+      // The accumulators are released only after the last commit has arrived.
+      if (last_commit >= 0) bar_wait(&done_bar[last_commit & 1], (last_commit >> 1) & 1, wait_limit);
     }
     __syncwarp();
-    // Every thread waits (bounded); the CTA leaves together if any gave up.
-    const bool arrived = bar_wait(&mma_bar, phase, wait_limit);
-    if (__syncthreads_or(!arrived)) {
-      if (tid == 0) atomicExch(err, 1);
-      ok = false;
-      break;
-    }
-    phase ^= 1u;
-    fence_after_sync();
-
-    // Epilogue: row r of tile (gi*J + j) is target i + (gi*J + j)*MT + r;
-    // accumulator lane 32*warp + lane holds row 32*warp + lane (MT = 128) or,
-    // for MT = 64, lanes 0-15 of each warp hold rows 16*warp + lane. Eight
-    // columns at a time: all loads of the old values first, then the stores.
-    const int r = MT == 128 ? 32 * warp + lane : 16 * warp + lane;
+  } else {
+    // ------------------------------------------------------------ drain
+    // Row r of tile (gi*J + j) is target i + (gi*J + j)*MT + r; lane 32q + x of
+    // the accumulator (q = warp % 4) holds row 32q + x (MT = 128) or, for
+    // MT = 64, rows 16q + x in lanes x < 16 of each quarter.
+    const int q = warp & 3;
+    const int r = MT == 128 ? 32 * q + lane : 16 * q + lane;
     const bool row_ok = MT == 128 || lane < 16;
-    for (int k = 0; k < nk; ++k) {
-      const long item = base + k;
-      const int l = (int)(item / g.D) + 1, d = (int)(item - (long)(l - 1) * g.D);
-      for (int c0 = 0; c0 < cols; c0 += 8) {
-        float v[8];
-        tmem_ld8(tmem + ((uint32_t)(32 * warp) << 16) + (uint32_t)(k * cols + c0), v);
-        if (!row_ok) continue;
-        float* dst[8];
-        float old[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const int c = c0 + e;
-          const int gi = c / NR, n = c - gi * NR;
-          dst[e] = nullptr;
-          if (n < J * g.B) {
-            const int j = n / g.B, b = n - j * g.B;
-            dst[e] = state + slot_index(g, l, d * g.B + b, i + (gi * J + j) * MT + r);
-          }
-          old[e] = (dst[e] && !overwrite) ? *dst[e] : 0.f;
-        }
-#pragma unroll
-        for (int e = 0; e < 8; ++e)
-          if (dst[e]) *dst[e] = old[e] + v[e];
+    for (int ps = 0; ps < npass; ++ps) {
+      const int st = ps & 1;
+      const long base = first + (long)ps * stride;
+      const int nk = (int)(items - base < IPC ? items - base : IPC);
+      // lanes of a warp leave together (the accumulator loads are warp-wide)
+      const bool arrived = bar_wait_or_abort(&done_bar[st], (ps >> 1) & 1, wait_limit, abort_flag);
+      if (!__all_sync(0xffffffffu, arrived)) {
+        if (lane == 0) give_up();
+        break;
       }
+      fence_after_sync();
+      for (int k = 0; k < nk; ++k) {
+        const long item = base + k;
+        const int l = (int)(item / g.D) + 1, d = (int)(item - (long)(l - 1) * g.D);
+        float* rowbase = state + slot_index(g, l, d * g.B, i + r);
+        for (int c0 = 0; c0 < cols; c0 += 8) {
+          float v[8];
+          tmem_ld8(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)((st * IPC + k) * cols + c0), v);
+          if (!row_ok) continue;
+          int ofs[8];
+          float old[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            ofs[e] = col_ofs[c0 + e];
+            old[e] = (ofs[e] >= 0 && !overwrite) ? rowbase[ofs[e]] : 0.f;
+          }
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            if (ofs[e] >= 0) rowbase[ofs[e]] = old[e] + v[e];
+        }
+      }
+      fence_before_sync();
+      bar_arrive(&empty_bar[st]);
     }
-    fence_before_sync();
-    __syncthreads();
   }
 
-  if (!ok) {
-    // The commit did not arrive in time: give the MMAs another bounded wait
-    // before the accumulator columns are released.
-    bar_wait(&mma_bar, phase, wait_limit);
-  }
   fence_before_sync();
   __syncthreads();
   fence_after_sync();
@@ -335,8 +425,9 @@ static cudaError_t tc_occupancy(const TcPlan& p, int device, int* per_sm) {
       (e = cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, device)) != cudaSuccess)
     return e;
   const size_t per_cta_smem = p.smem + fa.sharedSizeBytes + (size_t)reserved;
-  const int regs_cta = ((fa.numRegs * 32 + 255) / 256 * 256) * 4;   // 4 warps, 256-register allocation units
-  int n = sm_threads / 128;
+  const int warps = kTcThreads / 32;
+  const int regs_cta = ((fa.numRegs * 32 + 255) / 256 * 256) * warps;   // 256-register allocation units per warp
+  int n = sm_threads / kTcThreads;
   if (sm_blocks < n) n = sm_blocks;
   if (regs_cta > 0 && sm_regs / regs_cta < n) n = sm_regs / regs_cta;
   if ((int)(sm_smem / per_cta_smem) < n) n = (int)(sm_smem / per_cta_smem);
@@ -350,11 +441,22 @@ cudaError_t tc_prepare(const Dims& g, int U, int split, int num_sms, TcPlan* out
   p.U = U;
   p.MT = (U >= 128 && g.B % 16 == 0) ? 128 : 64;
   const int NT = U / p.MT;
-  // tiles per group: enough that N = B*J reaches 16 columns
-  int J = 1;
-  while (J < NT && g.B * J < 16) J <<= 1;
-  p.J = J;
+  int device = 0, smem_optin = 0;
+  cudaError_t e = cudaGetDevice(&device);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, device);
+  if (e != cudaSuccess) return e;
   const int mult = p.MT == 128 ? 16 : 8;
+  auto two_stage_bytes = [&](int J_) {   // two stages of one item's operands, plus slack
+    const int NR_ = (g.B * J_ + mult - 1) / mult * mult;
+    const size_t item = (size_t)(split ? 2 : 1) * ((size_t)32 * U + (size_t)NR_ * (U + (J_ - 1) * p.MT) * 2);
+    return 2 * (item + 127) / 128 * 128 + (size_t)NR_ * NR_ * 2 + 256 + 2048;
+  };
+  // tiles per group: enough that N = B*J reaches 16 columns, as long as two
+  // stages of operands fit in shared memory
+  int J = 1;
+  while (J < NT && g.B * J < 16 && two_stage_bytes(2 * J) <= (size_t)smem_optin) J <<= 1;
+  if (two_stage_bytes(J) > (size_t)smem_optin) return cudaErrorInvalidValue;
+  p.J = J;
   p.NR = (g.B * J + mult - 1) / mult * mult;
   if (p.NR > 256) return cudaErrorInvalidValue;
   p.K = U + (J - 1) * p.MT;
@@ -365,16 +467,14 @@ cudaError_t tc_prepare(const Dims& g, int U, int split, int num_sms, TcPlan* out
   // items share the smallest accumulator allocation (32 columns), within 64 KB.
   p.item_bytes = ((size_t)(split ? 2 : 1) * ((size_t)32 * U + (size_t)p.NR * p.K * 2) + 127) / 128 * 128;
   p.ipc = cols >= 32 ? 1 : 32 / cols;
-  while (p.ipc > 1 && (size_t)p.ipc * p.item_bytes > 64 * 1024) p.ipc >>= 1;
-  // Operands, plus slack past the last one: a B-operand read with its two
-  // strides exchanged would stay inside the allocation.
-  p.smem = (size_t)p.ipc * p.item_bytes + (size_t)p.NR * p.NR * 2 + 256;
-  const int cols_all = p.ipc * cols;
+  while (p.ipc > 1 && (size_t)p.ipc * p.item_bytes > 48 * 1024) p.ipc >>= 1;
+  if (2 * p.ipc * cols > 512) return cudaErrorInvalidValue;
+  // Two stages of operands, plus slack past the last one: a B-operand read
+  // with its two strides exchanged would stay inside the allocation.
+  p.smem = 2 * (size_t)p.ipc * p.item_bytes + (size_t)p.NR * p.NR * 2 + 256;
+  const int cols_all = 2 * p.ipc * cols;        // two stages of accumulators
   p.tmem_cols = pow2_at_least(cols_all < 32 ? 32 : cols_all);
   int occ = 0;
-  int device = 0;
-  cudaError_t e = cudaGetDevice(&device);
-  if (e != cudaSuccess) return e;
   e = p.MT == 128 ? (split ? tc_occupancy<128, true>(p, device, &occ) : tc_occupancy<128, false>(p, device, &occ))
                   : (split ? tc_occupancy<64, true>(p, device, &occ) : tc_occupancy<64, false>(p, device, &occ));
   if (e != cudaSuccess) return e;
@@ -395,11 +495,11 @@ cudaError_t launch_tile_tc(const Dims& g, float* state, const float* taps, const
   if ((i & -i) != p.U || p.grid < 1) return cudaErrorInvalidValue;
   const int ow = is_pow2(i) ? 1 : 0;
   if (p.MT == 128) {
-    if (p.split) k_tile_tc<128, true><<<p.grid, 128, p.smem, st>>>(g, state, taps, p, i, ow, err, wait_limit);
-    else k_tile_tc<128, false><<<p.grid, 128, p.smem, st>>>(g, state, taps, p, i, ow, err, wait_limit);
+    if (p.split) k_tile_tc<128, true><<<p.grid, kTcThreads, p.smem, st>>>(g, state, taps, p, i, ow, err, wait_limit);
+    else k_tile_tc<128, false><<<p.grid, kTcThreads, p.smem, st>>>(g, state, taps, p, i, ow, err, wait_limit);
   } else {
-    if (p.split) k_tile_tc<64, true><<<p.grid, 128, p.smem, st>>>(g, state, taps, p, i, ow, err, wait_limit);
-    else k_tile_tc<64, false><<<p.grid, 128, p.smem, st>>>(g, state, taps, p, i, ow, err, wait_limit);
+    if (p.split) k_tile_tc<64, true><<<p.grid, kTcThreads, p.smem, st>>>(g, state, taps, p, i, ow, err, wait_limit);
+    else k_tile_tc<64, false><<<p.grid, kTcThreads, p.smem, st>>>(g, state, taps, p, i, ow, err, wait_limit);
   }
   return cudaGetLastError();
 }
