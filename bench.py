@@ -92,7 +92,7 @@ def cost_model(w: synth.Workload, chunk: int, fft_from: int, fft_max: int = 1 <<
     return out, tot
 
 
-def survey_closed_form_bytes(w: synth.Workload) -> float:
+def closed_form_block_bytes(w: synth.Workload) -> float:
     """The schedule's block bytes in closed form, M*D*(L/2)*log2(L)*(8 + B(s_x+8))."""
     s = 2 if w.dtype == "bf16" else 4
     return w.layers * w.channels * (w.length / 2) * math.log2(w.length) * (8 + w.batch * (s + 8))

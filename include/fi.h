@@ -54,7 +54,7 @@ typedef enum {
   FI_E_CUDA = 3,        /* a CUDA runtime call or kernel launch failed */
   FI_E_STATE = 4,       /* not allowed in the current state (e.g. stepping past max_len) */
   FI_E_TIMEOUT = 5,     /* reserved: a bounded device-side wait gave up */
-  FI_E_UNSUPPORTED = 6  /* valid request outside what this build implements */
+  FI_E_UNSUPPORTED = 6  /* valid request outside what the library implements */
 } fi_status;
 
 typedef enum { FI_F32 = 0, FI_BF16 = 1 } fi_dtype;
