@@ -345,8 +345,11 @@ __global__ void __launch_bounds__(kTcThreads) k_tile_tc(Dims g, float* __restric
         mma_commit(&done_bar[st]);
         last_commit = ps;
       }
-      // The accumulators are released only after the last commit has arrived.
-      if (last_commit >= 0) bar_wait(&done_bar[last_commit & 1], (last_commit >> 1) & 1, wait_limit);
+      // The accumulators are released only after the last commit has arrived
+      // (a wait of its own, at least the default length: a caller's short wait
+      // limit must not release columns that MMAs still write).
+      if (last_commit >= 0)
+        bar_wait(&done_bar[last_commit & 1], (last_commit >> 1) & 1, wait_limit > kDefaultWaitLimit ? wait_limit : kDefaultWaitLimit);
     }
     __syncwarp();
   } else {

@@ -74,3 +74,28 @@ def test_tensor_core_blocks_above_fft_range(fi):
     h64 = oracle_filters(inp["h_np"], w.dtype)
     r = teacher_forced_errors(h64, acts, rec, [(b, d) for b in range(8) for d in range(4)], w.dtype)
     assert r["y"] <= 1e-5, r["y"]
+
+
+def test_tensor_core_bounded_waits_report_timeout(fi):
+    # With a wait limit of 0 the tensor-core kernel's pipeline waits give up at
+    # once: the MMA warp issues nothing, every role leaves its loop, the
+    # accumulator columns are released and fi_sync reports FI_E_TIMEOUT. With
+    # the default limit the same context then generates correctly.
+    w = synth.Workload("tc-timeout", 2, 4, 1024, 8, "bf16", 1e-5, 1e-3)
+    inp = gpu_inputs(w, 5)
+    ctx = fi.Context(inp["h"], w.batch, w.dtype, tc_max=256)
+    y = torch.empty((w.length, w.batch, w.channels), dtype=torch.float32, device="cuda")
+    ctx.set_wait_limit(0)
+    ctx.generate(w.length, inp["x0"], inp["eps"], y, 0.1)
+    with pytest.raises(fi.FiError) as e:
+        ctx.sync()
+    assert e.value.status == fi.FI_E_TIMEOUT
+    ctx.set_wait_limit(-1)
+    ctx.reset()
+    rec = torch.empty((w.layers, w.length, w.batch, w.channels), dtype=torch.float32, device="cuda")
+    ctx.generate(w.length, inp["x0"], inp["eps"], y, 0.1, rec)
+    ctx.sync()
+    acts = [a.cpu().numpy() for a in read_all_activations(ctx, w.length)]
+    h64 = oracle_filters(inp["h_np"], w.dtype)
+    r = teacher_forced_errors(h64, acts, rec.cpu().numpy(), [(b, d) for b in range(8) for d in range(4)], w.dtype)
+    assert r["y"] <= 1e-5, r["y"]
