@@ -67,7 +67,8 @@ typedef struct {
   int32_t dtype;     /* fi_dtype of filters and tokens; accumulation is always fp32 */
   int32_t chunk;     /* 0 = automatic; else block sides below this run on chip (power of two, 2..64) */
   int32_t fft_from;  /* 0 = automatic; else the smallest block side computed by FFT (power of two >= 64) */
-  int32_t tc_max;    /* 0 = automatic (sides 64..256 for bf16 with batch >= 32, else none), -1 = never;
+  int32_t tc_max;    /* 0 = automatic (bf16 with batch >= 32: sides 64..256, 64..512 from batch 64;
+                        otherwise none), -1 = never;
                         else block sides 64..tc_max (power of two >= 64) run on the tensor cores as
                         Toeplitz products (bf16 contexts: exact bf16 products; fp32 contexts: three
                         bf16 products of split operands), ahead of FFT */

@@ -233,14 +233,14 @@ fi_status fi_init(fi_ctx** out, const fi_config* cfg, const void* h, void* strea
   c->q_hi = g.P - 1 < kMaxFftLog2 ? g.P - 1 : kMaxFftLog2;
   if (c->q_lo < kMinFftLog2) c->q_lo = kMinFftLog2;
   // Tensor-core blocks from side 64 up to tc_max, ahead of FFT (the FFT range
-  // starts above them). Automatic: sides 64..256 for bf16 batches of 32 or
-  // more sequences, where they measured faster than the FFT blocks on B200
-  // (8 x 2048 channels, B = 64: 99.6 vs ~123 ms per generation for those
-  // sides; B = 8 and fp32 B = 4 stay on FFT); sides that cannot be planned
-  // are left to FFT.
+  // starts above them). Automatic: bf16 batches of 32 or more sequences, sides
+  // 64..256 (64..512 from B = 64), where they measured faster than the FFT
+  // blocks on B200 (8 x 2048 channels, L = 16384: B = 32 378 vs 391 ms per
+  // generation, B = 64 748 vs 779 ms; B = 8 and fp32 B = 4 stay on FFT);
+  // sides that cannot be planned are left to FFT.
   const bool tc_auto = cfg->tc_max == 0 && g.bf16 && g.B >= 32;
   if (cfg->tc_max > 0 || tc_auto) {
-    c->tc_q_hi = ilog2((uint32_t)(tc_auto ? 256 : cfg->tc_max));
+    c->tc_q_hi = ilog2((uint32_t)(tc_auto ? (g.B >= 64 ? 512 : 256) : cfg->tc_max));
     if (c->tc_q_hi > g.P - 1) c->tc_q_hi = g.P - 1;
     for (int q = kMinFftLog2; q <= c->tc_q_hi; ++q) {
       if ((e = tc_prepare(g, 1 << q, g.bf16 ? 0 : 1, c->num_sms, &c->tc[q])) != cudaSuccess) {

@@ -275,34 +275,53 @@ __global__ void __launch_bounds__(kTcThreads) k_tile_tc(Dims g, float* __restric
       // 8 consecutive sources of one sequence (one 32-byte sector) and writes
       // them as one 16-byte core-matrix row; consecutive threads take
       // consecutive sequences, so a warp's stores fill whole core matrices.
+      // Several tasks per round: all their global loads go out before the first
+      // conversion waits on data, so a thread keeps up to eight loads in flight.
       const int oct = U / 8;
-      for (int w = lt; w < nk * g.B * oct; w += 128) {
-        const int k = w / (g.B * oct), wr = w - k * (g.B * oct);
-        const int q8 = wr / g.B, b = wr - q8 * g.B;
-        const long item = base + k;
-        const int l = (int)(item / g.D) + 1, d = (int)(item - (long)(l - 1) * g.D);
-        const float4* src = reinterpret_cast<const float4*>(state + slot_index(g, l - 1, d * g.B + b, i - U) + 8 * q8);
-        const float4 v0 = src[0], v1 = src[1];
-        // source 8 q8 + e sits at kappa = U - 1 - 8 q8 - e: kappa kb + m holds element 7 - m
-        const int kb = U - 8 - 8 * q8;
-        const float vv[8] = {v1.w, v1.z, v1.y, v1.x, v0.w, v0.z, v0.y, v0.x};
-        uint32_t wh[4], wl[4];
+      const int ntask = nk * g.B * oct;
+      constexpr int kTasks = SPLIT ? 2 : 4;   // split operands need twice the registers per task
+      for (int w0 = lt; w0 < ntask; w0 += kTasks * 128) {
+        float4 v0[kTasks], v1[kTasks];
 #pragma unroll
-        for (int m = 0; m < 8; m += 2) {
-          uint16_t h0, l0, h1, l1;
-          if constexpr (SPLIT) {
-            split_bf16(vv[m], h0, l0);
-            split_bf16(vv[m + 1], h1, l1);
-          } else {
-            h0 = bf16_bits(vv[m]); h1 = bf16_bits(vv[m + 1]); l0 = l1 = 0;
+        for (int u = 0; u < kTasks; ++u) {
+          const int w = w0 + u * 128;
+          if (w < ntask) {
+            const int k = w / (g.B * oct), wr = w - k * (g.B * oct);
+            const int q8 = wr / g.B, b = wr - q8 * g.B;
+            const long item = base + k;
+            const int l = (int)(item / g.D) + 1, d = (int)(item - (long)(l - 1) * g.D);
+            const float4* src = reinterpret_cast<const float4*>(state + slot_index(g, l - 1, d * g.B + b, i - U) + 8 * q8);
+            v0[u] = src[0];
+            v1[u] = src[1];
           }
-          wh[m / 2] = (uint32_t)h0 | ((uint32_t)h1 << 16);
-          wl[m / 2] = (uint32_t)l0 | ((uint32_t)l1 << 16);
         }
-        for (int j = 0; j < J; ++j) {
-          const uint32_t off = tc_b_offset(NR, j * g.B + b, j * MT + kb);
-          *reinterpret_cast<uint4*>(x_hi(st, k) + off) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
-          if constexpr (SPLIT) *reinterpret_cast<uint4*>(x_lo(st, k) + off) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
+#pragma unroll
+        for (int u = 0; u < kTasks; ++u) {
+          const int w = w0 + u * 128;
+          if (w >= ntask) break;
+          const int k = w / (g.B * oct), wr = w - k * (g.B * oct);
+          const int q8 = wr / g.B, b = wr - q8 * g.B;
+          // source 8 q8 + e sits at kappa = U - 1 - 8 q8 - e: kappa kb + m holds element 7 - m
+          const int kb = U - 8 - 8 * q8;
+          const float vv[8] = {v1[u].w, v1[u].z, v1[u].y, v1[u].x, v0[u].w, v0[u].z, v0[u].y, v0[u].x};
+          uint32_t wh[4], wl[4];
+#pragma unroll
+          for (int m = 0; m < 8; m += 2) {
+            uint16_t h0, l0, h1, l1;
+            if constexpr (SPLIT) {
+              split_bf16(vv[m], h0, l0);
+              split_bf16(vv[m + 1], h1, l1);
+            } else {
+              h0 = bf16_bits(vv[m]); h1 = bf16_bits(vv[m + 1]); l0 = l1 = 0;
+            }
+            wh[m / 2] = (uint32_t)h0 | ((uint32_t)h1 << 16);
+            wl[m / 2] = (uint32_t)l0 | ((uint32_t)l1 << 16);
+          }
+          for (int j = 0; j < J; ++j) {
+            const uint32_t off = tc_b_offset(NR, j * g.B + b, j * MT + kb);
+            *reinterpret_cast<uint4*>(x_hi(st, k) + off) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
+            if constexpr (SPLIT) *reinterpret_cast<uint4*>(x_lo(st, k) + off) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
+          }
         }
       }
       fence_proxy_async();   // generic-proxy writes -> visible to the tensor core
@@ -375,20 +394,25 @@ __global__ void __launch_bounds__(kTcThreads) k_tile_tc(Dims g, float* __restric
         const long item = base + k;
         const int l = (int)(item / g.D) + 1, d = (int)(item - (long)(l - 1) * g.D);
         float* rowbase = state + slot_index(g, l, d * g.B, i + r);
-        for (int c0 = 0; c0 < cols; c0 += 8) {
-          float v[8];
-          tmem_ld8(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)((st * IPC + k) * cols + c0), v);
-          if (!row_ok) continue;
-          int ofs[8];
-          float old[8];
+        // 16 columns per round: the old accumulator values (independent of the
+        // tensor memory) are all requested first, then the two 8-column loads.
+        for (int c0 = 0; c0 < cols; c0 += 16) {
+          int ofs[16];
+          float old[16];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            ofs[e] = col_ofs[c0 + e];
+          for (int e = 0; e < 16; ++e) {
+            ofs[e] = (c0 + e < cols && row_ok) ? col_ofs[c0 + e] : -1;
             old[e] = (ofs[e] >= 0 && !overwrite) ? rowbase[ofs[e]] : 0.f;
           }
 #pragma unroll
-          for (int e = 0; e < 8; ++e)
-            if (ofs[e] >= 0) rowbase[ofs[e]] = old[e] + v[e];
+          for (int h = 0; h < 2; ++h) {
+            if (c0 + 8 * h >= cols) break;       // uniform across the warp
+            float v[8];
+            tmem_ld8(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)((st * IPC + k) * cols + c0 + 8 * h), v);
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              if (ofs[8 * h + e] >= 0) rowbase[ofs[8 * h + e]] = old[8 * h + e] + v[e];
+          }
         }
       }
       fence_before_sync();
