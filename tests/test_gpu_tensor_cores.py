@@ -14,6 +14,7 @@ target tiles per product (B < 16, including odd B and B = 1), 128-row tiles
 import numpy as np
 import pytest
 
+import oracle
 import synth
 from fi_testlib import TOL, gpu_inputs, oracle_filters, read_all_activations, sampler_error, teacher_forced_errors
 
@@ -99,3 +100,41 @@ def test_tensor_core_bounded_waits_report_timeout(fi):
     h64 = oracle_filters(inp["h_np"], w.dtype)
     r = teacher_forced_errors(h64, acts, rec.cpu().numpy(), [(b, d) for b in range(8) for d in range(4)], w.dtype)
     assert r["y"] <= 1e-5, r["y"]
+
+
+def test_tensor_core_blocks_with_steps_and_ragged_calls(fi):
+    # fi_step (one position per call, blocks launched per position) for the
+    # first 70 positions, then generation in calls that stop inside chunks: the
+    # tensor-core blocks of sides 64..256 run from both paths on one state.
+    w = synth.Workload("tc-mixed-calls", 2, 4, 1024, 8, "bf16", 1e-5, 1e-3)
+    inp = gpu_inputs(w, 9)
+    ctx = fi.Context(inp["h"], w.batch, w.dtype, tc_max=256)
+    toks = synth.token_stream(w, 9)
+    n_step = 70
+    ys = torch.empty((n_step, w.batch, w.channels), dtype=torch.float32, device="cuda")
+    tt = torch.from_numpy(toks).cuda().to(torch.bfloat16)
+    for t in range(n_step):
+        ctx.step(tt[t].contiguous(), ys[t])
+    rest = w.length - n_step
+    y = torch.empty((rest, w.batch, w.channels), dtype=torch.float32, device="cuda")
+    p = 0
+    x0 = tt[n_step].contiguous()
+    for m in (58, 1, 200, 3, rest - 262):
+        yk = torch.empty((m, w.batch, w.channels), dtype=torch.float32, device="cuda")
+        ctx.generate(m, x0, inp["eps"][n_step + p:n_step + p + m].contiguous(), yk, 0.1)
+        y[p:p + m] = yk
+        p += m
+        x0 = (torch.tanh(yk[-1].double()) + 0.1 * inp["eps"][n_step + p - 1].double()).to(torch.bfloat16)
+    ctx.sync()
+    assert ctx.position == w.length
+    acts = [a.cpu().numpy() for a in read_all_activations(ctx, w.length)]
+    h64 = oracle_filters(inp["h_np"], w.dtype)
+    # last layer's outputs: the steps' y and the generated y, against the oracle
+    # convolution of the recorded last-layer inputs
+    y_all = np.concatenate([ys.cpu().numpy(), y.cpu().numpy()])
+    worst = 0.0
+    for b in range(w.batch):
+        for d in range(w.channels):
+            ref = oracle.causal_conv(h64[-1, d], acts[-1][:, b, d].astype(np.float64))
+            worst = max(worst, oracle.stream_error(y_all[:, b, d], ref))
+    assert worst <= 1e-5, worst
