@@ -25,11 +25,13 @@
 // lo = bf16(v - hi), and add the three products hi*hi + hi*lo + lo*hi (the
 // dropped lo*lo term and the residuals are below 2^-16 relative per product).
 //
-// One CTA of 4 warps per (layer, channel) item at a time: all threads build the
-// table and the B operand in shared memory, one thread issues the MMAs of every
-// group (each group into its own accumulator columns), a commit arrives on an
-// mbarrier, and each warp reads its 32 accumulator lanes and adds them to the
-// targets in HBM. Every wait is bounded.
+// A CTA works through passes of one or more (layer, channel) items: operand
+// builder warps write the tables and B operands of a pass into shared memory,
+// one thread issues the MMAs of every item and group (each into its own
+// accumulator columns) and commits them to an mbarrier, and drain warps read
+// their 32 accumulator lanes and add them to the targets in HBM; two stages
+// let the three roles work on consecutive passes at once (details at the
+// kernel). Every wait is bounded.
 #include "fi_internal.cuh"
 
 namespace fi {
