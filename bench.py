@@ -245,34 +245,40 @@ def _oracle_job(args):
 
 
 def oracle_baseline(w: synth.Workload, seed: int, n_pos: int, streams_per_core: int, cores: int | None = None):
-    """Time the oracle on `cores` processes x streams_per_core streams x n_pos positions,
-    then extrapolate to the whole workload by its O(L^2) cost (work ~ streams * n^2)."""
+    """Time the oracle on `cores` processes x streams_per_core streams over two prefixes
+    (n_pos/4 and n_pos positions), fit time = a*n + b*n^2 (per-position overhead plus the
+    O(n^2) sums), and extrapolate to all L positions and all streams (streams are
+    independent, so the work scales with their number)."""
     cores = cores or os.cpu_count() or 1
     rng = np.random.default_rng(seed + 17)
-    jobs = []
-    for c in range(cores):
-        st = [(int(rng.integers(w.batch)), int(rng.integers(w.channels))) for _ in range(streams_per_core)]
-        jobs.append((w.name, seed, st, n_pos))
+    streams = [[(int(rng.integers(w.batch)), int(rng.integers(w.channels))) for _ in range(streams_per_core)]
+               for _ in range(cores)]
     ctx = mp.get_context("spawn")
+    n1, n2 = max(n_pos // 4, 1), n_pos
+    times = []
     t0 = time.perf_counter()
     with ctx.Pool(cores) as pool:
-        per = pool.map(_oracle_job, jobs)
+        for n in (n1, n2):
+            times.append(max(pool.map(_oracle_job, [(w.name, seed, st, n) for st in streams])))
     wall = time.perf_counter() - t0
-    compute = max(per)
+    A = np.array([[n1, n1 * n1], [n2, n2 * n2]], dtype=np.float64)
+    a_, b_ = np.linalg.solve(A, np.array(times))
+    if a_ < 0 or b_ < 0:                       # noisy fit: fall back to the pure n^2 law
+        a_, b_ = 0.0, times[1] / (n2 * n2)
     sample_streams = cores * streams_per_core
-    work_sample = sample_streams * n_pos * (n_pos + 1) / 2
-    work_full = w.streams * w.length * (w.length + 1) / 2
-    t_full = compute * work_full / work_sample
+    t_full = (a_ * w.length + b_ * w.length ** 2) * w.streams / sample_streams
     return {
         "value": w.batch * w.length / t_full,
         "unit": UNIT,
         "cores": cores,
         "kind": "oracle",
         "sample": (f"float64 oracle, all {w.layers} layers, {sample_streams} (sequence, channel) streams x first "
-                   f"{n_pos} positions ({cores} spawned processes, {compute:.1f} s compute, {wall:.1f} s wall); "
-                   f"extrapolated by streams x n^2 to {w.streams} streams x {w.length} positions"),
+                   f"{n1} and {n2} positions ({cores} spawned processes, {times[0]:.1f} + {times[1]:.1f} s compute, "
+                   f"{wall:.1f} s wall); time fitted as a*n + b*n^2 and extrapolated to {w.streams} streams x "
+                   f"{w.length} positions"),
         "extrapolated": True,
-        "seconds_sample": compute,
+        "seconds_sample": float(sum(times)),
+        "fit": {"a_s_per_position": float(a_), "b_s_per_position2": float(b_)},
     }
 
 

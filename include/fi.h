@@ -53,7 +53,7 @@ typedef enum {
   FI_E_OOM = 2,         /* a device or pinned-host allocation failed */
   FI_E_CUDA = 3,        /* a CUDA runtime call or kernel launch failed */
   FI_E_STATE = 4,       /* not allowed in the current state (e.g. stepping past max_len) */
-  FI_E_TIMEOUT = 5,     /* reserved: a bounded device-side wait gave up */
+  FI_E_TIMEOUT = 5,     /* a bounded device-side wait gave up (reported by fi_sync and the calls that synchronise) */
   FI_E_UNSUPPORTED = 6  /* valid request outside what the library implements */
 } fi_status;
 
@@ -99,13 +99,20 @@ FI_API fi_status fi_step(fi_ctx* ctx, const void* x_t, float* y_t);
 
 /* Closed-loop generation of n positions from the current position p on device:
  * x_p = x0, and for t >= p: x_{t+1} = R(tanh(y^M_t) + eps_scale * eps[t-p]).
- * x0:    device [B][D] of cfg->dtype.
+ * The page states the autoregressive loop (Algorithm 2: red cells and blocks
+ * per layer, then the sampler) but has no call that runs many positions at
+ * once: this one runs that loop on the device so that no host round trip sits
+ * between positions. The sampler rule is the workloads' (tanh of the last
+ * layer's output plus scaled noise; the page's synthetic sampler "adds noise",
+ * "Configurazione Sperimentale").
+ * x0:    device [B][D] of cfg->dtype; or NULL when p > 0, to continue with the
+ *        token the sampler produced at the end of the previous call.
  * eps:   device [n][B][D] fp32 sampler noise.
  * y_out: device [n][B][D] fp32, receives y^M_t for t = p..p+n-1.
  * rec:   NULL, or device [M][n][B][D] fp32 that receives y^l_t for every layer
  *        (test and inspection hook; costs one extra write per layer and position).
  * Leaves the context at position p+n with the same state fi_step would leave.
- * Errors: FI_E_INVALID (null, n < 0), FI_E_STATE (p + n > max_len). */
+ * Errors: FI_E_INVALID (null, x0 NULL at p = 0, n < 0), FI_E_STATE (p + n > max_len). */
 FI_API fi_status fi_generate(fi_ctx* ctx, int32_t n, const void* x0, const float* eps,
                       float eps_scale, float* y_out, float* rec);
 
@@ -131,14 +138,19 @@ FI_API fi_status fi_generate_lazy(fi_ctx* ctx, int32_t n, const void* x0, const 
 FI_API fi_status fi_sync(fi_ctx* ctx);
 
 /* Rewind to position 0. O(1): no memory is cleared, because every accumulator
- * is first written (not added to) by the block that first reaches it. */
+ * is first written (not added to) by the block that first reaches it.
+ * Not on the page (which runs one generation per model call); the filters and
+ * their precomputed spectra ("Precomputazione FFT") are kept. */
 FI_API fi_status fi_reset(fi_ctx* ctx);
 
 /* Current position (number of positions already produced). */
 FI_API fi_status fi_position(const fi_ctx* ctx, int32_t* pos);
 
 /* Copy the recorded activations a^layer_t for t < position into dst,
- * device [position][B][D] fp32; layer in [0, M-1] (layer 0 = the tokens). */
+ * device [position][B][D] fp32; layer in [0, M-1] (layer 0 = the tokens).
+ * These are the a^l_i the page keeps for every position ("Ottimizzazione della
+ * Memoria": the slot of a^l_i also holds b^l_i until it is consumed); reading
+ * them is a test hook, not on the page. */
 FI_API fi_status fi_read_activations(fi_ctx* ctx, int32_t layer, float* dst);
 
 /* Change the stream later calls run on. */
@@ -183,7 +195,10 @@ FI_API const char* fi_last_error(void);
  * returns FI_E_INVALID, with the sizes in fi_last_error(), when that is more.
  * All calls share the array and it keeps the last call's contents (each call
  * rewrites what it reads); calls whose work overlaps on the GPU race on it.
- * The first call on a device looks up the array's device address.
+ * The first call on a device, with that device current, looks up the array's
+ * device address and keeps it for the life of the process: make that first call
+ * before any stream capture, and do not call this entry point again after a
+ * cudaDeviceReset of that device (the kept address would no longer be valid).
  * Errors: FI_E_INVALID (NULL, sizes, L > 2^15), FI_E_CUDA, FI_E_TIMEOUT. */
 FI_API fi_status fi_generate_noalloc(const fi_config* cfg, const void* h, int32_t n, const void* x0,
                                      const float* eps, float eps_scale, float* y_out, void* stream);

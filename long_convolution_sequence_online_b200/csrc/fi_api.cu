@@ -361,7 +361,8 @@ fi_status fi_generate(fi_ctx* c, int32_t n, const void* x0, const float* eps, fl
   if (!c) return fail(FI_E_INVALID, "ctx is NULL");
   if (n < 0) return fail(FI_E_INVALID, "n < 0");
   if (n == 0) return FI_OK;
-  if (!x0 || !eps || !y_out) return fail(FI_E_INVALID, "NULL buffer");
+  if (!eps || !y_out) return fail(FI_E_INVALID, "NULL buffer");
+  if (!x0 && c->pos == 0) return fail(FI_E_INVALID, "x0 may be NULL only when continuing from a position > 0");
   if ((int64_t)c->pos + n > c->g.L) return fail(FI_E_STATE, "position + n > max_len");
   if (c->lazy_mode) return fail(FI_E_STATE, "context holds a lazy generation; call fi_reset");
   const int CH = c->chunk;

@@ -17,6 +17,8 @@
 // Thread roles: thread k owns the (layer, stream) rows k, k+T, ... for the gray
 // blocks (all U outputs of a row, with U sources and 2U-1 taps in registers);
 // threads [0, G) each carry one stream through the layers for the red cells.
+#include <mutex>
+
 #include "fi_internal.cuh"
 
 namespace fi {
@@ -433,11 +435,25 @@ int chunk_streams_per_cta(const Dims& g, int chunk, int num_sms, size_t max_smem
   return G;
 }
 
+// The dynamic shared-memory cap is one value per kernel function and device,
+// shared by every context in the process; it only ever grows here, so a small
+// configuration never lowers it under a live context that needs more.
+template <class K>
+static cudaError_t raise_smem_cap(K kernel, size_t smem) {
+  cudaFuncAttributes fa{};
+  cudaError_t e = cudaFuncGetAttributes(&fa, kernel);
+  if (e != cudaSuccess) return e;
+  if ((size_t)fa.maxDynamicSharedSizeBytes >= smem) return cudaSuccess;
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+}
+
 cudaError_t configure_chunk(size_t smem) {
-  cudaError_t e = cudaFuncSetAttribute(k_chunk<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e == cudaSuccess) e = cudaFuncSetAttribute(k_chunk<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e == cudaSuccess) e = cudaFuncSetAttribute(k_chunk<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e == cudaSuccess) e = cudaFuncSetAttribute(k_chunk<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  static std::mutex mu;
+  std::lock_guard<std::mutex> lock(mu);
+  cudaError_t e = raise_smem_cap(k_chunk<false, false>, smem);
+  if (e == cudaSuccess) e = raise_smem_cap(k_chunk<false, true>, smem);
+  if (e == cudaSuccess) e = raise_smem_cap(k_chunk<true, false>, smem);
+  if (e == cudaSuccess) e = raise_smem_cap(k_chunk<true, true>, smem);
   return e;
 }
 

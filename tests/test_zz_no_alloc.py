@@ -4,8 +4,11 @@ Such callers (a thread with a hard latency budget, a framework that owns all
 device memory, code running where allocation is not allowed) get their working
 memory from one fixed device array inside the library. This file checks, through
 the C-ABI, that two calls in a row give what the allocating path (fi_init +
-fi_generate) gives, within the fp32 / bf16 tolerances the other parity tests use,
-and that a configuration too large for the fixed array is refused cleanly.
+fi_generate) gives, within the fp32 / bf16 tolerances the other parity tests use;
+that the tiny workload matches the float64 oracle's own closed loop; that a second
+call leaves the device's free memory unchanged; that a call does not disturb a
+live context with a larger on-chip window; and that a configuration too large for
+the fixed array is refused cleanly.
 It sorts last so that a run stopping at its first failure has run everything else.
 """
 import numpy as np
@@ -13,7 +16,8 @@ import pytest
 
 import oracle
 import synth
-from fi_testlib import TOL, gpu_inputs
+from fi_testlib import (TOL, gpu_inputs, oracle_filters, read_all_activations,
+                        teacher_forced_errors)
 
 torch = pytest.importorskip("torch")
 
@@ -68,3 +72,59 @@ def test_noalloc_rejects_oversized_configuration(fi):
         fi.generate_noalloc(h, 1, 16, x0, eps, y)
     assert e.value.status == fi.FI_E_INVALID
     assert "floats of working memory" in str(e.value)
+
+
+@pytest.mark.gpu
+def test_noalloc_matches_oracle_closed_loop(fi):
+    # The tiny single-layer workload: short enough that the float64 oracle's own
+    # closed loop and the device's stay within the fp32 tolerance at every position.
+    w = synth.WORKLOADS["tiny-1x16-L1K"]
+    inp = gpu_inputs(w, 7)
+    h64 = oracle_filters(inp["h_np"], w.dtype)
+    d_of = np.arange(w.streams) % w.channels
+    y_ref, _ = oracle.online_lcsm(h64[:, d_of, :], inp["x0_np"].reshape(-1),
+                                  inp["eps_np"].reshape(w.length, w.streams))
+    for _ in range(2):
+        y = torch.full((w.length, w.batch, w.channels), float("nan"), dtype=torch.float32, device="cuda")
+        fi.generate_noalloc(inp["h"], w.batch, w.length, inp["x0"], inp["eps"], y, w.dtype)
+        torch.cuda.synchronize()
+        got = y.cpu().numpy().reshape(w.length, w.streams).T
+        assert oracle.stream_error(got, y_ref[-1]) <= TOL["f32"]
+
+
+@pytest.mark.gpu
+def test_noalloc_allocates_nothing(fi):
+    w = synth.Workload("noalloc-c", 2, 32, 512, 2, "f32", 1e-3, 1e-1)
+    inp = gpu_inputs(w, 11)
+    y = torch.empty((w.length, w.batch, w.channels), dtype=torch.float32, device="cuda")
+    fi.generate_noalloc(inp["h"], w.batch, w.length, inp["x0"], inp["eps"], y, w.dtype)   # warm-up call
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    fi.generate_noalloc(inp["h"], w.batch, w.length, inp["x0"], inp["eps"], y, w.dtype)
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert free1 == free0
+
+
+@pytest.mark.gpu
+def test_noalloc_leaves_a_wider_live_context_working(fi):
+    # A context whose on-chip window is wide (18 layers, 3456 streams) is created
+    # first; a small fixed-memory call in between must not shrink what its chunk
+    # kernel may use, and the context must still match the oracle afterwards.
+    big = synth.Workload("noalloc-live", 18, 864, 256, 4, "f32", 1e-3, 1e-1)
+    inp = gpu_inputs(big, 13)
+    ctx = fi.Context(inp["h"], big.batch, big.dtype)
+    small = synth.WORKLOADS["tiny-1x16-L1K"]
+    sinp = gpu_inputs(small, 14)
+    ys = torch.empty((small.length, small.batch, small.channels), dtype=torch.float32, device="cuda")
+    fi.generate_noalloc(sinp["h"], small.batch, small.length, sinp["x0"], sinp["eps"], ys, small.dtype)
+    y = torch.empty((big.length, big.batch, big.channels), dtype=torch.float32, device="cuda")
+    rec = torch.empty((big.layers, big.length, big.batch, big.channels), dtype=torch.float32, device="cuda")
+    ctx.generate(big.length, inp["x0"], inp["eps"], y, 0.1, rec)
+    ctx.sync()
+    acts = [a.cpu().numpy() for a in read_all_activations(ctx, big.length)]
+    ctx.close()
+    h64 = oracle_filters(inp["h_np"], big.dtype)
+    streams = [(0, 0), (1, 5), (3, 863), (2, 431)]
+    r = teacher_forced_errors(h64, acts, rec.cpu().numpy(), streams, big.dtype)
+    assert r["y"] <= TOL["f32"], r["y"]
