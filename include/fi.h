@@ -209,6 +209,17 @@ FI_API fi_status fi_generate_noalloc(const fi_config* cfg, const void* h, int32_
  * at once, which exercises the FI_E_TIMEOUT path of fi_sync without any wait. */
 FI_API fi_status fi_debug_set_wait_limit(fi_ctx* ctx, int32_t limit);
 
+/* Test hook (host only, no device work): the table of on-chip block pieces the
+ * chunk kernel runs for a chunk of `chunk` positions (a power of two, 2..64):
+ * retimed != 0 gives the table of a launch that covers a whole chunk (blocks of
+ * side 16 and 32 cut into pieces spread over neighbouring steps), 0 the page's
+ * tiling (the block of step r, side lowbit(r), at step r). Writes up to `cap`
+ * entries of 5 int32 (step, first source, sources, first target, targets;
+ * positions relative to the chunk start) to out and the entry count to *count.
+ * Errors: FI_E_INVALID (NULL, chunk). */
+FI_API fi_status fi_debug_chunk_schedule(int32_t chunk, int32_t retimed, int32_t* out, int32_t cap,
+                                         int32_t* count);
+
 /* Test hook: run the library's device FFT (the one its FFT blocks use) on
  * `count` complex sequences of length 2^log2n (6 <= log2n <= 14), interleaved
  * (re, im) fp32, device buffers in[count][2^log2n][2] -> out (may alias in).

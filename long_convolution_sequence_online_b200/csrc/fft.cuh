@@ -167,21 +167,24 @@ __device__ __forceinline__ void apply_twiddles(float2* v, const float2* __restri
 }
 
 // Shape of the transform: T threads, P = N/T points each, passes of radix
-// min(32, P) until the last pass takes what is left.
-template <int N, int T>
+// min(32, P); the pass that takes what is left (REM bits) comes last, or first
+// when REMF (a transform whose first pass must match the previous transform's
+// last one: the inverse of a convolution that keeps the forward's order).
+template <int N, int T, bool REMF = false>
 struct FftShape {
   static constexpr int LOGN = clog2(N);
   static constexpr int P = N / T;
   static constexpr int RBMAX = cmin(5, clog2(P));
-  static constexpr int rb(int done) { return cmin(RBMAX, LOGN - done); }
+  static constexpr int REM = LOGN % RBMAX;
+  static constexpr int rb(int done) { return (REMF && REM != 0 && done == 0) ? REM : cmin(RBMAX, LOGN - done); }
   static constexpr bool last(int done) { return done + rb(done) >= LOGN; }
 };
 
 // Twiddles and R-point DFTs of one pass on the P points a thread holds
 // (butterfly k in v[k*R .. k*R+R), butterfly index j = tid + k*T).
-template <int N, int T, bool INV, int DONE>
+template <int N, int T, bool INV, int DONE, bool REMF = false>
 __device__ __forceinline__ void pass_compute(float2* v, int tid, const float2* __restrict__ tw) {
-  using S = FftShape<N, T>;
+  using S = FftShape<N, T, REMF>;
   constexpr int R = 1 << S::rb(DONE);
   constexpr int Ns = 1 << DONE;
 #pragma unroll
@@ -196,9 +199,9 @@ __device__ __forceinline__ void pass_compute(float2* v, int tid, const float2* _
 }
 
 // Stockham load of one pass: value r of butterfly j sits at j + r*N/R.
-template <int N, int T, int DONE>
+template <int N, int T, int DONE, bool REMF = false>
 __device__ __forceinline__ void pass_load(const float2* sm, float2* v, int tid) {
-  using S = FftShape<N, T>;
+  using S = FftShape<N, T, REMF>;
   constexpr int R = 1 << S::rb(DONE);
 #pragma unroll
   for (int k = 0; k < S::P / R; ++k) {
@@ -208,9 +211,9 @@ __device__ __forceinline__ void pass_load(const float2* sm, float2* v, int tid) 
 }
 
 // Stockham store of one pass: output r of butterfly j goes to (j - kk)*R + kk + r*Ns.
-template <int N, int T, int DONE>
+template <int N, int T, int DONE, bool REMF = false>
 __device__ __forceinline__ void pass_store(float2* sm, const float2* v, int tid) {
-  using S = FftShape<N, T>;
+  using S = FftShape<N, T, REMF>;
   constexpr int R = 1 << S::rb(DONE);
   constexpr int Ns = 1 << DONE;
 #pragma unroll
@@ -225,28 +228,28 @@ __device__ __forceinline__ void pass_store(float2* sm, const float2* v, int tid)
 
 // Passes DONE.. that go shared memory -> shared memory, stopping before the
 // last pass when STOP_BEFORE_LAST (the caller finishes it with its own store).
-template <int N, int T, bool INV, int DONE, bool STOP_BEFORE_LAST, class Sync>
+template <int N, int T, bool INV, int DONE, bool STOP_BEFORE_LAST, bool REMF = false, class Sync>
 __device__ __forceinline__ void smem_passes(float2* sm, int tid, const float2* __restrict__ tw, Sync sync) {
-  using S = FftShape<N, T>;
+  using S = FftShape<N, T, REMF>;
   if constexpr (DONE < S::LOGN) {
     if constexpr (!(STOP_BEFORE_LAST && S::last(DONE))) {
       float2 v[S::P];
-      pass_load<N, T, DONE>(sm, v, tid);
-      pass_compute<N, T, INV, DONE>(v, tid, tw);
+      pass_load<N, T, DONE, REMF>(sm, v, tid);
+      pass_compute<N, T, INV, DONE, REMF>(v, tid, tw);
       sync();
-      pass_store<N, T, DONE>(sm, v, tid);
+      pass_store<N, T, DONE, REMF>(sm, v, tid);
       sync();
-      smem_passes<N, T, INV, DONE + S::rb(DONE), STOP_BEFORE_LAST>(sm, tid, tw, sync);
+      smem_passes<N, T, INV, DONE + S::rb(DONE), STOP_BEFORE_LAST, REMF>(sm, tid, tw, sync);
     }
   }
 }
 
 // Start of the last pass.
-template <int N, int T, int DONE = 0>
+template <int N, int T, int DONE = 0, bool REMF = false>
 constexpr int last_pass_done() {
-  using S = FftShape<N, T>;
+  using S = FftShape<N, T, REMF>;
   if constexpr (S::last(DONE)) return DONE;
-  else return last_pass_done<N, T, DONE + S::rb(DONE)>();
+  else return last_pass_done<N, T, DONE + S::rb(DONE), REMF>();
 }
 
 // In-place transform of sm[fft_pad<N, T>(0..N)) by the T threads with tid in [0, T).

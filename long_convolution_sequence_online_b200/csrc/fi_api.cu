@@ -494,6 +494,28 @@ fi_status fi_profile_read(fi_ctx* c, int32_t counts[FI_NUM_KERNEL_CLASSES], doub
   return FI_OK;
 }
 
+fi_status fi_debug_chunk_schedule(int32_t chunk, int32_t retimed, int32_t* out, int32_t cap, int32_t* count) {
+  if (!out || !count || cap < 0) return fail(FI_E_INVALID, "bad argument");
+  if (!pow2(chunk) || chunk < 2 || chunk > kChunkMaxSteps) return fail(FI_E_INVALID, "chunk must be a power of two in [2, 64]");
+  ChunkTable tab{};
+  if (!build_chunk_table(chunk, retimed != 0, &tab)) return fail(FI_E_UNSUPPORTED, "table too long");
+  *count = tab.n;
+  for (int j = 0; j < tab.n && j < cap; ++j) {
+    const uint32_t e = tab.e[j];
+    const int kind = (int)((e >> 21) & 15);
+    out[5 * j + 0] = (int32_t)(e & 127);
+    out[5 * j + 1] = (int32_t)((e >> 7) & 127);
+    out[5 * j + 2] = chunk_piece_sources(kind);
+    out[5 * j + 3] = (int32_t)((e >> 14) & 127);
+    out[5 * j + 4] = chunk_piece_targets(kind);
+  }
+  for (int r = 0; r < chunk; ++r) {
+    for (int j = tab.first[r]; j < tab.first[r + 1]; ++j)
+      if ((int)(tab.e[j] & 127) != r) return fail(FI_E_STATE, "step index does not match the entries");
+  }
+  return FI_OK;
+}
+
 fi_status fi_debug_set_wait_limit(fi_ctx* c, int32_t limit) {
   if (!c) return fail(FI_E_INVALID, "ctx is NULL");
   c->wait_limit = limit < 0 ? kDefaultWaitLimit : limit;

@@ -95,6 +95,24 @@ cudaError_t tc_prepare(const Dims& g, int U, int split, int num_sms, TcPlan* out
 cudaError_t launch_tile_tc(const Dims& g, float* state, const float* taps, const TcPlan& p, int i, int* err,
                            int wait_limit, cudaStream_t st);
 
+// Which on-chip block pieces run at which step of a chunk (built on the host):
+// entries sorted by step, e[first[r] .. first[r+1]) run at step r; entry =
+// step | s_lo << 7 | t_lo << 14 | kind << 21 (sources [s_lo, s_lo+ns) to
+// targets [t_lo, t_lo+nd), positions relative to the chunk start).
+constexpr int kChunkMaxSteps = 64;
+constexpr int kChunkMaxEntries = 128;
+struct ChunkTable {
+  int n;
+  uint16_t first[kChunkMaxSteps + 1];
+  uint32_t e[kChunkMaxEntries];
+};
+// retimed = the whole chunk runs in one launch: blocks of side 16 and 32 are cut
+// into pieces spread over neighbouring steps; else the page's blocks, one per step.
+bool build_chunk_table(int chunk, bool retimed, ChunkTable* tab);
+// Sources and targets of a piece kind (for the table's test hook).
+int chunk_piece_sources(int kind);
+int chunk_piece_targets(int kind);
+
 // The chunk kernel: positions [p0, p1) inside the aligned chunk [c, c+chunk),
 // small blocks (side < chunk) on chip, red cells, blocks and the sampler.
 struct ChunkArgs {
@@ -111,6 +129,7 @@ struct ChunkArgs {
   int last_done;         // last step whose blocks have reached HBM before this launch
   int* err;              // device flag set to 1 when a bounded wait gives up
   int wait_limit;        // barrier checks before a wait gives up
+  ChunkTable tab;        // filled by launch_chunk
 };
 
 // Default number of barrier checks before a device-side wait gives up (each

@@ -14,10 +14,28 @@
 // Streams are independent (the block and sampler act elementwise), so CTAs
 // never wait on each other.
 //
-// Thread roles: thread k owns the (layer, stream) rows k, k+T, ... for the gray
-// blocks (all U outputs of a row, with U sources and 2U-1 taps in registers);
-// threads [0, G) each carry one stream through the layers for the red cells.
+// Re-timed on-chip blocks. Inside the chunk every block is a direct sum, whose
+// cost is its area whatever the tiling, so the blocks of side >= 16 (the 16 x 16
+// and 32 x 32 blocks of the page's tiling, which would otherwise stall the
+// chain for thousands of cycles at their step) are cut into pieces that run
+// when their inputs exist and before their outputs are read: for the block of
+// step r and side U, with H = U/2,
+//   sources [r-U, r-H) -> targets [r, r+U)     run at steps r-H+1, r-H+3, ... < r,
+//   sources [r-H, r)   -> targets [r+H, r+U)   run at steps r+1, r+3, ...  < r+H,
+//   sources [r-H, r)   -> targets [r, r+H)     the same cut again, down to 8 x 8 at step r.
+// Every (source, target) pair of the chunk is still summed exactly once (the
+// host builds the table; tests/test_abi.py checks it). A launch that covers only
+// part of a chunk (a call boundary inside it) keeps the page's tiling unchanged,
+// so the state between calls is the same whichever call sequence produced it.
+//
+// Shared-memory window: position-major per layer, win[l][r][gg] (gg = stream in
+// the CTA), so the chain (one stream per lane) and the tile warps (one stream
+// per lane, sliding over positions) both touch 32 consecutive floats per warp
+// access, and the prologue and write-back move 16 contiguous bytes of a stream
+// per lane.
+#include <algorithm>
 #include <mutex>
+#include <vector>
 
 #include "fi_internal.cuh"
 
@@ -26,100 +44,169 @@ namespace fi {
 constexpr int kChunkMaxThreads = 512;
 constexpr int kChunkMaxStreams = 128;
 constexpr int kSuspendHintNs = 1000;   // longest a suspended barrier check may last
+constexpr int kLayersPerGroupMax = 12;  // layers whose accumulators the chain holds in registers at once
 
 struct ChunkShape {
-  int G, GdMax, CH, CHP, TPS, CW, NG, K;
-  size_t win, tp, h0, ep, ys, flags, total;  // float offsets / total floats
+  int G, GP, CH, LS, TPS, CW, GdMax, NG, K;
+  size_t win, tp, ep, flags, total;  // float offsets / total floats
 };
 
 __host__ __device__ inline ChunkShape chunk_shape(const Dims& g, int CH, int G) {
   ChunkShape c;
   c.G = G;
+  c.GP = G | 1;                    // odd: the prologue's transposing stores spread over banks
   c.CH = CH;
-  c.CHP = CH + 1;                  // odd strides: rows of different streams / channels fall in different banks
-  c.TPS = CH + 1;
+  c.LS = (CH + 1) * c.GP;          // floats per layer (one spare position for the next chunk's token)
+  c.TPS = CH + 1;                  // odd tap stride: lanes of different channels hit different banks
   c.CW = (G + 31) / 32;            // chain warps (one stream per lane)
   c.GdMax = (G - 1) / g.B + 2;     // channels a run of G consecutive streams can touch
+  c.NG = (g.M + kLayersPerGroupMax - 1) / kLayersPerGroupMax;   // layer groups per position
+  if (c.NG < 2 && g.M >= 2) c.NG = 2;
+  c.K = (g.M + c.NG - 1) / c.NG;   // layers per group
+  c.NG = (g.M + c.K - 1) / c.K;
   c.win = 0;
-  c.tp = c.win + (size_t)(g.M + 1) * G * c.CHP;
-  c.h0 = c.tp + (size_t)g.M * c.GdMax * c.TPS;
-  c.ep = c.h0 + (size_t)g.M * c.GdMax;
-  c.ys = c.ep + (size_t)CH * G;
-  c.flags = (c.ys + (size_t)CH * G + 1) & ~(size_t)1;   // 8-byte aligned mbarriers
-  c.NG = g.M >= 2 ? 2 : 1;                              // layer groups per position
-  c.K = (g.M + c.NG - 1) / c.NG;                        // layers per group
+  c.tp = c.win + (size_t)(g.M + 1) * c.LS;
+  c.ep = c.tp + (size_t)g.M * c.GdMax * c.TPS;
+  c.flags = (c.ep + (size_t)CH * G + 1) & ~(size_t)1;   // 8-byte aligned mbarriers
   c.total = c.flags + 2 * (size_t)(2 * c.NG) * c.CW;    // act_ready[NG][CW] + tile_done[NG][CW]
   return c;
 }
 
 __device__ __forceinline__ int highbit_dev(int t) { return 1 << (31 - __clz(t)); }
 
-// 4-byte asynchronous global -> shared copy; `valid` false writes 0 instead.
-__device__ __forceinline__ void cp_async4(float* dst, const float* src, bool valid) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
-               "l"(src), "r"(valid ? 4 : 0)
+// 4-byte asynchronous global -> shared copy.
+__device__ __forceinline__ void cp_async4(float* dst, const float* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+               "l"(src)
                : "memory");
 }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
-// Gray block of side U for one (layer, stream) row: dst[r+u'] += sum_u h[U+u'-u] src[r-U+u].
-// Outputs go in groups of OB; for a group the taps h[U+u'-u] form a window that
-// slides by one per source u, so each step loads one source and one new tap and
-// issues OB FMAs from registers.
-template <int U>
-__device__ __forceinline__ void small_block(const float* __restrict__ src, float* __restrict__ dst,
-                                            const float* __restrict__ taps, int r) {
-  constexpr int OB = U < 16 ? U : 16;
-  const float* x = src + r - U;
+// ---------------------------------------------------------------------------
+// Step table: which on-chip block pieces run at which step (host-built).
+// ---------------------------------------------------------------------------
+enum PieceKind { PK_SQ1 = 0, PK_SQ2, PK_SQ4, PK_SQ8, PK_SQ16, PK_SQ32, PK_R8x4, PK_R16x4, PK_COUNT };
+__host__ __device__ constexpr int piece_ns(int k) {
+  return k == PK_R8x4 ? 8 : k == PK_R16x4 ? 16 : 1 << k;
+}
+__host__ __device__ constexpr int piece_nd(int k) { return k >= PK_R8x4 ? 4 : 1 << k; }
+__host__ __device__ inline uint32_t piece_encode(int step, int s_lo, int t_lo, int kind) {
+  return (uint32_t)step | ((uint32_t)s_lo << 7) | ((uint32_t)t_lo << 14) | ((uint32_t)kind << 21);
+}
+
+// Block piece: dst[t] += sum_{s in [s_lo, s_lo+NS)} h[t-s] src[s] for t in
+// [t_lo, t_lo+ND), positions `stride` floats apart. Outputs go in groups of OB;
+// within a group the taps h[t-s] form a window that slides by one per source, so
+// each source costs one source load, one tap load and OB FMAs from registers.
+template <int NS, int ND>
+__device__ __forceinline__ void block_piece(const float* __restrict__ src, float* __restrict__ dst,
+                                            const float* __restrict__ taps, int s_lo, int t_lo, int stride) {
+  constexpr int OB = ND < 8 ? ND : 8;
+  const float* x = src + s_lo * stride;
 #pragma unroll
-  for (int up0 = 0; up0 < U; up0 += OB) {
+  for (int o0 = 0; o0 < ND; o0 += OB) {
+    const int lag0 = t_lo + o0 - s_lo;     // lag of output o0 + k for source 0 is lag0 + k
     float acc[OB], w[OB];
 #pragma unroll
     for (int k = 0; k < OB; ++k) {
       acc[k] = 0.f;
-      w[k] = taps[U + up0 + k];          // tap of output up0+k for source u = 0
+      w[k] = taps[lag0 + k];
     }
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const float xv = x[u];
+    for (int u = 0; u < NS; ++u) {
+      const float xv = x[u * stride];
 #pragma unroll
       for (int k = 0; k < OB; ++k) acc[k] = fmaf(w[k], xv, acc[k]);
-      if (u + 1 < U) {
+      if (u + 1 < NS) {
 #pragma unroll
         for (int k = OB - 1; k > 0; --k) w[k] = w[k - 1];
-        w[0] = taps[U + up0 - u - 1];
+        w[0] = taps[lag0 - u - 1];
       }
     }
+    float* out = dst + (t_lo + o0) * stride;
 #pragma unroll
-    for (int k = 0; k < OB; ++k) dst[r + up0 + k] += acc[k];
+    for (int k = 0; k < OB; ++k) out[k * stride] += acc[k];
   }
 }
 
-__device__ __forceinline__ void gray_block(int U, const float* src, float* dst, const float* taps, int r) {
-  switch (U) {
-    case 1: small_block<1>(src, dst, taps, r); break;
-    case 2: small_block<2>(src, dst, taps, r); break;
-    case 4: small_block<4>(src, dst, taps, r); break;
-    case 8: small_block<8>(src, dst, taps, r); break;
-    case 16: small_block<16>(src, dst, taps, r); break;
-    default: small_block<32>(src, dst, taps, r); break;
+__device__ __forceinline__ void run_piece(uint32_t e, const float* src, float* dst, const float* taps, int stride) {
+  const int s_lo = (e >> 7) & 127, t_lo = (e >> 14) & 127;
+  switch ((e >> 21) & 15) {
+    case PK_SQ1: block_piece<1, 1>(src, dst, taps, s_lo, t_lo, stride); break;
+    case PK_SQ2: block_piece<2, 2>(src, dst, taps, s_lo, t_lo, stride); break;
+    case PK_SQ4: block_piece<4, 4>(src, dst, taps, s_lo, t_lo, stride); break;
+    case PK_SQ8: block_piece<8, 8>(src, dst, taps, s_lo, t_lo, stride); break;
+    case PK_SQ16: block_piece<16, 16>(src, dst, taps, s_lo, t_lo, stride); break;
+    case PK_SQ32: block_piece<32, 32>(src, dst, taps, s_lo, t_lo, stride); break;
+    case PK_R8x4: block_piece<8, 4>(src, dst, taps, s_lo, t_lo, stride); break;
+    default: block_piece<16, 4>(src, dst, taps, s_lo, t_lo, stride); break;
   }
 }
 
+namespace {
+
+int kind_of_square(int U) { return U == 1 ? PK_SQ1 : U == 2 ? PK_SQ2 : U == 4 ? PK_SQ4 : U == 8 ? PK_SQ8 : U == 16 ? PK_SQ16 : PK_SQ32; }
+
+struct Piece { int step, s_lo, t_lo, kind; };
+
+// The block of step r and side U, cut so that at most an 8 x 8 square runs at
+// step r itself (see the file comment).
+void cut_block(int r, int U, std::vector<Piece>& out) {
+  if (U <= 8) {
+    out.push_back({r, r - U, r, kind_of_square(U)});
+    return;
+  }
+  const int H = U / 2;
+  const int kind = H == 8 ? PK_R8x4 : PK_R16x4;
+  for (int j = 0; j < U / 4; ++j) out.push_back({r - H + 1 + 2 * j, r - U, r + 4 * j, kind});
+  for (int j = 0; j < H / 4; ++j) out.push_back({r + 1 + 2 * j, r - H, r + H + 4 * j, kind});
+  cut_block(r, H, out);
+}
+
+}  // namespace
+
+int chunk_piece_sources(int kind) { return piece_ns(kind); }
+int chunk_piece_targets(int kind) { return piece_nd(kind); }
+
+bool build_chunk_table(int CH, bool retimed, ChunkTable* tab) {
+  std::vector<Piece> p;
+  for (int r = 1; r < CH; ++r) {
+    const int U = r & -r;
+    if (retimed && U >= 16 && U <= 32) cut_block(r, U, p);
+    else p.push_back({r, r - U, r, kind_of_square(U)});
+  }
+  if ((int)p.size() > kChunkMaxEntries) return false;
+  std::stable_sort(p.begin(), p.end(), [](const Piece& a, const Piece& b) { return a.step < b.step; });
+  tab->n = (int)p.size();
+  int k = 0;
+  for (int r = 0; r <= kChunkMaxSteps; ++r) {
+    while (k < tab->n && p[k].step < r) ++k;
+    tab->first[r] = (uint16_t)k;
+  }
+  for (int j = 0; j < tab->n; ++j) tab->e[j] = piece_encode(p[j].step, p[j].s_lo, p[j].t_lo, p[j].kind);
+  return true;
+}
+
+// ---------------------------------------------------------------------------
 // tanh for the block and the sampler, without branches (every lane of the chain
 // warp takes the same path).
 // fp32 activations: two forms evaluated side by side and selected by |y|.
-//  * |y| >= 0.55: tanh|y| = 1 - 2 / (1 + e^(2|y|)) with the hardware exp2 and
-//    reciprocal, e^(2|y|) = 2^(2 |y| log2 e) (overflow to +inf gives exactly 1),
-//    sign restored after. 2/(1+e) <= 0.5 here, so the subtraction loses nothing.
+//  * |y| >= 0.55: tanh y = 1 - 2 rc, rc = 1 / (1 + e^(2y)), with the hardware
+//    exp2 and reciprocal, e^(2y) = 2^(2y log2 e). For y >= 0.55, 2 rc <= 0.5 and
+//    the subtraction loses nothing; for y <= -0.55, |tanh y| >= 0.5 and the
+//    rounding of 2 rc is at most an ulp of 2. Overflow of e^(2y) to +inf gives
+//    rc = 0 (tanh = 1), underflow to 0 gives rc = 1 (tanh = -1).
 //  * |y| < 0.55: y * P(y^2), P a degree-5 polynomial fitted to tanh(y)/y by
 //    weighted least squares on that interval (fit error 1e-9).
 // Relative error within about 5e-7 for every y (1e-7 in the polynomial range).
-// The polynomial runs in parallel with the exp2/reciprocal chain, so the
-// critical path of a layer stays FMA, multiply, exp2, add, reciprocal, FMA,
-// sign, select.
+// The chain never forms tanh(y) on its critical path: the next layer's input
+// y' = h0' tanh(y) + acc' is taken straight from the parts, as
+// y' = (h0' + acc') - 2 h0' rc, or h0' (y P) + acc', so each layer costs the
+// exp2 / add / reciprocal / FMA / select chain (the polynomial runs beside it);
+// the argument of the next exp2 (2 log2 e y') comes out of the same FMAs.
 // bf16 activations: the hardware tanh approximation (relative error about 1e-5,
 // far below bfloat16's 2^-9), since the result is rounded to bf16 right after.
+// ---------------------------------------------------------------------------
 constexpr float kTwoLog2e = 2.88539008177792681f;
 
 __device__ __forceinline__ float ex2_approx(float x) {
@@ -137,27 +224,43 @@ __device__ __forceinline__ float tanh_approx(float x) {
   asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
-template <bool BF16>
-__device__ __forceinline__ float round_to(float v) {
-  if constexpr (BF16) return __bfloat162float(__float2bfloat16_rn(v));
-  else return v;
-}
+__device__ __forceinline__ float round_bf16(float v) { return __bfloat162float(__float2bfloat16_rn(v)); }
+
 constexpr float kTanhPolyMax = 0.55f;
 constexpr float kTanhP0 = 1.0f, kTanhP1 = -0.3333331048488617f, kTanhP2 = 0.1333247870206833f,
                 kTanhP3 = -0.05384441092610359f, kTanhP4 = 0.021046100184321404f,
                 kTanhP5 = -0.0062440442852675915f;
-template <bool BF16>
-__device__ __forceinline__ float block_tanh(float y) {
-  if constexpr (BF16) return tanh_approx(y);
-  const float ay = fabsf(y);
-  const float big = copysignf(fmaf(-2.0f, rcp_approx(1.0f + ex2_approx(ay * kTwoLog2e)), 1.0f), y);
+
+// tanh(y) in parts, from y and z = 2 log2(e) y.
+struct TanhParts {
+  float rc;    // 1 / (1 + e^(2y))
+  float tp;    // y P(y^2)
+  bool small;  // |y| < kTanhPolyMax: tanh y = tp, else 1 - 2 rc
+};
+__device__ __forceinline__ TanhParts tanh_parts(float y, float z) {
+  TanhParts p;
+  p.rc = rcp_approx(1.0f + ex2_approx(z));
   const float q = y * y;
-  float p = fmaf(kTanhP5, q, kTanhP4);
-  p = fmaf(p, q, kTanhP3);
-  p = fmaf(p, q, kTanhP2);
-  p = fmaf(p, q, kTanhP1);
-  p = fmaf(p, q, kTanhP0);
-  return ay < kTanhPolyMax ? y * p : big;
+  float pp = fmaf(kTanhP5, q, kTanhP4);
+  pp = fmaf(pp, q, kTanhP3);
+  pp = fmaf(pp, q, kTanhP2);
+  pp = fmaf(pp, q, kTanhP1);
+  pp = fmaf(pp, q, kTanhP0);
+  p.tp = y * pp;
+  p.small = fabsf(y) < kTanhPolyMax;
+  return p;
+}
+__device__ __forceinline__ float tanh_value(const TanhParts& p) { return p.small ? p.tp : fmaf(-2.0f, p.rc, 1.0f); }
+// y' = h0 tanh(y) + acc and z' = 2 log2(e) y', from the parts of tanh(y).
+__device__ __forceinline__ void next_input(const TanhParts& p, float h0, float acc, float& y, float& z) {
+  const float c1 = h0 + acc;
+  const float m2 = -2.0f * h0;
+  const float yb = fmaf(m2, p.rc, c1);
+  const float zb = fmaf(kTwoLog2e * m2, p.rc, kTwoLog2e * c1);
+  const float yp = fmaf(h0, p.tp, acc);
+  const float zp = fmaf(kTwoLog2e * h0, p.tp, kTwoLog2e * acc);
+  y = p.small ? yp : yb;
+  z = p.small ? zp : zb;
 }
 
 // Hardware barriers in shared memory (mbarrier): arrive has release semantics
@@ -200,10 +303,10 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, int parity, int* err, b
 // Warp roles. Chain warps (one stream per lane) run the red cells, blocks and
 // sampler position after position. The layers form NG groups of K; after group k
 // of position r every lane of chain warp c arrives on act_ready[k][c]. Tile warps
-// own row groups (layer l, chain warp c): the gray block of step r for layer l
-// needs a^{l-1} below r and must not run before the chain has consumed the
-// accumulator of (r-1, l), so it waits for act_ready[group(l)] of position r-1,
-// computes, and arrives on tile_done[group(l)][c] (which completes when every
+// own row groups (layer l, chain warp c): the pieces of step r for layer l need
+// a^{l-1} below r and must not run before the chain has consumed the
+// accumulator of (r-1, l), so they wait for act_ready[group(l)] of position r-1,
+// compute, and arrive on tile_done[group(l)][c] (which completes when every
 // layer of the group has arrived); the chain waits on tile_done before reading a
 // group's accumulators. Each barrier thus advances at most one phase ahead of
 // its waiters, parity waits are exact, and every wait is bounded.
@@ -211,12 +314,10 @@ template <bool BF16, bool REC>
 __global__ void __launch_bounds__(kChunkMaxThreads) k_chunk(Dims g, ChunkArgs a, int G) {
   extern __shared__ float csm[];
   const ChunkShape cs = chunk_shape(g, a.chunk, G);
-  const int CH = cs.CH, CHP = cs.CHP, TPS = cs.TPS, GdMax = cs.GdMax, CW = cs.CW;
-  float* win = csm + cs.win;   // [(M+1)][G][CHP]   slot window of positions [c, c+CH)
-  float* tp = csm + cs.tp;     // [M][GdMax][TPS]   taps h[0..CH)
-  float* h0s = csm + cs.h0;    // [M][GdMax]        h[0]
-  float* ep = csm + cs.ep;     // [CH][G]           sampler noise
-  float* ys = csm + cs.ys;     // [CH][G]           y^M of each position, written out at the end
+  const int CH = cs.CH, GP = cs.GP, LS = cs.LS, TPS = cs.TPS, GdMax = cs.GdMax, CW = cs.CW;
+  float* win = csm + cs.win;   // [(M+1)][CH+1][GP]   slot window of positions [c, c+CH]
+  float* tp = csm + cs.tp;     // [M][GdMax][TPS]     taps h[0..CH)
+  float* ep = csm + cs.ep;     // [CH][G]             sampler noise
   uint64_t* act_ready = reinterpret_cast<uint64_t*>(csm + cs.flags);   // [NG][CW]
   uint64_t* tile_done = act_ready + cs.NG * CW;                          // [NG][CW]
   const int K = cs.K, NG = cs.NG;
@@ -228,57 +329,98 @@ __global__ void __launch_bounds__(kChunkMaxThreads) k_chunk(Dims g, ChunkArgs a,
   const int tid = threadIdx.x, nt = blockDim.x;
   const int r0 = a.p0 - a.c, r1 = a.p1 - a.c;
 
-  // Prologue: every load is an asynchronous 4-byte copy into shared memory
-  // (zero-filled where the slot holds nothing yet), so the loads of a thread
-  // overlap instead of waiting one by one on HBM latency. Rows are spread over
-  // warps and positions over lanes, so index arithmetic is per row.
-  const int wid = tid >> 5, lid = tid & 31, nw = nt >> 5;
-  for (int row = wid; row < M * Gd; row += nw) {
-    const int l = row / Gd, dl = row - l * Gd;
-    const float* src = a.taps + ((size_t)l * g.D + d_lo + dl) * g.L;
-    float* dst = tp + (l * GdMax + dl) * TPS;
-    for (int j = lid; j < CH; j += 32) cp_async4(dst + j, src + j, true);
-  }
+  // ---------------------------------------------------------------- prologue
   // Slots already in HBM: tokens and activations below p0; the token at p0 when
   // no x0 is given; accumulators that some block has reached (the first block to
   // reach position t runs at step highbit(t)). Everything else starts at 0.
-  for (int row = wid; row < (M + 1) * Gc; row += nw) {
-    const int l = row / Gc, gg = row - l * Gc;
-    const float* src = a.state + slot_index(g, l, s0 + gg, 0);
-    float* dst = win + (l * G + gg) * CHP;
-    for (int r = lid; r < CH; r += 32) {
+  // Each lane moves 16 contiguous bytes (4 positions of one stream) and spreads
+  // them over the position-major window; loads are issued in batches of 8 so a
+  // thread has several in flight.
+  auto slot_valid = [&](int l, int t) {
+    if (t < a.p0) return true;
+    if (l == 0) return t == a.p0 && a.x0 == nullptr;
+    return t >= 1 && highbit_dev(t) <= a.last_done;
+  };
+  if (CH < 4) {
+    for (int idx = tid; idx < (M + 1) * Gc * CH; idx += nt) {
+      const int row = idx / CH, r = idx - row * CH;
+      const int l = row / Gc, gg = row - l * Gc;
       const int t = a.c + r;
-      bool valid = false;
-      if (t < g.L) {
-        valid = t < a.p0;
-        if (l == 0) valid = valid || (t == a.p0 && a.x0 == nullptr);
-        else valid = valid || (t >= 1 && highbit_dev(t) <= a.last_done);
+      win[l * LS + r * GP + gg] = slot_valid(l, t) ? a.state[slot_index(g, l, s0 + gg, t)] : 0.f;
+    }
+    for (int idx = tid; idx < M * Gd * CH; idx += nt) {
+      const int row = idx / CH, j = idx - row * CH;
+      const int l = row / Gd, dl = row - l * Gd;
+      tp[(l * GdMax + dl) * TPS + j] = a.taps[((size_t)l * g.D + d_lo + dl) * g.L + j];
+    }
+  } else {
+    const int vpr = CH >> 2;                          // float4 per (layer, stream) row
+    const int nwin = (M + 1) * Gc * vpr;
+    const int ntap = M * Gd * vpr;
+    constexpr int kBatch = 8;
+    for (int base = tid; base < nwin + ntap; base += nt * kBatch) {
+      float4 v[kBatch];
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int idx = base + u * nt;
+        v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (idx < nwin) {
+          const int row = idx / vpr, j = idx - row * vpr;
+          const int l = row / Gc, gg = row - l * Gc;
+          const int t = a.c + 4 * j;
+          if (slot_valid(l, t) || slot_valid(l, t + 1) || slot_valid(l, t + 2) || slot_valid(l, t + 3))
+            v[u] = __ldg(reinterpret_cast<const float4*>(a.state + slot_index(g, l, s0 + gg, t)));
+        } else if (idx < nwin + ntap) {
+          const int k = idx - nwin;
+          const int row = k / vpr, j = k - row * vpr;
+          const int l = row / Gd, dl = row - l * Gd;
+          v[u] = __ldg(reinterpret_cast<const float4*>(a.taps + ((size_t)l * g.D + d_lo + dl) * g.L + 4 * j));
+        }
       }
-      cp_async4(dst + r, src + (valid ? t : 0), valid);
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int idx = base + u * nt;
+        if (idx < nwin) {
+          const int row = idx / vpr, j = idx - row * vpr;
+          const int l = row / Gc, gg = row - l * Gc;
+          const int t = a.c + 4 * j;
+          float* w = win + l * LS + 4 * j * GP + gg;
+          w[0] = slot_valid(l, t) ? v[u].x : 0.f;
+          w[GP] = slot_valid(l, t + 1) ? v[u].y : 0.f;
+          w[2 * GP] = slot_valid(l, t + 2) ? v[u].z : 0.f;
+          w[3 * GP] = slot_valid(l, t + 3) ? v[u].w : 0.f;
+        } else if (idx < nwin + ntap) {
+          const int k = idx - nwin;
+          const int row = k / vpr, j = k - row * vpr;
+          float* w = tp + row / Gd * GdMax * TPS + (row % Gd) * TPS + 4 * j;
+          w[0] = v[u].x;
+          w[1] = v[u].y;
+          w[2] = v[u].z;
+          w[3] = v[u].w;
+        }
+      }
     }
   }
-  for (int r = r0 + wid; r < r1; r += nw) {
-    const float* src = a.eps + (size_t)(a.c + r - a.gen_base) * g.S;
-    for (int gg = lid; gg < Gc; gg += 32) {
-      const int s = s0 + gg, d = s / g.B, b = s - d * g.B;
-      cp_async4(ep + r * G + gg, src + (size_t)b * g.D + d, true);
+  {
+    const int wid = tid >> 5, lid = tid & 31, nw = nt >> 5;
+    for (int r = r0 + wid; r < r1; r += nw) {
+      const float* src = a.eps + (size_t)(a.c + r - a.gen_base) * g.S;
+      for (int gg = lid; gg < Gc; gg += 32) {
+        const int s = s0 + gg, d = s / g.B, b = s - d * g.B;
+        cp_async4(ep + r * G + gg, src + (size_t)b * g.D + d);
+      }
     }
-  }
-  cp_async_wait_all();
-  __syncthreads();
-  for (int k = tid; k < M * Gd; k += nt) {
-    const int dl = k % Gd, l = k / Gd;
-    h0s[l * GdMax + dl] = tp[(l * GdMax + dl) * TPS];
   }
   if (a.x0 != nullptr && tid < Gc) {
     const int s = s0 + tid, d = s / g.B, b = s - d * g.B;
-    win[tid * CHP + r0] = round_act(load_token(a.x0, (size_t)b * g.D + d, g.bf16), g.bf16);
+    win[r0 * GP + tid] = round_act(load_token(a.x0, (size_t)b * g.D + d, g.bf16), g.bf16);
   }
   for (int k = tid; k < NG * CW; k += nt) {
     const int grp = k / CW;
     mbar_init(act_ready + k, 32);
     mbar_init(tile_done + k, 32 * (min(M, (grp + 1) * K) - grp * K));   // one arrival per lane per layer
   }
+  cp_async_wait_all();
   __syncthreads();
 
   const int warp = tid >> 5, lane = tid & 31;
@@ -293,68 +435,133 @@ __global__ void __launch_bounds__(kChunkMaxThreads) k_chunk(Dims g, ChunkArgs a,
     const bool act = gg0 < Gc;
     const int gg = act ? gg0 : 0;
     const int s = s0 + gg, d = s / g.B, b = s - d * g.B;
-    const int c_dl = d - d_lo;
     const size_t c_io = (size_t)b * g.D + d;
-    const int lstride = G * CHP;                 // window floats per layer
-    float* wrow = win + gg * CHP;                // this stream's row of layer 0
-    const float* hrow = h0s + c_dl;              // h0 of layer l at (l-1)*GdMax
-    float av = wrow[r0];                         // the token of the current position
-    // Barrier tests run one group ahead (non-blocking), so their latency hides
-    // behind the previous group's layers; a test that comes back false is
-    // followed by a bounded wait.
-    bool ready = r0 == 0;                        // group 0 of position r0 needs no wait when r0 == 0
-    if (!ready) ready = mbar_test(&tile_done[warp], 0);
+    float* wcol = win + gg;                                  // slot (l, r) at wcol[l*LS + r*GP]
+    const float* hcol = tp + (d - d_lo) * TPS;               // h0 of layer l at hcol[(l-1)*GdMax*TPS]
+    const size_t y_stride = g.S;
+    // Accumulators and h0 of one layer group, in registers (loaded together once
+    // the group's blocks are done, so their latency is paid once per group).
+    float accA[kLayersPerGroupMax], h0A[kLayersPerGroupMax];
+    float accB[kLayersPerGroupMax], h0B[kLayersPerGroupMax];
+    auto load_group = [&](int grp, int r, float* acc, float* h0) {
+      const int lg0 = grp * K + 1;
+#pragma unroll
+      for (int k = 0; k < kLayersPerGroupMax; ++k) {
+        if (k < K && lg0 + k <= M) {
+          acc[k] = wcol[(lg0 + k) * LS + r * GP];
+          h0[k] = hcol[(lg0 + k - 1) * GdMax * TPS];
+        }
+      }
+    };
+    auto wait_group = [&](int grp, int r) {
+      if (r >= rs && ok) ok = mbar_wait(&tile_done[grp * CW + warp], (r - rs) & 1, err, true, a.wait_limit);
+    };
+    auto test_group = [&](int grp, int r) {
+      return r < rs || mbar_test(&tile_done[grp * CW + warp], (r - rs) & 1);
+    };
+
+    // Group 0 of the first position.
+    wait_group(0, r0);
+    load_group(0, r0, accA, h0A);
+    const float x_first = wcol[r0 * GP];
+    // The input of layer 1 as tanh parts (or the token itself at the first position).
+    TanhParts P{0.f, x_first, true};
+    float xb = x_first;          // bf16 path: the token
+    float epsk = 0.f;            // eps_scale * eps of the previous position (fp32 path)
+    bool loadedB = false;
     for (int r = r0; r < r1; ++r) {
       const int t = a.c + r;
-      const float epsv = ep[r * G + gg];
-      float y = 0.f;
-      for (int grp = 0; grp < NG; ++grp) {
-        const int lg0 = grp * K + 1, lg1 = min(M, (grp + 1) * K);
-        if (!ready && ok) ok = mbar_wait(&tile_done[grp * CW + warp], (r - rs) & 1, err, true, a.wait_limit);
-        const int lend = lg1 < M ? lg1 : M - 1;    // layers with a block (tanh) in this group
-        float acc = wrow[lg0 * lstride + r];
-        float h0 = hrow[(lg0 - 1) * GdMax];
-        auto layer = [&](int l) {
-          const int ln = l < lg1 ? l + 1 : l;      // prefetch the next layer of the group
-          const float acc_n = wrow[ln * lstride + r];
-          const float h0_n = hrow[(ln - 1) * GdMax];
-          y = fmaf(h0, av, acc);
-          if constexpr (REC) if (act) a.rec[((size_t)(l - 1) * a.n_gen + (t - a.gen_base)) * g.S + c_io] = y;
-          av = round_to<BF16>(block_tanh<BF16>(y));
-          if (act) wrow[l * lstride + r] = av;
-          acc = acc_n;
-          h0 = h0_n;
-        };
-        // Halfway through the group, test the next group's barrier (the next
-        // position's group 0 after the last group); by then its blocks are
-        // usually done, and the test's latency hides behind the second half.
-        const int lmid = lg0 + (lend - lg0 + 1) / 2;
-        for (int l = lg0; l < lmid; ++l) layer(l);
-        {
-          const int ng = grp + 1 < NG ? grp + 1 : 0;
-          const int nr = grp + 1 < NG ? r : r + 1;
-          ready = (nr == 0 || nr >= r1) ? true : mbar_test(&tile_done[ng * CW + warp], (nr - rs) & 1);
-        }
-        for (int l = lmid; l <= lend; ++l) layer(l);
-        if (lg1 == M) {                            // last layer: red cell only
-          y = fmaf(h0, av, acc);
-          if constexpr (REC) if (act) a.rec[((size_t)(M - 1) * a.n_gen + (t - a.gen_base)) * g.S + c_io] = y;
-        }
-        mbar_arrive(&act_ready[grp * CW + warp]);
+      float y, z = 0.f;
+      if constexpr (BF16) {
+        y = fmaf(h0A[0], xb, accA[0]);
+      } else {
+        next_input(P, h0A[0], fmaf(h0A[0], epsk, accA[0]), y, z);
       }
-      if (act) ys[r * G + gg] = y;
-      // x_{t+1}; for the last position of the chunk it lands in the row's spare
-      // column (index CH) and goes to HBM with the write-back.
-      av = round_to<BF16>(block_tanh<BF16>(y) + a.eps_scale * epsv);
-      if (act && t + 1 < g.L) wrow[r + 1] = av;
+      for (int grp = 0; grp < NG; ++grp) {
+        const int lg0 = grp * K + 1;
+        const int nk = min(M, lg0 + K - 1) - lg0 + 1;
+        const int kmid = nk / 2;
+        const bool last_grp = grp + 1 == NG;
+        // the barrier tested halfway through this group: the next group, or
+        // group 0 of the next position after the last group
+        const int ngrp = last_grp ? 0 : grp + 1;
+        const int nr = last_grp ? r + 1 : r;
+#pragma unroll
+        for (int k = 0; k < kLayersPerGroupMax; ++k) {
+          if (k < nk) {
+            const int l = lg0 + k;
+            if constexpr (REC) if (act) a.rec[((size_t)(l - 1) * a.n_gen + (t - a.gen_base)) * y_stride + c_io] = y;
+            if (k == kmid && !loadedB && nr < r1 && test_group(ngrp, nr)) {
+              load_group(ngrp, nr, accB, h0B);
+              loadedB = true;
+            }
+            if (l == M) break;
+            float av;
+            if constexpr (BF16) {
+              av = round_bf16(tanh_approx(y));
+            } else {
+              P = tanh_parts(y, z);
+              av = tanh_value(P);
+            }
+            if (act) wcol[l * LS + r * GP] = av;
+            if (k + 1 < nk) {
+              if constexpr (BF16) y = fmaf(h0A[k + 1], av, accA[k + 1]);
+              else next_input(P, h0A[k + 1], accA[k + 1], y, z);
+            } else {
+              // last layer of a group below M: hand the group to the tile
+              // warps, then continue into the next group
+              mbar_arrive(&act_ready[grp * CW + warp]);
+              if (!loadedB) {
+                wait_group(grp + 1, r);
+                load_group(grp + 1, r, accB, h0B);
+              }
+#pragma unroll
+              for (int q = 0; q < kLayersPerGroupMax; ++q) {
+                accA[q] = accB[q];
+                h0A[q] = h0B[q];
+              }
+              loadedB = false;
+              if constexpr (BF16) y = fmaf(h0A[0], av, accA[0]);
+              else next_input(P, h0A[0], accA[0], y, z);
+            }
+          }
+        }
+      }
+      // y = y^M_t: output, then the sampler x_{t+1} = R(tanh(y) + eps_scale eps_t)
+      mbar_arrive(&act_ready[(NG - 1) * CW + warp]);
+      if (act) a.y_out[(size_t)(t - a.gen_base) * y_stride + c_io] = y;
+      const float epsv = ep[r * G + gg];
+      float xn;
+      if constexpr (BF16) {
+        xn = round_bf16(tanh_approx(y) + a.eps_scale * epsv);
+        xb = xn;
+      } else {
+        P = tanh_parts(y, z);
+        epsk = a.eps_scale * epsv;
+        xn = tanh_value(P) + epsk;
+      }
+      // x_{t+1}; for the last position of the chunk it lands in the spare
+      // position CH and goes to HBM with the write-back.
+      if (act && t + 1 < g.L) wcol[(r + 1) * GP] = xn;
+      if (r + 1 < r1) {
+        if (!loadedB) {
+          wait_group(0, r + 1);
+          load_group(0, r + 1, accB, h0B);
+        }
+#pragma unroll
+        for (int q = 0; q < kLayersPerGroupMax; ++q) {
+          accA[q] = accB[q];
+          h0A[q] = h0B[q];
+        }
+        loadedB = false;
+      }
     }
   } else {
     // ---------------------------------------------------------------- tile warps
     // With a single chain warp, tile work stays off the scheduler that issues
     // for it (warp w issues on scheduler w % 4), so the latency-bound chain
-    // shares its issue slots with no busy warp; that leaves 12 of the 15 other
-    // warps for blocks (measured on the headline shape: 7.6 % fewer cycles per
-    // chunk). With more chain warps every warp takes blocks.
+    // shares its issue slots with no busy warp. With more chain warps every warp
+    // takes pieces.
     const int nwarps = nt / 32;
     const bool spare_sched = CW == 1 && nwarps - CW > 4;
     auto is_tile = [&](int w) { return w >= CW && (!spare_sched || (w & 3) >= CW); };
@@ -365,50 +572,68 @@ __global__ void __launch_bounds__(kChunkMaxThreads) k_chunk(Dims g, ChunkArgs a,
         ++ntw;
       }
     if (is_tile(warp))
-    for (int r = rs; r < r1; ++r) {
-      const int U = r & -r;
-      for (int k = tw; k < M * CW; k += ntw) {
-        const int l = k / CW + 1, c = k - (l - 1) * CW;
-        const int grp = (l - 1) / K;
-        if (r > r0 && ok) ok = mbar_wait(&act_ready[grp * CW + c], (r - 1 - r0) & 1, err, false, a.wait_limit);
-        const int gg = c * 32 + lane;
-        if (gg < Gc) {
-          const int dl = (s0 + gg) / g.B - d_lo;
-          gray_block(U, win + ((l - 1) * G + gg) * CHP, win + (l * G + gg) * CHP, tp + ((l - 1) * GdMax + dl) * TPS, r);
+      for (int r = rs; r < r1; ++r) {
+        const int e0 = a.tab.first[r], e1 = a.tab.first[r + 1];
+        for (int k = tw; k < M * CW; k += ntw) {
+          const int l = k / CW + 1, c = k - (l - 1) * CW;
+          const int grp = (l - 1) / K;
+          if (r > r0 && ok) ok = mbar_wait(&act_ready[grp * CW + c], (r - 1 - r0) & 1, err, false, a.wait_limit);
+          const int gg = c * 32 + lane;
+          if (gg < Gc) {
+            const int dl = (s0 + gg) / g.B - d_lo;
+            const float* src = win + (l - 1) * LS + gg;
+            float* dst = win + l * LS + gg;
+            const float* taps = tp + ((l - 1) * GdMax + dl) * TPS;
+            for (int e = e0; e < e1; ++e) run_piece(a.tab.e[e], src, dst, taps, GP);
+          }
+          mbar_arrive(&tile_done[grp * CW + c]);
         }
-        mbar_arrive(&tile_done[grp * CW + c]);
       }
-    }
   }
   __syncthreads();
 
-  // Outputs of the positions produced, then the next chunk's first token.
-  const int wid2 = tid >> 5, lid2 = tid & 31, nw2 = nt >> 5;
-  for (int r = r0 + wid2; r < r1; r += nw2) {
-    float* dst = a.y_out + (size_t)(a.c + r - a.gen_base) * g.S;
-    for (int gg = lid2; gg < Gc; gg += 32) {
-      const int s = s0 + gg, d = s / g.B, b = s - d * g.B;
-      dst[(size_t)b * g.D + d] = ys[r * G + gg];
-    }
-  }
-  if (r1 == CH && a.c + CH < g.L && tid < Gc) a.state[slot_index(g, 0, s0 + tid, a.c + CH)] = win[tid * CHP + CH];
-  // Write back positions [p0, c+CH) of layers 0..M-1: new tokens and
-  // activations below p1, accumulators (including the small blocks' partial
-  // sums) from p1 on. Layer M's slots below p1 were consumed and nothing reads
-  // them again; its accumulators from p1 on are still needed.
-  for (int row = wid2; row < (M + 1) * Gc; row += nw2) {
-    const int l = row / Gc, gg = row - l * Gc;
-    float* dst = a.state + slot_index(g, l, s0 + gg, a.c);
-    const float* src = win + (l * G + gg) * CHP;
-    const int rb = l == M ? r1 : r0;            // first slot to write
-    const int re = min(CH, g.L - a.c);          // past the last
-    if ((a.c & 3) == 0 && (rb & 3) == 0 && (re & 3) == 0) {
-      for (int q = (rb >> 2) + lid2; q < (re >> 2); q += 32) {
-        const int r = 4 * q;
-        reinterpret_cast<float4*>(dst)[q] = make_float4(src[r], src[r + 1], src[r + 2], src[r + 3]);
+  // ---------------------------------------------------------------- write-back
+  // The next chunk's first token, then positions [p0, c+CH) of layers 0..M-1:
+  // new tokens and activations below p1, accumulators (including the on-chip
+  // blocks' partial sums) from p1 on. Layer M's slots below p1 were consumed and
+  // nothing reads them again; its accumulators from p1 on are still needed.
+  if (r1 == CH && a.c + CH < g.L && tid < Gc) a.state[slot_index(g, 0, s0 + tid, a.c + CH)] = win[CH * GP + tid];
+  const int re = min(CH, g.L - a.c);
+  if (r0 == 0 && (re & 3) == 0) {
+    const int vpr = re >> 2;
+    const int nrow_full = M * Gc;                       // layers 0..M-1 from position 0
+    const int nrow_last = (r1 & 3) == 0 ? Gc : 0;       // layer M from p1, when aligned
+    const int v_last = (re - r1) >> 2;
+    const int n1 = nrow_full * vpr, n2 = nrow_last * v_last;
+    for (int idx = tid; idx < n1 + n2; idx += nt) {
+      int l, gg, j;
+      if (idx < n1) {
+        const int row = idx / vpr;
+        j = idx - row * vpr;
+        l = row / Gc;
+        gg = row - l * Gc;
+      } else {
+        const int k = idx - n1;
+        gg = k / v_last;
+        j = (r1 >> 2) + (k - gg * v_last);
+        l = M;
       }
-    } else {
-      for (int r = rb + lid2; r < re; r += 32) dst[r] = src[r];
+      const float* w = win + l * LS + 4 * j * GP + gg;
+      *reinterpret_cast<float4*>(a.state + slot_index(g, l, s0 + gg, a.c + 4 * j)) =
+          make_float4(w[0], w[GP], w[2 * GP], w[3 * GP]);
+    }
+    if (nrow_last == 0) {
+      for (int idx = tid; idx < Gc * (re - r1); idx += nt) {
+        const int gg = idx / (re - r1), r = r1 + idx % (re - r1);
+        a.state[slot_index(g, M, s0 + gg, a.c + r)] = win[M * LS + r * GP + gg];
+      }
+    }
+  } else {
+    for (int idx = tid; idx < (M + 1) * Gc * CH; idx += nt) {
+      const int row = idx / CH, r = idx - row * CH;
+      const int l = row / Gc, gg = row - l * Gc;
+      const int rb = l == M ? r1 : r0;
+      if (r >= rb && r < re) a.state[slot_index(g, l, s0 + gg, a.c + r)] = win[l * LS + r * GP + gg];
     }
   }
 }
@@ -457,7 +682,13 @@ cudaError_t configure_chunk(size_t smem) {
   return e;
 }
 
-cudaError_t launch_chunk(const Dims& g, const ChunkArgs& a, int G, cudaStream_t st) {
+cudaError_t launch_chunk(const Dims& g, const ChunkArgs& a_in, int G, cudaStream_t st) {
+  if (a_in.chunk < 2 || (a_in.chunk & (a_in.chunk - 1)) || a_in.chunk > kChunkMaxSteps) return cudaErrorInvalidValue;
+  ChunkArgs a = a_in;
+  // A launch over a whole chunk runs the re-timed pieces; one over part of a
+  // chunk keeps the page's blocks, so the state at a call boundary is canonical.
+  const bool whole = a.p0 == a.c && a.p1 == a.c + a.chunk;
+  if (!build_chunk_table(a.chunk, whole, &a.tab)) return cudaErrorInvalidValue;
   const size_t smem = chunk_smem_bytes(g, a.chunk, G);
   const int blocks = (g.S + G - 1) / G;
   const int nt = chunk_threads(g, G);

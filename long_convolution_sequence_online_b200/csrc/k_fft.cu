@@ -252,6 +252,140 @@ k_tile_fft(Dims g, float* __restrict__ state, const float2* __restrict__ spec,
   else tile_fft_body<N, T>(sm, ds, tid, active, src, dst, H, tw, overwrite, SyncBlock());
 }
 
+// ---------------------------------------------------------------------------
+// Paired FFT blocks (even batch): two sequences b, b+1 of one (layer, channel)
+// share the filter, so their sources go into one complex sequence
+// z[m] = x_b[m] + i x_{b+1}[m] (m < U, zero above) of N2 = 2U points. Its DFT is
+// X_b + i X_{b+1}; multiplied by the filter's 2U-point spectrum H (the same
+// spectrum for both, and H[2U-k] = conj H[k] because h is real) it becomes
+// Y_b + i Y_{b+1}, whose inverse carries y_b in the real part and y_{b+1} in the
+// imaginary part. The product is pointwise, so no real-FFT split is needed and
+// the forward transform's last pass, the product and the inverse's first pass
+// run on the same registers: the Stockham last pass leaves thread j holding
+// points j + r N2/R, which is exactly what the inverse's first pass of the same
+// radix reads (the inverse takes its passes in the opposite radix order).
+// ---------------------------------------------------------------------------
+template <int N2, int T>
+__device__ __forceinline__ void tile_fft2_body(float2* sm, float* ds, int tid, bool active,
+                                               const float* __restrict__ src1, const float* __restrict__ src2,
+                                               float* __restrict__ dst1, float* __restrict__ dst2,
+                                               const float2* __restrict__ H, const float2* __restrict__ tw,
+                                               int overwrite) {
+  constexpr int U = N2 / 2;
+  using SF = FftShape<N2, T, false>;
+  using SI = FftShape<N2, T, true>;
+  auto sync = [] {
+    if constexpr (T <= 32) __syncwarp();
+    else __syncthreads();
+  };
+  // accumulators of both sequences travel to shared memory meanwhile
+  if (active && !overwrite) {
+    for (int q = tid; q < U / 4; q += T) {
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(ds + 4 * q))),
+                   "l"(dst1 + 4 * q) : "memory");
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(ds + U + 4 * q))),
+                   "l"(dst2 + 4 * q) : "memory");
+    }
+  }
+  asm volatile("cp.async.commit_group;" ::: "memory");
+  float2 v[SF::P];
+  {
+    // forward pass 0 straight from HBM; points m >= U are the zero padding
+    constexpr int R = 1 << SF::rb(0);
+#pragma unroll
+    for (int k = 0; k < SF::P / R; ++k) {
+      const int j = tid + k * T;
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        const int m = j + r * (N2 / R);
+        v[k * R + r] = (active && r < R / 2) ? make_float2(__ldg(src1 + m), __ldg(src2 + m)) : make_float2(0.f, 0.f);
+      }
+    }
+    pass_compute<N2, T, false, 0, false>(v, tid, tw);
+    if constexpr (!SF::last(0)) {
+      pass_store<N2, T, 0, false>(sm, v, tid);
+      sync();
+      smem_passes<N2, T, false, SF::rb(0), true, false>(sm, tid, tw, sync);
+      constexpr int DL = last_pass_done<N2, T, 0, false>();
+      pass_load<N2, T, DL, false>(sm, v, tid);
+      pass_compute<N2, T, false, DL, false>(v, tid, tw);
+    }
+  }
+  {
+    // spectrum product on the points this thread holds: j + r N2/R
+    constexpr int R = 1 << SF::rb(last_pass_done<N2, T, 0, false>());
+    static_assert(R == (1 << SI::rb(0)), "inverse must start with the forward's last radix");
+#pragma unroll
+    for (int k = 0; k < SF::P / R; ++k) {
+      const int j = tid + k * T;
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        const int kk = j + r * (N2 / R);
+        float2 h = __ldg(H + (kk <= U ? kk : N2 - kk));
+        if (kk > U) h.y = -h.y;
+        v[k * R + r] = cmul(v[k * R + r], h);
+      }
+    }
+  }
+  // inverse, first pass in registers
+  pass_compute<N2, T, true, 0, true>(v, tid, tw);
+  if constexpr (!SI::last(0)) {
+    sync();   // every thread is done reading sm in the forward's last pass
+    pass_store<N2, T, 0, true>(sm, v, tid);
+    sync();
+    smem_passes<N2, T, true, SI::rb(0), true, true>(sm, tid, tw, sync);
+    constexpr int DL = last_pass_done<N2, T, 0, true>();
+    pass_load<N2, T, DL, true>(sm, v, tid);
+    pass_compute<N2, T, true, DL, true>(v, tid, tw);
+  }
+  asm volatile("cp.async.wait_all;" ::: "memory");
+  sync();
+  if (active) {
+    constexpr int R = 1 << SI::rb(last_pass_done<N2, T, 0, true>());
+#pragma unroll
+    for (int k = 0; k < SI::P / R; ++k) {
+      const int j = tid + k * T;
+#pragma unroll
+      for (int r = R / 2; r < R; ++r) {
+        const int m = j + r * (N2 / R) - U;
+        const float2 o = v[k * R + r];
+        if (overwrite) {
+          dst1[m] = o.x;
+          dst2[m] = o.y;
+        } else {
+          dst1[m] = ds[m] + o.x;
+          dst2[m] = ds[U + m] + o.y;
+        }
+      }
+    }
+  }
+}
+
+// item = pair ((l-1)*S/2 + p): sequences s = 2p and 2p+1 (same channel, B even).
+template <int N2, int T>
+__global__ void __launch_bounds__(T >= 128 ? T : 128)
+k_tile_fft2(Dims g, float* __restrict__ state, const float2* __restrict__ spec, const float2* __restrict__ tw, int i,
+            int overwrite) {
+  constexpr int U = N2 / 2;
+  constexpr int F = T >= 128 ? 1 : 128 / T;
+  extern __shared__ float2 fsm[];
+  const int sub = threadIdx.x / T, tid = threadIdx.x - sub * T;
+  float2* sm = fsm + sub * fft_smem_elems(N2);
+  float* ds = reinterpret_cast<float*>(fsm + F * fft_smem_elems(N2)) + sub * 2 * U;
+  const long item = (long)blockIdx.x * F + sub;
+  const int half = g.S / 2;
+  const bool active = item < (long)g.M * half;
+  const int l = active ? (int)(item / half) + 1 : 1;
+  const int s1 = active ? 2 * (int)(item % half) : 0;
+  const int d = s1 / g.B;
+  const float* src1 = state + slot_index(g, l - 1, s1, i - U);
+  const float* src2 = state + slot_index(g, l - 1, s1 + 1, i - U);
+  float* dst1 = state + slot_index(g, l, s1, i);
+  float* dst2 = state + slot_index(g, l, s1 + 1, i);
+  const float2* H = spec + ((size_t)(l - 1) * g.D + d) * (U + 1);
+  tile_fft2_body<N2, T>(sm, ds, tid, active, src1, src2, dst1, dst2, H, tw, overwrite);
+}
+
 // Spectrum of h[0..2N) / (2N) for one (layer, channel): item = l*D + d.
 template <int N>
 __global__ void __launch_bounds__(fft_cta_threads(N))
@@ -338,6 +472,24 @@ static cudaError_t tile_fft_n(const Dims& g, float* state, const float2* spec, c
   return cudaGetLastError();
 }
 
+// Points per thread of the paired blocks (N2 = 2U points per pair).
+__host__ __device__ constexpr int fft2_points(int n2) { return (n2 == 1024 || n2 == 16384) ? 32 : 16; }
+
+template <int N2, int P = fft2_points(N2)>
+static cudaError_t tile_fft2_n(const Dims& g, float* state, const float2* spec, const float2* tw, int i,
+                               cudaStream_t st) {
+  constexpr int T = N2 / P;
+  constexpr int F = T >= 128 ? 1 : 128 / T;
+  const size_t smem = (size_t)F * (fft_smem_elems(N2) * sizeof(float2) + (size_t)N2 * sizeof(float));
+  cudaError_t e = prepare(k_tile_fft2<N2, T>, smem);
+  if (e != cudaSuccess) return e;
+  const long items = (long)g.M * (g.S / 2);
+  const long blocks = (items + F - 1) / F;
+  const int overwrite = is_pow2(i) ? 1 : 0;
+  k_tile_fft2<N2, T><<<(unsigned)blocks, T * F, smem, st>>>(g, state, spec, tw, i, overwrite);
+  return cudaGetLastError();
+}
+
 template <int N>
 static cudaError_t spectra_n(const Dims& g, const float* taps, float2* spec, const float2* tw, int nseg,
                              cudaStream_t st) {
@@ -379,6 +531,22 @@ cudaError_t launch_tile_fft(const Dims& g, float* state, const float2* spectrum_
                             cudaStream_t st) {
   const int U = i & -i;
   const int q = ilog2((uint32_t)U);
+  if (g.B % 2 == 0 && q <= kMaxFftLog2 - 1) {
+    // two sequences of a channel per complex transform of 2U points
+#define CALL(n) tile_fft2_n<2 * (n)>(g, state, spectrum_q, twiddle, i, st)
+    switch (q) {
+      case 6: return CALL(64);
+      case 7: return CALL(128);
+      case 8: return CALL(256);
+      case 9: return CALL(512);
+      case 10: return CALL(1024);
+      case 11: return CALL(2048);
+      case 12: return CALL(4096);
+      case 13: return CALL(8192);
+      default: return cudaErrorInvalidValue;
+    }
+#undef CALL
+  }
 #define CALL(n) tile_fft_n<n>(g, state, spectrum_q, twiddle, i, st)
   FI_FFT_SWITCH(q, CALL)
 #undef CALL

@@ -22,7 +22,7 @@ KERNEL_CLASSES = ("chunk", "direct", "fft", "token", "lazy", "tc")
 EXPORTED = ("fi_init", "fi_step", "fi_generate", "fi_generate_host", "fi_generate_lazy", "fi_sync", "fi_reset",
             "fi_position", "fi_read_activations", "fi_set_stream", "fi_get_plan", "fi_profile",
             "fi_profile_read", "fi_destroy", "fi_status_str", "fi_last_error", "fi_debug_fft",
-            "fi_generate_noalloc", "fi_debug_set_wait_limit")
+            "fi_generate_noalloc", "fi_debug_set_wait_limit", "fi_debug_chunk_schedule")
 
 
 class FiError(RuntimeError):
@@ -61,6 +61,7 @@ def _load():
         "fi_debug_fft": [i32, i32, vp, vp, i32, vp],
         "fi_generate_noalloc": [ctypes.POINTER(Config), vp, i32, vp, vp, f32, vp, vp],
         "fi_debug_set_wait_limit": [vp, i32],
+        "fi_debug_chunk_schedule": [i32, i32, vp, i32, ctypes.POINTER(i32)],
     }
     for name, args in sig.items():
         fn = getattr(lib, name)
@@ -207,6 +208,17 @@ def generate_noalloc(h, batch: int, n: int, x0, eps, y_out, dtype: str = "f32", 
     cfg = Config(M, D, L, int(batch), FI_BF16 if dtype == "bf16" else FI_F32, chunk, 0)
     _check(lib.fi_generate_noalloc(ctypes.byref(cfg), _ptr(h), n, _ptr(x0), _ptr(eps), eps_scale, _ptr(y_out),
                                    _stream(stream)), "fi_generate_noalloc")
+
+
+def chunk_schedule(chunk: int, retimed: bool):
+    """The chunk kernel's table of on-chip block pieces (host only): a list of
+    (step, first source, sources, first target, targets), chunk-relative."""
+    cap = 4 * chunk
+    out = (ctypes.c_int32 * (5 * cap))()
+    n = ctypes.c_int32()
+    _check(lib.fi_debug_chunk_schedule(chunk, 1 if retimed else 0, ctypes.cast(out, ctypes.c_void_p), cap,
+                                       ctypes.byref(n)), "fi_debug_chunk_schedule")
+    return [tuple(out[5 * j: 5 * j + 5]) for j in range(min(n.value, cap))]
 
 
 def status_str(s: int) -> str:

@@ -99,3 +99,40 @@ def test_python_binding_refuses_cpu_tensors():
     from long_convolution_sequence_online_b200 import fi
     with pytest.raises(ValueError):
         fi._ptr(torch.zeros(4))
+
+
+@pytest.mark.parametrize("chunk", [2, 4, 8, 16, 32, 64])
+@pytest.mark.parametrize("retimed", [False, True])
+def test_chunk_piece_table_covers_every_pair_once_in_time(chunk, retimed):
+    """The on-chip pieces of a chunk sum every (source s, target t) pair with
+    s < t inside the chunk exactly once; a piece at step r reads only sources
+    below r (final once position r-1 is done) and writes only targets >= r (the
+    chain reads target t after the pieces of step t); lags stay in 1..chunk-1
+    (the taps the kernel holds). The page's tiling (retimed=False) is one square
+    block of side lowbit(r) per step r; the re-timed one runs at most an 8 x 8
+    square plus pieces of at most 16 x 4 at any step."""
+    from long_convolution_sequence_online_b200 import fi
+    tab = fi.chunk_schedule(chunk, retimed)
+    count = {}
+    per_step = {}
+    for step, s_lo, ns, t_lo, nd in tab:
+        assert 1 <= step < chunk
+        assert s_lo >= 0 and s_lo + ns <= step, (step, s_lo, ns)
+        assert t_lo >= step and t_lo + nd <= chunk, (step, t_lo, nd)
+        assert t_lo - (s_lo + ns - 1) >= 1 and (t_lo + nd - 1) - s_lo <= chunk - 1
+        per_step.setdefault(step, []).append((s_lo, ns, t_lo, nd))
+        for s in range(s_lo, s_lo + ns):
+            for t in range(t_lo, t_lo + nd):
+                count[(s, t)] = count.get((s, t), 0) + 1
+    want = {(s, t) for t in range(chunk) for s in range(t)}
+    assert set(count) == want
+    assert all(v == 1 for v in count.values())
+    assert [step for step, *_ in tab] == sorted(step for step, *_ in tab)
+    for r in range(1, chunk):
+        U = r & -r
+        pieces = per_step[r]
+        if not retimed or U <= 8:
+            assert (r - U, U, r, U) in pieces
+        if retimed:
+            assert max(ns * nd for _, ns, _, nd in pieces) <= 64
+            assert sum(ns * nd for _, ns, _, nd in pieces) <= 64 + 2 * 64
