@@ -382,9 +382,25 @@ def gpu_arm(args, world, rank, local):
         for _ in range(args.e2e_steps):
             e2e_step()
         e2e_s = reduce_max(time.perf_counter() - t0, device)
+        # the host-link share: the same copies alone, from and to the same pinned buffers
+        eps_tmp = torch.empty_like(eps_d)
+        c0, c1, c2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        torch.cuda.synchronize(device)
+        c0.record(stream)
+        eps_tmp.copy_(eps_h, non_blocking=True)
+        c1.record(stream)
+        y_h.copy_(y_d, non_blocking=True)
+        c2.record(stream)
+        torch.cuda.synchronize(device)
+        h2d_ms, d2h_ms = c0.elapsed_time(c1), c1.elapsed_time(c2)
+        del eps_tmp
+        h2d_b = int(x0_h.numel() * x0_h.element_size() + eps_h.numel() * 4)
+        d2h_b = int(y_h.numel() * 4)
         e2e = {"value": world * tokens_per_step * args.e2e_steps / e2e_s, "unit": UNIT,
-               "h2d_bytes_per_step": int(x0_h.numel() * x0_h.element_size() + eps_h.numel() * 4),
-               "d2h_bytes_per_step": int(y_h.numel() * 4),
+               "h2d_bytes_per_step": h2d_b, "d2h_bytes_per_step": d2h_b,
+               "ms_per_step": 1e3 * e2e_s / args.e2e_steps,
+               "copies_alone_ms": {"h2d": h2d_ms, "d2h": d2h_ms,
+                                   "h2d_gbs": h2d_b / h2d_ms / 1e6, "d2h_gbs": d2h_b / d2h_ms / 1e6},
                "timing": "host wall clock around fi_generate_host (synchronous), max over ranks"}
 
     # --- roofline: dominant kernel class during the timed steps
@@ -465,7 +481,9 @@ def gpu_arm(args, world, rank, local):
                    "batch": w.batch, "global_batch": w.batch * world, "tokens_per_step": tokens_per_step,
                    "parallelism": f"dp{world}" if world > 1 else "single",
                    "plan": {"chunk": chunk, "fft_from": fft_from, "fft_max": 1 << 14, "tc_max": tc_max},
-                   "l2": "inputs larger than L2 (state 8.6 GB streamed every step)",
+                   "l2": (f"inputs larger than L2 (state {4 * (w.layers + 1) * w.streams * w.length / 1e9:.1f} GB "
+                          "streamed every step)") if 4 * (w.layers + 1) * w.streams * w.length > L2_BYTES
+                         else "state fits in L2 (latency-bound workload)",
                    "step": "fi_reset + fi_generate over all L positions, closed loop",
                    "init_s": t_init},
         "roofline": roof,

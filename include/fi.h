@@ -116,6 +116,24 @@ FI_API fi_status fi_step(fi_ctx* ctx, const void* x_t, float* y_t);
 FI_API fi_status fi_generate(fi_ctx* ctx, int32_t n, const void* x0, const float* eps,
                       float eps_scale, float* y_out, float* rec);
 
+/* Prompt prefill (page, "Limitazioni" 4, Fase di Prompt: with a long prompt the
+ * prefill dominates, and every prompt position is known at once). Starts a
+ * sequence from position 0 with the p prompt tokens x[p][B][D] (device, of
+ * cfg->dtype) and computes, layer by layer, the offline causal convolution of
+ * the whole prompt by one FFT per (layer, sequence, channel) with the filter's
+ * spectrum zero-padded to twice the transform, then the block. It leaves the
+ * context at position p with the state p calls of fi_step would leave (the
+ * blocks of steps below p whose targets reach past the prompt are added for
+ * their targets >= p), so fi_generate (with the token at p as x0) or fi_step
+ * continue from there.
+ * y_out: NULL or device [p][B][D] fp32, receives y^M_t for t < p.
+ * rec:   NULL or device [M][p][B][D] fp32, receives y^l_t for every layer.
+ * Allocates scratch for the padded spectra (M*D*(2^ceil(log2 p)+1) complex) on
+ * first use and keeps it.
+ * Errors: FI_E_INVALID (NULL, p out of [1, max_len]), FI_E_STATE (position != 0),
+ * FI_E_UNSUPPORTED (p > 16384), FI_E_OOM. */
+FI_API fi_status fi_prefill(fi_ctx* ctx, int32_t p, const void* x, float* y_out, float* rec);
+
 /* fi_generate with HOST buffers: copies x0_host and eps_host to the device,
  * generates, copies y^M back to y_out_host, and returns when the copy is done.
  * Host buffers may be pageable or pinned (pinned is faster). Staging device

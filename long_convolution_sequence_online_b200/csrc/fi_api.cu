@@ -60,6 +60,8 @@ struct fi_ctx {
   int wait_limit = kDefaultWaitLimit;
   size_t spec_off[32] = {};
   float2* part_xs = nullptr;       // forward spectra of source sub-blocks (blocks wider than one transform)
+  float2* pf_spec = nullptr;       // prompt prefill: padded filter spectra (allocated on first use)
+  size_t pf_spec_n = 0;
   // staging for fi_generate_host
   void* d_x0 = nullptr;
   float* d_eps = nullptr;
@@ -80,6 +82,7 @@ void free_ctx(fi_ctx* c) {
   cudaFree(c->taps);
   cudaFree(c->spectra);
   cudaFree(c->part_xs);
+  cudaFree(c->pf_spec);
   cudaFree(c->twiddle);
   cudaFree(c->err);
   cudaFree(c->d_x0);
@@ -126,24 +129,30 @@ fi_status timed(fi_ctx* c, int cls, F&& launch, const char* what) {
 }
 
 // The block of step i (side U = lowbit(i)), read from and written to HBM.
-fi_status run_block(fi_ctx* c, int i) {
+// Targets below t_min are left alone (t_min <= i: the whole block); such
+// partial blocks never go to the tensor cores.
+fi_status run_block(fi_ctx* c, int i, int t_min = 0) {
   const int U = i & -i;
   const int q = ilog2((uint32_t)U);
   if (q > kMaxFftLog2 && c->q_lo <= kMaxFftLog2) {
     return timed(c, KC_FFT,
-                 [&] { return launch_part_block(c->g, c->state, c->part_xs, c->spectra + c->spec_off[q], c->twiddle, i, c->st); },
+                 [&] {
+                   return launch_part_block(c->g, c->state, c->part_xs, c->spectra + c->spec_off[q], c->twiddle, i,
+                                            t_min, c->st);
+                 },
                  "partitioned FFT block launch");
   }
-  if (q >= kMinFftLog2 && q <= c->tc_q_hi) {
+  if (q >= kMinFftLog2 && q <= c->tc_q_hi && t_min <= i) {
     return timed(c, KC_TC,
                  [&] { return launch_tile_tc(c->g, c->state, c->taps, c->tc[q], i, c->err, c->wait_limit, c->st); },
                  "tensor-core block launch");
   }
   if (q >= c->q_lo && q <= c->q_hi) {
-    return timed(c, KC_FFT, [&] { return launch_tile_fft(c->g, c->state, c->spectra + c->spec_off[q], c->twiddle, i, c->st); },
+    return timed(c, KC_FFT,
+                 [&] { return launch_tile_fft(c->g, c->state, c->spectra + c->spec_off[q], c->twiddle, i, t_min, c->st); },
                  "FFT block launch");
   }
-  return timed(c, KC_DIRECT, [&] { return launch_tile_direct(c->g, c->state, c->taps, i, c->st); },
+  return timed(c, KC_DIRECT, [&] { return launch_tile_direct(c->g, c->state, c->taps, i, t_min, c->st); },
                "direct block launch");
 }
 
@@ -399,6 +408,39 @@ fi_status fi_generate(fi_ctx* c, int32_t n, const void* x0, const float* eps, fl
     p = p1;
   }
   c->pos = end;
+  return FI_OK;
+}
+
+fi_status fi_prefill(fi_ctx* c, int32_t p, const void* x, float* y_out, float* rec) {
+  if (!c || !x) return fail(FI_E_INVALID, "NULL argument");
+  if (p < 1 || p > c->g.L) return fail(FI_E_INVALID, "p must be in [1, max_len]");
+  if (p > (1 << kMaxFftLog2))
+    return fail(FI_E_UNSUPPORTED, "prompts longer than " + std::to_string(1 << kMaxFftLog2) + " positions");
+  if (c->pos != 0) return fail(FI_E_STATE, "fi_prefill starts a sequence: call fi_reset first");
+  if (c->lazy_mode) return fail(FI_E_STATE, "context holds a lazy generation; call fi_reset");
+  const Dims& g = c->g;
+  const int q = prefix_transform_log2(p);
+  const size_t need = (size_t)g.M * g.D * ((size_t(1) << q) + 1);
+  if (need > c->pf_spec_n) {
+    FI_CUDA(cudaStreamSynchronize(c->st), "synchronize");
+    cudaFree(c->pf_spec);
+    c->pf_spec = nullptr;
+    c->pf_spec_n = 0;
+    fi_status s = dev_alloc((void**)&c->pf_spec, need * sizeof(float2), "prefill spectra");
+    if (s != FI_OK) return s;
+    c->pf_spec_n = need;
+  }
+  fi_status s = timed(c, KC_FFT,
+                      [&] { return launch_prefix(g, c->state, c->taps, c->pf_spec, c->twiddle, p, x, y_out, rec, c->st); },
+                      "prefill launch");
+  if (s != FI_OK) return s;
+  // Blocks of steps i < p whose targets reach past the prompt (i + lowbit(i) > p):
+  // their parts at targets >= p are what p calls of fi_step would have added
+  // there. Increasing steps, so the first block to reach a target (a power-of-two
+  // step) stores before the others add.
+  for (int i = 1; i < p; ++i)
+    if (i + (i & -i) > p && (s = run_block(c, i, p)) != FI_OK) return s;
+  c->pos = p;
   return FI_OK;
 }
 

@@ -64,12 +64,13 @@ cudaError_t launch_token(const Dims& g, float* state, const float* taps, int t, 
 
 // Direct block of step i (side U = lowbit(i)) from HBM for all layers and streams;
 // overwrite = the block is the first to reach its targets (i a power of two).
+// Block launchers take t_min: targets below it are not written (t_min <= i: all).
 cudaError_t launch_tile_direct(const Dims& g, float* state, const float* taps, int i,
-                               cudaStream_t st);
+                               int t_min, cudaStream_t st);
 
 // FFT block of step i (side U = lowbit(i), 2^kMinFftLog2 <= U <= 2^kMaxFftLog2).
 cudaError_t launch_tile_fft(const Dims& g, float* state, const float2* spectrum_q,
-                            const float2* twiddle, int i, cudaStream_t st);
+                            const float2* twiddle, int i, int t_min, cudaStream_t st);
 
 // Spectra of one level q for all (layer, channel).
 cudaError_t launch_spectra(const Dims& g, const float* taps, float2* spectrum_q,
@@ -81,7 +82,7 @@ cudaError_t launch_spectra(const Dims& g, const float* taps, float2* spectrum_q,
 cudaError_t launch_part_spectra(const Dims& g, const float* taps, float2* gspec, const float2* twiddle, int m,
                                 cudaStream_t st);
 cudaError_t launch_part_block(const Dims& g, float* state, float2* xs, const float2* gspec, const float2* twiddle,
-                              int i, cudaStream_t st);
+                              int i, int t_min, cudaStream_t st);
 
 // Tensor-core block of side U (k_tile_tc.cu): M-tile rows MT (64 or 128), J
 // target tiles per product, NR operand rows (B*J padded), K steps of 16 over
@@ -142,6 +143,15 @@ size_t chunk_smem_bytes(const Dims& g, int chunk, int streams_per_cta);
 
 // Lazy sums of position t for all layers: slot(l, s, t) = sum_{s' < t} h^l[t-s'] a^{l-1}_{s'}.
 cudaError_t launch_lazy_sums(const Dims& g, float* state, const float* taps, int t, cudaStream_t st);
+
+// Prompt prefill: tokens x[p][B][D] into layer 0, then for every layer the
+// offline causal convolution of the prompt (FFT of 2N points, N = 2^q >= p with
+// q = prefix_transform_log2(p) <= kMaxFftLog2) and the block; spec is scratch
+// for M*D*(N+1) complex values. y_out [p][B][D] (layer M) and rec [M][p][B][D]
+// may be NULL.
+int prefix_transform_log2(int p);
+cudaError_t launch_prefix(const Dims& g, float* state, const float* taps, float2* spec, const float2* twiddle, int p,
+                          const void* x, float* y_out, float* rec, cudaStream_t st);
 
 // Debug: batch of complex FFTs with the tile FFT code.
 cudaError_t launch_debug_fft(int log2n, int count, const float2* in, float2* out, int inverse,

@@ -132,7 +132,7 @@ fi_status fi_generate_noalloc(const fi_config* cfg, const void* h, int32_t n, co
     const int p1 = (cst + CH < n) ? cst + CH : n;
     int last_done = p - 1;
     if (cst > 0) {
-      if ((e = launch_tile_direct(g, state, taps, cst, st)) != cudaSuccess)
+      if ((e = launch_tile_direct(g, state, taps, cst, cst, st)) != cudaSuccess)
         return noalloc_fail(FI_E_CUDA, std::string("direct block launch: ") + cudaGetErrorString(e));
       last_done = cst;
     }

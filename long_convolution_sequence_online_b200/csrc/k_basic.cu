@@ -57,7 +57,7 @@ cudaError_t launch_token(const Dims& g, float* state, const float* taps, int t, 
 // reach its targets and stores instead of adding.
 // ---------------------------------------------------------------------------
 __global__ void k_tile_direct(Dims g, float* __restrict__ state, const float* __restrict__ taps, int i, int U,
-                              int overwrite) {
+                              int overwrite, int t_min) {
   extern __shared__ float dsm[];
   float* hs = dsm;          // taps h[0..2U)
   float* xs = dsm + 2 * U;  // sources a[i-U..i)
@@ -74,6 +74,7 @@ __global__ void k_tile_direct(Dims g, float* __restrict__ state, const float* __
   __syncthreads();
   float* dp = state + slot_index(g, l, s, i);
   for (int up = threadIdx.x; up < U; up += blockDim.x) {
+    if (i + up < t_min) continue;
     float sum = 0.f;
     for (int u = 0; u < U; ++u) sum = fmaf(hs[U + up - u], xs[u], sum);
     dp[up] = overwrite ? sum : dp[up] + sum;
@@ -84,7 +85,7 @@ __global__ void k_tile_direct(Dims g, float* __restrict__ state, const float* __
 // taps and sources are read through the cache (every thread of the CTA reads the
 // same source at the same time, and neighbouring threads neighbouring taps).
 __global__ void k_tile_direct_big(Dims g, float* __restrict__ state, const float* __restrict__ taps, int i, int U,
-                                  int overwrite) {
+                                  int overwrite, int t_min) {
   const long cta = blockIdx.x;          // ((l-1)*D + d)*B + b
   const int b = (int)(cta % g.B);
   const long ld = cta / g.B;
@@ -95,17 +96,18 @@ __global__ void k_tile_direct_big(Dims g, float* __restrict__ state, const float
   const float* xp = state + slot_index(g, l - 1, s, i - U);
   float* dp = state + slot_index(g, l, s, i);
   for (int up = threadIdx.x; up < U; up += blockDim.x) {
+    if (i + up < t_min) continue;
     float sum = 0.f;
     for (int u = 0; u < U; ++u) sum = fmaf(__ldg(hp + U + up - u), __ldg(xp + u), sum);
     dp[up] = overwrite ? sum : dp[up] + sum;
   }
 }
 
-cudaError_t launch_tile_direct(const Dims& g, float* state, const float* taps, int i, cudaStream_t st) {
+cudaError_t launch_tile_direct(const Dims& g, float* state, const float* taps, int i, int t_min, cudaStream_t st) {
   const int U = i & -i;
   const long blocks_big = (long)g.M * g.D * g.B;
   if (U > 8192) {
-    k_tile_direct_big<<<(unsigned)blocks_big, 256, 0, st>>>(g, state, taps, i, U, is_pow2(i) ? 1 : 0);
+    k_tile_direct_big<<<(unsigned)blocks_big, 256, 0, st>>>(g, state, taps, i, U, is_pow2(i) ? 1 : 0, t_min);
     return cudaGetLastError();
   }
   const size_t smem = (size_t)3 * U * sizeof(float);
@@ -115,7 +117,7 @@ cudaError_t launch_tile_direct(const Dims& g, float* state, const float* taps, i
   }
   const long blocks = (long)g.M * g.D * g.B;
   const int threads = U >= 256 ? 256 : (U < 32 ? 32 : U);
-  k_tile_direct<<<(unsigned)blocks, threads, smem, st>>>(g, state, taps, i, U, is_pow2(i) ? 1 : 0);
+  k_tile_direct<<<(unsigned)blocks, threads, smem, st>>>(g, state, taps, i, U, is_pow2(i) ? 1 : 0, t_min);
   return cudaGetLastError();
 }
 

@@ -44,7 +44,7 @@ namespace fi {
 constexpr int kChunkMaxThreads = 512;
 constexpr int kChunkMaxStreams = 128;
 constexpr int kSuspendHintNs = 1000;   // longest a suspended barrier check may last
-constexpr int kLayersPerGroupMax = 12;  // layers whose accumulators the chain holds in registers at once
+constexpr int kLayersPerGroupMax = 12;  // most layers per barrier group
 
 struct ChunkShape {
   int G, GP, CH, LS, TPS, CW, GdMax, NG, K;
@@ -357,7 +357,7 @@ __global__ void __launch_bounds__(kChunkMaxThreads) k_chunk(Dims g, ChunkArgs a,
     const int vpr = CH >> 2;                          // float4 per (layer, stream) row
     const int nwin = (M + 1) * Gc * vpr;
     const int ntap = M * Gd * vpr;
-    constexpr int kBatch = 8;
+    constexpr int kBatch = 12;
     for (int base = tid; base < nwin + ntap; base += nt * kBatch) {
       float4 v[kBatch];
 #pragma unroll
@@ -367,9 +367,9 @@ __global__ void __launch_bounds__(kChunkMaxThreads) k_chunk(Dims g, ChunkArgs a,
         if (idx < nwin) {
           const int row = idx / vpr, j = idx - row * vpr;
           const int l = row / Gc, gg = row - l * Gc;
-          const int t = a.c + 4 * j;
-          if (slot_valid(l, t) || slot_valid(l, t + 1) || slot_valid(l, t + 2) || slot_valid(l, t + 3))
-            v[u] = __ldg(reinterpret_cast<const float4*>(a.state + slot_index(g, l, s0 + gg, t)));
+          // every slot of the window lies inside the state, so the load is
+          // always in bounds; slots holding nothing yet are zeroed below
+          v[u] = __ldg(reinterpret_cast<const float4*>(a.state + slot_index(g, l, s0 + gg, a.c + 4 * j)));
         } else if (idx < nwin + ntap) {
           const int k = idx - nwin;
           const int row = k / vpr, j = k - row * vpr;
@@ -436,101 +436,81 @@ __global__ void __launch_bounds__(kChunkMaxThreads) k_chunk(Dims g, ChunkArgs a,
     const int gg = act ? gg0 : 0;
     const int s = s0 + gg, d = s / g.B, b = s - d * g.B;
     const size_t c_io = (size_t)b * g.D + d;
-    float* wcol = win + gg;                                  // slot (l, r) at wcol[l*LS + r*GP]
-    const float* hcol = tp + (d - d_lo) * TPS;               // h0 of layer l at hcol[(l-1)*GdMax*TPS]
     const size_t y_stride = g.S;
-    // Accumulators and h0 of one layer group, in registers (loaded together once
-    // the group's blocks are done, so their latency is paid once per group).
-    float accA[kLayersPerGroupMax], h0A[kLayersPerGroupMax];
-    float accB[kLayersPerGroupMax], h0B[kLayersPerGroupMax];
-    auto load_group = [&](int grp, int r, float* acc, float* h0) {
-      const int lg0 = grp * K + 1;
-#pragma unroll
-      for (int k = 0; k < kLayersPerGroupMax; ++k) {
-        if (k < K && lg0 + k <= M) {
-          acc[k] = wcol[(lg0 + k) * LS + r * GP];
-          h0[k] = hcol[(lg0 + k - 1) * GdMax * TPS];
-        }
-      }
-    };
+    float* wcol = win + gg;                          // slot (l, r) at wcol[l*LS + r*GP]
+    const float* hcol = tp + (d - d_lo) * TPS;       // h0 of layer l at hcol[(l-1)*HS]
+    const int HS = GdMax * TPS;
+    // The tile_done barrier of (group, position) is tested one step ahead
+    // (halfway through the previous group) without blocking; a test that came
+    // back false is followed by a bounded wait when the group starts.
     auto wait_group = [&](int grp, int r) {
       if (r >= rs && ok) ok = mbar_wait(&tile_done[grp * CW + warp], (r - rs) & 1, err, true, a.wait_limit);
     };
-    auto test_group = [&](int grp, int r) {
-      return r < rs || mbar_test(&tile_done[grp * CW + warp], (r - rs) & 1);
-    };
+    auto test_group = [&](int grp, int r) { return r < rs || mbar_test(&tile_done[grp * CW + warp], (r - rs) & 1); };
 
-    // Group 0 of the first position.
-    wait_group(0, r0);
-    load_group(0, r0, accA, h0A);
+    // layer 1 of the first position: the token itself
+    if (!test_group(0, r0)) wait_group(0, r0);
     const float x_first = wcol[r0 * GP];
-    // The input of layer 1 as tanh parts (or the token itself at the first position).
-    TanhParts P{0.f, x_first, true};
-    float xb = x_first;          // bf16 path: the token
-    float epsk = 0.f;            // eps_scale * eps of the previous position (fp32 path)
-    bool loadedB = false;
+    TanhParts P{0.f, x_first, true};   // the input of layer 1 as tanh parts (here: the token)
+    float xb = x_first;                // bf16 path: the token
+    float epsk = 0.f;                  // eps_scale * eps of the previous position (fp32 path)
+    float acc_n = wcol[LS + r0 * GP];  // operands of the next layer to enter
+    float h0_n = hcol[0];
+    bool ready = false;                // the barrier of the next group to enter has completed
     for (int r = r0; r < r1; ++r) {
       const int t = a.c + r;
       float y, z = 0.f;
-      if constexpr (BF16) {
-        y = fmaf(h0A[0], xb, accA[0]);
-      } else {
-        next_input(P, h0A[0], fmaf(h0A[0], epsk, accA[0]), y, z);
-      }
-      for (int grp = 0; grp < NG; ++grp) {
-        const int lg0 = grp * K + 1;
-        const int nk = min(M, lg0 + K - 1) - lg0 + 1;
-        const int kmid = nk / 2;
-        const bool last_grp = grp + 1 == NG;
-        // the barrier tested halfway through this group: the next group, or
-        // group 0 of the next position after the last group
-        const int ngrp = last_grp ? 0 : grp + 1;
-        const int nr = last_grp ? r + 1 : r;
-#pragma unroll
-        for (int k = 0; k < kLayersPerGroupMax; ++k) {
-          if (k < nk) {
-            const int l = lg0 + k;
-            if constexpr (REC) if (act) a.rec[((size_t)(l - 1) * a.n_gen + (t - a.gen_base)) * y_stride + c_io] = y;
-            if (k == kmid && !loadedB && nr < r1 && test_group(ngrp, nr)) {
-              load_group(ngrp, nr, accB, h0B);
-              loadedB = true;
-            }
-            if (l == M) break;
-            float av;
-            if constexpr (BF16) {
-              av = round_bf16(tanh_approx(y));
-            } else {
-              P = tanh_parts(y, z);
-              av = tanh_value(P);
-            }
-            if (act) wcol[l * LS + r * GP] = av;
-            if (k + 1 < nk) {
-              if constexpr (BF16) y = fmaf(h0A[k + 1], av, accA[k + 1]);
-              else next_input(P, h0A[k + 1], accA[k + 1], y, z);
-            } else {
-              // last layer of a group below M: hand the group to the tile
-              // warps, then continue into the next group
-              mbar_arrive(&act_ready[grp * CW + warp]);
-              if (!loadedB) {
-                wait_group(grp + 1, r);
-                load_group(grp + 1, r, accB, h0B);
-              }
-#pragma unroll
-              for (int q = 0; q < kLayersPerGroupMax; ++q) {
-                accA[q] = accB[q];
-                h0A[q] = h0B[q];
-              }
-              loadedB = false;
-              if constexpr (BF16) y = fmaf(h0A[0], av, accA[0]);
-              else next_input(P, h0A[0], accA[0], y, z);
-            }
-          }
+      if constexpr (BF16) y = fmaf(h0_n, xb, acc_n);
+      else next_input(P, h0_n, fmaf(h0_n, epsk, acc_n), y, z);
+      int grp = 0, lg_end = K;         // current group and its last layer
+      const int kmid = K / 2;
+      for (int l = 1;; ++l) {
+        if constexpr (REC) if (act) a.rec[((size_t)(l - 1) * a.n_gen + (t - a.gen_base)) * y_stride + c_io] = y;
+        if (l == M) break;
+        const bool boundary = l == lg_end;         // layer l closes its group
+        if (!boundary) {
+          // next layer's operands, issued before this layer's exp2/reciprocal so
+          // their latency hides behind them
+          acc_n = wcol[(l + 1) * LS + r * GP];
+          h0_n = hcol[l * HS];
         }
+        if (l == grp * K + kmid) {
+          // halfway through the group: test the next one's barrier (group 0 of
+          // the next position after the last group)
+          const bool last = grp + 1 == NG;
+          ready = last ? (r + 1 >= r1 || test_group(0, r + 1)) : test_group(grp + 1, r);
+        }
+        float av;
+        if constexpr (BF16) {
+          av = round_bf16(tanh_approx(y));
+        } else {
+          P = tanh_parts(y, z);
+          av = tanh_value(P);
+        }
+        if (act) wcol[l * LS + r * GP] = av;
+        if (boundary) {
+          // hand the group to the tile warps, then enter the next one
+          mbar_arrive(&act_ready[grp * CW + warp]);
+          ++grp;
+          lg_end = min(M, lg_end + K);
+          if (!ready) wait_group(grp, r);
+          ready = false;
+          acc_n = wcol[(l + 1) * LS + r * GP];
+          h0_n = hcol[l * HS];
+        }
+        if constexpr (BF16) y = fmaf(h0_n, av, acc_n);
+        else next_input(P, h0_n, acc_n, y, z);
       }
       // y = y^M_t: output, then the sampler x_{t+1} = R(tanh(y) + eps_scale eps_t)
       mbar_arrive(&act_ready[(NG - 1) * CW + warp]);
       if (act) a.y_out[(size_t)(t - a.gen_base) * y_stride + c_io] = y;
       const float epsv = ep[r * G + gg];
+      if (r + 1 < r1) {
+        if (!ready) wait_group(0, r + 1);
+        acc_n = wcol[LS + (r + 1) * GP];
+        h0_n = hcol[0];
+      }
+      ready = false;
       float xn;
       if constexpr (BF16) {
         xn = round_bf16(tanh_approx(y) + a.eps_scale * epsv);
@@ -543,18 +523,6 @@ __global__ void __launch_bounds__(kChunkMaxThreads) k_chunk(Dims g, ChunkArgs a,
       // x_{t+1}; for the last position of the chunk it lands in the spare
       // position CH and goes to HBM with the write-back.
       if (act && t + 1 < g.L) wcol[(r + 1) * GP] = xn;
-      if (r + 1 < r1) {
-        if (!loadedB) {
-          wait_group(0, r + 1);
-          load_group(0, r + 1, accB, h0B);
-        }
-#pragma unroll
-        for (int q = 0; q < kLayersPerGroupMax; ++q) {
-          accA[q] = accB[q];
-          h0A[q] = h0B[q];
-        }
-        loadedB = false;
-      }
     }
   } else {
     // ---------------------------------------------------------------- tile warps

@@ -93,7 +93,7 @@ __device__ __forceinline__ void fwd_from_global(float2* sm, int tid, bool active
 template <int N, int T, class Sync>
 __device__ __forceinline__ void inv_to_global(float2* sm, const float2* ds, int tid, bool active,
                                               float2* __restrict__ dst, const float2* __restrict__ tw, int overwrite,
-                                              Sync sync) {
+                                              int w_min, Sync sync) {
   using S = FftShape<N, T>;
   smem_passes<N, T, true, 0, true>(sm, tid, tw, sync);
   constexpr int DL = last_pass_done<N, T>();
@@ -111,12 +111,14 @@ __device__ __forceinline__ void inv_to_global(float2* sm, const float2* ds, int 
       for (int r = R / 2; r < R; ++r) {
         const int m = j + r * (N / R) - N / 2;
         const float2 o = v[k * R + r];
-        if (overwrite) {
-          dst[m] = o;
-        } else {
+        float2 val = o;
+        if (!overwrite) {
           const float2 p = ds[m];
-          dst[m] = make_float2(p.x + o.x, p.y + o.y);
+          val = make_float2(p.x + o.x, p.y + o.y);
         }
+        // targets below w_min (relative to dst) are left alone: positions 2m, 2m+1
+        if (2 * m >= w_min) dst[m] = val;
+        else if (2 * m + 1 >= w_min) reinterpret_cast<float*>(dst)[2 * m + 1] = val.y;
       }
     }
   }
@@ -125,12 +127,12 @@ __device__ __forceinline__ void inv_to_global(float2* sm, const float2* ds, int 
 template <int N, int T, class Sync>
 __device__ __forceinline__ void tile_fft_body(float2* sm, float2* ds, int tid, bool active, const float2* __restrict__ src,
                                               float2* __restrict__ dst, const float2* __restrict__ H,
-                                              const float2* __restrict__ tw, int overwrite, Sync sync) {
+                                              const float2* __restrict__ tw, int overwrite, int w_min, Sync sync) {
   stage_dst<N, T>(ds, tid, active, dst, overwrite);
   fwd_from_global<N, T>(sm, tid, active, src, tw, sync);
   spectral_product<N, T>(sm, tid, H, tw);
   sync();
-  inv_to_global<N, T>(sm, ds, tid, active, dst, tw, overwrite, sync);
+  inv_to_global<N, T>(sm, ds, tid, active, dst, tw, overwrite, w_min, sync);
 }
 
 // ---------------------------------------------------------------------------
@@ -185,7 +187,7 @@ k_part_fwd(Dims g, const float* __restrict__ state, float2* __restrict__ xs, con
 template <int N>
 __global__ void __launch_bounds__(fft_cta_threads(N))
 k_part_inv(Dims g, float* __restrict__ state, const float2* __restrict__ xs, const float2* __restrict__ gspec,
-           const float2* __restrict__ tw, int i, int m, int overwrite) {
+           const float2* __restrict__ tw, int i, int m, int overwrite, int t_min) {
   constexpr int T = fft_threads(N), F = fft_per_cta(N);
   constexpr int twstep = kTwiddleN / (2 * N);
   extern __shared__ float2 fsm[];
@@ -221,10 +223,10 @@ k_part_inv(Dims g, float* __restrict__ state, const float2* __restrict__ xs, con
   }
   if constexpr (T <= 32) {
     __syncwarp();
-    inv_to_global<N, T>(sm, ds, tid, active, dst, tw, overwrite, SyncWarp());
+    inv_to_global<N, T>(sm, ds, tid, active, dst, tw, overwrite, t_min - (i + k * N), SyncWarp());
   } else {
     __syncthreads();
-    inv_to_global<N, T>(sm, ds, tid, active, dst, tw, overwrite, SyncBlock());
+    inv_to_global<N, T>(sm, ds, tid, active, dst, tw, overwrite, t_min - (i + k * N), SyncBlock());
   }
 }
 
@@ -233,7 +235,7 @@ k_part_inv(Dims g, float* __restrict__ state, const float2* __restrict__ xs, con
 template <int N, int T = fft_threads(N)>
 __global__ void __launch_bounds__(T >= 128 ? T : 128)
 k_tile_fft(Dims g, float* __restrict__ state, const float2* __restrict__ spec,
-           const float2* __restrict__ tw, int i, int overwrite) {
+           const float2* __restrict__ tw, int i, int overwrite, int t_min) {
   constexpr int F = T >= 128 ? 1 : 128 / T;
   extern __shared__ float2 fsm[];
   const int sub = threadIdx.x / T, tid = threadIdx.x - sub * T;
@@ -248,8 +250,8 @@ k_tile_fft(Dims g, float* __restrict__ state, const float2* __restrict__ spec,
   const float2* src = reinterpret_cast<const float2*>(state + slot_index(g, l - 1, s, i - N));
   float2* dst = reinterpret_cast<float2*>(state + slot_index(g, l, s, i));
   const float2* H = spec + ((size_t)(l - 1) * g.D + d) * (N + 1);
-  if constexpr (T <= 32) tile_fft_body<N, T>(sm, ds, tid, active, src, dst, H, tw, overwrite, SyncWarp());
-  else tile_fft_body<N, T>(sm, ds, tid, active, src, dst, H, tw, overwrite, SyncBlock());
+  if constexpr (T <= 32) tile_fft_body<N, T>(sm, ds, tid, active, src, dst, H, tw, overwrite, t_min - i, SyncWarp());
+  else tile_fft_body<N, T>(sm, ds, tid, active, src, dst, H, tw, overwrite, t_min - i, SyncBlock());
 }
 
 // ---------------------------------------------------------------------------
@@ -270,7 +272,7 @@ __device__ __forceinline__ void tile_fft2_body(float2* sm, float* ds, int tid, b
                                                const float* __restrict__ src1, const float* __restrict__ src2,
                                                float* __restrict__ dst1, float* __restrict__ dst2,
                                                const float2* __restrict__ H, const float2* __restrict__ tw,
-                                               int overwrite) {
+                                               int overwrite, int w_min) {
   constexpr int U = N2 / 2;
   using SF = FftShape<N2, T, false>;
   using SI = FftShape<N2, T, true>;
@@ -349,6 +351,7 @@ __device__ __forceinline__ void tile_fft2_body(float2* sm, float* ds, int tid, b
       for (int r = R / 2; r < R; ++r) {
         const int m = j + r * (N2 / R) - U;
         const float2 o = v[k * R + r];
+        if (m < w_min) continue;
         if (overwrite) {
           dst1[m] = o.x;
           dst2[m] = o.y;
@@ -365,7 +368,7 @@ __device__ __forceinline__ void tile_fft2_body(float2* sm, float* ds, int tid, b
 template <int N2, int T>
 __global__ void __launch_bounds__(T >= 128 ? T : 128)
 k_tile_fft2(Dims g, float* __restrict__ state, const float2* __restrict__ spec, const float2* __restrict__ tw, int i,
-            int overwrite) {
+            int overwrite, int t_min) {
   constexpr int U = N2 / 2;
   constexpr int F = T >= 128 ? 1 : 128 / T;
   extern __shared__ float2 fsm[];
@@ -383,14 +386,104 @@ k_tile_fft2(Dims g, float* __restrict__ state, const float2* __restrict__ spec, 
   float* dst1 = state + slot_index(g, l, s1, i);
   float* dst2 = state + slot_index(g, l, s1 + 1, i);
   const float2* H = spec + ((size_t)(l - 1) * g.D + d) * (U + 1);
-  tile_fft2_body<N2, T>(sm, ds, tid, active, src1, src2, dst1, dst2, H, tw, overwrite);
+  tile_fft2_body<N2, T>(sm, ds, tid, active, src1, src2, dst1, dst2, H, tw, overwrite, t_min - i);
+}
+
+// ---------------------------------------------------------------------------
+// Prompt prefill (summary page, Limitazioni 4, "Fase di Prompt": the prompt's
+// positions are all known, so each layer is one offline causal convolution).
+// For a prompt of p <= N positions (N a power of two), y^l_t for t < p is the
+// causal convolution of a^{l-1}_0..p-1 with h^l, computed by one real FFT of
+// length 2N against the spectrum of h[0..N) zero-padded to 2N: both sequences
+// have support [0, N), so the circular convolution of length 2N has no
+// wrap-around and its first N outputs are the causal convolution (lag 0, the
+// red cell, included). One launch per layer, one transform per stream; the
+// block (tanh, bf16 rounding) is applied on the way out.
+// ---------------------------------------------------------------------------
+template <int N, int T = fft_threads(N)>
+__global__ void __launch_bounds__(T >= 128 ? T : 128)
+k_prefix_conv(Dims g, float* __restrict__ state, const float2* __restrict__ spec, const float2* __restrict__ tw,
+              int l, int p, float* __restrict__ y_out, float* __restrict__ rec, int n_rec) {
+  constexpr int F = T >= 128 ? 1 : 128 / T;
+  using S = FftShape<N, T>;
+  extern __shared__ float2 fsm[];
+  const int sub = threadIdx.x / T, tid = threadIdx.x - sub * T;
+  float2* sm = fsm + sub * fft_smem_elems(N);
+  const long item = (long)blockIdx.x * F + sub;
+  const bool active = item < g.S;
+  const int s = active ? (int)item : 0, d = s / g.B, b = s - d * g.B;
+  const float* src = state + slot_index(g, l - 1, s, 0);
+  const float2* H = spec + ((size_t)(l - 1) * g.D + d) * (N + 1);
+  auto sync = [] {
+    if constexpr (T <= 32) __syncwarp();
+    else __syncthreads();
+  };
+  {
+    // forward pass 0 from HBM: z[m] = (a[2m], a[2m+1]), zero at positions >= p
+    constexpr int R = 1 << S::rb(0);
+    float2 v[S::P];
+#pragma unroll
+    for (int k = 0; k < S::P / R; ++k) {
+      const int j = tid + k * T;
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        const int t0 = 2 * (j + r * (N / R));
+        v[k * R + r] = (active && r < R / 2)
+                           ? make_float2(t0 < p ? src[t0] : 0.f, t0 + 1 < p ? src[t0 + 1] : 0.f)
+                           : make_float2(0.f, 0.f);
+      }
+    }
+    pass_compute<N, T, false, 0>(v, tid, tw);
+    pass_store<N, T, 0>(sm, v, tid);
+    sync();
+  }
+  smem_passes<N, T, false, S::rb(0), false>(sm, tid, tw, sync);
+  spectral_product<N, T>(sm, tid, H, tw);
+  sync();
+  smem_passes<N, T, true, 0, true>(sm, tid, tw, sync);
+  constexpr int DL = last_pass_done<N, T>();
+  constexpr int R = 1 << S::rb(DL);
+  float2 v[S::P];
+  pass_load<N, T, DL>(sm, v, tid);
+  pass_compute<N, T, true, DL>(v, tid, tw);
+  if (!active) return;
+  const size_t io = (size_t)b * g.D + d;
+  float* dst = state + slot_index(g, l, s, 0);
+#pragma unroll
+  for (int k = 0; k < S::P / R; ++k) {
+    const int j = tid + k * T;
+#pragma unroll
+    for (int r = 0; r < R / 2; ++r) {
+      const int t0 = 2 * (j + r * (N / R));
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        const int t = t0 + q;
+        if (t >= p) continue;
+        const float y = q ? v[k * R + r].y : v[k * R + r].x;
+        if (rec) rec[((size_t)(l - 1) * n_rec + t) * g.S + io] = y;
+        if (l < g.M) dst[t] = round_act(tanhf(y), g.bf16);
+        else if (y_out) y_out[(size_t)t * g.S + io] = y;
+      }
+    }
+  }
+}
+
+// Prompt tokens x[t][b][d] into the layer-0 slots.
+__global__ void k_store_tokens(Dims g, float* __restrict__ state, const void* __restrict__ x, int p) {
+  const size_t total = (size_t)p * g.S;
+  for (size_t k = (size_t)blockIdx.x * blockDim.x + threadIdx.x; k < total; k += (size_t)gridDim.x * blockDim.x) {
+    const int t = (int)(k / g.S);
+    const int r = (int)(k - (size_t)t * g.S);   // r = b*D + d
+    const int b = r / g.D, d = r - b * g.D;
+    state[slot_index(g, 0, d * g.B + b, t)] = round_act(load_token(x, k, g.bf16), g.bf16);
+  }
 }
 
 // Spectrum of h[0..2N) / (2N) for one (layer, channel): item = l*D + d.
 template <int N>
 __global__ void __launch_bounds__(fft_cta_threads(N))
 k_spectra(Dims g, const float* __restrict__ taps, float2* __restrict__ spec, const float2* __restrict__ tw, int off,
-          int nseg, int seg0) {
+          int nseg, int seg0, int pad) {
   constexpr int T = fft_threads(N), F = fft_per_cta(N);
   constexpr int twstep = kTwiddleN / (2 * N);
   extern __shared__ float2 fsm[];
@@ -402,7 +495,9 @@ k_spectra(Dims g, const float* __restrict__ taps, float2* __restrict__ spec, con
   const long ld = active ? item / nseg : 0;
   const int e = active ? (int)(item - ld * nseg) : 0;
   const float2* src = reinterpret_cast<const float2*>(taps + (size_t)ld * g.L + off + (size_t)(seg0 + e) * N);
-  for (int m = tid; m < N; m += T) sm[fft_pad<N, T>(m)] = active ? src[m] : make_float2(0.f, 0.f);
+  // pad: only h[0..N) (complex points m < N/2), zero above
+  for (int m = tid; m < N; m += T)
+    sm[fft_pad<N, T>(m)] = (active && (!pad || m < N / 2)) ? src[m] : make_float2(0.f, 0.f);
   if constexpr (T <= 32) {
     __syncwarp();
     fft_smem<N, T, false>(sm, tid, tw, SyncWarp());
@@ -460,7 +555,7 @@ static cudaError_t prepare(K kernel, size_t smem) {
 
 template <int N, int T = fft_threads(N)>
 static cudaError_t tile_fft_n(const Dims& g, float* state, const float2* spec, const float2* tw, int i,
-                              cudaStream_t st) {
+                              int t_min, cudaStream_t st) {
   constexpr int F = T >= 128 ? 1 : 128 / T;
   const size_t smem = (size_t)F * (fft_smem_elems(N) + N / 2) * sizeof(float2);
   cudaError_t e = prepare(k_tile_fft<N, T>, smem);
@@ -468,16 +563,20 @@ static cudaError_t tile_fft_n(const Dims& g, float* state, const float2* spec, c
   const long items = (long)g.M * g.S;
   const long blocks = (items + F - 1) / F;
   const int overwrite = is_pow2(i) ? 1 : 0;
-  k_tile_fft<N, T><<<(unsigned)blocks, T * F, smem, st>>>(g, state, spec, tw, i, overwrite);
+  k_tile_fft<N, T><<<(unsigned)blocks, T * F, smem, st>>>(g, state, spec, tw, i, overwrite, t_min);
   return cudaGetLastError();
 }
 
-// Points per thread of the paired blocks (N2 = 2U points per pair).
-__host__ __device__ constexpr int fft2_points(int n2) { return (n2 == 1024 || n2 == 16384) ? 32 : 16; }
+// Points per thread of the paired blocks (N2 = 2U points per pair): the choice
+// that avoids a radix-2 pass (radix 32 where log2 N2 = 9, 10, 13, 14; radix 16
+// where it is 7, 8, 11, 12).
+__host__ __device__ constexpr int fft2_points(int n2) {
+  return (n2 == 512 || n2 == 1024 || n2 == 8192 || n2 == 16384) ? 32 : 16;
+}
 
 template <int N2, int P = fft2_points(N2)>
 static cudaError_t tile_fft2_n(const Dims& g, float* state, const float2* spec, const float2* tw, int i,
-                               cudaStream_t st) {
+                               int t_min, cudaStream_t st) {
   constexpr int T = N2 / P;
   constexpr int F = T >= 128 ? 1 : 128 / T;
   const size_t smem = (size_t)F * (fft_smem_elems(N2) * sizeof(float2) + (size_t)N2 * sizeof(float));
@@ -486,19 +585,19 @@ static cudaError_t tile_fft2_n(const Dims& g, float* state, const float2* spec, 
   const long items = (long)g.M * (g.S / 2);
   const long blocks = (items + F - 1) / F;
   const int overwrite = is_pow2(i) ? 1 : 0;
-  k_tile_fft2<N2, T><<<(unsigned)blocks, T * F, smem, st>>>(g, state, spec, tw, i, overwrite);
+  k_tile_fft2<N2, T><<<(unsigned)blocks, T * F, smem, st>>>(g, state, spec, tw, i, overwrite, t_min);
   return cudaGetLastError();
 }
 
 template <int N>
 static cudaError_t spectra_n(const Dims& g, const float* taps, float2* spec, const float2* tw, int nseg,
-                             cudaStream_t st) {
+                             cudaStream_t st, int pad = 0) {
   const size_t smem = fft_smem_bytes<N>();
   cudaError_t e = prepare(k_spectra<N>, smem);
   if (e != cudaSuccess) return e;
   const long items = (long)g.M * g.D * nseg;
   const long blocks = (items + fft_per_cta(N) - 1) / fft_per_cta(N);
-  k_spectra<N><<<(unsigned)blocks, fft_cta_threads(N), smem, st>>>(g, taps, spec, tw, 0, nseg, 0);
+  k_spectra<N><<<(unsigned)blocks, fft_cta_threads(N), smem, st>>>(g, taps, spec, tw, 0, nseg, 0, pad);
   return cudaGetLastError();
 }
 
@@ -528,12 +627,12 @@ static cudaError_t debug_fft_n(int count, const float2* in, float2* out, int inv
   }
 
 cudaError_t launch_tile_fft(const Dims& g, float* state, const float2* spectrum_q, const float2* twiddle, int i,
-                            cudaStream_t st) {
+                            int t_min, cudaStream_t st) {
   const int U = i & -i;
   const int q = ilog2((uint32_t)U);
   if (g.B % 2 == 0 && q <= kMaxFftLog2 - 1) {
     // two sequences of a channel per complex transform of 2U points
-#define CALL(n) tile_fft2_n<2 * (n)>(g, state, spectrum_q, twiddle, i, st)
+#define CALL(n) tile_fft2_n<2 * (n)>(g, state, spectrum_q, twiddle, i, t_min, st)
     switch (q) {
       case 6: return CALL(64);
       case 7: return CALL(128);
@@ -547,7 +646,7 @@ cudaError_t launch_tile_fft(const Dims& g, float* state, const float2* spectrum_
     }
 #undef CALL
   }
-#define CALL(n) tile_fft_n<n>(g, state, spectrum_q, twiddle, i, st)
+#define CALL(n) tile_fft_n<n>(g, state, spectrum_q, twiddle, i, t_min, st)
   FI_FFT_SWITCH(q, CALL)
 #undef CALL
 }
@@ -565,7 +664,7 @@ cudaError_t launch_part_spectra(const Dims& g, const float* taps, float2* gspec,
 }
 
 cudaError_t launch_part_block(const Dims& g, float* state, float2* xs, const float2* gspec, const float2* twiddle,
-                              int i, cudaStream_t st) {
+                              int i, int t_min, cudaStream_t st) {
   constexpr int N = 1 << kMaxFftLog2;
   const int m = (i & -i) / N;
   const long items = (long)g.M * g.S * m;
@@ -578,7 +677,7 @@ cudaError_t launch_part_block(const Dims& g, float* state, float2* xs, const flo
   smem += (size_t)fft_per_cta(N) * (N / 2) * sizeof(float2);
   if ((e = prepare(k_part_inv<N>, smem)) != cudaSuccess) return e;
   k_part_inv<N><<<(unsigned)blocks, fft_cta_threads(N), smem, st>>>(g, state, xs, gspec, twiddle, i, m,
-                                                                   is_pow2(i) ? 1 : 0);
+                                                                   is_pow2(i) ? 1 : 0, t_min);
   return cudaGetLastError();
 }
 
@@ -586,6 +685,38 @@ cudaError_t launch_debug_fft(int log2n, int count, const float2* in, float2* out
                              const float2* twiddle, cudaStream_t st) {
 #define CALL(n) debug_fft_n<n>(count, in, out, inverse, twiddle, st)
   FI_FFT_SWITCH(log2n, CALL)
+#undef CALL
+}
+
+template <int N>
+static cudaError_t prefix_n(const Dims& g, float* state, const float* taps, float2* spec, const float2* tw, int p,
+                            const void* x, float* y_out, float* rec, cudaStream_t st) {
+  cudaError_t e = spectra_n<N>(g, taps, spec, tw, 1, st, 1);
+  if (e != cudaSuccess) return e;
+  k_store_tokens<<<148 * 4, 256, 0, st>>>(g, state, x, p);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  constexpr int T = fft_threads(N), F = T >= 128 ? 1 : 128 / T;
+  const size_t smem = (size_t)F * fft_smem_elems(N) * sizeof(float2);
+  if ((e = prepare(k_prefix_conv<N>, smem)) != cudaSuccess) return e;
+  const long blocks = ((long)g.S + F - 1) / F;
+  for (int l = 1; l <= g.M; ++l) {
+    k_prefix_conv<N><<<(unsigned)blocks, T * F, smem, st>>>(g, state, spec, tw, l, p, y_out, rec, p);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+int prefix_transform_log2(int p) {
+  int q = kMinFftLog2;
+  while ((1 << q) < p) ++q;
+  return q;
+}
+
+cudaError_t launch_prefix(const Dims& g, float* state, const float* taps, float2* spec, const float2* twiddle, int p,
+                          const void* x, float* y_out, float* rec, cudaStream_t st) {
+  const int q = prefix_transform_log2(p);
+#define CALL(n) prefix_n<n>(g, state, taps, spec, twiddle, p, x, y_out, rec, st)
+  FI_FFT_SWITCH(q, CALL)
 #undef CALL
 }
 

@@ -22,7 +22,7 @@ KERNEL_CLASSES = ("chunk", "direct", "fft", "token", "lazy", "tc")
 EXPORTED = ("fi_init", "fi_step", "fi_generate", "fi_generate_host", "fi_generate_lazy", "fi_sync", "fi_reset",
             "fi_position", "fi_read_activations", "fi_set_stream", "fi_get_plan", "fi_profile",
             "fi_profile_read", "fi_destroy", "fi_status_str", "fi_last_error", "fi_debug_fft",
-            "fi_generate_noalloc", "fi_debug_set_wait_limit", "fi_debug_chunk_schedule")
+            "fi_generate_noalloc", "fi_debug_set_wait_limit", "fi_debug_chunk_schedule", "fi_prefill")
 
 
 class FiError(RuntimeError):
@@ -62,6 +62,7 @@ def _load():
         "fi_generate_noalloc": [ctypes.POINTER(Config), vp, i32, vp, vp, f32, vp, vp],
         "fi_debug_set_wait_limit": [vp, i32],
         "fi_debug_chunk_schedule": [i32, i32, vp, i32, ctypes.POINTER(i32)],
+        "fi_prefill": [vp, i32, vp, vp, vp],
     }
     for name, args in sig.items():
         fn = getattr(lib, name)
@@ -147,6 +148,9 @@ class Context:
 
     def generate(self, n: int, x0, eps, y_out, eps_scale: float = 0.1, rec=None):
         _check(lib.fi_generate(self._h, n, _ptr(x0), _ptr(eps), eps_scale, _ptr(y_out), _ptr(rec)), "fi_generate")
+
+    def prefill(self, p: int, x, y_out=None, rec=None):
+        _check(lib.fi_prefill(self._h, p, _ptr(x), _ptr(y_out), _ptr(rec)), "fi_prefill")
 
     def generate_host(self, n: int, x0: np.ndarray, eps: np.ndarray, y_out: np.ndarray, eps_scale: float = 0.1):
         for a in (x0, eps, y_out):

@@ -21,6 +21,7 @@ from .lcsm import (  # noqa: F401
     dft,
     lowbit,
     online_lcsm,
+    prompt_lcsm,
     relaxed_online,
     relaxed_tiles,
     stream_error,

@@ -156,6 +156,30 @@ def online_lcsm(h: np.ndarray, x0: np.ndarray, eps: np.ndarray, eps_scale: float
     return y, a
 
 
+def prompt_lcsm(h: np.ndarray, x: np.ndarray, bf16: bool = False):
+    """The stack on a prompt whose tokens are all given (summary page,
+    "Limitazioni" 4, Fase di Prompt: every prompt position is known up front).
+
+    a^0 = R(x); for each layer y^l = causal convolution of a^{l-1} with h^l over
+    the prompt, a^l = R(tanh(y^l)). No sampler: the tokens are the prompt's.
+    h: [M][S][L] filters (per stream), x: [S][p] tokens.
+    Returns (y, a) with y[l-1] = y^l and a[l] = a^l, each [M][S][p].
+    """
+    h = np.asarray(h, dtype=np.float64)
+    M, S, L = h.shape
+    x = np.asarray(x, dtype=np.float64)
+    p = x.shape[-1]
+    R = bf16_round if bf16 else _identity
+    a = np.zeros((M, S, p), dtype=np.float64)
+    y = np.zeros((M, S, p), dtype=np.float64)
+    a[0] = R(x)
+    for l in range(M):
+        y[l] = causal_conv(h[l, :, :p], a[l])
+        if l + 1 < M:
+            a[l + 1] = R(np.tanh(y[l]))
+    return y, a
+
+
 def relaxed_online(h: np.ndarray, x0: np.ndarray, eps: np.ndarray, eps_scale: float = 0.1,
                    bf16: bool = False, n: int | None = None):
     """The same generation, computed in the order of the page's Algorithm 2.

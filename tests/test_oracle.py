@@ -329,3 +329,44 @@ def test_stream_error_definition():
 
 def test_oracle_header_marks_test_infrastructure():
     assert "TEST INFRASTRUCTURE ONLY" in oracle.__doc__
+
+
+# --------------------------------------------------------------------------- prompt (prefill)
+def test_prompt_single_layer_matches_numpy_convolve():
+    r = np.random.default_rng(31)
+    h = r.standard_normal((1, 3, 40))
+    x = r.standard_normal((3, 25))
+    y, a = oracle.prompt_lcsm(h, x)
+    for s in range(3):
+        assert np.allclose(y[0, s], np.convolve(h[0, s, :25], x[s])[:25], rtol=1e-12, atol=1e-12)
+    assert np.array_equal(a[0], x)
+
+
+def test_prompt_of_closed_loop_tokens_reproduces_the_closed_loop():
+    # Feeding a closed-loop trajectory's own tokens as a prompt gives back its
+    # outputs and activations (the online model is the prompt model on the
+    # tokens it generates).
+    r = np.random.default_rng(32)
+    M, S, L = 3, 4, 48
+    h = r.standard_normal((M, S, L)) * np.exp(-0.05 * np.arange(L))
+    x0 = r.standard_normal(S)
+    eps = r.standard_normal((L, S))
+    for bf16 in (False, True):
+        hh = oracle.bf16_round(h) if bf16 else h
+        y_ref, a_ref = oracle.online_lcsm(hh, x0, eps, 0.1, bf16)
+        y, a = oracle.prompt_lcsm(hh, a_ref[0], bf16)
+        assert np.allclose(y, y_ref, rtol=0, atol=1e-12)
+        assert np.allclose(a, a_ref, rtol=0, atol=1e-12)
+
+
+def test_prompt_identity_filter_is_iterated_tanh():
+    # h = delta: every layer's output is its own input, so y^l = tanh^(l-1)(x).
+    M, S, p = 4, 2, 10
+    h = np.zeros((M, S, 16))
+    h[:, :, 0] = 1.0
+    x = np.linspace(-2, 2, S * p).reshape(S, p)
+    y, _ = oracle.prompt_lcsm(h, x)
+    want = x.copy()
+    for l in range(M):
+        assert np.allclose(y[l], want, atol=1e-15)
+        want = np.tanh(want)

@@ -76,17 +76,25 @@ def test_noalloc_rejects_oversized_configuration(fi):
 
 @pytest.mark.gpu
 def test_noalloc_matches_oracle_closed_loop(fi):
-    # The tiny single-layer workload: short enough that the float64 oracle's own
-    # closed loop and the device's stay within the fp32 tolerance at every position.
-    w = synth.WORKLOADS["tiny-1x16-L1K"]
-    inp = gpu_inputs(w, 7)
-    h64 = oracle_filters(inp["h_np"], w.dtype)
+    # Closed loop against the float64 oracle's own closed loop. The feedback of
+    # the standard workloads is chaotic (rounding differences grow), so this case
+    # uses short, scaled-down filters (decay rates 0.1..0.5, taps x 0.1) whose
+    # loop gain is below one: differences stay at rounding level over all 1024
+    # positions (a relative perturbation of 1e-6 moves the oracle's output by
+    # 3e-6), and every position can be held to the fp32 tolerance.
+    w = synth.Workload("noalloc-contractive", 2, 16, 1024, 2, "f32", 0.1, 0.5)
+    h = (synth.filters(w, 9) * np.float32(0.1)).astype(np.float32)
+    x0 = synth.first_token(w, 9)
+    eps = synth.noise(w, 9)
     d_of = np.arange(w.streams) % w.channels
-    y_ref, _ = oracle.online_lcsm(h64[:, d_of, :], inp["x0_np"].reshape(-1),
-                                  inp["eps_np"].reshape(w.length, w.streams))
+    y_ref, _ = oracle.online_lcsm(h.astype(np.float64)[:, d_of, :], x0.reshape(-1).astype(np.float64),
+                                  eps.reshape(w.length, w.streams).astype(np.float64))
+    h_d = torch.from_numpy(h).cuda()
+    x0_d = torch.from_numpy(x0).cuda()
+    eps_d = torch.from_numpy(eps).cuda()
     for _ in range(2):
         y = torch.full((w.length, w.batch, w.channels), float("nan"), dtype=torch.float32, device="cuda")
-        fi.generate_noalloc(inp["h"], w.batch, w.length, inp["x0"], inp["eps"], y, w.dtype)
+        fi.generate_noalloc(h_d, w.batch, w.length, x0_d, eps_d, y, w.dtype)
         torch.cuda.synchronize()
         got = y.cpu().numpy().reshape(w.length, w.streams).T
         assert oracle.stream_error(got, y_ref[-1]) <= TOL["f32"]
