@@ -44,7 +44,6 @@ namespace fi {
 constexpr int kChunkMaxThreads = 512;
 constexpr int kChunkMaxStreams = 128;
 constexpr int kSuspendHintNs = 1000;   // longest a suspended barrier check may last
-constexpr int kLayersPerGroupMax = 12;  // most layers per barrier group
 
 struct ChunkShape {
   int G, GP, CH, LS, TPS, CW, GdMax, NG, K;
@@ -60,15 +59,13 @@ __host__ __device__ inline ChunkShape chunk_shape(const Dims& g, int CH, int G) 
   c.TPS = CH + 1;                  // odd tap stride: lanes of different channels hit different banks
   c.CW = (G + 31) / 32;            // chain warps (one stream per lane)
   c.GdMax = (G - 1) / g.B + 2;     // channels a run of G consecutive streams can touch
-  c.NG = (g.M + kLayersPerGroupMax - 1) / kLayersPerGroupMax;   // layer groups per position
-  if (c.NG < 2 && g.M >= 2) c.NG = 2;
-  c.K = (g.M + c.NG - 1) / c.NG;   // layers per group
-  c.NG = (g.M + c.K - 1) / c.K;
+  c.NG = 1;                        // one hand-off per position (both ways)
+  c.K = g.M;
   c.win = 0;
   c.tp = c.win + (size_t)(g.M + 1) * c.LS;
   c.ep = c.tp + (size_t)g.M * c.GdMax * c.TPS;
   c.flags = (c.ep + (size_t)CH * G + 1) & ~(size_t)1;   // 8-byte aligned mbarriers
-  c.total = c.flags + 2 * (size_t)(2 * c.NG) * c.CW;    // act_ready[NG][CW] + tile_done[NG][CW]
+  c.total = c.flags + 2 * (size_t)4 * c.CW;            // act_ready[2][CW] + tile_done[2][CW]
   return c;
 }
 
@@ -85,11 +82,11 @@ __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wai
 // ---------------------------------------------------------------------------
 // Step table: which on-chip block pieces run at which step (host-built).
 // ---------------------------------------------------------------------------
-enum PieceKind { PK_SQ1 = 0, PK_SQ2, PK_SQ4, PK_SQ8, PK_SQ16, PK_SQ32, PK_R8x4, PK_R16x4, PK_COUNT };
+enum PieceKind { PK_SQ1 = 0, PK_SQ2, PK_SQ4, PK_SQ8, PK_SQ16, PK_SQ32, PK_R8x4, PK_R16x4, PK_R16x2, PK_COUNT };
 __host__ __device__ constexpr int piece_ns(int k) {
-  return k == PK_R8x4 ? 8 : k == PK_R16x4 ? 16 : 1 << k;
+  return k == PK_R8x4 ? 8 : (k == PK_R16x4 || k == PK_R16x2) ? 16 : 1 << k;
 }
-__host__ __device__ constexpr int piece_nd(int k) { return k >= PK_R8x4 ? 4 : 1 << k; }
+__host__ __device__ constexpr int piece_nd(int k) { return k == PK_R16x2 ? 2 : k >= PK_R8x4 ? 4 : 1 << k; }
 __host__ __device__ inline uint32_t piece_encode(int step, int s_lo, int t_lo, int kind) {
   return (uint32_t)step | ((uint32_t)s_lo << 7) | ((uint32_t)t_lo << 14) | ((uint32_t)kind << 21);
 }
@@ -139,7 +136,8 @@ __device__ __forceinline__ void run_piece(uint32_t e, const float* src, float* d
     case PK_SQ16: block_piece<16, 16>(src, dst, taps, s_lo, t_lo, stride); break;
     case PK_SQ32: block_piece<32, 32>(src, dst, taps, s_lo, t_lo, stride); break;
     case PK_R8x4: block_piece<8, 4>(src, dst, taps, s_lo, t_lo, stride); break;
-    default: block_piece<16, 4>(src, dst, taps, s_lo, t_lo, stride); break;
+    case PK_R16x4: block_piece<16, 4>(src, dst, taps, s_lo, t_lo, stride); break;
+    default: block_piece<16, 2>(src, dst, taps, s_lo, t_lo, stride); break;
   }
 }
 
@@ -149,18 +147,50 @@ int kind_of_square(int U) { return U == 1 ? PK_SQ1 : U == 2 ? PK_SQ2 : U == 4 ? 
 
 struct Piece { int step, s_lo, t_lo, kind; };
 
-// The block of step r and side U, cut so that at most an 8 x 8 square runs at
-// step r itself (see the file comment).
-void cut_block(int r, int U, std::vector<Piece>& out) {
-  if (U <= 8) {
-    out.push_back({r, r - U, r, kind_of_square(U)});
+// The block of step r and side U (sources [r-U, r), targets from r + sh), cut
+// so that at most a 4 x 4 square is bound to step r itself (see the file
+// comment): with H = U/2, sources [r-U, r-H) to every target, sources [r-H, r)
+// to the targets past r+H+sh, and the square [r-H, r) x [r+sh, r+H+sh) cut
+// again. The other pieces get a step later (balance_pieces).
+void cut_block(int r, int U, int sh, std::vector<Piece>& out) {
+  if (U <= 4) {
+    out.push_back({r, r - U, r + sh, kind_of_square(U)});
     return;
   }
   const int H = U / 2;
-  const int kind = H == 8 ? PK_R8x4 : PK_R16x4;
-  for (int j = 0; j < U / 4; ++j) out.push_back({r - H + 1 + 2 * j, r - U, r + 4 * j, kind});
-  for (int j = 0; j < H / 4; ++j) out.push_back({r + 1 + 2 * j, r - H, r + H + 4 * j, kind});
-  cut_block(r, H, out);
+  const int kind = H == 16 ? PK_R16x2 : H == 8 ? PK_R8x4 : PK_SQ4;   // 32, 32, 16 products per row
+  const int nd = piece_nd(kind);
+  for (int t = r + sh; t < r + sh + U; t += nd) out.push_back({-1, r - U, t, kind});
+  for (int t = r + H + sh; t < r + U + sh; t += nd) out.push_back({-1, r - H, t, kind});
+  cut_block(r, H, sh, out);
+}
+
+// A piece reading sources [s_lo, s_lo+ns) and writing targets from t_lo may run
+// at any step k with s_lo + ns <= k <= t_lo - sh. Pieces with a step already
+// fixed keep it; each other piece, the tightest windows first, goes to the
+// least loaded step of its window (load = products per row plus a fixed cost
+// per piece), so every step carries about the same work.
+void balance_pieces(std::vector<Piece>& p, int CH, int sh) {
+  constexpr int kPieceCost = 8;
+  std::vector<int> load(CH + 1, 0);
+  for (const Piece& x : p)
+    if (x.step >= 0) load[x.step] += piece_ns(x.kind) * piece_nd(x.kind) + kPieceCost;
+  std::vector<Piece*> free_p;
+  for (Piece& x : p)
+    if (x.step < 0) free_p.push_back(&x);
+  auto lo = [](const Piece* x) { return x->s_lo + piece_ns(x->kind); };
+  auto hi = [&](const Piece* x) { return x->t_lo - sh; };
+  std::stable_sort(free_p.begin(), free_p.end(), [&](const Piece* a, const Piece* b) {
+    const int wa = hi(a) - lo(a), wb = hi(b) - lo(b);
+    return wa != wb ? wa < wb : lo(a) < lo(b);
+  });
+  for (Piece* x : free_p) {
+    int best = lo(x);
+    for (int k = lo(x); k <= hi(x) && k < CH; ++k)
+      if (load[k] < load[best]) best = k;
+    x->step = best;
+    load[best] += piece_ns(x->kind) * piece_nd(x->kind) + kPieceCost;
+  }
 }
 
 }  // namespace
@@ -170,14 +200,23 @@ int chunk_piece_targets(int kind) { return piece_nd(kind); }
 
 bool build_chunk_table(int CH, bool retimed, ChunkTable* tab) {
   std::vector<Piece> p;
+  const int sh = retimed ? 1 : 0;   // retimed: targets one position later (lag-1 terms in the chain)
   for (int r = 1; r < CH; ++r) {
     const int U = r & -r;
-    if (retimed && U >= 16 && U <= 32) cut_block(r, U, p);
-    else p.push_back({r, r - U, r, kind_of_square(U)});
+    std::vector<Piece> q;
+    if (retimed) cut_block(r, U, sh, q);
+    else q.push_back({r, r - U, r, kind_of_square(U)});
+    // pieces whose targets all lie past the chunk are dropped; one that reaches
+    // past it writes its last targets into the window's spare position (CH),
+    // which nothing reads
+    for (const Piece& x : q)
+      if (x.t_lo < CH) p.push_back(x);
   }
+  if (retimed) balance_pieces(p, CH, sh);
   if ((int)p.size() > kChunkMaxEntries) return false;
   std::stable_sort(p.begin(), p.end(), [](const Piece& a, const Piece& b) { return a.step < b.step; });
   tab->n = (int)p.size();
+  tab->lag1 = retimed ? 1 : 0;
   int k = 0;
   for (int r = 0; r <= kChunkMaxSteps; ++r) {
     while (k < tab->n && p[k].step < r) ++k;
@@ -318,9 +357,11 @@ __global__ void __launch_bounds__(kChunkMaxThreads) k_chunk(Dims g, ChunkArgs a,
   float* win = csm + cs.win;   // [(M+1)][CH+1][GP]   slot window of positions [c, c+CH]
   float* tp = csm + cs.tp;     // [M][GdMax][TPS]     taps h[0..CH)
   float* ep = csm + cs.ep;     // [CH][G]             sampler noise
-  uint64_t* act_ready = reinterpret_cast<uint64_t*>(csm + cs.flags);   // [NG][CW]
-  uint64_t* tile_done = act_ready + cs.NG * CW;                          // [NG][CW]
-  const int K = cs.K, NG = cs.NG;
+  // Double-buffered hand-off barriers (index = ordinal & 1): act_ready[k][c]
+  // completes when chain warp c has finished a position, tile_done[k][c] when
+  // every layer's pieces of a step are done for chain warp c's streams.
+  uint64_t* act_ready = reinterpret_cast<uint64_t*>(csm + cs.flags);   // [2][CW]
+  uint64_t* tile_done = act_ready + 2 * CW;                              // [2][CW]
   const int M = g.M;
   const int s0 = blockIdx.x * G;
   const int Gc = min(G, g.S - s0);
@@ -354,45 +395,51 @@ __global__ void __launch_bounds__(kChunkMaxThreads) k_chunk(Dims g, ChunkArgs a,
       tp[(l * GdMax + dl) * TPS + j] = a.taps[((size_t)l * g.D + d_lo + dl) * g.L + j];
     }
   } else {
-    const int vpr = CH >> 2;                          // float4 per (layer, stream) row
-    const int nwin = (M + 1) * Gc * vpr;
-    const int ntap = M * Gd * vpr;
+    // Items: float4 j (4 positions or taps) of row `row` (a stream, or a
+    // channel for the taps) of a layer, numbered with the rows padded to a
+    // power of two, so a thread finds its item with shifts alone. Each thread
+    // issues kBatch loads before storing any.
+    const int vpr = CH >> 2;                          // float4 per row
+    const int lv = 31 - __clz(vpr);
+    const int lw = lv + (Gc > 1 ? 32 - __clz(Gc - 1) : 0);   // log2 items per window layer
+    const int lt = lv + (Gd > 1 ? 32 - __clz(Gd - 1) : 0);   // log2 items per tap layer
+    const int nwin = (M + 1) << lw, nall = nwin + (M << lt);
     constexpr int kBatch = 12;
-    for (int base = tid; base < nwin + ntap; base += nt * kBatch) {
+    for (int base = tid; base < nall; base += nt * kBatch) {
       float4 v[kBatch];
 #pragma unroll
       for (int u = 0; u < kBatch; ++u) {
         const int idx = base + u * nt;
-        v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (idx < nwin) {
-          const int row = idx / vpr, j = idx - row * vpr;
-          const int l = row / Gc, gg = row - l * Gc;
-          // every slot of the window lies inside the state, so the load is
-          // always in bounds; slots holding nothing yet are zeroed below
-          v[u] = __ldg(reinterpret_cast<const float4*>(a.state + slot_index(g, l, s0 + gg, a.c + 4 * j)));
-        } else if (idx < nwin + ntap) {
-          const int k = idx - nwin;
-          const int row = k / vpr, j = k - row * vpr;
-          const int l = row / Gd, dl = row - l * Gd;
-          v[u] = __ldg(reinterpret_cast<const float4*>(a.taps + ((size_t)l * g.D + d_lo + dl) * g.L + 4 * j));
-        }
+        const bool is_win = idx < nwin;
+        const int k = is_win ? idx : idx - nwin;
+        const int sh = is_win ? lw : lt;
+        const int l = k >> sh, rem = k & ((1 << sh) - 1);
+        const int row = rem >> lv, j = rem & (vpr - 1);
+        // every slot of the window lies inside the state, so the load is in
+        // bounds; slots that hold nothing yet are zeroed below
+        if (idx < nall && row < (is_win ? Gc : Gd))
+          v[u] = __ldg(reinterpret_cast<const float4*>(
+              is_win ? a.state + slot_index(g, l, s0 + row, a.c + 4 * j)
+                     : a.taps + ((size_t)l * g.D + d_lo + row) * g.L + 4 * j));
       }
 #pragma unroll
       for (int u = 0; u < kBatch; ++u) {
         const int idx = base + u * nt;
-        if (idx < nwin) {
-          const int row = idx / vpr, j = idx - row * vpr;
-          const int l = row / Gc, gg = row - l * Gc;
+        const bool is_win = idx < nwin;
+        const int k = is_win ? idx : idx - nwin;
+        const int sh = is_win ? lw : lt;
+        const int l = k >> sh, rem = k & ((1 << sh) - 1);
+        const int row = rem >> lv, j = rem & (vpr - 1);
+        if (idx >= nall || row >= (is_win ? Gc : Gd)) continue;
+        if (is_win) {
           const int t = a.c + 4 * j;
-          float* w = win + l * LS + 4 * j * GP + gg;
+          float* w = win + l * LS + 4 * j * GP + row;
           w[0] = slot_valid(l, t) ? v[u].x : 0.f;
           w[GP] = slot_valid(l, t + 1) ? v[u].y : 0.f;
           w[2 * GP] = slot_valid(l, t + 2) ? v[u].z : 0.f;
           w[3 * GP] = slot_valid(l, t + 3) ? v[u].w : 0.f;
-        } else if (idx < nwin + ntap) {
-          const int k = idx - nwin;
-          const int row = k / vpr, j = k - row * vpr;
-          float* w = tp + row / Gd * GdMax * TPS + (row % Gd) * TPS + 4 * j;
+        } else {
+          float* w = tp + (l * GdMax + row) * TPS + 4 * j;
           w[0] = v[u].x;
           w[1] = v[u].y;
           w[2] = v[u].z;
@@ -415,16 +462,26 @@ __global__ void __launch_bounds__(kChunkMaxThreads) k_chunk(Dims g, ChunkArgs a,
     const int s = s0 + tid, d = s / g.B, b = s - d * g.B;
     win[r0 * GP + tid] = round_act(load_token(a.x0, (size_t)b * g.D + d, g.bf16), g.bf16);
   }
-  for (int k = tid; k < NG * CW; k += nt) {
-    const int grp = k / CW;
+  // tp[.][CH]: the tap one past the window, zero (pieces that reach the spare
+  // position read it)
+  for (int k = tid; k < M * GdMax; k += nt) tp[k * TPS + CH] = 0.f;
+  for (int k = tid; k < 2 * CW; k += nt) {
     mbar_init(act_ready + k, 32);
-    mbar_init(tile_done + k, 32 * (min(M, (grp + 1) * K) - grp * K));   // one arrival per lane per layer
+    mbar_init(tile_done + k, 32 * M);   // one arrival per lane per layer
   }
   cp_async_wait_all();
   __syncthreads();
 
   const int warp = tid >> 5, lane = tid & 31;
-  const int rs = r0 > 0 ? r0 : 1;   // first position of this launch with an on-chip gray block
+  // Hand-off. In the re-timed table (lag1) the chain adds every lag-1 term
+  // h^l[1] a^{l-1}_{t-1} itself and the pieces of step i (sources below i,
+  // targets from i+1) run while the chain is at position i, needed at position
+  // i+1: the tile warps have a whole position of slack. Otherwise (a launch
+  // over part of a chunk) the pieces of step i have targets from i and the
+  // chain at position i waits for them.
+  const bool lag1 = a.tab.lag1 != 0;
+  const int rs = r0 > 0 ? r0 : 1;                 // first tile step
+  const int s_last = lag1 ? CH - 2 : r1 - 1;      // last tile step
   int* err = a.err;
   bool ok = true;
   if (warp < CW) {
@@ -438,47 +495,44 @@ __global__ void __launch_bounds__(kChunkMaxThreads) k_chunk(Dims g, ChunkArgs a,
     const size_t c_io = (size_t)b * g.D + d;
     const size_t y_stride = g.S;
     float* wcol = win + gg;                          // slot (l, r) at wcol[l*LS + r*GP]
-    const float* hcol = tp + (d - d_lo) * TPS;       // h0 of layer l at hcol[(l-1)*HS]
+    const float* hcol = tp + (d - d_lo) * TPS;       // h^l[k] at hcol[(l-1)*HS + k]
     const int HS = GdMax * TPS;
-    // The tile_done barrier of (group, position) is tested one step ahead
-    // (halfway through the previous group) without blocking; a test that came
-    // back false is followed by a bounded wait when the group starts.
-    auto wait_group = [&](int grp, int r) {
-      if (r >= rs && ok) ok = mbar_wait(&tile_done[grp * CW + warp], (r - rs) & 1, err, true, a.wait_limit);
-    };
-    auto test_group = [&](int grp, int r) { return r < rs || mbar_test(&tile_done[grp * CW + warp], (r - rs) & 1); };
-
-    // layer 1 of the first position: the token itself
-    if (!test_group(0, r0)) wait_group(0, r0);
-    const float x_first = wcol[r0 * GP];
-    TanhParts P{0.f, x_first, true};   // the input of layer 1 as tanh parts (here: the token)
-    float xb = x_first;                // bf16 path: the token
-    float epsk = 0.f;                  // eps_scale * eps of the previous position (fp32 path)
-    float acc_n = wcol[LS + r0 * GP];  // operands of the next layer to enter
-    float h0_n = hcol[0];
-    bool ready = false;                // the barrier of the next group to enter has completed
+    float x_cur = wcol[r0 * GP];                     // token of the current position (first: as loaded)
+    TanhParts P{0.f, 0.f, true};
+    float epsk = 0.f;                                // eps_scale * eps of the previous position
+    bool from_parts = false;                         // layer 1's input is P (+ epsk), else x_cur
     for (int r = r0; r < r1; ++r) {
       const int t = a.c + r;
+      // the pieces this position needs (lag1: step r-1, else step r)
+      const int need = lag1 ? r - 1 : r;
+      if (need >= rs && need <= s_last && ok) {
+        const int j = need - rs;
+        ok = mbar_wait(&tile_done[(j & 1) * CW + warp], (j >> 1) & 1, err, true, a.wait_limit);
+      }
+      const bool use_lag1 = lag1 && r >= 1;
+      // operands of layer 1
+      float h0_n = hcol[0];
+      float acc_n = wcol[LS + r * GP];
+      if (use_lag1) acc_n = fmaf(hcol[1], wcol[(r - 1) * GP], acc_n);
       float y, z = 0.f;
-      if constexpr (BF16) y = fmaf(h0_n, xb, acc_n);
-      else next_input(P, h0_n, fmaf(h0_n, epsk, acc_n), y, z);
-      int grp = 0, lg_end = K;         // current group and its last layer
-      const int kmid = K / 2;
+      if (from_parts) {
+        if constexpr (BF16) y = fmaf(h0_n, x_cur, acc_n);
+        else next_input(P, h0_n, fmaf(h0_n, epsk, acc_n), y, z);
+      } else {
+        y = fmaf(h0_n, x_cur, acc_n);
+        z = kTwoLog2e * y;
+      }
       for (int l = 1;; ++l) {
         if constexpr (REC) if (act) a.rec[((size_t)(l - 1) * a.n_gen + (t - a.gen_base)) * y_stride + c_io] = y;
         if (l == M) break;
-        const bool boundary = l == lg_end;         // layer l closes its group
-        if (!boundary) {
-          // next layer's operands, issued before this layer's exp2/reciprocal so
-          // their latency hides behind them
-          acc_n = wcol[(l + 1) * LS + r * GP];
-          h0_n = hcol[l * HS];
-        }
-        if (l == grp * K + kmid) {
-          // halfway through the group: test the next one's barrier (group 0 of
-          // the next position after the last group)
-          const bool last = grp + 1 == NG;
-          ready = last ? (r + 1 >= r1 || test_group(0, r + 1)) : test_group(grp + 1, r);
+        // next layer's operands, issued before this layer's exp2/reciprocal so
+        // their latency hides behind them
+        h0_n = hcol[l * HS];
+        acc_n = wcol[(l + 1) * LS + r * GP];
+        float hp = 0.f, ap = 0.f;
+        if (use_lag1) {
+          hp = hcol[l * HS + 1];
+          ap = wcol[l * LS + (r - 1) * GP];
         }
         float av;
         if constexpr (BF16) {
@@ -488,37 +542,28 @@ __global__ void __launch_bounds__(kChunkMaxThreads) k_chunk(Dims g, ChunkArgs a,
           av = tanh_value(P);
         }
         if (act) wcol[l * LS + r * GP] = av;
-        if (boundary) {
-          // hand the group to the tile warps, then enter the next one
-          mbar_arrive(&act_ready[grp * CW + warp]);
-          ++grp;
-          lg_end = min(M, lg_end + K);
-          if (!ready) wait_group(grp, r);
-          ready = false;
-          acc_n = wcol[(l + 1) * LS + r * GP];
-          h0_n = hcol[l * HS];
-        }
+        acc_n = fmaf(hp, ap, acc_n);
         if constexpr (BF16) y = fmaf(h0_n, av, acc_n);
         else next_input(P, h0_n, acc_n, y, z);
       }
-      // y = y^M_t: output, then the sampler x_{t+1} = R(tanh(y) + eps_scale eps_t)
-      mbar_arrive(&act_ready[(NG - 1) * CW + warp]);
+      // y = y^M_t: hand the position to the tile warps, output, then the sampler
+      // x_{t+1} = R(tanh(y) + eps_scale eps_t)
+      {
+        const int jp = r - r0;
+        mbar_arrive(&act_ready[(jp & 1) * CW + warp]);
+      }
       if (act) a.y_out[(size_t)(t - a.gen_base) * y_stride + c_io] = y;
       const float epsv = ep[r * G + gg];
-      if (r + 1 < r1) {
-        if (!ready) wait_group(0, r + 1);
-        acc_n = wcol[LS + (r + 1) * GP];
-        h0_n = hcol[0];
-      }
-      ready = false;
       float xn;
       if constexpr (BF16) {
         xn = round_bf16(tanh_approx(y) + a.eps_scale * epsv);
-        xb = xn;
+        x_cur = xn;
       } else {
         P = tanh_parts(y, z);
         epsk = a.eps_scale * epsv;
         xn = tanh_value(P) + epsk;
+        x_cur = xn;
+        from_parts = true;
       }
       // x_{t+1}; for the last position of the chunk it lands in the spare
       // position CH and goes to HBM with the write-back.
@@ -540,12 +585,13 @@ __global__ void __launch_bounds__(kChunkMaxThreads) k_chunk(Dims g, ChunkArgs a,
         ++ntw;
       }
     if (is_tile(warp))
-      for (int r = rs; r < r1; ++r) {
-        const int e0 = a.tab.first[r], e1 = a.tab.first[r + 1];
+      for (int i = rs; i <= s_last; ++i) {
+        // step i reads sources below i: position i-1 must be finished
+        const int e0 = a.tab.first[i], e1 = a.tab.first[i + 1];
+        const int j = i - rs, jp = i - 1 - r0;
         for (int k = tw; k < M * CW; k += ntw) {
           const int l = k / CW + 1, c = k - (l - 1) * CW;
-          const int grp = (l - 1) / K;
-          if (r > r0 && ok) ok = mbar_wait(&act_ready[grp * CW + c], (r - 1 - r0) & 1, err, false, a.wait_limit);
+          if (jp >= 0 && ok) ok = mbar_wait(&act_ready[(jp & 1) * CW + c], (jp >> 1) & 1, err, false, a.wait_limit);
           const int gg = c * 32 + lane;
           if (gg < Gc) {
             const int dl = (s0 + gg) / g.B - d_lo;
@@ -554,7 +600,7 @@ __global__ void __launch_bounds__(kChunkMaxThreads) k_chunk(Dims g, ChunkArgs a,
             const float* taps = tp + ((l - 1) * GdMax + dl) * TPS;
             for (int e = e0; e < e1; ++e) run_piece(a.tab.e[e], src, dst, taps, GP);
           }
-          mbar_arrive(&tile_done[grp * CW + c]);
+          mbar_arrive(&tile_done[(j & 1) * CW + c]);
         }
       }
   }
@@ -567,33 +613,20 @@ __global__ void __launch_bounds__(kChunkMaxThreads) k_chunk(Dims g, ChunkArgs a,
   // nothing reads them again; its accumulators from p1 on are still needed.
   if (r1 == CH && a.c + CH < g.L && tid < Gc) a.state[slot_index(g, 0, s0 + tid, a.c + CH)] = win[CH * GP + tid];
   const int re = min(CH, g.L - a.c);
-  if (r0 == 0 && (re & 3) == 0) {
+  if (r0 == 0 && (re & 3) == 0 && (r1 & 3) == 0) {
+    // one warp per layer: layers 0..M-1 from position 0, layer M from p1
     const int vpr = re >> 2;
-    const int nrow_full = M * Gc;                       // layers 0..M-1 from position 0
-    const int nrow_last = (r1 & 3) == 0 ? Gc : 0;       // layer M from p1, when aligned
-    const int v_last = (re - r1) >> 2;
-    const int n1 = nrow_full * vpr, n2 = nrow_last * v_last;
-    for (int idx = tid; idx < n1 + n2; idx += nt) {
-      int l, gg, j;
-      if (idx < n1) {
-        const int row = idx / vpr;
-        j = idx - row * vpr;
-        l = row / Gc;
-        gg = row - l * Gc;
-      } else {
-        const int k = idx - n1;
-        gg = k / v_last;
-        j = (r1 >> 2) + (k - gg * v_last);
-        l = M;
-      }
-      const float* w = win + l * LS + 4 * j * GP + gg;
-      *reinterpret_cast<float4*>(a.state + slot_index(g, l, s0 + gg, a.c + 4 * j)) =
-          make_float4(w[0], w[GP], w[2 * GP], w[3 * GP]);
-    }
-    if (nrow_last == 0) {
-      for (int idx = tid; idx < Gc * (re - r1); idx += nt) {
-        const int gg = idx / (re - r1), r = r1 + idx % (re - r1);
-        a.state[slot_index(g, M, s0 + gg, a.c + r)] = win[M * LS + r * GP + gg];
+    const int lv = 31 - __clz(vpr);
+    const int wid = tid >> 5, lid = tid & 31, nw = nt >> 5;
+    for (int l = wid; l <= M; l += nw) {
+      const int j0 = l == M ? (r1 >> 2) : 0;
+      const int nk = Gc << lv;
+      for (int k = lid; k < nk; k += 32) {
+        const int row = k >> lv, j = k & (vpr - 1);
+        if (j < j0) continue;
+        const float* w = win + l * LS + 4 * j * GP + row;
+        *reinterpret_cast<float4*>(a.state + slot_index(g, l, s0 + row, a.c + 4 * j)) =
+            make_float4(w[0], w[GP], w[2 * GP], w[3 * GP]);
       }
     }
   } else {

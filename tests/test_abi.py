@@ -104,35 +104,45 @@ def test_python_binding_refuses_cpu_tensors():
 @pytest.mark.parametrize("chunk", [2, 4, 8, 16, 32, 64])
 @pytest.mark.parametrize("retimed", [False, True])
 def test_chunk_piece_table_covers_every_pair_once_in_time(chunk, retimed):
-    """The on-chip pieces of a chunk sum every (source s, target t) pair with
-    s < t inside the chunk exactly once; a piece at step r reads only sources
-    below r (final once position r-1 is done) and writes only targets >= r (the
-    chain reads target t after the pieces of step t); lags stay in 1..chunk-1
-    (the taps the kernel holds). The page's tiling (retimed=False) is one square
-    block of side lowbit(r) per step r; the re-timed one runs at most an 8 x 8
-    square plus pieces of at most 16 x 4 at any step."""
+    """The on-chip pieces of a chunk and the chain together sum every (source s,
+    target t) pair with s < t inside the chunk exactly once.
+
+    Page's tiling (retimed=False): one square block of side lowbit(r) per step r,
+    sources [r-U, r), targets [r, r+U); a piece at step r reads sources below r
+    (final once position r-1 is done) and writes targets >= r (the chain reads
+    target t after the pieces of step t).
+    Re-timed (the whole chunk in one launch): the chain adds the lag-1 pairs
+    (t-1, t) itself, and the pieces cover every pair with t - s >= 2 with the
+    page's tiling shifted by one target (the chain reads target t after the
+    pieces of step t-1, so a piece at step r writes targets >= r+1); a piece may
+    also reach the window's spare position t = chunk (never read). Lags stay in
+    1..chunk (tap `chunk` is held as zero); the re-timed pieces hold at most 32
+    products per row each and are spread so that no step carries more than 64."""
     from long_convolution_sequence_online_b200 import fi
     tab = fi.chunk_schedule(chunk, retimed)
+    sh = 1 if retimed else 0
     count = {}
     per_step = {}
     for step, s_lo, ns, t_lo, nd in tab:
         assert 1 <= step < chunk
         assert s_lo >= 0 and s_lo + ns <= step, (step, s_lo, ns)
-        assert t_lo >= step and t_lo + nd <= chunk, (step, t_lo, nd)
-        assert t_lo - (s_lo + ns - 1) >= 1 and (t_lo + nd - 1) - s_lo <= chunk - 1
+        assert t_lo >= step + sh and t_lo < chunk and t_lo + nd <= chunk + sh, (step, t_lo, nd)
+        assert t_lo - (s_lo + ns - 1) >= 1 + sh and (t_lo + nd - 1) - s_lo <= chunk
         per_step.setdefault(step, []).append((s_lo, ns, t_lo, nd))
         for s in range(s_lo, s_lo + ns):
-            for t in range(t_lo, t_lo + nd):
+            for t in range(t_lo, min(t_lo + nd, chunk)):
                 count[(s, t)] = count.get((s, t), 0) + 1
-    want = {(s, t) for t in range(chunk) for s in range(t)}
+    want = {(s, t) for t in range(chunk) for s in range(t) if t - s >= 1 + sh}
     assert set(count) == want
     assert all(v == 1 for v in count.values())
     assert [step for step, *_ in tab] == sorted(step for step, *_ in tab)
-    for r in range(1, chunk):
+    for r in range(1, chunk - sh):
         U = r & -r
-        pieces = per_step[r]
-        if not retimed or U <= 8:
-            assert (r - U, U, r, U) in pieces
-        if retimed:
-            assert max(ns * nd for _, ns, _, nd in pieces) <= 64
-            assert sum(ns * nd for _, ns, _, nd in pieces) <= 64 + 2 * 64
+        pieces = per_step.get(r, [])
+        if not retimed:
+            assert pieces == [(r - U, U, r, U)]
+        else:
+            if U <= 4 and r + 1 < chunk:
+                assert (r - U, U, r + 1, U) in pieces
+            assert max(ns * nd for _, ns, _, nd in pieces) <= 32
+            assert sum(ns * nd for _, ns, _, nd in pieces) <= 64
