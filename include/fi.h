@@ -191,6 +191,11 @@ FI_API fi_status fi_get_plan(const fi_ctx* ctx, int32_t* chunk, int32_t* fft_fro
 FI_API fi_status fi_profile(fi_ctx* ctx, int32_t enable);
 FI_API fi_status fi_profile_read(fi_ctx* ctx, int32_t counts[FI_NUM_KERNEL_CLASSES],
                           double ms[FI_NUM_KERNEL_CLASSES]);
+/* fi_profile_read, plus the block launches (direct, FFT, tensor-core) split by
+ * block side: side_counts[q] and side_ms[q] for side 2^q (either may be NULL). */
+FI_API fi_status fi_profile_read_sides(fi_ctx* ctx, int32_t counts[FI_NUM_KERNEL_CLASSES],
+                                       double ms[FI_NUM_KERNEL_CLASSES], int32_t side_counts[32],
+                                       double side_ms[32]);
 
 /* Release everything the context owns (synchronises its stream first). NULL is allowed. */
 FI_API fi_status fi_destroy(fi_ctx* ctx);
@@ -229,14 +234,17 @@ FI_API fi_status fi_debug_set_wait_limit(fi_ctx* ctx, int32_t limit);
 
 /* Test hook (host only, no device work): the table of on-chip block pieces the
  * chunk kernel runs for a chunk of `chunk` positions (a power of two, 2..64):
- * retimed != 0 gives the table of a launch that covers a whole chunk (blocks of
- * side 16 and 32 cut into pieces spread over neighbouring steps), 0 the page's
- * tiling (the block of step r, side lowbit(r), at step r). Writes up to `cap`
- * entries of 5 int32 (step, first source, sources, first target, targets;
- * positions relative to the chunk start) to out and the entry count to *count.
+ * retimed != 0 gives the table of a launch that covers a whole chunk (the chain
+ * adds the terms of the first *chain_lags lags itself; the page's tiling of the
+ * other pairs is shifted that many positions later, and its blocks are cut into
+ * pieces spread over steps), 0 the page's tiling (the block of step r, side
+ * lowbit(r), at step r; *chain_lags = 0). Writes up to `cap` entries of 5 int32
+ * (step, first source, sources, first target, targets; positions relative to
+ * the chunk start) to out, the entry count to *count, the lags to *chain_lags
+ * (may be NULL).
  * Errors: FI_E_INVALID (NULL, chunk). */
 FI_API fi_status fi_debug_chunk_schedule(int32_t chunk, int32_t retimed, int32_t* out, int32_t cap,
-                                         int32_t* count);
+                                         int32_t* count, int32_t* chain_lags);
 
 /* Test hook: run the library's device FFT (the one its FFT blocks use) on
  * `count` complex sequences of length 2^log2n (6 <= log2n <= 14), interleaved

@@ -34,6 +34,7 @@ fi_status cuda_fail(cudaError_t e, const char* what) {
 struct EventPair {
   cudaEvent_t a, b;
   int cls;
+  int side_q;   // log2 of the block side for block launches, else -1
 };
 
 }  // namespace
@@ -106,7 +107,7 @@ fi_status dev_alloc(void** p, size_t bytes, const char* what) {
 
 // Kernel launch wrapped in profiling events when enabled.
 template <class F>
-fi_status timed(fi_ctx* c, int cls, F&& launch, const char* what) {
+fi_status timed(fi_ctx* c, int cls, F&& launch, const char* what, int side_q = -1) {
   EventPair ep{};
   if (c->prof) {
     if (!c->ev_free.empty()) {
@@ -117,6 +118,7 @@ fi_status timed(fi_ctx* c, int cls, F&& launch, const char* what) {
       FI_CUDA(cudaEventCreate(&ep.b), "cudaEventCreate");
     }
     ep.cls = cls;
+    ep.side_q = side_q;
     FI_CUDA(cudaEventRecord(ep.a, c->st), "cudaEventRecord");
   }
   cudaError_t e = launch();
@@ -140,20 +142,20 @@ fi_status run_block(fi_ctx* c, int i, int t_min = 0) {
                    return launch_part_block(c->g, c->state, c->part_xs, c->spectra + c->spec_off[q], c->twiddle, i,
                                             t_min, c->st);
                  },
-                 "partitioned FFT block launch");
+                 "partitioned FFT block launch", q);
   }
   if (q >= kMinFftLog2 && q <= c->tc_q_hi && t_min <= i) {
     return timed(c, KC_TC,
                  [&] { return launch_tile_tc(c->g, c->state, c->taps, c->tc[q], i, c->err, c->wait_limit, c->st); },
-                 "tensor-core block launch");
+                 "tensor-core block launch", q);
   }
   if (q >= c->q_lo && q <= c->q_hi) {
     return timed(c, KC_FFT,
                  [&] { return launch_tile_fft(c->g, c->state, c->spectra + c->spec_off[q], c->twiddle, i, t_min, c->st); },
-                 "FFT block launch");
+                 "FFT block launch", q);
   }
   return timed(c, KC_DIRECT, [&] { return launch_tile_direct(c->g, c->state, c->taps, i, t_min, c->st); },
-               "direct block launch");
+               "direct block launch", q);
 }
 
 // Synchronise the context's stream and report a device-side wait that gave up.
@@ -519,29 +521,44 @@ fi_status fi_profile(fi_ctx* c, int32_t enable) {
 }
 
 fi_status fi_profile_read(fi_ctx* c, int32_t counts[FI_NUM_KERNEL_CLASSES], double ms[FI_NUM_KERNEL_CLASSES]) {
+  return fi_profile_read_sides(c, counts, ms, nullptr, nullptr);
+}
+
+fi_status fi_profile_read_sides(fi_ctx* c, int32_t counts[FI_NUM_KERNEL_CLASSES], double ms[FI_NUM_KERNEL_CLASSES],
+                                int32_t side_counts[32], double side_ms[32]) {
   if (!c || !counts || !ms) return fail(FI_E_INVALID, "NULL argument");
   FI_CUDA(cudaStreamSynchronize(c->st), "profile synchronize");
   for (int k = 0; k < FI_NUM_KERNEL_CLASSES; ++k) {
     counts[k] = 0;
     ms[k] = 0.0;
   }
+  for (int k = 0; k < 32; ++k) {
+    if (side_counts) side_counts[k] = 0;
+    if (side_ms) side_ms[k] = 0.0;
+  }
   for (auto& e : c->ev_live) {
     float t = 0.f;
     FI_CUDA(cudaEventElapsedTime(&t, e.a, e.b), "cudaEventElapsedTime");
     counts[e.cls] += 1;
     ms[e.cls] += t;
+    if (e.side_q >= 0 && e.side_q < 32) {
+      if (side_counts) side_counts[e.side_q] += 1;
+      if (side_ms) side_ms[e.side_q] += t;
+    }
     c->ev_free.push_back(e);
   }
   c->ev_live.clear();
   return FI_OK;
 }
 
-fi_status fi_debug_chunk_schedule(int32_t chunk, int32_t retimed, int32_t* out, int32_t cap, int32_t* count) {
+fi_status fi_debug_chunk_schedule(int32_t chunk, int32_t retimed, int32_t* out, int32_t cap, int32_t* count,
+                                  int32_t* chain_lags) {
   if (!out || !count || cap < 0) return fail(FI_E_INVALID, "bad argument");
   if (!pow2(chunk) || chunk < 2 || chunk > kChunkMaxSteps) return fail(FI_E_INVALID, "chunk must be a power of two in [2, 64]");
   ChunkTable tab{};
   if (!build_chunk_table(chunk, retimed != 0, &tab)) return fail(FI_E_UNSUPPORTED, "table too long");
   *count = tab.n;
+  if (chain_lags) *chain_lags = tab.lag1;
   for (int j = 0; j < tab.n && j < cap; ++j) {
     const uint32_t e = tab.e[j];
     const int kind = (int)((e >> 21) & 15);

@@ -101,17 +101,18 @@ cudaError_t launch_tile_tc(const Dims& g, float* state, const float* taps, const
 // step | s_lo << 7 | t_lo << 14 | kind << 21 (sources [s_lo, s_lo+ns) to
 // targets [t_lo, t_lo+nd), positions relative to the chunk start).
 constexpr int kChunkMaxSteps = 64;
+constexpr int kChainLags = 2;   // re-timed chunks: lags the chain adds itself (pieces take the rest)
 constexpr int kChunkMaxEntries = 192;
 struct ChunkTable {
   int n;
-  int lag1;      // 1: the chain adds every lag-1 term itself, pieces cover lags >= 2
+  int lag1;      // lags 1..lag1 are added by the chain itself (0 or kChainLags); pieces cover the rest
   uint16_t first[kChunkMaxSteps + 1];
   uint32_t e[kChunkMaxEntries];
 };
-// retimed = the whole chunk runs in one launch: the chain takes the lag-1 terms,
-// the page's tiling of the remaining pairs runs one position ahead (its targets
-// shifted by one), with blocks of side 16 and 32 cut into pieces spread over
-// neighbouring steps; else the page's blocks, one per step.
+// retimed = the whole chunk runs in one launch: the chain takes the terms of
+// lags 1..kChainLags, the page's tiling of the remaining pairs runs kChainLags
+// positions ahead (its targets shifted by kChainLags), with blocks of side 8 and
+// up cut into pieces spread over steps; else the page's blocks, one per step.
 bool build_chunk_table(int chunk, bool retimed, ChunkTable* tab);
 // Sources and targets of a piece kind (for the table's test hook).
 int chunk_piece_sources(int kind);

@@ -44,6 +44,7 @@ namespace fi {
 constexpr int kChunkMaxThreads = 512;
 constexpr int kChunkMaxStreams = 128;
 constexpr int kSuspendHintNs = 1000;   // longest a suspended barrier check may last
+constexpr int kRing = 4;                // depth of the hand-off barrier rings
 
 struct ChunkShape {
   int G, GP, CH, LS, TPS, CW, GdMax, NG, K;
@@ -55,8 +56,10 @@ __host__ __device__ inline ChunkShape chunk_shape(const Dims& g, int CH, int G) 
   c.G = G;
   c.GP = G | 1;                    // odd: the prologue's transposing stores spread over banks
   c.CH = CH;
-  c.LS = (CH + 1) * c.GP;          // floats per layer (one spare position for the next chunk's token)
-  c.TPS = CH + 1;                  // odd tap stride: lanes of different channels hit different banks
+  // floats per layer: the chunk's positions plus kChainLags spare ones (the next
+  // chunk's token, and targets of pieces that reach past the chunk)
+  c.LS = (CH + kChainLags) * c.GP;
+  c.TPS = (CH + kChainLags) | 1;   // odd tap stride: lanes of different channels hit different banks
   c.CW = (G + 31) / 32;            // chain warps (one stream per lane)
   c.GdMax = (G - 1) / g.B + 2;     // channels a run of G consecutive streams can touch
   c.NG = 1;                        // one hand-off per position (both ways)
@@ -65,7 +68,7 @@ __host__ __device__ inline ChunkShape chunk_shape(const Dims& g, int CH, int G) 
   c.tp = c.win + (size_t)(g.M + 1) * c.LS;
   c.ep = c.tp + (size_t)g.M * c.GdMax * c.TPS;
   c.flags = (c.ep + (size_t)CH * G + 1) & ~(size_t)1;   // 8-byte aligned mbarriers
-  c.total = c.flags + 2 * (size_t)4 * c.CW;            // act_ready[2][CW] + tile_done[2][CW]
+  c.total = c.flags + 2 * (size_t)(2 * kRing) * c.CW;  // act_ready[kRing][CW] + tile_done[kRing][CW]
   return c;
 }
 
@@ -126,6 +129,74 @@ __device__ __forceinline__ void block_piece(const float* __restrict__ src, float
   }
 }
 
+__device__ __forceinline__ void run_piece(uint32_t e, const float* src, float* dst, const float* taps, int stride);
+
+// The same piece for two rows (two layers of one stream) at once: two
+// independent FMA chains per output group, so a warp with two rows pays the
+// latency of one.
+template <int NS, int ND>
+__device__ __forceinline__ void block_piece2(const float* __restrict__ srcA, float* __restrict__ dstA,
+                                             const float* __restrict__ tapsA, const float* __restrict__ srcB,
+                                             float* __restrict__ dstB, const float* __restrict__ tapsB, int s_lo,
+                                             int t_lo, int stride) {
+  constexpr int OB = ND < 8 ? ND : 8;
+  const float* xA = srcA + s_lo * stride;
+  const float* xB = srcB + s_lo * stride;
+#pragma unroll
+  for (int o0 = 0; o0 < ND; o0 += OB) {
+    const int lag0 = t_lo + o0 - s_lo;
+    float accA[OB], wA[OB], accB[OB], wB[OB];
+#pragma unroll
+    for (int k = 0; k < OB; ++k) {
+      accA[k] = 0.f;
+      accB[k] = 0.f;
+      wA[k] = tapsA[lag0 + k];
+      wB[k] = tapsB[lag0 + k];
+    }
+#pragma unroll
+    for (int u = 0; u < NS; ++u) {
+      const float xa = xA[u * stride], xb = xB[u * stride];
+#pragma unroll
+      for (int k = 0; k < OB; ++k) {
+        accA[k] = fmaf(wA[k], xa, accA[k]);
+        accB[k] = fmaf(wB[k], xb, accB[k]);
+      }
+      if (u + 1 < NS) {
+#pragma unroll
+        for (int k = OB - 1; k > 0; --k) {
+          wA[k] = wA[k - 1];
+          wB[k] = wB[k - 1];
+        }
+        wA[0] = tapsA[lag0 - u - 1];
+        wB[0] = tapsB[lag0 - u - 1];
+      }
+    }
+    float* outA = dstA + (t_lo + o0) * stride;
+    float* outB = dstB + (t_lo + o0) * stride;
+#pragma unroll
+    for (int k = 0; k < OB; ++k) {
+      outA[k * stride] += accA[k];
+      outB[k * stride] += accB[k];
+    }
+  }
+}
+
+__device__ __forceinline__ void run_piece2(uint32_t e, const float* srcA, float* dstA, const float* tapsA,
+                                           const float* srcB, float* dstB, const float* tapsB, int stride) {
+  const int s_lo = (e >> 7) & 127, t_lo = (e >> 14) & 127;
+  switch ((e >> 21) & 15) {
+    case PK_SQ1: block_piece2<1, 1>(srcA, dstA, tapsA, srcB, dstB, tapsB, s_lo, t_lo, stride); break;
+    case PK_SQ2: block_piece2<2, 2>(srcA, dstA, tapsA, srcB, dstB, tapsB, s_lo, t_lo, stride); break;
+    case PK_SQ4: block_piece2<4, 4>(srcA, dstA, tapsA, srcB, dstB, tapsB, s_lo, t_lo, stride); break;
+    case PK_R8x4: block_piece2<8, 4>(srcA, dstA, tapsA, srcB, dstB, tapsB, s_lo, t_lo, stride); break;
+    case PK_R16x2: block_piece2<16, 2>(srcA, dstA, tapsA, srcB, dstB, tapsB, s_lo, t_lo, stride); break;
+    default:   // kinds only the one-row path uses (page's tiling of a partial chunk)
+      run_piece(e, srcA, dstA, tapsA, stride);
+      run_piece(e, srcB, dstB, tapsB, stride);
+      break;
+  }
+}
+
 __device__ __forceinline__ void run_piece(uint32_t e, const float* src, float* dst, const float* taps, int stride) {
   const int s_lo = (e >> 7) & 127, t_lo = (e >> 14) & 127;
   switch ((e >> 21) & 15) {
@@ -172,7 +243,7 @@ void cut_block(int r, int U, int sh, std::vector<Piece>& out) {
 // per piece), so every step carries about the same work.
 void balance_pieces(std::vector<Piece>& p, int CH, int sh) {
   constexpr int kPieceCost = 8;
-  std::vector<int> load(CH + 1, 0);
+  std::vector<int> load(CH + kChainLags, 0);
   for (const Piece& x : p)
     if (x.step >= 0) load[x.step] += piece_ns(x.kind) * piece_nd(x.kind) + kPieceCost;
   std::vector<Piece*> free_p;
@@ -200,15 +271,15 @@ int chunk_piece_targets(int kind) { return piece_nd(kind); }
 
 bool build_chunk_table(int CH, bool retimed, ChunkTable* tab) {
   std::vector<Piece> p;
-  const int sh = retimed ? 1 : 0;   // retimed: targets one position later (lag-1 terms in the chain)
+  const int sh = retimed ? kChainLags : 0;   // retimed: the chain takes lags 1..sh, pieces the rest
   for (int r = 1; r < CH; ++r) {
     const int U = r & -r;
     std::vector<Piece> q;
     if (retimed) cut_block(r, U, sh, q);
     else q.push_back({r, r - U, r, kind_of_square(U)});
     // pieces whose targets all lie past the chunk are dropped; one that reaches
-    // past it writes its last targets into the window's spare position (CH),
-    // which nothing reads
+    // past it writes its last targets into the window's spare positions (CH and
+    // up), which nothing reads
     for (const Piece& x : q)
       if (x.t_lo < CH) p.push_back(x);
   }
@@ -216,7 +287,7 @@ bool build_chunk_table(int CH, bool retimed, ChunkTable* tab) {
   if ((int)p.size() > kChunkMaxEntries) return false;
   std::stable_sort(p.begin(), p.end(), [](const Piece& a, const Piece& b) { return a.step < b.step; });
   tab->n = (int)p.size();
-  tab->lag1 = retimed ? 1 : 0;
+  tab->lag1 = sh;
   int k = 0;
   for (int r = 0; r <= kChunkMaxSteps; ++r) {
     while (k < tab->n && p[k].step < r) ++k;
@@ -355,13 +426,16 @@ __global__ void __launch_bounds__(kChunkMaxThreads) k_chunk(Dims g, ChunkArgs a,
   const ChunkShape cs = chunk_shape(g, a.chunk, G);
   const int CH = cs.CH, GP = cs.GP, LS = cs.LS, TPS = cs.TPS, GdMax = cs.GdMax, CW = cs.CW;
   float* win = csm + cs.win;   // [(M+1)][CH+1][GP]   slot window of positions [c, c+CH]
-  float* tp = csm + cs.tp;     // [M][GdMax][TPS]     taps h[0..CH)
+  float* tp = csm + cs.tp;     // [M][GdMax][TPS]     taps h[0..CH), zero above
   float* ep = csm + cs.ep;     // [CH][G]             sampler noise
-  // Double-buffered hand-off barriers (index = ordinal & 1): act_ready[k][c]
-  // completes when chain warp c has finished a position, tile_done[k][c] when
-  // every layer's pieces of a step are done for chain warp c's streams.
-  uint64_t* act_ready = reinterpret_cast<uint64_t*>(csm + cs.flags);   // [2][CW]
-  uint64_t* tile_done = act_ready + 2 * CW;                              // [2][CW]
+  // Hand-off barrier rings (ordinal o uses slot o % kRing, phase parity
+  // (o / kRing) & 1): act_ready[k][c] completes when chain warp c has finished a
+  // position, tile_done[k][c] when every layer's pieces of a step are done for
+  // chain warp c's streams. The chain runs at most kChainLags + 1 positions
+  // ahead of the tile warps and they at most one step ahead of it, so a ring
+  // slot never gets two phases ahead of its waiters.
+  uint64_t* act_ready = reinterpret_cast<uint64_t*>(csm + cs.flags);   // [kRing][CW]
+  uint64_t* tile_done = act_ready + kRing * CW;                          // [kRing][CW]
   const int M = g.M;
   const int s0 = blockIdx.x * G;
   const int Gc = min(G, g.S - s0);
@@ -464,8 +538,8 @@ __global__ void __launch_bounds__(kChunkMaxThreads) k_chunk(Dims g, ChunkArgs a,
   }
   // tp[.][CH]: the tap one past the window, zero (pieces that reach the spare
   // position read it)
-  for (int k = tid; k < M * GdMax; k += nt) tp[k * TPS + CH] = 0.f;
-  for (int k = tid; k < 2 * CW; k += nt) {
+  for (int k = tid; k < M * GdMax * (TPS - CH); k += nt) tp[(k / (TPS - CH)) * TPS + CH + k % (TPS - CH)] = 0.f;
+  for (int k = tid; k < kRing * CW; k += nt) {
     mbar_init(act_ready + k, 32);
     mbar_init(tile_done + k, 32 * M);   // one arrival per lane per layer
   }
@@ -473,15 +547,15 @@ __global__ void __launch_bounds__(kChunkMaxThreads) k_chunk(Dims g, ChunkArgs a,
   __syncthreads();
 
   const int warp = tid >> 5, lane = tid & 31;
-  // Hand-off. In the re-timed table (lag1) the chain adds every lag-1 term
-  // h^l[1] a^{l-1}_{t-1} itself and the pieces of step i (sources below i,
-  // targets from i+1) run while the chain is at position i, needed at position
-  // i+1: the tile warps have a whole position of slack. Otherwise (a launch
-  // over part of a chunk) the pieces of step i have targets from i and the
-  // chain at position i waits for them.
-  const bool lag1 = a.tab.lag1 != 0;
+  // Hand-off. In the re-timed table the chain adds the terms of lags
+  // 1..nlag (h^l[k] a^{l-1}_{t-k}) itself and the pieces of step i (sources
+  // below i, targets from i+nlag) run while the chain is at positions i..,
+  // needed at position i+nlag: the tile warps have nlag positions of slack.
+  // Otherwise (a launch over part of a chunk, nlag = 0) the pieces of step i
+  // have targets from i and the chain at position i waits for them.
+  const int nlag = a.tab.lag1;
   const int rs = r0 > 0 ? r0 : 1;                 // first tile step
-  const int s_last = lag1 ? CH - 2 : r1 - 1;      // last tile step
+  const int s_last = nlag ? CH - 1 - nlag : r1 - 1;   // last tile step
   int* err = a.err;
   bool ok = true;
   if (warp < CW) {
@@ -503,37 +577,45 @@ __global__ void __launch_bounds__(kChunkMaxThreads) k_chunk(Dims g, ChunkArgs a,
     bool from_parts = false;                         // layer 1's input is P (+ epsk), else x_cur
     for (int r = r0; r < r1; ++r) {
       const int t = a.c + r;
-      // the pieces this position needs (lag1: step r-1, else step r)
-      const int need = lag1 ? r - 1 : r;
+      // the pieces this position needs: step r - nlag
+      const int need = r - nlag;
       if (need >= rs && need <= s_last && ok) {
         const int j = need - rs;
-        ok = mbar_wait(&tile_done[(j & 1) * CW + warp], (j >> 1) & 1, err, true, a.wait_limit);
+        ok = mbar_wait(&tile_done[(j % kRing) * CW + warp], (j / kRing) & 1, err, true, a.wait_limit);
       }
-      const bool use_lag1 = lag1 && r >= 1;
-      // operands of layer 1
-      float h0_n = hcol[0];
-      float acc_n = wcol[LS + r * GP];
-      if (use_lag1) acc_n = fmaf(hcol[1], wcol[(r - 1) * GP], acc_n);
+      // lags the chain adds here (sources inside the chunk: earlier ones came
+      // with the blocks from HBM)
+      const int nl = min(nlag, r);
+      // Operands of layer m at this position: h^m[0] and the accumulator, plus
+      // the lag terms h^m[k] a^{m-1}_{r-k}. They are loaded two layers ahead of
+      // use, so their latency hides behind two exp2/reciprocal chains.
+      struct Ops { float h0, acc, h1, a1, h2, a2; };
+      auto load_ops = [&](int m, Ops& o) {
+        const float* hm = hcol + (m - 1) * HS;
+        const float* am = wcol + (m - 1) * LS;
+        o.h0 = hm[0];
+        o.acc = wcol[m * LS + r * GP];
+        o.h1 = 0.f; o.a1 = 0.f; o.h2 = 0.f; o.a2 = 0.f;
+        if (nl >= 1) { o.h1 = hm[1]; o.a1 = am[(r - 1) * GP]; }
+        if (nl >= 2) { o.h2 = hm[2]; o.a2 = am[(r - 2) * GP]; }
+      };
+      auto acc_of = [](const Ops& o) { return fmaf(o.h2, o.a2, fmaf(o.h1, o.a1, o.acc)); };
+      Ops cur, nxt;
+      load_ops(1, cur);
+      if (M >= 2) load_ops(2, nxt);
       float y, z = 0.f;
       if (from_parts) {
-        if constexpr (BF16) y = fmaf(h0_n, x_cur, acc_n);
-        else next_input(P, h0_n, fmaf(h0_n, epsk, acc_n), y, z);
+        if constexpr (BF16) y = fmaf(cur.h0, x_cur, acc_of(cur));
+        else next_input(P, cur.h0, fmaf(cur.h0, epsk, acc_of(cur)), y, z);
       } else {
-        y = fmaf(h0_n, x_cur, acc_n);
+        y = fmaf(cur.h0, x_cur, acc_of(cur));
         z = kTwoLog2e * y;
       }
+      cur = nxt;                                   // operands of layer 2
       for (int l = 1;; ++l) {
         if constexpr (REC) if (act) a.rec[((size_t)(l - 1) * a.n_gen + (t - a.gen_base)) * y_stride + c_io] = y;
         if (l == M) break;
-        // next layer's operands, issued before this layer's exp2/reciprocal so
-        // their latency hides behind them
-        h0_n = hcol[l * HS];
-        acc_n = wcol[(l + 1) * LS + r * GP];
-        float hp = 0.f, ap = 0.f;
-        if (use_lag1) {
-          hp = hcol[l * HS + 1];
-          ap = wcol[l * LS + (r - 1) * GP];
-        }
+        if (l + 2 <= M) load_ops(l + 2, nxt);     // two layers ahead
         float av;
         if constexpr (BF16) {
           av = round_bf16(tanh_approx(y));
@@ -542,15 +624,15 @@ __global__ void __launch_bounds__(kChunkMaxThreads) k_chunk(Dims g, ChunkArgs a,
           av = tanh_value(P);
         }
         if (act) wcol[l * LS + r * GP] = av;
-        acc_n = fmaf(hp, ap, acc_n);
-        if constexpr (BF16) y = fmaf(h0_n, av, acc_n);
-        else next_input(P, h0_n, acc_n, y, z);
+        if constexpr (BF16) y = fmaf(cur.h0, av, acc_of(cur));
+        else next_input(P, cur.h0, acc_of(cur), y, z);
+        cur = nxt;
       }
       // y = y^M_t: hand the position to the tile warps, output, then the sampler
       // x_{t+1} = R(tanh(y) + eps_scale eps_t)
       {
         const int jp = r - r0;
-        mbar_arrive(&act_ready[(jp & 1) * CW + warp]);
+        mbar_arrive(&act_ready[(jp % kRing) * CW + warp]);
       }
       if (act) a.y_out[(size_t)(t - a.gen_base) * y_stride + c_io] = y;
       const float epsv = ep[r * G + gg];
@@ -589,18 +671,46 @@ __global__ void __launch_bounds__(kChunkMaxThreads) k_chunk(Dims g, ChunkArgs a,
         // step i reads sources below i: position i-1 must be finished
         const int e0 = a.tab.first[i], e1 = a.tab.first[i + 1];
         const int j = i - rs, jp = i - 1 - r0;
-        for (int k = tw; k < M * CW; k += ntw) {
+        // row groups k (layer k / CW + 1, chain warp k % CW), two at a time when
+        // they belong to the same chain warp
+        for (int k = tw; k < M * CW; k += 2 * ntw) {
+          const int kB = k + ntw;
           const int l = k / CW + 1, c = k - (l - 1) * CW;
-          if (jp >= 0 && ok) ok = mbar_wait(&act_ready[(jp & 1) * CW + c], (jp >> 1) & 1, err, false, a.wait_limit);
+          const bool two = kB < M * CW && kB % CW == c;
+          const int lB = two ? kB / CW + 1 : l;
+          if (jp >= 0 && ok) ok = mbar_wait(&act_ready[(jp % kRing) * CW + c], (jp / kRing) & 1, err, false, a.wait_limit);
           const int gg = c * 32 + lane;
           if (gg < Gc) {
             const int dl = (s0 + gg) / g.B - d_lo;
             const float* src = win + (l - 1) * LS + gg;
             float* dst = win + l * LS + gg;
             const float* taps = tp + ((l - 1) * GdMax + dl) * TPS;
-            for (int e = e0; e < e1; ++e) run_piece(a.tab.e[e], src, dst, taps, GP);
+            if (two) {
+              const float* srcB = win + (lB - 1) * LS + gg;
+              float* dstB = win + lB * LS + gg;
+              const float* tapsB = tp + ((lB - 1) * GdMax + dl) * TPS;
+              for (int e = e0; e < e1; ++e) run_piece2(a.tab.e[e], src, dst, taps, srcB, dstB, tapsB, GP);
+            } else {
+              for (int e = e0; e < e1; ++e) run_piece(a.tab.e[e], src, dst, taps, GP);
+            }
           }
-          mbar_arrive(&tile_done[(j & 1) * CW + c]);
+          mbar_arrive(&tile_done[(j % kRing) * CW + c]);
+          if (two) mbar_arrive(&tile_done[(j % kRing) * CW + c]);
+          else if (kB < M * CW) {
+            // the second row group belongs to another chain warp: on its own
+            const int lb = kB / CW + 1, cb = kB - (lb - 1) * CW;
+            if (jp >= 0 && ok)
+              ok = mbar_wait(&act_ready[(jp % kRing) * CW + cb], (jp / kRing) & 1, err, false, a.wait_limit);
+            const int ggb = cb * 32 + lane;
+            if (ggb < Gc) {
+              const int dlb = (s0 + ggb) / g.B - d_lo;
+              const float* srcb = win + (lb - 1) * LS + ggb;
+              float* dstb = win + lb * LS + ggb;
+              const float* tapsb = tp + ((lb - 1) * GdMax + dlb) * TPS;
+              for (int e = e0; e < e1; ++e) run_piece(a.tab.e[e], srcb, dstb, tapsb, GP);
+            }
+            mbar_arrive(&tile_done[(j % kRing) * CW + cb]);
+          }
         }
       }
   }

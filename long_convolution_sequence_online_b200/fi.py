@@ -22,7 +22,7 @@ KERNEL_CLASSES = ("chunk", "direct", "fft", "token", "lazy", "tc")
 EXPORTED = ("fi_init", "fi_step", "fi_generate", "fi_generate_host", "fi_generate_lazy", "fi_sync", "fi_reset",
             "fi_position", "fi_read_activations", "fi_set_stream", "fi_get_plan", "fi_profile",
             "fi_profile_read", "fi_destroy", "fi_status_str", "fi_last_error", "fi_debug_fft",
-            "fi_generate_noalloc", "fi_debug_set_wait_limit", "fi_debug_chunk_schedule", "fi_prefill")
+            "fi_generate_noalloc", "fi_debug_set_wait_limit", "fi_debug_chunk_schedule", "fi_prefill", "fi_profile_read_sides")
 
 
 class FiError(RuntimeError):
@@ -61,8 +61,10 @@ def _load():
         "fi_debug_fft": [i32, i32, vp, vp, i32, vp],
         "fi_generate_noalloc": [ctypes.POINTER(Config), vp, i32, vp, vp, f32, vp, vp],
         "fi_debug_set_wait_limit": [vp, i32],
-        "fi_debug_chunk_schedule": [i32, i32, vp, i32, ctypes.POINTER(i32)],
+        "fi_debug_chunk_schedule": [i32, i32, vp, i32, ctypes.POINTER(i32), ctypes.POINTER(i32)],
         "fi_prefill": [vp, i32, vp, vp, vp],
+        "fi_profile_read_sides": [vp, ctypes.POINTER(i32), ctypes.POINTER(ctypes.c_double), ctypes.POINTER(i32),
+                                  ctypes.POINTER(ctypes.c_double)],
     }
     for name, args in sig.items():
         fn = getattr(lib, name)
@@ -198,6 +200,16 @@ class Context:
         _check(lib.fi_profile_read(self._h, counts, ms), "fi_profile_read")
         return {KERNEL_CLASSES[k]: (counts[k], ms[k]) for k in range(NUM_KERNEL_CLASSES)}
 
+    def profile_read_sides(self):
+        """(per-class dict as profile_read, {block side: (launches, ms)})."""
+        counts = (ctypes.c_int32 * NUM_KERNEL_CLASSES)()
+        ms = (ctypes.c_double * NUM_KERNEL_CLASSES)()
+        sc = (ctypes.c_int32 * 32)()
+        sm = (ctypes.c_double * 32)()
+        _check(lib.fi_profile_read_sides(self._h, counts, ms, sc, sm), "fi_profile_read_sides")
+        return ({KERNEL_CLASSES[k]: (counts[k], ms[k]) for k in range(NUM_KERNEL_CLASSES)},
+                {1 << q: (sc[q], sm[q]) for q in range(32) if sc[q]})
+
 
 def debug_fft(log2n: int, x, out, inverse: bool = False, stream=None):
     """The library's device FFT on x (complex64 CUDA tensor [count][2^log2n]) into out."""
@@ -215,14 +227,15 @@ def generate_noalloc(h, batch: int, n: int, x0, eps, y_out, dtype: str = "f32", 
 
 
 def chunk_schedule(chunk: int, retimed: bool):
-    """The chunk kernel's table of on-chip block pieces (host only): a list of
-    (step, first source, sources, first target, targets), chunk-relative."""
+    """The chunk kernel's table of on-chip block pieces (host only): (lags the
+    chain adds itself, [(step, first source, sources, first target, targets)]),
+    chunk-relative."""
     cap = 4 * chunk
     out = (ctypes.c_int32 * (5 * cap))()
-    n = ctypes.c_int32()
+    n, lags = ctypes.c_int32(), ctypes.c_int32()
     _check(lib.fi_debug_chunk_schedule(chunk, 1 if retimed else 0, ctypes.cast(out, ctypes.c_void_p), cap,
-                                       ctypes.byref(n)), "fi_debug_chunk_schedule")
-    return [tuple(out[5 * j: 5 * j + 5]) for j in range(min(n.value, cap))]
+                                       ctypes.byref(n), ctypes.byref(lags)), "fi_debug_chunk_schedule")
+    return lags.value, [tuple(out[5 * j: 5 * j + 5]) for j in range(min(n.value, cap))]
 
 
 def status_str(s: int) -> str:

@@ -111,23 +111,24 @@ def test_chunk_piece_table_covers_every_pair_once_in_time(chunk, retimed):
     sources [r-U, r), targets [r, r+U); a piece at step r reads sources below r
     (final once position r-1 is done) and writes targets >= r (the chain reads
     target t after the pieces of step t).
-    Re-timed (the whole chunk in one launch): the chain adds the lag-1 pairs
-    (t-1, t) itself, and the pieces cover every pair with t - s >= 2 with the
-    page's tiling shifted by one target (the chain reads target t after the
-    pieces of step t-1, so a piece at step r writes targets >= r+1); a piece may
-    also reach the window's spare position t = chunk (never read). Lags stay in
-    1..chunk (tap `chunk` is held as zero); the re-timed pieces hold at most 32
-    products per row each and are spread so that no step carries more than 64."""
+    Re-timed (the whole chunk in one launch): the chain adds the pairs of lags
+    1 and 2 itself, and the pieces cover every pair with t - s >= 3 with the
+    page's tiling shifted by two targets (the chain reads target t after the
+    pieces of step t-2, so a piece at step r writes targets >= r+2); a piece may
+    also reach the window's spare positions t = chunk, chunk+1 (never read).
+    Lags stay below chunk+2 (taps from `chunk` up are held as zero); the
+    re-timed pieces hold at most 32 products per row each and are spread so that
+    no step carries more than 64."""
     from long_convolution_sequence_online_b200 import fi
-    tab = fi.chunk_schedule(chunk, retimed)
-    sh = 1 if retimed else 0
+    sh, tab = fi.chunk_schedule(chunk, retimed)
+    assert sh == (2 if retimed else 0)
     count = {}
     per_step = {}
     for step, s_lo, ns, t_lo, nd in tab:
         assert 1 <= step < chunk
         assert s_lo >= 0 and s_lo + ns <= step, (step, s_lo, ns)
         assert t_lo >= step + sh and t_lo < chunk and t_lo + nd <= chunk + sh, (step, t_lo, nd)
-        assert t_lo - (s_lo + ns - 1) >= 1 + sh and (t_lo + nd - 1) - s_lo <= chunk
+        assert t_lo - (s_lo + ns - 1) >= 1 + sh and (t_lo + nd - 1) - s_lo <= chunk + sh - 1
         per_step.setdefault(step, []).append((s_lo, ns, t_lo, nd))
         for s in range(s_lo, s_lo + ns):
             for t in range(t_lo, min(t_lo + nd, chunk)):
@@ -142,7 +143,7 @@ def test_chunk_piece_table_covers_every_pair_once_in_time(chunk, retimed):
         if not retimed:
             assert pieces == [(r - U, U, r, U)]
         else:
-            if U <= 4 and r + 1 < chunk:
-                assert (r - U, U, r + 1, U) in pieces
+            if U <= 4 and r + sh < chunk:
+                assert (r - U, U, r + sh, U) in pieces
             assert max(ns * nd for _, ns, _, nd in pieces) <= 32
             assert sum(ns * nd for _, ns, _, nd in pieces) <= 64
