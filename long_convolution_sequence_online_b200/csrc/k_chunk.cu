@@ -48,7 +48,7 @@ constexpr int kRing = 4;                // depth of the hand-off barrier rings
 
 struct ChunkShape {
   int G, GP, CH, LS, TPS, CW, GdMax, NG, K;
-  size_t win, tp, ep, flags, total;  // float offsets / total floats
+  size_t win, tp, hv, ep, flags, total;  // float offsets / total floats
 };
 
 __host__ __device__ inline ChunkShape chunk_shape(const Dims& g, int CH, int G) {
@@ -66,7 +66,8 @@ __host__ __device__ inline ChunkShape chunk_shape(const Dims& g, int CH, int G) 
   c.K = g.M;
   c.win = 0;
   c.tp = c.win + (size_t)(g.M + 1) * c.LS;
-  c.ep = c.tp + (size_t)g.M * c.GdMax * c.TPS;
+  c.hv = (c.tp + (size_t)g.M * c.GdMax * c.TPS + 3) & ~(size_t)3;   // 16-byte aligned
+  c.ep = c.hv + (size_t)4 * g.M * c.GdMax;
   c.flags = (c.ep + (size_t)CH * G + 1) & ~(size_t)1;   // 8-byte aligned mbarriers
   c.total = c.flags + 2 * (size_t)(2 * kRing) * c.CW;  // act_ready[kRing][CW] + tile_done[kRing][CW]
   return c;
@@ -428,6 +429,7 @@ __global__ void __launch_bounds__(kChunkMaxThreads) k_chunk(Dims g, ChunkArgs a,
   float* win = csm + cs.win;   // [(M+1)][CH+1][GP]   slot window of positions [c, c+CH]
   float* tp = csm + cs.tp;     // [M][GdMax][TPS]     taps h[0..CH), zero above
   float* ep = csm + cs.ep;     // [CH][G]             sampler noise
+  float4* hv4 = reinterpret_cast<float4*>(csm + cs.hv);   // [M][GdMax] (h[0], h[1], h[2], h[3]) for the chain
   // Hand-off barrier rings (ordinal o uses slot o % kRing, phase parity
   // (o / kRing) & 1): act_ready[k][c] completes when chain warp c has finished a
   // position, tile_done[k][c] when every layer's pieces of a step are done for
@@ -539,6 +541,12 @@ __global__ void __launch_bounds__(kChunkMaxThreads) k_chunk(Dims g, ChunkArgs a,
   // tp[.][CH]: the tap one past the window, zero (pieces that reach the spare
   // position read it)
   for (int k = tid; k < M * GdMax * (TPS - CH); k += nt) tp[(k / (TPS - CH)) * TPS + CH + k % (TPS - CH)] = 0.f;
+  for (int k = tid; k < M * Gd; k += nt) {
+    const int l = k / Gd, dl = k - l * Gd;
+    const float* hrow = a.taps + ((size_t)l * g.D + d_lo + dl) * g.L;
+    hv4[l * GdMax + dl] = g.L >= 4 ? __ldg(reinterpret_cast<const float4*>(hrow))
+                                   : make_float4(hrow[0], g.L > 1 ? hrow[1] : 0.f, 0.f, 0.f);
+  }
   for (int k = tid; k < kRing * CW; k += nt) {
     mbar_init(act_ready + k, 32);
     mbar_init(tile_done + k, 32 * M);   // one arrival per lane per layer
@@ -569,8 +577,8 @@ __global__ void __launch_bounds__(kChunkMaxThreads) k_chunk(Dims g, ChunkArgs a,
     const size_t c_io = (size_t)b * g.D + d;
     const size_t y_stride = g.S;
     float* wcol = win + gg;                          // slot (l, r) at wcol[l*LS + r*GP]
-    const float* hcol = tp + (d - d_lo) * TPS;       // h^l[k] at hcol[(l-1)*HS + k]
-    const int HS = GdMax * TPS;
+    const float4* hv = hv4 + (d - d_lo);             // (h^l[0], h^l[1], h^l[2], .) at hv[(l-1)*HV]
+    const int HV = GdMax;
     float x_cur = wcol[r0 * GP];                     // token of the current position (first: as loaded)
     TanhParts P{0.f, 0.f, true};
     float epsk = 0.f;                                // eps_scale * eps of the previous position
@@ -583,39 +591,42 @@ __global__ void __launch_bounds__(kChunkMaxThreads) k_chunk(Dims g, ChunkArgs a,
         const int j = need - rs;
         ok = mbar_wait(&tile_done[(j % kRing) * CW + warp], (j / kRing) & 1, err, true, a.wait_limit);
       }
-      // lags the chain adds here (sources inside the chunk: earlier ones came
-      // with the blocks from HBM)
-      const int nl = min(nlag, r);
-      // Operands of layer m at this position: h^m[0] and the accumulator, plus
-      // the lag terms h^m[k] a^{m-1}_{r-k}. They are loaded two layers ahead of
-      // use, so their latency hides behind two exp2/reciprocal chains.
-      struct Ops { float h0, acc, h1, a1, h2, a2; };
-      auto load_ops = [&](int m, Ops& o) {
-        const float* hm = hcol + (m - 1) * HS;
-        const float* am = wcol + (m - 1) * LS;
-        o.h0 = hm[0];
-        o.acc = wcol[m * LS + r * GP];
-        o.h1 = 0.f; o.a1 = 0.f; o.h2 = 0.f; o.a2 = 0.f;
-        if (nl >= 1) { o.h1 = hm[1]; o.a1 = am[(r - 1) * GP]; }
-        if (nl >= 2) { o.h2 = hm[2]; o.a2 = am[(r - 2) * GP]; }
+      // Lag terms the chain adds here: lag k only when its source lies in this
+      // chunk (r >= k; earlier sources came with the blocks from HBM), applied
+      // through 0/1 multipliers so the layer loop has no branch. The operands of
+      // layer m (h^m[0..2] as one 16-byte load, the accumulator, a^{m-1} at
+      // r-1 and r-2) are loaded two layers ahead of use, so their latency hides
+      // behind two exp2/reciprocal chains.
+      const float m1 = (nlag >= 1 && r >= 1) ? 1.f : 0.f;
+      const float m2 = (nlag >= 2 && r >= 2) ? 1.f : 0.f;
+      const int o1 = max(r - 1, 0) * GP, o2 = max(r - 2, 0) * GP, o0 = r * GP;
+      float4 Hc = hv[0];
+      float accc = wcol[LS + o0], a1c = wcol[o1], a2c = wcol[o2];
+      const int m_n = M >= 2 ? 2 : 1;
+      float4 Hn = hv[(m_n - 1) * HV];
+      float accn = wcol[m_n * LS + o0], a1n = wcol[(m_n - 1) * LS + o1], a2n = wcol[(m_n - 1) * LS + o2];
+      auto acc_eff = [&](const float4& H, float acc, float a1, float a2) {
+        return fmaf(m2 * H.z, a2, fmaf(m1 * H.y, a1, acc));
       };
-      auto acc_of = [](const Ops& o) { return fmaf(o.h2, o.a2, fmaf(o.h1, o.a1, o.acc)); };
-      Ops cur, nxt;
-      load_ops(1, cur);
-      if (M >= 2) load_ops(2, nxt);
       float y, z = 0.f;
       if (from_parts) {
-        if constexpr (BF16) y = fmaf(cur.h0, x_cur, acc_of(cur));
-        else next_input(P, cur.h0, fmaf(cur.h0, epsk, acc_of(cur)), y, z);
+        if constexpr (BF16) y = fmaf(Hc.x, x_cur, acc_eff(Hc, accc, a1c, a2c));
+        else next_input(P, Hc.x, fmaf(Hc.x, epsk, acc_eff(Hc, accc, a1c, a2c)), y, z);
       } else {
-        y = fmaf(cur.h0, x_cur, acc_of(cur));
+        y = fmaf(Hc.x, x_cur, acc_eff(Hc, accc, a1c, a2c));
         z = kTwoLog2e * y;
       }
-      cur = nxt;                                   // operands of layer 2
+      Hc = Hn; accc = accn; a1c = a1n; a2c = a2n;   // layer 2
       for (int l = 1;; ++l) {
         if constexpr (REC) if (act) a.rec[((size_t)(l - 1) * a.n_gen + (t - a.gen_base)) * y_stride + c_io] = y;
         if (l == M) break;
-        if (l + 2 <= M) load_ops(l + 2, nxt);     // two layers ahead
+        {
+          const int m = min(l + 2, M);   // two layers ahead (the last layers reload layer M: harmless)
+          Hn = hv[(m - 1) * HV];
+          accn = wcol[m * LS + o0];
+          a1n = wcol[(m - 1) * LS + o1];
+          a2n = wcol[(m - 1) * LS + o2];
+        }
         float av;
         if constexpr (BF16) {
           av = round_bf16(tanh_approx(y));
@@ -623,10 +634,10 @@ __global__ void __launch_bounds__(kChunkMaxThreads) k_chunk(Dims g, ChunkArgs a,
           P = tanh_parts(y, z);
           av = tanh_value(P);
         }
-        if (act) wcol[l * LS + r * GP] = av;
-        if constexpr (BF16) y = fmaf(cur.h0, av, acc_of(cur));
-        else next_input(P, cur.h0, acc_of(cur), y, z);
-        cur = nxt;
+        if (act) wcol[l * LS + o0] = av;
+        if constexpr (BF16) y = fmaf(Hc.x, av, acc_eff(Hc, accc, a1c, a2c));
+        else next_input(P, Hc.x, acc_eff(Hc, accc, a1c, a2c), y, z);
+        Hc = Hn; accc = accn; a1c = a1n; a2c = a2n;
       }
       // y = y^M_t: hand the position to the tile warps, output, then the sampler
       // x_{t+1} = R(tanh(y) + eps_scale eps_t)
