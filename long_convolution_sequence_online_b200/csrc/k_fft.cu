@@ -365,8 +365,14 @@ __device__ __forceinline__ void tile_fft2_body(float2* sm, float* ds, int tid, b
 }
 
 // item = pair ((l-1)*S/2 + p): sequences s = 2p and 2p+1 (same channel, B even).
+// CTAs per SM the paired blocks ask the compiler to fit (register budget),
+// from a B200 sweep of 1..3 at the 18 x 3456-row batch: 3 for side 256
+// (91 -> 74 us per launch), 2 for side 2048 (965 -> 730 us); more hurt the
+// sides that hold 32 points per thread (8192: 4.1 -> 6.5 ms).
+__host__ __device__ constexpr int fft2_min_blocks(int n2) { return n2 == 512 ? 3 : n2 == 4096 ? 2 : 1; }
+
 template <int N2, int T>
-__global__ void __launch_bounds__(T >= 128 ? T : 128)
+__global__ void __launch_bounds__(T >= 128 ? T : 128, fft2_min_blocks(N2))
 k_tile_fft2(Dims g, float* __restrict__ state, const float2* __restrict__ spec, const float2* __restrict__ tw, int i,
             int overwrite, int t_min) {
   constexpr int U = N2 / 2;
