@@ -346,8 +346,6 @@ def gpu_arm(args, world, rank, local):
     torch.cuda.synchronize(device)
 
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    ctx.profile(True)
-    ctx.profile_read()
     with ClockSampler(local) as clocks:
         barrier(device)
         torch.cuda.synchronize(device)
@@ -357,7 +355,14 @@ def gpu_arm(args, world, rank, local):
             ev[k][1].record(stream)
         torch.cuda.synchronize(device)
         barrier(device)
-    prof = ctx.profile_read()
+    # Per-kernel times: the same number of steps again with CUDA events around
+    # every launch (the events themselves cost about 5 % of a step, so they stay
+    # out of the region `value` is timed on).
+    ctx.profile(True)
+    ctx.profile_read()
+    for _ in range(args.steps):
+        step()
+    prof, sides = ctx.profile_read_sides()
     ctx.profile(False)
     step_ms = [a.elapsed_time(b) for a, b in ev]
     total_ms = reduce_max(float(sum(step_ms)), device)
@@ -489,6 +494,8 @@ def gpu_arm(args, world, rank, local):
         "roofline": roof,
         "step_roofline": step_roof,
         "kernels": classes,
+        "block_sides_ms_per_step": {str(k): ms / args.steps for k, (n, ms) in sorted(sides.items())},
+        "kernels_timing": "CUDA events around every launch, on as many further steps as timed (same stream)",
         "e2e": e2e,
         "gpu_launches": int(round(launches_per_step * args.steps)),
         "clocks": clk,

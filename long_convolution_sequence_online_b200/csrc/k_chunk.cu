@@ -191,6 +191,8 @@ __device__ __forceinline__ void run_piece2(uint32_t e, const float* srcA, float*
     case PK_SQ4: block_piece2<4, 4>(srcA, dstA, tapsA, srcB, dstB, tapsB, s_lo, t_lo, stride); break;
     case PK_R8x4: block_piece2<8, 4>(srcA, dstA, tapsA, srcB, dstB, tapsB, s_lo, t_lo, stride); break;
     case PK_R16x2: block_piece2<16, 2>(srcA, dstA, tapsA, srcB, dstB, tapsB, s_lo, t_lo, stride); break;
+    case PK_SQ8: block_piece2<8, 8>(srcA, dstA, tapsA, srcB, dstB, tapsB, s_lo, t_lo, stride); break;
+    case PK_R16x4: block_piece2<16, 4>(srcA, dstA, tapsA, srcB, dstB, tapsB, s_lo, t_lo, stride); break;
     default:   // kinds only the one-row path uses (page's tiling of a partial chunk)
       run_piece(e, srcA, dstA, tapsA, stride);
       run_piece(e, srcB, dstB, tapsB, stride);
@@ -230,7 +232,9 @@ void cut_block(int r, int U, int sh, std::vector<Piece>& out) {
     return;
   }
   const int H = U / 2;
-  const int kind = H == 16 ? PK_R16x2 : H == 8 ? PK_R8x4 : PK_SQ4;   // 32, 32, 16 products per row
+  // 64, 64, 16 products per row (measured on B200: pieces of 32 products took
+  // more steps' worth of per-piece latency than they saved)
+  const int kind = H == 16 ? PK_R16x4 : H == 8 ? PK_SQ8 : PK_SQ4;
   const int nd = piece_nd(kind);
   for (int t = r + sh; t < r + sh + U; t += nd) out.push_back({-1, r - U, t, kind});
   for (int t = r + H + sh; t < r + U + sh; t += nd) out.push_back({-1, r - H, t, kind});

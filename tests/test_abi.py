@@ -117,8 +117,8 @@ def test_chunk_piece_table_covers_every_pair_once_in_time(chunk, retimed):
     pieces of step t-2, so a piece at step r writes targets >= r+2); a piece may
     also reach the window's spare positions t = chunk, chunk+1 (never read).
     Lags stay below chunk+2 (taps from `chunk` up are held as zero); the
-    re-timed pieces hold at most 32 products per row each and are spread so that
-    no step carries more than 64."""
+    re-timed pieces hold at most 64 products per row each and are spread so that
+    no step carries more than 96."""
     from long_convolution_sequence_online_b200 import fi
     sh, tab = fi.chunk_schedule(chunk, retimed)
     assert sh == (2 if retimed else 0)
@@ -145,5 +145,5 @@ def test_chunk_piece_table_covers_every_pair_once_in_time(chunk, retimed):
         else:
             if U <= 4 and r + sh < chunk:
                 assert (r - U, U, r + sh, U) in pieces
-            assert max(ns * nd for _, ns, _, nd in pieces) <= 32
-            assert sum(ns * nd for _, ns, _, nd in pieces) <= 64
+            assert max(ns * nd for _, ns, _, nd in pieces) <= 64
+            assert sum(ns * nd for _, ns, _, nd in pieces) <= 96
