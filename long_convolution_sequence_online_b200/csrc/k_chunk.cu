@@ -45,6 +45,8 @@ constexpr int kChunkMaxThreads = 512;
 constexpr int kChunkMaxStreams = 128;
 constexpr int kSuspendHintNs = 1000;   // longest a suspended barrier check may last
 constexpr int kRing = 4;                // depth of the hand-off barrier rings
+static_assert(kChainLags >= 1 && kChainLags <= 3, "the chain holds h[0..3] in one 16-byte load");
+static_assert(kRing >= kChainLags + 1, "a ring slot must never get two phases ahead of its waiter");
 
 struct ChunkShape {
   int G, GP, CH, LS, TPS, CW, GdMax, NG, K;
@@ -603,24 +605,28 @@ __global__ void __launch_bounds__(kChunkMaxThreads) k_chunk(Dims g, ChunkArgs a,
       // behind two exp2/reciprocal chains.
       const float m1 = (nlag >= 1 && r >= 1) ? 1.f : 0.f;
       const float m2 = (nlag >= 2 && r >= 2) ? 1.f : 0.f;
-      const int o1 = max(r - 1, 0) * GP, o2 = max(r - 2, 0) * GP, o0 = r * GP;
+      const float m3 = (nlag >= 3 && r >= 3) ? 1.f : 0.f;
+      const int o1 = max(r - 1, 0) * GP, o2 = max(r - 2, 0) * GP, o3 = max(r - 3, 0) * GP, o0 = r * GP;
       float4 Hc = hv[0];
-      float accc = wcol[LS + o0], a1c = wcol[o1], a2c = wcol[o2];
+      float accc = wcol[LS + o0], a1c = wcol[o1], a2c = wcol[o2], a3c = kChainLags >= 3 ? wcol[o3] : 0.f;
       const int m_n = M >= 2 ? 2 : 1;
       float4 Hn = hv[(m_n - 1) * HV];
       float accn = wcol[m_n * LS + o0], a1n = wcol[(m_n - 1) * LS + o1], a2n = wcol[(m_n - 1) * LS + o2];
-      auto acc_eff = [&](const float4& H, float acc, float a1, float a2) {
-        return fmaf(m2 * H.z, a2, fmaf(m1 * H.y, a1, acc));
+      float a3n = kChainLags >= 3 ? wcol[(m_n - 1) * LS + o3] : 0.f;
+      auto acc_eff = [&](const float4& H, float acc, float a1, float a2, float a3) {
+        float v = fmaf(m2 * H.z, a2, fmaf(m1 * H.y, a1, acc));
+        if constexpr (kChainLags >= 3) v = fmaf(m3 * H.w, a3, v);
+        return v;
       };
       float y, z = 0.f;
       if (from_parts) {
-        if constexpr (BF16) y = fmaf(Hc.x, x_cur, acc_eff(Hc, accc, a1c, a2c));
-        else next_input(P, Hc.x, fmaf(Hc.x, epsk, acc_eff(Hc, accc, a1c, a2c)), y, z);
+        if constexpr (BF16) y = fmaf(Hc.x, x_cur, acc_eff(Hc, accc, a1c, a2c, a3c));
+        else next_input(P, Hc.x, fmaf(Hc.x, epsk, acc_eff(Hc, accc, a1c, a2c, a3c)), y, z);
       } else {
-        y = fmaf(Hc.x, x_cur, acc_eff(Hc, accc, a1c, a2c));
+        y = fmaf(Hc.x, x_cur, acc_eff(Hc, accc, a1c, a2c, a3c));
         z = kTwoLog2e * y;
       }
-      Hc = Hn; accc = accn; a1c = a1n; a2c = a2n;   // layer 2
+      Hc = Hn; accc = accn; a1c = a1n; a2c = a2n; a3c = a3n;   // layer 2
       for (int l = 1;; ++l) {
         if constexpr (REC) if (act) a.rec[((size_t)(l - 1) * a.n_gen + (t - a.gen_base)) * y_stride + c_io] = y;
         if (l == M) break;
@@ -630,6 +636,7 @@ __global__ void __launch_bounds__(kChunkMaxThreads) k_chunk(Dims g, ChunkArgs a,
           accn = wcol[m * LS + o0];
           a1n = wcol[(m - 1) * LS + o1];
           a2n = wcol[(m - 1) * LS + o2];
+          if constexpr (kChainLags >= 3) a3n = wcol[(m - 1) * LS + o3];
         }
         float av;
         if constexpr (BF16) {
@@ -639,9 +646,9 @@ __global__ void __launch_bounds__(kChunkMaxThreads) k_chunk(Dims g, ChunkArgs a,
           av = tanh_value(P);
         }
         if (act) wcol[l * LS + o0] = av;
-        if constexpr (BF16) y = fmaf(Hc.x, av, acc_eff(Hc, accc, a1c, a2c));
-        else next_input(P, Hc.x, acc_eff(Hc, accc, a1c, a2c), y, z);
-        Hc = Hn; accc = accn; a1c = a1n; a2c = a2n;
+        if constexpr (BF16) y = fmaf(Hc.x, av, acc_eff(Hc, accc, a1c, a2c, a3c));
+        else next_input(P, Hc.x, acc_eff(Hc, accc, a1c, a2c, a3c), y, z);
+        Hc = Hn; accc = accn; a1c = a1n; a2c = a2n; a3c = a3n;
       }
       // y = y^M_t: hand the position to the tile warps, output, then the sampler
       // x_{t+1} = R(tanh(y) + eps_scale eps_t)
