@@ -36,7 +36,16 @@ if ROOT not in sys.path:
 
 import synth  # noqa: E402
 
-METRIC = "mixer tokens/s at 18x864, L=32K on 1 B200"
+METRIC = "mixer tokens/s at 18\u00d7864, L=32K on 1 B200; % of roofline; speedup vs O(L\u00b2)"
+
+
+def metric_name(w: synth.Workload, api: str = "generate") -> str:
+    """The headline metric's name for the headline workload, the same form for the others."""
+    if w.name == synth.HEADLINE and api == "generate":
+        return METRIC
+    kind = "mixer tokens/s" if api == "generate" else "mixer tokens/s through fi_step (one call per position)"
+    return (f"{kind} at {w.layers}\u00d7{w.channels}, L={w.length}, B={w.batch} {w.dtype} on 1 B200; "
+            "% of roofline; speedup vs O(L\u00b2)")
 UNIT = "tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 NOMINAL_HBM_GBS = 8000.0            # the HBM figure the roofline target is quoted against
@@ -68,6 +77,7 @@ def cost_model(w: synth.Workload, chunk: int, fft_from: int, fft_max: int = 1 <<
     output (s_x + 4 + 4). Flops: direct block 2U^2, FFT block fft_flops(U), red cell 3.
     Tensor-core blocks (sides 64..tc_max) count like direct ones: taps, sources,
     accumulators, 2U^2 flops per row (the Toeplitz product, not the padded MMA work).
+    Blocks wider than fft_max are partitioned FFT blocks (fft class).
     """
     M, D, L, B = w.layers, w.channels, w.length, w.batch
     s = 2 if w.dtype == "bf16" else 4
@@ -77,16 +87,25 @@ def cost_model(w: synth.Workload, chunk: int, fft_from: int, fft_max: int = 1 <<
             cls = "chunk"
         elif 64 <= U <= tc_max:
             cls = "tc"
-        elif fft_from and fft_from <= U <= fft_max:
+        elif fft_from and fft_from <= U:
             cls = "fft"
         else:
             cls = "direct"
-        per_ld = (U + 1) * 8 if cls == "fft" else (2 * U - 1) * s
+        m = U // fft_max if (cls == "fft" and U > fft_max) else 0
+        if m:
+            # partitioned: m sub-blocks of side fft_max; 2m-1 segment spectra per
+            # (layer, channel); per row m forward and m inverse transforms and m^2
+            # spectrum products of fft_max + 1 points (8 flops each)
+            per_ld = (2 * m - 1) * (fft_max + 1) * 8
+            row_flops = m * fft_flops(fft_max) + 8.0 * m * m * (fft_max + 1)
+        else:
+            per_ld = (U + 1) * 8 if cls == "fft" else (2 * U - 1) * s
+            row_flops = fft_flops(U) if cls == "fft" else 2.0 * U * U
         per_lbd = U * s + 2 * U * 4
         out[cls]["bytes"] += n * (M * D * per_ld + M * B * D * per_lbd)
         if cls == "chunk":
             out[cls]["block_bytes"] = out[cls].get("block_bytes", 0.0) + n * (M * D * per_ld + M * B * D * per_lbd)
-        out[cls]["flops"] += n * M * B * D * (fft_flops(U) if cls == "fft" else 2.0 * U * U)
+        out[cls]["flops"] += n * M * B * D * row_flops
         out[cls]["blocks"] += n
     out["chunk"]["bytes"] += L * (M * B * D * (4 + s) + B * D * (s + 8))
     out["chunk"]["flops"] += L * M * B * D * 3.0
@@ -144,12 +163,26 @@ class ClockSampler:
             self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}",
                                           "--format=csv,noheader,nounits", "-lms", "200"],
                                          stdout=self.fh, stderr=subprocess.DEVNULL)
+            self._wait_lines(1, 5.0)      # the sampler is live before the region starts
         except Exception:
             self.proc = None
         return self
 
+    def _lines(self) -> int:
+        self.fh.flush()
+        with open(self.path) as f:
+            return sum(1 for _ in f)
+
+    def _wait_lines(self, n: int, limit_s: float):
+        t0 = time.perf_counter()
+        while self._lines() < n and time.perf_counter() - t0 < limit_s:
+            time.sleep(0.02)
+
     def __exit__(self, *exc):
         if self.proc is not None:
+            # one more sample after the region, so that a region shorter than the
+            # sampling period still has one taken while or right after it ran
+            self._wait_lines(self._lines() + 1, 1.0)
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
@@ -337,9 +370,22 @@ def gpu_arm(args, world, rank, local):
     del h_d
     chunk, fft_from, tc_max = ctx.plan()
 
+    step_api = args.api == "step"
+    if step_api:
+        # one fi_step call per position on given tokens (the noise stands in for them),
+        # each position's output written to its row of y
+        tok_d = eps_d.to(td).contiguous()
+        row_x = tok_d[0].numel() * tok_d.element_size()
+        row_y = w.batch * w.channels * 4
+        x_base, y_base = tok_d.data_ptr(), y_d.data_ptr()
+
     def step():
         ctx.reset()
-        ctx.generate(w.length, x0_d, eps_d, y_d, 0.1)
+        if step_api:
+            for t in range(w.length):
+                ctx.step_ptr(x_base + t * row_x, y_base + t * row_y)
+        else:
+            ctx.generate(w.length, x0_d, eps_d, y_d, 0.1)
 
     for _ in range(args.warmup):
         step()
@@ -380,7 +426,7 @@ def gpu_arm(args, world, rank, local):
         ctx.generate_host_ptr(w.length, x0_h.data_ptr(), eps_h.data_ptr(), y_h.data_ptr(), 0.1)
 
     e2e = None
-    if args.e2e_steps > 0:
+    if args.e2e_steps > 0 and not step_api:
         e2e_step()
         barrier(device)
         t0 = time.perf_counter()
@@ -411,9 +457,12 @@ def gpu_arm(args, world, rank, local):
     # --- roofline: dominant kernel class during the timed steps
     peaks = measured_peaks()
     clk = clocks.summary()
-    model, tot = cost_model(w, chunk, fft_from, tc_max=tc_max)
+    # fi_step computes every block from HBM (no on-chip chunk) and each position's red
+    # cells in k_token, so the per-position bytes and flops belong to "token" there
+    model, tot = cost_model(w, 1 if step_api else chunk, fft_from, tc_max=tc_max)
+    model["token"] = model["chunk"] if step_api else {"bytes": 0.0, "flops": 0.0}
     classes = {}
-    for cls in ("chunk", "direct", "fft", "tc"):
+    for cls in ("chunk", "direct", "fft", "tc", "token"):
         n, ms = prof[cls]
         if n == 0:
             continue
@@ -456,8 +505,9 @@ def gpu_arm(args, world, rank, local):
 
     # --- quadratic Lazy baseline on the GPU: measured on two prefixes, extrapolated a*n + b*n^2/2
     lazy = None
-    if args.lazy_prefix > 0 and rank == 0:
-        n1, n2 = args.lazy_prefix // 4, args.lazy_prefix
+    if args.lazy_prefix > 0 and rank == 0 and not step_api:
+        n2 = min(args.lazy_prefix, w.length)
+        n1 = n2 // 4
         times = []
         for n in (n1, n2):
             ctx.reset()
@@ -479,7 +529,7 @@ def gpu_arm(args, world, rank, local):
 
     launches_per_step = sum(prof[k][0] for k in prof) / args.steps
     res = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "metric": metric_name(w, args.api), "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32" if w.dtype == "f32" else "bf16", "data": "synthetic",
         "config": {"workload": w.name, "layers": w.layers, "channels": w.channels, "seq_len": w.length,
@@ -489,7 +539,9 @@ def gpu_arm(args, world, rank, local):
                    "l2": (f"inputs larger than L2 (state {4 * (w.layers + 1) * w.streams * w.length / 1e9:.1f} GB "
                           "streamed every step)") if 4 * (w.layers + 1) * w.streams * w.length > L2_BYTES
                          else "state fits in L2 (latency-bound workload)",
-                   "step": "fi_reset + fi_generate over all L positions, closed loop",
+                   "step": ("fi_reset + one fi_step per position over all L given tokens (host loop)" if step_api
+                            else "fi_reset + fi_generate over all L positions, closed loop"),
+                   "api": args.api,
                    "init_s": t_init},
         "roofline": roof,
         "step_roofline": step_roof,
@@ -518,6 +570,8 @@ def main():
     ap.add_argument("--fft-from", dest="fft_from", type=int, default=0)
     ap.add_argument("--tc-max", dest="tc_max", type=int, default=0,
                     help="largest block side on the tensor cores (0 = automatic, -1 = none)")
+    ap.add_argument("--api", default="generate", choices=["generate", "step"],
+                    help="generate: closed-loop fi_generate per step; step: one fi_step call per position")
     ap.add_argument("--e2e-steps", dest="e2e_steps", type=int, default=3)
     ap.add_argument("--lazy-prefix", dest="lazy_prefix", type=int, default=4096)
     ap.add_argument("--oracle-positions", dest="oracle_positions", type=int, default=6144)
@@ -543,7 +597,7 @@ def main():
         cpu = {k: per[-1][k] for k in ("unit", "cores", "kind", "sample")}
         cpu["value"] = value
         print(json.dumps({
-            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "metric": metric_name(w, args.api), "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": 1e3 * t_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
             "config": {"workload": w.name, "layers": w.layers, "channels": w.channels, "seq_len": w.length,

@@ -119,15 +119,21 @@ __device__ __forceinline__ void dft_reg(float2* v) {
 struct SyncWarp { __device__ __forceinline__ void operator()() const { __syncwarp(); } };
 struct SyncBlock { __device__ __forceinline__ void operator()() const { __syncthreads(); } };
 
-// v[r] *= w^r for r = 1..R-1 (w = W_{Ns R}^{kk}, forward sign; conjugated for the
-// inverse). w, w^4, w^8 (and w^16) come from the table; the other powers are
-// products of at most four table values, so each carries a few roundings at most.
-template <int R, bool INV>
-__device__ __forceinline__ void apply_twiddles(float2* v, const float2* __restrict__ tw, int base) {
+// v[r] *= w^r for r = 1..R-1 (w = W_{NSR}^{kk}, NSR = Ns R, forward sign;
+// conjugated for the inverse). w, w^4, w^8 (and w^16) come from the hardware
+// sine/cosine (__sincosf, absolute error about 2^-21 on [-pi, pi]) with the angle
+// reduced to that range; the other powers are products of at most four of them.
+// Measured on B200, this beats loading the four values from a table by 9-19 % per
+// FFT block: the table loads of a pass are strided over a 256 KB table, so each
+// warp load touched 16-32 sectors.
+template <int R, int NSR, bool INV>
+__device__ __forceinline__ void apply_twiddles(float2* v, int kk) {
   auto ld = [&](int r) {
-    float2 w = __ldg(tw + r * base);
-    if (INV) w.y = -w.y;
-    return w;
+    int m = r * kk;                        // in [0, NSR)
+    if (2 * m > NSR) m -= NSR;             // angle in (-pi, pi]
+    float sn, cs;
+    __sincosf((float)m * (-6.28318530717958647692f / (float)NSR), &sn, &cs);
+    return make_float2(cs, INV ? -sn : sn);
   };
   const float2 w1 = ld(1);
   v[1] = cmul(v[1], w1);
@@ -166,25 +172,39 @@ __device__ __forceinline__ void apply_twiddles(float2* v, const float2* __restri
   }
 }
 
-// Shape of the transform: T threads, P = N/T points each, passes of radix
-// min(32, P); the pass that takes what is left (REM bits) comes last, or first
-// when REMF (a transform whose first pass must match the previous transform's
-// last one: the inverse of a convolution that keeps the forward's order).
-template <int N, int T, bool REMF = false>
+// Shape of the transform: T threads, P = N/T points each. SH = (PL << 4) | REV.
+// With PL = 0 the passes have radix min(32, P) and the pass that takes what is
+// left (REM bits) comes last, or first when REV (a transform whose first pass
+// must match the previous transform's last one: the inverse of a convolution
+// that keeps the forward's order). Otherwise PL lists the passes' radix bits,
+// one hex digit each, the first pass in the lowest digit, taken in reverse order
+// when REV (so the inverse again starts with the forward's last radix).
+template <int N, int T, int SH = 0>
 struct FftShape {
   static constexpr int LOGN = clog2(N);
   static constexpr int P = N / T;
   static constexpr int RBMAX = cmin(5, clog2(P));
   static constexpr int REM = LOGN % RBMAX;
-  static constexpr int rb(int done) { return (REMF && REM != 0 && done == 0) ? REM : cmin(RBMAX, LOGN - done); }
+  static constexpr int PL = SH >> 4;
+  static constexpr bool REV = (SH & 1) != 0;
+  static constexpr int ndig(int p) { return p ? 1 + ndig(p >> 4) : 0; }
+  static constexpr int ND = ndig(PL);
+  static constexpr int digit(int k) { return REV ? (PL >> (4 * (ND - 1 - k))) & 15 : (PL >> (4 * k)) & 15; }
+  static constexpr int plan_rb(int done, int k = 0) { return done == 0 ? digit(k) : plan_rb(done - digit(k), k + 1); }
+  static constexpr int plan_sum(int k = 0) { return k == ND ? 0 : digit(k) + plan_sum(k + 1); }
+  static constexpr bool plan_ok(int k = 0) { return k == ND ? true : (digit(k) >= 1 && digit(k) <= clog2(P) && plan_ok(k + 1)); }
+  static_assert(PL == 0 || (plan_sum() == LOGN && plan_ok()), "pass plan must cover log2 N with radices <= P");
+  static constexpr int rb(int done) {
+    return PL ? plan_rb(done) : (REV && REM != 0 && done == 0) ? REM : cmin(RBMAX, LOGN - done);
+  }
   static constexpr bool last(int done) { return done + rb(done) >= LOGN; }
 };
 
 // Twiddles and R-point DFTs of one pass on the P points a thread holds
 // (butterfly k in v[k*R .. k*R+R), butterfly index j = tid + k*T).
-template <int N, int T, bool INV, int DONE, bool REMF = false>
-__device__ __forceinline__ void pass_compute(float2* v, int tid, const float2* __restrict__ tw) {
-  using S = FftShape<N, T, REMF>;
+template <int N, int T, bool INV, int DONE, int SH = 0>
+__device__ __forceinline__ void pass_compute(float2* v, int tid) {
+  using S = FftShape<N, T, SH>;
   constexpr int R = 1 << S::rb(DONE);
   constexpr int Ns = 1 << DONE;
 #pragma unroll
@@ -192,16 +212,16 @@ __device__ __forceinline__ void pass_compute(float2* v, int tid, const float2* _
     if constexpr (Ns > 1) {
       const int j = tid + k * T;
       const int kk = j & (Ns - 1);
-      apply_twiddles<R, INV>(v + k * R, tw, kk * (kTwiddleN / (Ns * R)));
+      apply_twiddles<R, Ns * R, INV>(v + k * R, kk);
     }
     dft_reg<R, INV>(v + k * R);
   }
 }
 
 // Stockham load of one pass: value r of butterfly j sits at j + r*N/R.
-template <int N, int T, int DONE, bool REMF = false>
+template <int N, int T, int DONE, int SH = 0>
 __device__ __forceinline__ void pass_load(const float2* sm, float2* v, int tid) {
-  using S = FftShape<N, T, REMF>;
+  using S = FftShape<N, T, SH>;
   constexpr int R = 1 << S::rb(DONE);
 #pragma unroll
   for (int k = 0; k < S::P / R; ++k) {
@@ -211,9 +231,9 @@ __device__ __forceinline__ void pass_load(const float2* sm, float2* v, int tid) 
 }
 
 // Stockham store of one pass: output r of butterfly j goes to (j - kk)*R + kk + r*Ns.
-template <int N, int T, int DONE, bool REMF = false>
+template <int N, int T, int DONE, int SH = 0>
 __device__ __forceinline__ void pass_store(float2* sm, const float2* v, int tid) {
-  using S = FftShape<N, T, REMF>;
+  using S = FftShape<N, T, SH>;
   constexpr int R = 1 << S::rb(DONE);
   constexpr int Ns = 1 << DONE;
 #pragma unroll
@@ -228,36 +248,36 @@ __device__ __forceinline__ void pass_store(float2* sm, const float2* v, int tid)
 
 // Passes DONE.. that go shared memory -> shared memory, stopping before the
 // last pass when STOP_BEFORE_LAST (the caller finishes it with its own store).
-template <int N, int T, bool INV, int DONE, bool STOP_BEFORE_LAST, bool REMF = false, class Sync>
-__device__ __forceinline__ void smem_passes(float2* sm, int tid, const float2* __restrict__ tw, Sync sync) {
-  using S = FftShape<N, T, REMF>;
+template <int N, int T, bool INV, int DONE, bool STOP_BEFORE_LAST, int SH = 0, class Sync>
+__device__ __forceinline__ void smem_passes(float2* sm, int tid, Sync sync) {
+  using S = FftShape<N, T, SH>;
   if constexpr (DONE < S::LOGN) {
     if constexpr (!(STOP_BEFORE_LAST && S::last(DONE))) {
       float2 v[S::P];
-      pass_load<N, T, DONE, REMF>(sm, v, tid);
-      pass_compute<N, T, INV, DONE, REMF>(v, tid, tw);
+      pass_load<N, T, DONE, SH>(sm, v, tid);
+      pass_compute<N, T, INV, DONE, SH>(v, tid);
       sync();
-      pass_store<N, T, DONE, REMF>(sm, v, tid);
+      pass_store<N, T, DONE, SH>(sm, v, tid);
       sync();
-      smem_passes<N, T, INV, DONE + S::rb(DONE), STOP_BEFORE_LAST, REMF>(sm, tid, tw, sync);
+      smem_passes<N, T, INV, DONE + S::rb(DONE), STOP_BEFORE_LAST, SH>(sm, tid, sync);
     }
   }
 }
 
 // Start of the last pass.
-template <int N, int T, int DONE = 0, bool REMF = false>
+template <int N, int T, int DONE = 0, int SH = 0>
 constexpr int last_pass_done() {
-  using S = FftShape<N, T, REMF>;
+  using S = FftShape<N, T, SH>;
   if constexpr (S::last(DONE)) return DONE;
-  else return last_pass_done<N, T, DONE + S::rb(DONE), REMF>();
+  else return last_pass_done<N, T, DONE + S::rb(DONE), SH>();
 }
 
 // In-place transform of sm[fft_pad<N, T>(0..N)) by the T threads with tid in [0, T).
 // Callers synchronise before (data written) and may read results right after.
 template <int N, int T, bool INV, class Sync>
-__device__ __forceinline__ void fft_smem(float2* sm, int tid, const float2* __restrict__ tw, Sync sync) {
+__device__ __forceinline__ void fft_smem(float2* sm, int tid, Sync sync) {
   static_assert((N & (N - 1)) == 0 && N >= 2 * T, "bad FFT shape");
-  smem_passes<N, T, INV, 0, false>(sm, tid, tw, sync);
+  smem_passes<N, T, INV, 0, false>(sm, tid, sync);
 }
 
 // Threads per transform: 16 or 32 points per thread, whichever measured faster

@@ -358,9 +358,12 @@ fi_status fi_step(fi_ctx* c, const void* x_t, float* y_t) {
   if (c->pos >= c->g.L) return fail(FI_E_STATE, "position == max_len");
   if (c->lazy_mode) return fail(FI_E_STATE, "context holds a lazy generation; call fi_reset");
   fi_status s;
-  if (c->pos >= 1 && (s = run_block(c, c->pos)) != FI_OK) return s;
   const int t = c->pos;
-  if ((s = timed(c, KC_TOKEN, [&] { return launch_token(c->g, c->state, c->taps, t, x_t, nullptr, 0.f, y_t, c->st); },
+  // small blocks (direct, side <= kTokenBlockMax) run inside the red-cell launch
+  const int fused_u = (t >= 1 && token_block_fused(c->g, lowbit(t))) ? lowbit(t) : 0;
+  if (t >= 1 && !fused_u && (s = run_block(c, t)) != FI_OK) return s;
+  if ((s = timed(c, KC_TOKEN,
+                 [&] { return launch_token(c->g, c->state, c->taps, t, x_t, nullptr, 0.f, y_t, c->st, fused_u); },
                  "red-cell launch")) != FI_OK)
     return s;
   c->pos++;

@@ -58,9 +58,15 @@ inline int highbit(int i) { int r = 1; while ((int64_t)r * 2 <= i) r *= 2; retur
 // ---------------------------------------------------------------- launchers (kernels/*.cu)
 // All return cudaSuccess or the launch error.
 
-// Red cells + blocks of one position for all streams (fi_step, lazy).
+// Red cells + blocks of one position for all streams (fi_step, lazy). block_u > 0
+// (1, 2, 4 or kTokenBlockMax) also adds the direct block of step t (side
+// block_u = lowbit(t)) in the same launch, before the red cells; it needs
+// M <= kTokenMaxLayers (token_block_fused says whether a shape qualifies).
+constexpr int kTokenBlockMax = 8;
+constexpr int kTokenMaxLayers = 32;
+inline bool token_block_fused(const Dims& g, int U) { return g.M <= kTokenMaxLayers && U >= 1 && U <= kTokenBlockMax; }
 cudaError_t launch_token(const Dims& g, float* state, const float* taps, int t, const void* x_t,
-                         const float* eps_t, float eps_scale, float* y_t, cudaStream_t st);
+                         const float* eps_t, float eps_scale, float* y_t, cudaStream_t st, int block_u = 0);
 
 // Direct block of step i (side U = lowbit(i)) from HBM for all layers and streams;
 // overwrite = the block is the first to reach its targets (i a power of two).

@@ -26,15 +26,103 @@ __global__ void k_token(Dims g, float* __restrict__ state, const float* __restri
   } else {
     a = state[slot_index(g, 0, s, t)];
   }
+  // The layers' accumulators and h_0 taps do not depend on the chain, so they are
+  // loaded a group of layers at a time, all in flight together, before the group's
+  // dependent red cells run.
+  constexpr int kGroup = 8;
+  float y = 0.f;
+  for (int l0 = 1; l0 <= g.M; l0 += kGroup) {
+    float acc[kGroup], h0[kGroup];
+#pragma unroll
+    for (int j = 0; j < kGroup; ++j) {
+      const int l = l0 + j;
+      acc[j] = 0.f;
+      h0[j] = 0.f;
+      if (l <= g.M) {
+        if (t > 0) acc[j] = state[slot_index(g, l, s, t)];
+        h0[j] = __ldg(taps + ((size_t)(l - 1) * g.D + d) * g.L);
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < kGroup; ++j) {
+      const int l = l0 + j;
+      if (l > g.M) break;
+      y = fmaf(h0[j], a, acc[j]);
+      if (l < g.M) {
+        a = round_act(tanhf(y), g.bf16);
+        state[slot_index(g, l, s, t)] = a;
+      }
+    }
+  }
+  y_t[io] = y;
+  if (eps_t && t + 1 < g.L) state[slot_index(g, 0, s, t + 1)] = round_act(tanhf(y) + eps_scale * eps_t[io], g.bf16);
+}
+
+// The same position with one thread per (stream, layer): a CTA holds 32 streams
+// and all M layers (32*M threads), so every layer's accumulator, h_0 tap and
+// (U > 0) direct block of step t are fetched and computed in parallel, and only
+// the red-cell chain is serial (one warp, through shared memory). The block of
+// step t, side U = lowbit(t), adds sum_{u<U} h^l[U+u'-u] a^{l-1}_{t-U+u} to the
+// targets t+u' (u' < U) of layer l (stored, not added, when t is a power of two,
+// the first block to reach them): target t's part goes straight into the chain,
+// the others back to the state, as the direct block kernel would leave them.
+template <int U>
+__global__ void k_token_par(Dims g, float* __restrict__ state, const float* __restrict__ taps, int t,
+                            const void* __restrict__ x_t, const float* __restrict__ eps_t, float eps_scale,
+                            float* __restrict__ y_t) {
+  extern __shared__ float tsm[];
+  float* accs = tsm;               // [M][32] accumulator of (layer, lane) at t
+  float* h0s = tsm + g.M * 32;     // [M][32] h^l_0 of the lane's channel
+  const int lane = threadIdx.x & 31, li = threadIdx.x >> 5;
+  const int s = blockIdx.x * 32 + lane;
+  const bool ok = s < g.S;
+  const int d = ok ? s / g.B : 0;
+  if (ok) {
+    const int l = li + 1;
+    const float* hp = taps + ((size_t)(l - 1) * g.D + d) * g.L;
+    h0s[li * 32 + lane] = __ldg(hp);
+    float* dp = state + slot_index(g, l, s, t);
+    float acc;
+    if constexpr (U == 0) {
+      acc = (t == 0) ? 0.f : dp[0];
+    } else {
+      const bool overwrite = (t == U);   // lowbit(t) == t: t is a power of two
+      const float* xp = state + slot_index(g, l - 1, s, t - U);
+      float x[U], hw[2 * U - 1], cur[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) x[u] = xp[u];
+#pragma unroll
+      for (int k = 0; k < 2 * U - 1; ++k) hw[k] = __ldg(hp + 1 + k);   // h[1 .. 2U-1]
+#pragma unroll
+      for (int up = 0; up < U; ++up) cur[up] = overwrite ? 0.f : dp[up];
+#pragma unroll
+      for (int up = 0; up < U; ++up) {
+#pragma unroll
+        for (int u = 0; u < U; ++u) cur[up] = fmaf(hw[U + up - u - 1], x[u], cur[up]);
+      }
+      acc = cur[0];
+#pragma unroll
+      for (int up = 1; up < U; ++up) dp[up] = cur[up];
+    }
+    accs[li * 32 + lane] = acc;
+  }
+  __syncthreads();
+  if (li != 0 || !ok) return;
+  const int b = s - d * g.B;
+  const size_t io = (size_t)b * g.D + d;
+  float a;
+  if (x_t) {
+    a = round_act(load_token(x_t, io, g.bf16), g.bf16);
+    state[slot_index(g, 0, s, t)] = a;
+  } else {
+    a = state[slot_index(g, 0, s, t)];
+  }
   float y = 0.f;
   for (int l = 1; l <= g.M; ++l) {
-    const size_t si = slot_index(g, l, s, t);
-    const float acc = (t == 0) ? 0.f : state[si];
-    const float h0 = taps[((size_t)(l - 1) * g.D + d) * g.L];
-    y = fmaf(h0, a, acc);
+    y = fmaf(h0s[(l - 1) * 32 + lane], a, accs[(l - 1) * 32 + lane]);
     if (l < g.M) {
       a = round_act(tanhf(y), g.bf16);
-      state[si] = a;
+      state[slot_index(g, l, s, t)] = a;
     }
   }
   y_t[io] = y;
@@ -42,7 +130,24 @@ __global__ void k_token(Dims g, float* __restrict__ state, const float* __restri
 }
 
 cudaError_t launch_token(const Dims& g, float* state, const float* taps, int t, const void* x_t,
-                         const float* eps_t, float eps_scale, float* y_t, cudaStream_t st) {
+                         const float* eps_t, float eps_scale, float* y_t, cudaStream_t st, int block_u) {
+  if (g.M <= kTokenMaxLayers) {
+    const unsigned blocks = (unsigned)((g.S + 31) / 32);
+    const unsigned threads = 32u * (unsigned)g.M;
+    const size_t smem = (size_t)2 * g.M * 32 * sizeof(float);
+#define FI_TOKEN_PAR(UU) k_token_par<UU><<<blocks, threads, smem, st>>>(g, state, taps, t, x_t, eps_t, eps_scale, y_t)
+    switch (block_u) {
+      case 0: FI_TOKEN_PAR(0); break;
+      case 1: FI_TOKEN_PAR(1); break;
+      case 2: FI_TOKEN_PAR(2); break;
+      case 4: FI_TOKEN_PAR(4); break;
+      case kTokenBlockMax: FI_TOKEN_PAR(kTokenBlockMax); break;
+      default: return cudaErrorInvalidValue;
+    }
+#undef FI_TOKEN_PAR
+    return cudaGetLastError();
+  }
+  if (block_u != 0) return cudaErrorInvalidValue;
   const int threads = 128;
   k_token<<<(g.S + threads - 1) / threads, threads, 0, st>>>(g, state, taps, t, x_t, eps_t, eps_scale, y_t);
   return cudaGetLastError();
@@ -81,6 +186,31 @@ __global__ void k_tile_direct(Dims g, float* __restrict__ state, const float* __
   }
 }
 
+// The same block for small sides (U <= 32, the blocks fi_step takes from HBM at
+// most positions): one thread per (row, target), U threads per row, so a launch
+// is a few waves of short threads instead of one CTA per row. Taps h[U+u'-u] are
+// contiguous across a row's threads; its sources are the same for all of them.
+__global__ void k_tile_direct_small(Dims g, float* __restrict__ state, const float* __restrict__ taps, int i,
+                                    int log2u, int overwrite, int t_min) {
+  const int U = 1 << log2u;
+  const long gid = (long)blockIdx.x * blockDim.x + threadIdx.x;
+  const long row = gid >> log2u;        // ((l-1)*D + d)*B + b
+  if (row >= (long)g.M * g.S) return;
+  const int up = (int)(gid & (U - 1));
+  if (i + up < t_min) return;
+  const int b = (int)(row % g.B);
+  const long ld = row / g.B;
+  const int d = (int)(ld % g.D);
+  const int l = (int)(ld / g.D) + 1;
+  const int s = d * g.B + b;
+  const float* hp = taps + ((size_t)(l - 1) * g.D + d) * g.L + U + up;
+  const float* xp = state + slot_index(g, l - 1, s, i - U);
+  float sum = 0.f;
+  for (int u = 0; u < U; ++u) sum = fmaf(__ldg(hp - u), __ldg(xp + u), sum);
+  float* dp = state + slot_index(g, l, s, i + up);
+  *dp = overwrite ? sum : *dp + sum;
+}
+
 // The same block for sides whose taps and sources do not fit in shared memory:
 // taps and sources are read through the cache (every thread of the CTA reads the
 // same source at the same time, and neighbouring threads neighbouring taps).
@@ -108,6 +238,13 @@ cudaError_t launch_tile_direct(const Dims& g, float* state, const float* taps, i
   const long blocks_big = (long)g.M * g.D * g.B;
   if (U > 8192) {
     k_tile_direct_big<<<(unsigned)blocks_big, 256, 0, st>>>(g, state, taps, i, U, is_pow2(i) ? 1 : 0, t_min);
+    return cudaGetLastError();
+  }
+  if (U <= 32) {
+    const long threads_total = (long)g.M * g.S * U;
+    const int threads = 256;
+    k_tile_direct_small<<<(unsigned)((threads_total + threads - 1) / threads), threads, 0, st>>>(
+        g, state, taps, i, ilog2(U), is_pow2(i) ? 1 : 0, t_min);
     return cudaGetLastError();
   }
   const size_t smem = (size_t)3 * U * sizeof(float);

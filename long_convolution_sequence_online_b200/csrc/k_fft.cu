@@ -22,19 +22,34 @@
 
 namespace fi {
 
+// W_{2N}^k = exp(-i pi k / N) (0 <= k <= N/2) for the split and pack of a real FFT
+// of length 2N: from the table where consecutive k are consecutive entries (N of
+// 2^14 and 2^13), else from the hardware sine/cosine (absolute error about 2^-21),
+// since a warp's table loads at a stride of 2^15/(2N) entries touch one sector each.
+template <int N>
+__device__ __forceinline__ float2 split_twiddle(const float2* __restrict__ tw, int k) {
+  constexpr int twstep = kTwiddleN / (2 * N);
+  if constexpr (twstep <= 2) {
+    return __ldg(tw + k * twstep);
+  } else {
+    float sn, cs;
+    __sincosf((float)k * (3.14159265358979323846f / (float)N), &sn, &cs);
+    return make_float2(cs, -sn);
+  }
+}
+
 // Spectrum split + product + inverse pack, in place on sm (N complex points).
 // H: N+1 spectrum values. Threads [0, T) of the transform.
 template <int N, int T>
 __device__ __forceinline__ void spectral_product(float2* sm, int tid, const float2* __restrict__ H,
                                                  const float2* __restrict__ tw) {
-  constexpr int twstep = kTwiddleN / (2 * N);
 #pragma unroll
   for (int k = tid; k <= N / 2; k += T) {
     const int kk = (N - k) & (N - 1);
     const float2 zk = sm[fft_pad<N, T>(k)], zn = sm[fft_pad<N, T>(kk)];
     const float2 E = make_float2(0.5f * (zk.x + zn.x), 0.5f * (zk.y - zn.y));
     const float2 O = make_float2(0.5f * (zk.y + zn.y), -0.5f * (zk.x - zn.x));
-    const float2 W = __ldg(tw + k * twstep);
+    const float2 W = split_twiddle<N>(tw, k);
     const float2 WO = cmul(W, O);
     const float2 Xk = cadd(E, WO);
     const float2 Xn = cconj(csub(E, WO));
@@ -68,7 +83,7 @@ __device__ __forceinline__ void stage_dst(float2* ds, int tid, bool active, cons
 // its first pass read straight from HBM; the result is left in sm.
 template <int N, int T, class Sync>
 __device__ __forceinline__ void fwd_from_global(float2* sm, int tid, bool active, const float2* __restrict__ src,
-                                                const float2* __restrict__ tw, Sync sync) {
+                                                Sync sync) {
   using S = FftShape<N, T>;
   {
     constexpr int R = 1 << S::rb(0);
@@ -80,11 +95,11 @@ __device__ __forceinline__ void fwd_from_global(float2* sm, int tid, bool active
       for (int r = 0; r < R; ++r)
         v[k * R + r] = (active && r < R / 2) ? src[j + r * (N / R)] : make_float2(0.f, 0.f);
     }
-    pass_compute<N, T, false, 0>(v, tid, tw);
+    pass_compute<N, T, false, 0>(v, tid);
     pass_store<N, T, 0>(sm, v, tid);
     sync();
   }
-  smem_passes<N, T, false, S::rb(0), false>(sm, tid, tw, sync);
+  smem_passes<N, T, false, S::rb(0), false>(sm, tid, sync);
 }
 
 // Inverse transform of the packed spectrum in sm, its last pass written straight
@@ -92,15 +107,14 @@ __device__ __forceinline__ void fwd_from_global(float2* sm, int tid, bool active
 // staged accumulators (or stored, for the first block to reach them).
 template <int N, int T, class Sync>
 __device__ __forceinline__ void inv_to_global(float2* sm, const float2* ds, int tid, bool active,
-                                              float2* __restrict__ dst, const float2* __restrict__ tw, int overwrite,
-                                              int w_min, Sync sync) {
+                                              float2* __restrict__ dst, int overwrite, int w_min, Sync sync) {
   using S = FftShape<N, T>;
-  smem_passes<N, T, true, 0, true>(sm, tid, tw, sync);
+  smem_passes<N, T, true, 0, true>(sm, tid, sync);
   constexpr int DL = last_pass_done<N, T>();
   constexpr int R = 1 << S::rb(DL);
   float2 v[S::P];
   pass_load<N, T, DL>(sm, v, tid);
-  pass_compute<N, T, true, DL>(v, tid, tw);
+  pass_compute<N, T, true, DL>(v, tid);
   asm volatile("cp.async.wait_all;" ::: "memory");
   sync();
   if (active) {
@@ -129,10 +143,10 @@ __device__ __forceinline__ void tile_fft_body(float2* sm, float2* ds, int tid, b
                                               float2* __restrict__ dst, const float2* __restrict__ H,
                                               const float2* __restrict__ tw, int overwrite, int w_min, Sync sync) {
   stage_dst<N, T>(ds, tid, active, dst, overwrite);
-  fwd_from_global<N, T>(sm, tid, active, src, tw, sync);
+  fwd_from_global<N, T>(sm, tid, active, src, sync);
   spectral_product<N, T>(sm, tid, H, tw);
   sync();
-  inv_to_global<N, T>(sm, ds, tid, active, dst, tw, overwrite, w_min, sync);
+  inv_to_global<N, T>(sm, ds, tid, active, dst, overwrite, w_min, sync);
 }
 
 // ---------------------------------------------------------------------------
@@ -150,13 +164,12 @@ __device__ __forceinline__ void tile_fft_body(float2* sm, float2* ds, int tid, b
 template <int N, int T>
 __device__ __forceinline__ void store_half_spectrum(const float2* sm, int tid, float2* __restrict__ out,
                                                     const float2* __restrict__ tw) {
-  constexpr int twstep = kTwiddleN / (2 * N);
   for (int k = tid; k <= N / 2; k += T) {
     const int kk = (N - k) & (N - 1);
     const float2 zk = sm[fft_pad<N, T>(k)], zn = sm[fft_pad<N, T>(kk)];
     const float2 E = make_float2(0.5f * (zk.x + zn.x), 0.5f * (zk.y - zn.y));
     const float2 O = make_float2(0.5f * (zk.y + zn.y), -0.5f * (zk.x - zn.x));
-    const float2 WO = cmul(__ldg(tw + k * twstep), O);
+    const float2 WO = cmul(split_twiddle<N>(tw, k), O);
     out[k] = cadd(E, WO);
     if (k != N / 2) out[N - k] = cconj(csub(E, WO));
   }
@@ -178,8 +191,8 @@ k_part_fwd(Dims g, const float* __restrict__ state, float2* __restrict__ xs, con
   const int l = (int)(row / g.S) + 1, s = (int)(row % g.S);
   const int U = m * N;
   const float2* src = reinterpret_cast<const float2*>(state + slot_index(g, l - 1, s, i - U + j * N));
-  if constexpr (T <= 32) fwd_from_global<N, T>(sm, tid, active, src, tw, SyncWarp());
-  else fwd_from_global<N, T>(sm, tid, active, src, tw, SyncBlock());
+  if constexpr (T <= 32) fwd_from_global<N, T>(sm, tid, active, src, SyncWarp());
+  else fwd_from_global<N, T>(sm, tid, active, src, SyncBlock());
   if (active) store_half_spectrum<N, T>(sm, tid, xs + (size_t)item * (N + 1), tw);
 }
 
@@ -189,7 +202,6 @@ __global__ void __launch_bounds__(fft_cta_threads(N))
 k_part_inv(Dims g, float* __restrict__ state, const float2* __restrict__ xs, const float2* __restrict__ gspec,
            const float2* __restrict__ tw, int i, int m, int overwrite, int t_min) {
   constexpr int T = fft_threads(N), F = fft_per_cta(N);
-  constexpr int twstep = kTwiddleN / (2 * N);
   extern __shared__ float2 fsm[];
   const int sub = threadIdx.x / T, tid = threadIdx.x - sub * T;
   float2* sm = fsm + sub * fft_smem_elems(N);
@@ -215,7 +227,7 @@ k_part_inv(Dims g, float* __restrict__ state, const float2* __restrict__ xs, con
       yf = cadd(yf, a);
       yn = cadd(yn, b);
     }
-    const float2 W = __ldg(tw + f * twstep);
+    const float2 W = split_twiddle<N>(tw, f);
     const float2 A = cadd(yf, cconj(yn));
     const float2 Bv = cmul(csub(yf, cconj(yn)), cconj(W));
     sm[fft_pad<N, T>(f & (N - 1))] = make_float2(A.x - Bv.y, A.y + Bv.x);
@@ -223,10 +235,10 @@ k_part_inv(Dims g, float* __restrict__ state, const float2* __restrict__ xs, con
   }
   if constexpr (T <= 32) {
     __syncwarp();
-    inv_to_global<N, T>(sm, ds, tid, active, dst, tw, overwrite, t_min - (i + k * N), SyncWarp());
+    inv_to_global<N, T>(sm, ds, tid, active, dst, overwrite, t_min - (i + k * N), SyncWarp());
   } else {
     __syncthreads();
-    inv_to_global<N, T>(sm, ds, tid, active, dst, tw, overwrite, t_min - (i + k * N), SyncBlock());
+    inv_to_global<N, T>(sm, ds, tid, active, dst, overwrite, t_min - (i + k * N), SyncBlock());
   }
 }
 
@@ -267,15 +279,16 @@ k_tile_fft(Dims g, float* __restrict__ state, const float2* __restrict__ spec,
 // points j + r N2/R, which is exactly what the inverse's first pass of the same
 // radix reads (the inverse takes its passes in the opposite radix order).
 // ---------------------------------------------------------------------------
-template <int N2, int T>
+template <int N2, int T, int PL = 0>
 __device__ __forceinline__ void tile_fft2_body(float2* sm, float* ds, int tid, bool active,
                                                const float* __restrict__ src1, const float* __restrict__ src2,
                                                float* __restrict__ dst1, float* __restrict__ dst2,
-                                               const float2* __restrict__ H, const float2* __restrict__ tw,
+                                               const float2* __restrict__ H,
                                                int overwrite, int w_min) {
   constexpr int U = N2 / 2;
-  using SF = FftShape<N2, T, false>;
-  using SI = FftShape<N2, T, true>;
+  constexpr int SHF = PL << 4, SHI = (PL << 4) | 1;   // forward plan; the inverse takes it reversed
+  using SF = FftShape<N2, T, SHF>;
+  using SI = FftShape<N2, T, SHI>;
   auto sync = [] {
     if constexpr (T <= 32) __syncwarp();
     else __syncthreads();
@@ -303,19 +316,19 @@ __device__ __forceinline__ void tile_fft2_body(float2* sm, float* ds, int tid, b
         v[k * R + r] = (active && r < R / 2) ? make_float2(__ldg(src1 + m), __ldg(src2 + m)) : make_float2(0.f, 0.f);
       }
     }
-    pass_compute<N2, T, false, 0, false>(v, tid, tw);
+    pass_compute<N2, T, false, 0, SHF>(v, tid);
     if constexpr (!SF::last(0)) {
-      pass_store<N2, T, 0, false>(sm, v, tid);
+      pass_store<N2, T, 0, SHF>(sm, v, tid);
       sync();
-      smem_passes<N2, T, false, SF::rb(0), true, false>(sm, tid, tw, sync);
-      constexpr int DL = last_pass_done<N2, T, 0, false>();
-      pass_load<N2, T, DL, false>(sm, v, tid);
-      pass_compute<N2, T, false, DL, false>(v, tid, tw);
+      smem_passes<N2, T, false, SF::rb(0), true, SHF>(sm, tid, sync);
+      constexpr int DL = last_pass_done<N2, T, 0, SHF>();
+      pass_load<N2, T, DL, SHF>(sm, v, tid);
+      pass_compute<N2, T, false, DL, SHF>(v, tid);
     }
   }
   {
     // spectrum product on the points this thread holds: j + r N2/R
-    constexpr int R = 1 << SF::rb(last_pass_done<N2, T, 0, false>());
+    constexpr int R = 1 << SF::rb(last_pass_done<N2, T, 0, SHF>());
     static_assert(R == (1 << SI::rb(0)), "inverse must start with the forward's last radix");
 #pragma unroll
     for (int k = 0; k < SF::P / R; ++k) {
@@ -330,20 +343,20 @@ __device__ __forceinline__ void tile_fft2_body(float2* sm, float* ds, int tid, b
     }
   }
   // inverse, first pass in registers
-  pass_compute<N2, T, true, 0, true>(v, tid, tw);
+  pass_compute<N2, T, true, 0, SHI>(v, tid);
   if constexpr (!SI::last(0)) {
     sync();   // every thread is done reading sm in the forward's last pass
-    pass_store<N2, T, 0, true>(sm, v, tid);
+    pass_store<N2, T, 0, SHI>(sm, v, tid);
     sync();
-    smem_passes<N2, T, true, SI::rb(0), true, true>(sm, tid, tw, sync);
-    constexpr int DL = last_pass_done<N2, T, 0, true>();
-    pass_load<N2, T, DL, true>(sm, v, tid);
-    pass_compute<N2, T, true, DL, true>(v, tid, tw);
+    smem_passes<N2, T, true, SI::rb(0), true, SHI>(sm, tid, sync);
+    constexpr int DL = last_pass_done<N2, T, 0, SHI>();
+    pass_load<N2, T, DL, SHI>(sm, v, tid);
+    pass_compute<N2, T, true, DL, SHI>(v, tid);
   }
   asm volatile("cp.async.wait_all;" ::: "memory");
   sync();
   if (active) {
-    constexpr int R = 1 << SI::rb(last_pass_done<N2, T, 0, true>());
+    constexpr int R = 1 << SI::rb(last_pass_done<N2, T, 0, SHI>());
 #pragma unroll
     for (int k = 0; k < SI::P / R; ++k) {
       const int j = tid + k * T;
@@ -371,9 +384,9 @@ __device__ __forceinline__ void tile_fft2_body(float2* sm, float* ds, int tid, b
 // sides that hold 32 points per thread (8192: 4.1 -> 6.5 ms).
 __host__ __device__ constexpr int fft2_min_blocks(int n2) { return n2 == 512 ? 3 : n2 == 4096 ? 2 : 1; }
 
-template <int N2, int T>
+template <int N2, int T, int PL = 0>
 __global__ void __launch_bounds__(T >= 128 ? T : 128, fft2_min_blocks(N2))
-k_tile_fft2(Dims g, float* __restrict__ state, const float2* __restrict__ spec, const float2* __restrict__ tw, int i,
+k_tile_fft2(Dims g, float* __restrict__ state, const float2* __restrict__ spec, int i,
             int overwrite, int t_min) {
   constexpr int U = N2 / 2;
   constexpr int F = T >= 128 ? 1 : 128 / T;
@@ -392,7 +405,7 @@ k_tile_fft2(Dims g, float* __restrict__ state, const float2* __restrict__ spec, 
   float* dst1 = state + slot_index(g, l, s1, i);
   float* dst2 = state + slot_index(g, l, s1 + 1, i);
   const float2* H = spec + ((size_t)(l - 1) * g.D + d) * (U + 1);
-  tile_fft2_body<N2, T>(sm, ds, tid, active, src1, src2, dst1, dst2, H, tw, overwrite, t_min - i);
+  tile_fft2_body<N2, T, PL>(sm, ds, tid, active, src1, src2, dst1, dst2, H, overwrite, t_min - i);
 }
 
 // ---------------------------------------------------------------------------
@@ -439,19 +452,19 @@ k_prefix_conv(Dims g, float* __restrict__ state, const float2* __restrict__ spec
                            : make_float2(0.f, 0.f);
       }
     }
-    pass_compute<N, T, false, 0>(v, tid, tw);
+    pass_compute<N, T, false, 0>(v, tid);
     pass_store<N, T, 0>(sm, v, tid);
     sync();
   }
-  smem_passes<N, T, false, S::rb(0), false>(sm, tid, tw, sync);
+  smem_passes<N, T, false, S::rb(0), false>(sm, tid, sync);
   spectral_product<N, T>(sm, tid, H, tw);
   sync();
-  smem_passes<N, T, true, 0, true>(sm, tid, tw, sync);
+  smem_passes<N, T, true, 0, true>(sm, tid, sync);
   constexpr int DL = last_pass_done<N, T>();
   constexpr int R = 1 << S::rb(DL);
   float2 v[S::P];
   pass_load<N, T, DL>(sm, v, tid);
-  pass_compute<N, T, true, DL>(v, tid, tw);
+  pass_compute<N, T, true, DL>(v, tid);
   if (!active) return;
   const size_t io = (size_t)b * g.D + d;
   float* dst = state + slot_index(g, l, s, 0);
@@ -506,10 +519,10 @@ k_spectra(Dims g, const float* __restrict__ taps, float2* __restrict__ spec, con
     sm[fft_pad<N, T>(m)] = (active && (!pad || m < N / 2)) ? src[m] : make_float2(0.f, 0.f);
   if constexpr (T <= 32) {
     __syncwarp();
-    fft_smem<N, T, false>(sm, tid, tw, SyncWarp());
+    fft_smem<N, T, false>(sm, tid, SyncWarp());
   } else {
     __syncthreads();
-    fft_smem<N, T, false>(sm, tid, tw, SyncBlock());
+    fft_smem<N, T, false>(sm, tid, SyncBlock());
   }
   if (!active) return;
   float2* H = spec + (size_t)item * (N + 1);
@@ -527,8 +540,7 @@ k_spectra(Dims g, const float* __restrict__ taps, float2* __restrict__ spec, con
 
 template <int N>
 __global__ void __launch_bounds__(fft_cta_threads(N))
-k_debug_fft(int count, const float2* __restrict__ in, float2* __restrict__ out, int inverse,
-            const float2* __restrict__ tw) {
+k_debug_fft(int count, const float2* __restrict__ in, float2* __restrict__ out, int inverse) {
   constexpr int T = fft_threads(N), F = fft_per_cta(N);
   extern __shared__ float2 fsm[];
   const int sub = threadIdx.x / T, tid = threadIdx.x - sub * T;
@@ -538,12 +550,12 @@ k_debug_fft(int count, const float2* __restrict__ in, float2* __restrict__ out, 
   for (int m = tid; m < N; m += T) sm[fft_pad<N, T>(m)] = active ? in[item * N + m] : make_float2(0.f, 0.f);
   if constexpr (T <= 32) {
     __syncwarp();
-    if (inverse) fft_smem<N, T, true>(sm, tid, tw, SyncWarp());
-    else fft_smem<N, T, false>(sm, tid, tw, SyncWarp());
+    if (inverse) fft_smem<N, T, true>(sm, tid, SyncWarp());
+    else fft_smem<N, T, false>(sm, tid, SyncWarp());
   } else {
     __syncthreads();
-    if (inverse) fft_smem<N, T, true>(sm, tid, tw, SyncBlock());
-    else fft_smem<N, T, false>(sm, tid, tw, SyncBlock());
+    if (inverse) fft_smem<N, T, true>(sm, tid, SyncBlock());
+    else fft_smem<N, T, false>(sm, tid, SyncBlock());
   }
   if (!active) return;
   for (int m = tid; m < N; m += T) out[item * N + m] = sm[fft_pad<N, T>(m)];
@@ -579,19 +591,21 @@ static cudaError_t tile_fft_n(const Dims& g, float* state, const float2* spec, c
 __host__ __device__ constexpr int fft2_points(int n2) {
   return (n2 == 512 || n2 == 1024 || n2 == 8192 || n2 == 16384) ? 32 : 16;
 }
+// Pass plan of the paired blocks (FftShape's PL; 0 = radix min(32, P) passes).
+__host__ __device__ constexpr int fft2_plan(int /*n2*/) { return 0; }
 
-template <int N2, int P = fft2_points(N2)>
+template <int N2, int P = fft2_points(N2), int PL = fft2_plan(N2)>
 static cudaError_t tile_fft2_n(const Dims& g, float* state, const float2* spec, const float2* tw, int i,
                                int t_min, cudaStream_t st) {
   constexpr int T = N2 / P;
   constexpr int F = T >= 128 ? 1 : 128 / T;
   const size_t smem = (size_t)F * (fft_smem_elems(N2) * sizeof(float2) + (size_t)N2 * sizeof(float));
-  cudaError_t e = prepare(k_tile_fft2<N2, T>, smem);
+  cudaError_t e = prepare(k_tile_fft2<N2, T, PL>, smem);
   if (e != cudaSuccess) return e;
   const long items = (long)g.M * (g.S / 2);
   const long blocks = (items + F - 1) / F;
   const int overwrite = is_pow2(i) ? 1 : 0;
-  k_tile_fft2<N2, T><<<(unsigned)blocks, T * F, smem, st>>>(g, state, spec, tw, i, overwrite, t_min);
+  k_tile_fft2<N2, T, PL><<<(unsigned)blocks, T * F, smem, st>>>(g, state, spec, i, overwrite, t_min);
   return cudaGetLastError();
 }
 
@@ -614,7 +628,7 @@ static cudaError_t debug_fft_n(int count, const float2* in, float2* out, int inv
   cudaError_t e = prepare(k_debug_fft<N>, smem);
   if (e != cudaSuccess) return e;
   const long blocks = ((long)count + fft_per_cta(N) - 1) / fft_per_cta(N);
-  k_debug_fft<N><<<(unsigned)blocks, fft_cta_threads(N), smem, st>>>(count, in, out, inverse, tw);
+  k_debug_fft<N><<<(unsigned)blocks, fft_cta_threads(N), smem, st>>>(count, in, out, inverse);
   return cudaGetLastError();
 }
 

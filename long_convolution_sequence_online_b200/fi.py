@@ -148,6 +148,10 @@ class Context:
     def step(self, x_t, y_t):
         _check(lib.fi_step(self._h, _ptr(x_t), _ptr(y_t)), "fi_step")
 
+    def step_ptr(self, x_ptr: int, y_ptr: int):
+        """fi_step on raw device addresses (a loop over positions without tensor views)."""
+        _check(lib.fi_step(self._h, x_ptr, y_ptr), "fi_step")
+
     def generate(self, n: int, x0, eps, y_out, eps_scale: float = 0.1, rec=None):
         _check(lib.fi_generate(self._h, n, _ptr(x0), _ptr(eps), eps_scale, _ptr(y_out), _ptr(rec)), "fi_generate")
 

@@ -73,6 +73,9 @@ WORKLOADS["hyena-18x864-L2K-B4"] = Workload("hyena-18x864-L2K-B4", 18, 864, 2048
 WORKLOADS["hyena-18x64-L32K-B4"] = Workload("hyena-18x64-L32K-B4", 18, 64, 32768, 4, "f32", 1e-3, 1e-1)
 # ... and of the batched bf16 stack (8 layers, B = 64): 128 channels at L = 4096.
 WORKLOADS["sweep-8x128-L4K-bf16-B64"] = Workload("sweep-8x128-L4K-bf16-B64", 8, 128, 4096, 64, "bf16", 1e-3, 1e-1)
+# ... and of the long-range stack: 64 channels at the full L = 131072 (which reaches the
+# partitioned blocks of sides 32768 and 65536; 0.2 GB of state).
+WORKLOADS["longrange-4x64-L128K-bf16"] = Workload("longrange-4x64-L128K-bf16", 4, 64, 131072, 1, "bf16", 1e-5, 1e-3)
 
 HEADLINE = "hyena-18x864-L32K-B4"
 

@@ -162,6 +162,40 @@ def test_step_api_teacher_forced(fi):
         ctx.step(tt[0].contiguous(), ys[0])
 
 
+@pytest.mark.parametrize("M,D,L,B,dtype", [(1, 8, 256, 1, "f32"), (3, 6, 1024, 2, "f32"), (18, 4, 512, 3, "f32"),
+                                           (2, 8, 512, 2, "bf16"), (33, 2, 128, 1, "f32")])
+def test_step_api_every_position(fi, M, D, L, B, dtype):
+    # fi_step for every position on given tokens: the red cells with the small
+    # direct blocks fused into the same launch (M <= 32; M = 33 takes the
+    # one-thread-per-stream kernel and separate block launches), every layer
+    # checked against the oracle's causal convolution of the recorded inputs.
+    w = synth.Workload(f"step-{M}x{D}-L{L}", M, D, L, B, dtype, 1e-3, 1e-1)
+    inp = gpu_inputs(w, 21)
+    ctx = fi.Context(inp["h"], w.batch, w.dtype)
+    toks = synth.token_stream(w, 21)
+    td = torch.bfloat16 if dtype == "bf16" else torch.float32
+    tt = torch.from_numpy(toks).cuda().to(td)
+    ys = torch.empty((L, B, D), dtype=torch.float32, device="cuda")
+    for t in range(L):
+        ctx.step(tt[t].contiguous(), ys[t])
+    torch.cuda.synchronize()
+    acts = [a.cpu().numpy() for a in read_all_activations(ctx, L)]
+    ctx.close()
+    h64 = oracle_filters(inp["h_np"], dtype)
+    R = oracle.bf16_round if dtype == "bf16" else (lambda v: v)
+    tol = TOL[dtype]
+    y_np = ys.cpu().numpy()
+    for b in range(B):
+        for d in range(D):
+            for l in range(M):
+                yl = oracle.causal_conv(h64[l, d], acts[l][:, b, d].astype(np.float64))
+                if l + 1 < M:
+                    want = R(np.tanh(yl))
+                    assert np.max(np.abs(acts[l + 1][:, b, d] - want)) <= (2e-2 if dtype == "bf16" else 1e-5)
+                else:
+                    assert oracle.stream_error(y_np[:, b, d], yl) <= tol
+
+
 def test_bf16_small(fi):
     w = _workload(3, 8, 512, 2, dtype="bf16", lam=(1e-5, 1e-3))
     ctx, inp, y, rec, acts = _run_generate(fi, w, seed=3, chunk=16, fft_from=64)
