@@ -55,6 +55,15 @@ inline bool is_pow2(int64_t v) { return v > 0 && (v & (v - 1)) == 0; }
 inline int lowbit(int i) { return i & -i; }
 inline int highbit(int i) { int r = 1; while ((int64_t)r * 2 <= i) r *= 2; return r; }
 
+// Programmatic dependent launch. Block kernels call pdl_launch_dependents() on
+// entry, so that the next launch on the stream, the chunk kernel (launched with
+// programmatic stream serialization), may start once every block CTA is
+// running; the chunk kernel loads what no block writes (taps, noise) and then
+// calls pdl_wait_primary(), which returns when the preceding grid has completed
+// and its writes are visible. Both are no-ops for a launch without the attribute.
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait_primary() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ---------------------------------------------------------------- launchers (kernels/*.cu)
 // All return cudaSuccess or the launch error.
 

@@ -163,6 +163,7 @@ cudaError_t launch_token(const Dims& g, float* state, const float* taps, int t, 
 // ---------------------------------------------------------------------------
 __global__ void k_tile_direct(Dims g, float* __restrict__ state, const float* __restrict__ taps, int i, int U,
                               int overwrite, int t_min) {
+  pdl_launch_dependents();
   extern __shared__ float dsm[];
   float* hs = dsm;          // taps h[0..2U)
   float* xs = dsm + 2 * U;  // sources a[i-U..i)
@@ -192,6 +193,7 @@ __global__ void k_tile_direct(Dims g, float* __restrict__ state, const float* __
 // contiguous across a row's threads; its sources are the same for all of them.
 __global__ void k_tile_direct_small(Dims g, float* __restrict__ state, const float* __restrict__ taps, int i,
                                     int log2u, int overwrite, int t_min) {
+  pdl_launch_dependents();
   const int U = 1 << log2u;
   const long gid = (long)blockIdx.x * blockDim.x + threadIdx.x;
   const long row = gid >> log2u;        // ((l-1)*D + d)*B + b
@@ -216,6 +218,7 @@ __global__ void k_tile_direct_small(Dims g, float* __restrict__ state, const flo
 // same source at the same time, and neighbouring threads neighbouring taps).
 __global__ void k_tile_direct_big(Dims g, float* __restrict__ state, const float* __restrict__ taps, int i, int U,
                                   int overwrite, int t_min) {
+  pdl_launch_dependents();
   const long cta = blockIdx.x;          // ((l-1)*D + d)*B + b
   const int b = (int)(cta % g.B);
   const long ld = cta / g.B;

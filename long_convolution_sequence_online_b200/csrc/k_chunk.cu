@@ -464,17 +464,40 @@ __global__ void __launch_bounds__(kChunkMaxThreads) k_chunk(Dims g, ChunkArgs a,
     if (l == 0) return t == a.p0 && a.x0 == nullptr;
     return t >= 1 && highbit_dev(t) <= a.last_done;
   };
+  {
+    const int wid = tid >> 5, lid = tid & 31, nw = nt >> 5;
+    for (int r = r0 + wid; r < r1; r += nw) {
+      const float* src = a.eps + (size_t)(a.c + r - a.gen_base) * g.S;
+      for (int gg = lid; gg < Gc; gg += 32) {
+        const int s = s0 + gg, d = s / g.B, b = s - d * g.B;
+        cp_async4(ep + r * G + gg, src + (size_t)b * g.D + d);
+      }
+    }
+  }
+  // tp[.][CH]: the tap one past the window, zero (pieces that reach the spare
+  // position read it)
+  for (int k = tid; k < M * GdMax * (TPS - CH); k += nt) tp[(k / (TPS - CH)) * TPS + CH + k % (TPS - CH)] = 0.f;
+  for (int k = tid; k < M * Gd; k += nt) {
+    const int l = k / Gd, dl = k - l * Gd;
+    const float* hrow = a.taps + ((size_t)l * g.D + d_lo + dl) * g.L;
+    hv4[l * GdMax + dl] = g.L >= 4 ? __ldg(reinterpret_cast<const float4*>(hrow))
+                                   : make_float4(hrow[0], g.L > 1 ? hrow[1] : 0.f, 0.f, 0.f);
+  }
+  // The taps and the noise are inputs no block writes, so they are fetched
+  // before pdl_wait_primary() (while the preceding block launch drains); the
+  // window, which that block writes, after it.
   if (CH < 4) {
+    for (int idx = tid; idx < M * Gd * CH; idx += nt) {
+      const int row = idx / CH, j = idx - row * CH;
+      const int l = row / Gd, dl = row - l * Gd;
+      tp[(l * GdMax + dl) * TPS + j] = a.taps[((size_t)l * g.D + d_lo + dl) * g.L + j];
+    }
+    pdl_wait_primary();
     for (int idx = tid; idx < (M + 1) * Gc * CH; idx += nt) {
       const int row = idx / CH, r = idx - row * CH;
       const int l = row / Gc, gg = row - l * Gc;
       const int t = a.c + r;
       win[l * LS + r * GP + gg] = slot_valid(l, t) ? a.state[slot_index(g, l, s0 + gg, t)] : 0.f;
-    }
-    for (int idx = tid; idx < M * Gd * CH; idx += nt) {
-      const int row = idx / CH, j = idx - row * CH;
-      const int l = row / Gd, dl = row - l * Gd;
-      tp[(l * GdMax + dl) * TPS + j] = a.taps[((size_t)l * g.D + d_lo + dl) * g.L + j];
     }
   } else {
     // Items: float4 j (4 positions or taps) of row `row` (a stream, or a
@@ -487,71 +510,57 @@ __global__ void __launch_bounds__(kChunkMaxThreads) k_chunk(Dims g, ChunkArgs a,
     const int lt = lv + (Gd > 1 ? 32 - __clz(Gd - 1) : 0);   // log2 items per tap layer
     const int nwin = (M + 1) << lw, nall = nwin + (M << lt);
     constexpr int kBatch = 12;
-    for (int base = tid; base < nall; base += nt * kBatch) {
-      float4 v[kBatch];
+    // items [nwin, nall) (taps) first, then [0, nwin) (window) after the wait
+    for (int pass = 0; pass < 2; ++pass) {
+      const int beg = pass == 0 ? nwin : 0, end = pass == 0 ? nall : nwin;
+      if (pass == 1) pdl_wait_primary();
+      for (int base = beg + tid; base < end; base += nt * kBatch) {
+        float4 v[kBatch];
 #pragma unroll
-      for (int u = 0; u < kBatch; ++u) {
-        const int idx = base + u * nt;
-        const bool is_win = idx < nwin;
-        const int k = is_win ? idx : idx - nwin;
-        const int sh = is_win ? lw : lt;
-        const int l = k >> sh, rem = k & ((1 << sh) - 1);
-        const int row = rem >> lv, j = rem & (vpr - 1);
-        // every slot of the window lies inside the state, so the load is in
-        // bounds; slots that hold nothing yet are zeroed below
-        if (idx < nall && row < (is_win ? Gc : Gd))
-          v[u] = __ldg(reinterpret_cast<const float4*>(
-              is_win ? a.state + slot_index(g, l, s0 + row, a.c + 4 * j)
-                     : a.taps + ((size_t)l * g.D + d_lo + row) * g.L + 4 * j));
-      }
-#pragma unroll
-      for (int u = 0; u < kBatch; ++u) {
-        const int idx = base + u * nt;
-        const bool is_win = idx < nwin;
-        const int k = is_win ? idx : idx - nwin;
-        const int sh = is_win ? lw : lt;
-        const int l = k >> sh, rem = k & ((1 << sh) - 1);
-        const int row = rem >> lv, j = rem & (vpr - 1);
-        if (idx >= nall || row >= (is_win ? Gc : Gd)) continue;
-        if (is_win) {
-          const int t = a.c + 4 * j;
-          float* w = win + l * LS + 4 * j * GP + row;
-          w[0] = slot_valid(l, t) ? v[u].x : 0.f;
-          w[GP] = slot_valid(l, t + 1) ? v[u].y : 0.f;
-          w[2 * GP] = slot_valid(l, t + 2) ? v[u].z : 0.f;
-          w[3 * GP] = slot_valid(l, t + 3) ? v[u].w : 0.f;
-        } else {
-          float* w = tp + (l * GdMax + row) * TPS + 4 * j;
-          w[0] = v[u].x;
-          w[1] = v[u].y;
-          w[2] = v[u].z;
-          w[3] = v[u].w;
+        for (int u = 0; u < kBatch; ++u) {
+          const int idx = base + u * nt;
+          const bool is_win = idx < nwin;
+          const int k = is_win ? idx : idx - nwin;
+          const int sh = is_win ? lw : lt;
+          const int l = k >> sh, rem = k & ((1 << sh) - 1);
+          const int row = rem >> lv, j = rem & (vpr - 1);
+          // every slot of the window lies inside the state, so the load is in
+          // bounds; slots that hold nothing yet are zeroed below
+          if (idx < end && row < (is_win ? Gc : Gd))
+            v[u] = __ldg(reinterpret_cast<const float4*>(
+                is_win ? a.state + slot_index(g, l, s0 + row, a.c + 4 * j)
+                       : a.taps + ((size_t)l * g.D + d_lo + row) * g.L + 4 * j));
         }
-      }
-    }
-  }
-  {
-    const int wid = tid >> 5, lid = tid & 31, nw = nt >> 5;
-    for (int r = r0 + wid; r < r1; r += nw) {
-      const float* src = a.eps + (size_t)(a.c + r - a.gen_base) * g.S;
-      for (int gg = lid; gg < Gc; gg += 32) {
-        const int s = s0 + gg, d = s / g.B, b = s - d * g.B;
-        cp_async4(ep + r * G + gg, src + (size_t)b * g.D + d);
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+          const int idx = base + u * nt;
+          const bool is_win = idx < nwin;
+          const int k = is_win ? idx : idx - nwin;
+          const int sh = is_win ? lw : lt;
+          const int l = k >> sh, rem = k & ((1 << sh) - 1);
+          const int row = rem >> lv, j = rem & (vpr - 1);
+          if (idx >= end || row >= (is_win ? Gc : Gd)) continue;
+          if (is_win) {
+            const int t = a.c + 4 * j;
+            float* w = win + l * LS + 4 * j * GP + row;
+            w[0] = slot_valid(l, t) ? v[u].x : 0.f;
+            w[GP] = slot_valid(l, t + 1) ? v[u].y : 0.f;
+            w[2 * GP] = slot_valid(l, t + 2) ? v[u].z : 0.f;
+            w[3 * GP] = slot_valid(l, t + 3) ? v[u].w : 0.f;
+          } else {
+            float* w = tp + (l * GdMax + row) * TPS + 4 * j;
+            w[0] = v[u].x;
+            w[1] = v[u].y;
+            w[2] = v[u].z;
+            w[3] = v[u].w;
+          }
+        }
       }
     }
   }
   if (a.x0 != nullptr && tid < Gc) {
     const int s = s0 + tid, d = s / g.B, b = s - d * g.B;
     win[r0 * GP + tid] = round_act(load_token(a.x0, (size_t)b * g.D + d, g.bf16), g.bf16);
-  }
-  // tp[.][CH]: the tap one past the window, zero (pieces that reach the spare
-  // position read it)
-  for (int k = tid; k < M * GdMax * (TPS - CH); k += nt) tp[(k / (TPS - CH)) * TPS + CH + k % (TPS - CH)] = 0.f;
-  for (int k = tid; k < M * Gd; k += nt) {
-    const int l = k / Gd, dl = k - l * Gd;
-    const float* hrow = a.taps + ((size_t)l * g.D + d_lo + dl) * g.L;
-    hv4[l * GdMax + dl] = g.L >= 4 ? __ldg(reinterpret_cast<const float4*>(hrow))
-                                   : make_float4(hrow[0], g.L > 1 ? hrow[1] : 0.f, 0.f, 0.f);
   }
   for (int k = tid; k < kRing * CW; k += nt) {
     mbar_init(act_ready + k, 32);
@@ -825,14 +834,24 @@ cudaError_t launch_chunk(const Dims& g, const ChunkArgs& a_in, int G, cudaStream
   const size_t smem = chunk_smem_bytes(g, a.chunk, G);
   const int blocks = (g.S + G - 1) / G;
   const int nt = chunk_threads(g, G);
+  // programmatic stream serialization: the launch may begin while the block
+  // kernel before it drains (the kernel waits for it before reading the state)
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)blocks);
+  cfg.blockDim = dim3((unsigned)nt);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   if (g.bf16) {
-    if (a.rec) k_chunk<true, true><<<blocks, nt, smem, st>>>(g, a, G);
-    else k_chunk<true, false><<<blocks, nt, smem, st>>>(g, a, G);
-  } else {
-    if (a.rec) k_chunk<false, true><<<blocks, nt, smem, st>>>(g, a, G);
-    else k_chunk<false, false><<<blocks, nt, smem, st>>>(g, a, G);
+    if (a.rec) return cudaLaunchKernelEx(&cfg, k_chunk<true, true>, g, a, G);
+    return cudaLaunchKernelEx(&cfg, k_chunk<true, false>, g, a, G);
   }
-  return cudaGetLastError();
+  if (a.rec) return cudaLaunchKernelEx(&cfg, k_chunk<false, true>, g, a, G);
+  return cudaLaunchKernelEx(&cfg, k_chunk<false, false>, g, a, G);
 }
 
 }  // namespace fi

@@ -201,6 +201,7 @@ template <int N>
 __global__ void __launch_bounds__(fft_cta_threads(N))
 k_part_inv(Dims g, float* __restrict__ state, const float2* __restrict__ xs, const float2* __restrict__ gspec,
            const float2* __restrict__ tw, int i, int m, int overwrite, int t_min) {
+  pdl_launch_dependents();
   constexpr int T = fft_threads(N), F = fft_per_cta(N);
   extern __shared__ float2 fsm[];
   const int sub = threadIdx.x / T, tid = threadIdx.x - sub * T;
@@ -248,6 +249,7 @@ template <int N, int T = fft_threads(N)>
 __global__ void __launch_bounds__(T >= 128 ? T : 128)
 k_tile_fft(Dims g, float* __restrict__ state, const float2* __restrict__ spec,
            const float2* __restrict__ tw, int i, int overwrite, int t_min) {
+  pdl_launch_dependents();
   constexpr int F = T >= 128 ? 1 : 128 / T;
   extern __shared__ float2 fsm[];
   const int sub = threadIdx.x / T, tid = threadIdx.x - sub * T;
@@ -388,6 +390,7 @@ template <int N2, int T, int PL = 0>
 __global__ void __launch_bounds__(T >= 128 ? T : 128, fft2_min_blocks(N2))
 k_tile_fft2(Dims g, float* __restrict__ state, const float2* __restrict__ spec, int i,
             int overwrite, int t_min) {
+  pdl_launch_dependents();
   constexpr int U = N2 / 2;
   constexpr int F = T >= 128 ? 1 : 128 / T;
   extern __shared__ float2 fsm[];

@@ -164,6 +164,7 @@ __device__ __forceinline__ bool bar_wait_or_abort(uint64_t* bar, uint32_t parity
 template <int MT, bool SPLIT>
 __global__ void __launch_bounds__(kTcThreads) k_tile_tc(Dims g, float* __restrict__ state, const float* __restrict__ taps,
                                                         TcPlan p, int i, int overwrite, int* err, int wait_limit) {
+  pdl_launch_dependents();
   extern __shared__ __align__(1024) unsigned char tsm[];
   __shared__ uint64_t full_bar[2], done_bar[2], empty_bar[2];
   __shared__ uint32_t tmem_base_s;
