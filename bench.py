@@ -287,7 +287,8 @@ def oracle_baseline(w: synth.Workload, seed: int, n_pos: int, streams_per_core: 
     streams = [[(int(rng.integers(w.batch)), int(rng.integers(w.channels))) for _ in range(streams_per_core)]
                for _ in range(cores)]
     ctx = mp.get_context("spawn")
-    n1, n2 = max(n_pos // 4, 1), n_pos
+    n2 = min(n_pos, w.length)
+    n1 = max(n2 // 4, 1)
     times = []
     t0 = time.perf_counter()
     with ctx.Pool(cores) as pool:
