@@ -697,53 +697,68 @@ __global__ void __launch_bounds__(kChunkMaxThreads) k_chunk(Dims g, ChunkArgs a,
         if (w < warp) ++tw;
         ++ntw;
       }
-    if (is_tile(warp))
+    if (is_tile(warp)) {
+      // A row group k is (layer k / CW + 1, chain warp k % CW); this warp takes
+      // k = tw, tw + ntw (two at a time when they share a chain warp), then
+      // tw + 2 ntw, ... Everything about a row group but the step is resolved
+      // once here for the first pair (the only one in most shapes), so a step
+      // costs its waits and pieces alone.
+      struct Grp {
+        const float* src;
+        float* dst;
+        const float* taps;
+        int c;
+        bool act;
+      };
+      auto resolve = [&](int k) {
+        Grp q;
+        const int l = k / CW + 1;
+        q.c = k - (l - 1) * CW;
+        const int gg = q.c * 32 + lane;
+        q.act = gg < Gc;
+        const int ggs = q.act ? gg : 0;
+        const int dl = (s0 + ggs) / g.B - d_lo;
+        q.src = win + (l - 1) * LS + ggs;
+        q.dst = win + l * LS + ggs;
+        q.taps = tp + ((l - 1) * GdMax + dl) * TPS;
+        return q;
+      };
+      const int MC = M * CW;
+      const Grp gA0 = resolve(tw < MC ? tw : 0);
+      const Grp gB0 = resolve(tw + ntw < MC ? tw + ntw : 0);
       for (int i = rs; i <= s_last; ++i) {
         // step i reads sources below i: position i-1 must be finished
         const int e0 = a.tab.first[i], e1 = a.tab.first[i + 1];
         const int j = i - rs, jp = i - 1 - r0;
-        // row groups k (layer k / CW + 1, chain warp k % CW), two at a time when
-        // they belong to the same chain warp
-        for (int k = tw; k < M * CW; k += 2 * ntw) {
+        for (int k = tw; k < MC; k += 2 * ntw) {
           const int kB = k + ntw;
-          const int l = k / CW + 1, c = k - (l - 1) * CW;
-          const bool two = kB < M * CW && kB % CW == c;
-          const int lB = two ? kB / CW + 1 : l;
-          if (jp >= 0 && ok) ok = mbar_wait(&act_ready[(jp % kRing) * CW + c], (jp / kRing) & 1, err, false, a.wait_limit);
-          const int gg = c * 32 + lane;
-          if (gg < Gc) {
-            const int dl = (s0 + gg) / g.B - d_lo;
-            const float* src = win + (l - 1) * LS + gg;
-            float* dst = win + l * LS + gg;
-            const float* taps = tp + ((l - 1) * GdMax + dl) * TPS;
+          const Grp gA = k == tw ? gA0 : resolve(k);
+          const bool hasB = kB < MC;
+          const Grp gB = !hasB ? gA : (k == tw ? gB0 : resolve(kB));
+          const bool two = hasB && gB.c == gA.c;
+          if (jp >= 0 && ok)
+            ok = mbar_wait(&act_ready[(jp % kRing) * CW + gA.c], (jp / kRing) & 1, err, false, a.wait_limit);
+          if (gA.act) {
             if (two) {
-              const float* srcB = win + (lB - 1) * LS + gg;
-              float* dstB = win + lB * LS + gg;
-              const float* tapsB = tp + ((lB - 1) * GdMax + dl) * TPS;
-              for (int e = e0; e < e1; ++e) run_piece2(a.tab.e[e], src, dst, taps, srcB, dstB, tapsB, GP);
+              for (int e = e0; e < e1; ++e) run_piece2(a.tab.e[e], gA.src, gA.dst, gA.taps, gB.src, gB.dst, gB.taps, GP);
             } else {
-              for (int e = e0; e < e1; ++e) run_piece(a.tab.e[e], src, dst, taps, GP);
+              for (int e = e0; e < e1; ++e) run_piece(a.tab.e[e], gA.src, gA.dst, gA.taps, GP);
             }
           }
-          mbar_arrive(&tile_done[(j % kRing) * CW + c]);
-          if (two) mbar_arrive(&tile_done[(j % kRing) * CW + c]);
-          else if (kB < M * CW) {
+          mbar_arrive(&tile_done[(j % kRing) * CW + gA.c]);
+          if (two) {
+            mbar_arrive(&tile_done[(j % kRing) * CW + gA.c]);
+          } else if (hasB) {
             // the second row group belongs to another chain warp: on its own
-            const int lb = kB / CW + 1, cb = kB - (lb - 1) * CW;
             if (jp >= 0 && ok)
-              ok = mbar_wait(&act_ready[(jp % kRing) * CW + cb], (jp / kRing) & 1, err, false, a.wait_limit);
-            const int ggb = cb * 32 + lane;
-            if (ggb < Gc) {
-              const int dlb = (s0 + ggb) / g.B - d_lo;
-              const float* srcb = win + (lb - 1) * LS + ggb;
-              float* dstb = win + lb * LS + ggb;
-              const float* tapsb = tp + ((lb - 1) * GdMax + dlb) * TPS;
-              for (int e = e0; e < e1; ++e) run_piece(a.tab.e[e], srcb, dstb, tapsb, GP);
-            }
-            mbar_arrive(&tile_done[(j % kRing) * CW + cb]);
+              ok = mbar_wait(&act_ready[(jp % kRing) * CW + gB.c], (jp / kRing) & 1, err, false, a.wait_limit);
+            if (gB.act)
+              for (int e = e0; e < e1; ++e) run_piece(a.tab.e[e], gB.src, gB.dst, gB.taps, GP);
+            mbar_arrive(&tile_done[(j % kRing) * CW + gB.c]);
           }
         }
       }
+    }
   }
   __syncthreads();
 
