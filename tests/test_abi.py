@@ -143,7 +143,7 @@ def test_chunk_piece_table_covers_every_pair_once_in_time(chunk, retimed):
         if not retimed:
             assert pieces == [(r - U, U, r, U)]
         else:
-            if U <= 4 and r + sh < chunk:
+            if U <= 8 and r + sh < chunk:
                 assert (r - U, U, r + sh, U) in pieces
             assert max(ns * nd for _, ns, _, nd in pieces) <= 64
             assert sum(ns * nd for _, ns, _, nd in pieces) <= 96
