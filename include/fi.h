@@ -237,8 +237,9 @@ FI_API fi_status fi_debug_set_wait_limit(fi_ctx* ctx, int32_t limit);
  * retimed != 0 gives the table of a launch that covers a whole chunk (the chain
  * adds the terms of the first *chain_lags lags itself; the page's tiling of the
  * other pairs is shifted that many positions later, and its blocks are cut into
- * pieces spread over steps), 0 the page's tiling (the block of step r, side
- * lowbit(r), at step r; *chain_lags = 0). Writes up to `cap` entries of 5 int32
+ * pieces spread over steps; retimed == 2: the coarser cut used for stacks of at
+ * most 8 layers), 0 the page's tiling (the block of step r, side lowbit(r), at
+ * step r; *chain_lags = 0). Writes up to `cap` entries of 5 int32
  * (step, first source, sources, first target, targets; positions relative to
  * the chunk start) to out, the entry count to *count, the lags to *chain_lags
  * (may be NULL).

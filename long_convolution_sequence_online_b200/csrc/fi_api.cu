@@ -559,7 +559,7 @@ fi_status fi_debug_chunk_schedule(int32_t chunk, int32_t retimed, int32_t* out, 
   if (!out || !count || cap < 0) return fail(FI_E_INVALID, "bad argument");
   if (!pow2(chunk) || chunk < 2 || chunk > kChunkMaxSteps) return fail(FI_E_INVALID, "chunk must be a power of two in [2, 64]");
   ChunkTable tab{};
-  if (!build_chunk_table(chunk, retimed != 0, &tab)) return fail(FI_E_UNSUPPORTED, "table too long");
+  if (!build_chunk_table(chunk, retimed != 0, &tab, retimed == 2)) return fail(FI_E_UNSUPPORTED, "table too long");
   *count = tab.n;
   if (chain_lags) *chain_lags = tab.lag1;
   for (int j = 0; j < tab.n && j < cap; ++j) {

@@ -128,7 +128,10 @@ struct ChunkTable {
 // lags 1..kChainLags, the page's tiling of the remaining pairs runs kChainLags
 // positions ahead (its targets shifted by kChainLags), with blocks of side 8 and
 // up cut into pieces spread over steps; else the page's blocks, one per step.
-bool build_chunk_table(int chunk, bool retimed, ChunkTable* tab);
+// coarse: the 16-source halves of the side-32 blocks stay 16 x 16 pieces
+// (fewer pieces; measured faster when the chain is short, M <= kCoarseMaxLayers).
+constexpr int kCoarseMaxLayers = 8;
+bool build_chunk_table(int chunk, bool retimed, ChunkTable* tab, bool coarse = false);
 // Sources and targets of a piece kind (for the table's test hook).
 int chunk_piece_sources(int kind);
 int chunk_piece_targets(int kind);

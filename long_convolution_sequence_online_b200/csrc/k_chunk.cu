@@ -230,19 +230,20 @@ struct Piece { int step, s_lo, t_lo, kind; };
 // again. The other pieces get a step later (balance_pieces). Blocks of side 8
 // stay whole: each piece costs a fixed ~200 cycles on top of its products
 // (measured with clock stamps on B200), so one 64-product piece beats four of 16.
-void cut_block(int r, int U, int sh, std::vector<Piece>& out) {
+void cut_block(int r, int U, int sh, bool coarse, std::vector<Piece>& out) {
   if (U <= 8) {
     out.push_back({r, r - U, r + sh, kind_of_square(U)});
     return;
   }
   const int H = U / 2;
-  // 64, 64, 16 products per row (measured on B200: pieces of 32 products took
-  // more steps' worth of per-piece latency than they saved)
-  const int kind = H == 16 ? PK_R16x4 : H == 8 ? PK_SQ8 : PK_SQ4;
+  // 64 products per row (measured on B200: pieces of 32 products took more
+  // steps' worth of per-piece latency than they saved); with a short chain
+  // (few layers) the tile warps set the pace and 16 x 16 pieces measured faster
+  const int kind = H == 16 ? (coarse ? PK_SQ16 : PK_R16x4) : H == 8 ? PK_SQ8 : PK_SQ4;
   const int nd = piece_nd(kind);
   for (int t = r + sh; t < r + sh + U; t += nd) out.push_back({-1, r - U, t, kind});
   for (int t = r + H + sh; t < r + U + sh; t += nd) out.push_back({-1, r - H, t, kind});
-  cut_block(r, H, sh, out);
+  cut_block(r, H, sh, coarse, out);
 }
 
 // A piece reading sources [s_lo, s_lo+ns) and writing targets from t_lo may run
@@ -278,13 +279,13 @@ void balance_pieces(std::vector<Piece>& p, int CH, int sh) {
 int chunk_piece_sources(int kind) { return piece_ns(kind); }
 int chunk_piece_targets(int kind) { return piece_nd(kind); }
 
-bool build_chunk_table(int CH, bool retimed, ChunkTable* tab) {
+bool build_chunk_table(int CH, bool retimed, ChunkTable* tab, bool coarse) {
   std::vector<Piece> p;
   const int sh = retimed ? kChainLags : 0;   // retimed: the chain takes lags 1..sh, pieces the rest
   for (int r = 1; r < CH; ++r) {
     const int U = r & -r;
     std::vector<Piece> q;
-    if (retimed) cut_block(r, U, sh, q);
+    if (retimed) cut_block(r, U, sh, coarse, q);
     else q.push_back({r, r - U, r, kind_of_square(U)});
     // pieces whose targets all lie past the chunk are dropped; one that reaches
     // past it writes its last targets into the window's spare positions (CH and
@@ -848,7 +849,7 @@ cudaError_t launch_chunk(const Dims& g, const ChunkArgs& a_in, int G, cudaStream
   // A launch over a whole chunk runs the re-timed pieces; one over part of a
   // chunk keeps the page's blocks, so the state at a call boundary is canonical.
   const bool whole = a.p0 == a.c && a.p1 == a.c + a.chunk;
-  if (!build_chunk_table(a.chunk, whole, &a.tab)) return cudaErrorInvalidValue;
+  if (!build_chunk_table(a.chunk, whole, &a.tab, g.M <= kCoarseMaxLayers)) return cudaErrorInvalidValue;
   const size_t smem = chunk_smem_bytes(g, a.chunk, G);
   const int blocks = (g.S + G - 1) / G;
   const int nt = chunk_threads(g, G);

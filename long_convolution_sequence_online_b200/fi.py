@@ -230,14 +230,15 @@ def generate_noalloc(h, batch: int, n: int, x0, eps, y_out, dtype: str = "f32", 
                                    _stream(stream)), "fi_generate_noalloc")
 
 
-def chunk_schedule(chunk: int, retimed: bool):
+def chunk_schedule(chunk: int, retimed: bool, coarse: bool = False):
     """The chunk kernel's table of on-chip block pieces (host only): (lags the
     chain adds itself, [(step, first source, sources, first target, targets)]),
-    chunk-relative."""
+    chunk-relative. coarse: the cut used for stacks of at most 8 layers."""
     cap = 4 * chunk
     out = (ctypes.c_int32 * (5 * cap))()
     n, lags = ctypes.c_int32(), ctypes.c_int32()
-    _check(lib.fi_debug_chunk_schedule(chunk, 1 if retimed else 0, ctypes.cast(out, ctypes.c_void_p), cap,
+    mode = (2 if coarse else 1) if retimed else 0
+    _check(lib.fi_debug_chunk_schedule(chunk, mode, ctypes.cast(out, ctypes.c_void_p), cap,
                                        ctypes.byref(n), ctypes.byref(lags)), "fi_debug_chunk_schedule")
     return lags.value, [tuple(out[5 * j: 5 * j + 5]) for j in range(min(n.value, cap))]
 

@@ -102,8 +102,8 @@ def test_python_binding_refuses_cpu_tensors():
 
 
 @pytest.mark.parametrize("chunk", [2, 4, 8, 16, 32, 64])
-@pytest.mark.parametrize("retimed", [False, True])
-def test_chunk_piece_table_covers_every_pair_once_in_time(chunk, retimed):
+@pytest.mark.parametrize("retimed,coarse", [(False, False), (True, False), (True, True)])
+def test_chunk_piece_table_covers_every_pair_once_in_time(chunk, retimed, coarse):
     """The on-chip pieces of a chunk and the chain together sum every (source s,
     target t) pair with s < t inside the chunk exactly once.
 
@@ -118,9 +118,10 @@ def test_chunk_piece_table_covers_every_pair_once_in_time(chunk, retimed):
     also reach the window's spare positions t = chunk, chunk+1 (never read).
     Lags stay below chunk+2 (taps from `chunk` up are held as zero); the
     re-timed pieces hold at most 64 products per row each and are spread so that
-    no step carries more than 96."""
+    no step carries more than 96 (the coarse cut for short stacks: 16 x 16 pieces,
+    at most 256 and 320)."""
     from long_convolution_sequence_online_b200 import fi
-    sh, tab = fi.chunk_schedule(chunk, retimed)
+    sh, tab = fi.chunk_schedule(chunk, retimed, coarse)
     assert sh == (2 if retimed else 0)
     count = {}
     per_step = {}
@@ -145,5 +146,5 @@ def test_chunk_piece_table_covers_every_pair_once_in_time(chunk, retimed):
         else:
             if U <= 8 and r + sh < chunk:
                 assert (r - U, U, r + sh, U) in pieces
-            assert max(ns * nd for _, ns, _, nd in pieces) <= 64
-            assert sum(ns * nd for _, ns, _, nd in pieces) <= 96
+            assert max(ns * nd for _, ns, _, nd in pieces) <= (256 if coarse else 64)
+            assert sum(ns * nd for _, ns, _, nd in pieces) <= (320 if coarse else 96)
