@@ -799,11 +799,23 @@ __global__ void __launch_bounds__(kChunkMaxThreads) k_chunk(Dims g, ChunkArgs a,
 
 size_t chunk_smem_bytes(const Dims& g, int chunk, int G) { return chunk_shape(g, chunk, G).total * sizeof(float); }
 
+// Warps per CTA: the chain warps, then enough warps for one tile warp per row
+// group (layer, chain warp) up to the CTA's limit. With a single chain warp and
+// more than four warps the kernel leaves scheduler 0 to the chain (warps
+// 4, 8, 12 take no tile work), so those warps are added on top.
 static int chunk_threads(const Dims& g, int G) {
-  const int cw = (G + 31) / 32;
-  int tile_warps = g.M * cw;
-  if (tile_warps > kChunkMaxThreads / 32 - cw) tile_warps = kChunkMaxThreads / 32 - cw;
-  return 32 * (cw + tile_warps);
+  const int cw = (G + 31) / 32, max_w = kChunkMaxThreads / 32;
+  const int want = g.M * cw;
+  if (cw == 1) {
+    int nw = 1, tiles = 0;
+    while (tiles < want && nw < max_w) {
+      if ((nw & 3) != 0) ++tiles;
+      ++nw;
+    }
+    if (nw - cw <= 4) return 32 * (cw + (want < max_w - cw ? want : max_w - cw));   // no spare scheduler
+    return 32 * nw;
+  }
+  return 32 * (cw + (want < max_w - cw ? want : max_w - cw));
 }
 
 int chunk_streams_per_cta(const Dims& g, int chunk, int num_sms, size_t max_smem) {
