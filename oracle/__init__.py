@@ -19,8 +19,11 @@ from .lcsm import (  # noqa: F401
     causal_conv,
     causal_conv_at,
     dft,
+    gelu,
     lowbit,
+    mlp_block,
     online_lcsm,
+    online_lcsm_mlp,
     prompt_lcsm,
     relaxed_online,
     relaxed_tiles,

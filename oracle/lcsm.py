@@ -9,7 +9,8 @@ Notation (0-indexed positions t = 0..L-1, layers l = 1..M, streams s = (b, d)):
 * mixer of one layer (Flash Inference summary page, "Architettura del Modello",
   LCSM definition): y^l_t = sum_{s <= t} a^{l-1}_s * h^l_{t-s}, elementwise
   (Hadamard) over channels, so every channel is an independent 1-D sequence;
-* block: a^l_t = R(tanh(y^l_t)) (the synthetic workloads' elementwise block);
+* block: a^l_t = R(tanh(y^l_t)) (the synthetic workloads' elementwise block),
+  or the channel-mixing MLP + GELU block (online_lcsm_mlp);
 * sampler: x_{t+1} = a^0_{t+1} = R(tanh(y^M_t) + 0.1 * eps_t);
 * R is the identity for fp32 workloads and round-to-nearest-even to bfloat16
   for bf16 workloads.
@@ -153,6 +154,66 @@ def online_lcsm(h: np.ndarray, x0: np.ndarray, eps: np.ndarray, eps_scale: float
                 below = a[l + 1, :, : t + 1]
         if t + 1 < n:
             a[0, :, t + 1] = R(np.tanh(y[M - 1, :, t]) + eps_scale * eps[t])
+    return y, a
+
+
+# ----------------------------------------------------------------------------
+# Channel-mixing block (summary page, "Architettura del Modello": block^l maps
+# R^D to R^D and includes an MLP; "Configurazione Sperimentale", synthetic
+# setting: the blocks are MLP + GELU and the sampler adds noise). Reading: one
+# hidden layer of width Dh, block^l(y) = W2^l GELU(W1^l y + b1^l) + b2^l per
+# sequence, GELU in its exact form x * Phi(x) (Phi the standard normal CDF).
+# ----------------------------------------------------------------------------
+_erf = np.vectorize(__import__("math").erf, otypes=[np.float64])
+
+
+def gelu(x) -> np.ndarray:
+    """GELU(x) = x Phi(x) = x (1 + erf(x / sqrt 2)) / 2, float64."""
+    x = np.asarray(x, dtype=np.float64)
+    return 0.5 * x * (1.0 + _erf(x / np.sqrt(2.0)))
+
+
+def mlp_block(y: np.ndarray, w1: np.ndarray, b1: np.ndarray, w2: np.ndarray, b2: np.ndarray) -> np.ndarray:
+    """block(y) = w2 @ gelu(w1 @ y + b1) + b2 along the channel axis.
+
+    y: [..., D]; w1: [Dh][D]; b1: [Dh]; w2: [D][Dh]; b2: [D]. Returns [..., D].
+    """
+    y = np.asarray(y, dtype=np.float64)
+    z = gelu(y @ np.asarray(w1, np.float64).T + np.asarray(b1, np.float64))
+    return z @ np.asarray(w2, np.float64).T + np.asarray(b2, np.float64)
+
+
+def online_lcsm_mlp(h: np.ndarray, w1: np.ndarray, b1: np.ndarray, w2: np.ndarray, b2: np.ndarray,
+                    x0: np.ndarray, eps: np.ndarray, eps_scale: float = 0.1, bf16: bool = False,
+                    n: int | None = None):
+    """Closed-loop generation with the channel-mixing block after every layer.
+
+    h: [M][D][L] filters (rounded by the caller in bf16 mode); w1: [M][Dh][D];
+    b1: [M][Dh]; w2: [M][D][Dh]; b2: [M][D]; x0: [B][D]; eps: [n][B][D].
+    Per position t, layer by layer: y^l_t = sum_{s <= t} h^l_{t-s} a^{l-1}_s
+    (per channel), a^l_t = R(block^l(y^l_t)) (across channels, per sequence);
+    then x_{t+1} = R(a^M_t + eps_scale eps_t), with a^M_t the last layer's
+    block output before rounding.
+    Returns (y, a): y[l-1] = y^l, shape [M][B][D][n]; a[l] = a^l for l = 0..M-1.
+    """
+    h = np.asarray(h, dtype=np.float64)
+    M, D, L = h.shape
+    B = np.asarray(x0).shape[0]
+    n = L if n is None else n
+    R = bf16_round if bf16 else _identity
+    eps = np.asarray(eps, dtype=np.float64)
+    a = np.zeros((M, B, D, n), dtype=np.float64)
+    y = np.zeros((M, B, D, n), dtype=np.float64)
+    a[0, :, :, 0] = R(x0)
+    for t in range(n):
+        for l in range(M):
+            # y^{l+1}_t = sum_{s <= t} h^{l+1}_{t-s} a^l_s, per (b, d)
+            y[l, :, :, t] = np.sum(h[l][None, :, t::-1] * a[l, :, :, : t + 1], axis=-1)
+            out = mlp_block(y[l, :, :, t], w1[l], b1[l], w2[l], b2[l])
+            if l + 1 < M:
+                a[l + 1, :, :, t] = R(out)
+            elif t + 1 < n:
+                a[0, :, :, t + 1] = R(out + eps_scale * eps[t])
     return y, a
 
 

@@ -370,3 +370,84 @@ def test_prompt_identity_filter_is_iterated_tanh():
     for l in range(M):
         assert np.allclose(y[l], want, atol=1e-15)
         want = np.tanh(want)
+
+
+# ---------------------------------------------------------------------------- channel-mixing block
+def test_gelu_is_x_times_normal_cdf():
+    # GELU(x) = x Phi(x), Phi from scipy's normal distribution (an independent
+    # implementation), and the identity GELU(x) - GELU(-x) = x (Phi(x) + Phi(-x) = 1)
+    import scipy.stats
+    x = np.linspace(-8, 8, 2001)
+    ref = x * scipy.stats.norm.cdf(x)
+    assert np.max(np.abs(oracle.gelu(x) - ref)) <= 1e-15 * 8
+    assert np.max(np.abs(oracle.gelu(x) - oracle.gelu(-x) - x)) <= 1e-14
+    assert oracle.gelu(0.0) == 0.0
+
+
+def test_mlp_block_matches_index_loops():
+    rng = np.random.default_rng(3)
+    B, D, Dh = 2, 5, 7
+    y = rng.standard_normal((B, D))
+    w1, b1 = rng.standard_normal((Dh, D)), rng.standard_normal(Dh)
+    w2, b2 = rng.standard_normal((D, Dh)), rng.standard_normal(D)
+    out = oracle.mlp_block(y, w1, b1, w2, b2)
+    import math
+    for b in range(B):
+        z = []
+        for k in range(Dh):
+            u = b1[k] + sum(w1[k, d] * y[b, d] for d in range(D))
+            z.append(0.5 * u * (1 + math.erf(u / math.sqrt(2))))
+        for d in range(D):
+            want = b2[d] + sum(w2[d, k] * z[k] for k in range(Dh))
+            assert abs(out[b, d] - want) <= 1e-12 * max(1.0, abs(want))
+
+
+def _mlp_setup(M, B, D, Dh, L, seed):
+    rng = np.random.default_rng(seed)
+    h = rng.standard_normal((M, D, L)) * np.exp(-0.05 * np.arange(L))
+    w1 = rng.standard_normal((M, Dh, D)) / np.sqrt(D)
+    b1 = 0.1 * rng.standard_normal((M, Dh))
+    w2 = rng.standard_normal((M, D, Dh)) / np.sqrt(Dh)
+    b2 = 0.1 * rng.standard_normal((M, D))
+    x0 = rng.standard_normal((B, D))
+    eps = rng.standard_normal((L, B, D))
+    return h, w1, b1, w2, b2, x0, eps
+
+
+def test_mlp_constant_block_closed_form():
+    # W2 = 0: every block outputs b2, so layers 2..M see a constant input and
+    # y^l_t = b2^{l-1}_d * sum_{k <= t} h^l_k (prefix sums of the filter), and the
+    # sampler's tokens are x_{t+1} = b2^M + eps_scale eps_t.
+    M, B, D, Dh, L = 3, 2, 4, 3, 24
+    h, w1, b1, w2, b2, x0, eps = _mlp_setup(M, B, D, Dh, L, 5)
+    w2 = np.zeros_like(w2)
+    y, a = oracle.online_lcsm_mlp(h, w1, b1, w2, b2, x0, eps, 0.25)
+    for l in range(1, M):
+        want = b2[l - 1][None, :, None] * np.cumsum(h[l], axis=-1)[None, :, :]
+        assert np.max(np.abs(y[l] - want)) <= 1e-12
+    toks = np.concatenate([x0[:, :, None], (b2[M - 1][None, :, None] + 0.25 * eps[:-1].transpose(1, 2, 0))], axis=-1)
+    assert np.max(np.abs(a[0] - toks)) <= 1e-12
+    assert np.max(np.abs(y[0] - np.stack([[causal_conv(h[0, d], toks[b, d]) for d in range(D)] for b in range(B)]))) <= 1e-12
+
+
+@pytest.mark.parametrize("bf16", [False, True])
+def test_mlp_online_equals_offline_of_final_sequence(bf16):
+    # Each layer's outputs are the causal convolutions of its recorded inputs,
+    # and each recorded input is the block of the layer below at the same position.
+    M, B, D, Dh, L = 3, 2, 4, 6, 32
+    h, w1, b1, w2, b2, x0, eps = _mlp_setup(M, B, D, Dh, L, 7)
+    if bf16:
+        h = bf16_round(h)
+    R = bf16_round if bf16 else (lambda v: v)
+    y, a = oracle.online_lcsm_mlp(h, w1, b1, w2, b2, x0, eps, 0.1, bf16=bf16)
+    for l in range(M):
+        for b in range(B):
+            for d in range(D):
+                assert np.max(np.abs(y[l, b, d] - causal_conv(h[l, d], a[l, b, d]))) <= 1e-10
+    for l in range(1, M):
+        for t in range(L):
+            want = R(oracle.mlp_block(y[l - 1, :, :, t], w1[l - 1], b1[l - 1], w2[l - 1], b2[l - 1]))
+            assert np.max(np.abs(a[l, :, :, t] - want)) <= 1e-12
+    for t in range(L - 1):
+        want = R(oracle.mlp_block(y[M - 1, :, :, t], w1[M - 1], b1[M - 1], w2[M - 1], b2[M - 1]) + 0.1 * eps[t])
+        assert np.max(np.abs(a[0, :, :, t + 1] - want)) <= 1e-12
