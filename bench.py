@@ -39,11 +39,13 @@ import synth  # noqa: E402
 METRIC = "mixer tokens/s at 18\u00d7864, L=32K on 1 B200; % of roofline; speedup vs O(L\u00b2)"
 
 
-def metric_name(w: synth.Workload, api: str = "generate") -> str:
+def metric_name(w: synth.Workload, api: str = "generate", block: str = "tanh") -> str:
     """The headline metric's name for the headline workload, the same form for the others."""
-    if w.name == synth.HEADLINE and api == "generate":
+    if w.name == synth.HEADLINE and api == "generate" and block == "tanh":
         return METRIC
     kind = "mixer tokens/s" if api == "generate" else "mixer tokens/s through fi_step (one call per position)"
+    if block == "mlp":
+        kind += " with MLP + GELU blocks"
     return (f"{kind} at {w.layers}\u00d7{w.channels}, L={w.length}, B={w.batch} {w.dtype} on 1 B200; "
             "% of roofline; speedup vs O(L\u00b2)")
 UNIT = "tokens/s"
@@ -370,6 +372,17 @@ def gpu_arm(args, world, rank, local):
     t_init = time.perf_counter() - t_init
     del h_d
     chunk, fft_from, tc_max = ctx.plan()
+    mlp_hidden = 0
+    if args.block == "mlp":
+        # channel-mixing block after every layer: random weights of the stated shape
+        mlp_hidden = args.hidden or w.channels
+        r = np.random.default_rng(seed + 7)
+        ws = [r.standard_normal((w.layers, mlp_hidden, w.channels)) * (0.3 / np.sqrt(w.channels)),
+              0.1 * r.standard_normal((w.layers, mlp_hidden)),
+              r.standard_normal((w.layers, w.channels, mlp_hidden)) * (0.3 / np.sqrt(mlp_hidden)),
+              0.1 * r.standard_normal((w.layers, w.channels))]
+        ctx.set_mlp_block(*(torch.from_numpy(a.astype(np.float32)).to(device) for a in ws))
+        del ws
 
     step_api = args.api == "step"
     if step_api:
@@ -458,10 +471,20 @@ def gpu_arm(args, world, rank, local):
     # --- roofline: dominant kernel class during the timed steps
     peaks = measured_peaks()
     clk = clocks.summary()
-    # fi_step computes every block from HBM (no on-chip chunk) and each position's red
-    # cells in k_token, so the per-position bytes and flops belong to "token" there
-    model, tot = cost_model(w, 1 if step_api else chunk, fft_from, tc_max=tc_max)
-    model["token"] = model["chunk"] if step_api else {"bytes": 0.0, "flops": 0.0}
+    # fi_step (and any generation with the channel-mixing block) computes every block
+    # from HBM (no on-chip chunk) and each position's red cells in the per-position
+    # kernels, so the per-position bytes and flops belong to "token" there; the block's
+    # two products add their weights (read once per position) and 2 * 2 * D * Dh flops
+    # per (layer, sequence)
+    per_pos = step_api or mlp_hidden > 0
+    model, tot = cost_model(w, 1 if per_pos else chunk, fft_from, tc_max=tc_max)
+    model["token"] = dict(model["chunk"]) if per_pos else {"bytes": 0.0, "flops": 0.0}
+    if mlp_hidden:
+        extra_b = w.length * w.layers * (2.0 * w.channels * mlp_hidden + mlp_hidden + w.channels) * 4
+        extra_f = w.length * w.layers * w.batch * 4.0 * w.channels * mlp_hidden
+        model["token"]["bytes"] += extra_b
+        model["token"]["flops"] += extra_f
+        tot = {"bytes": tot["bytes"] + extra_b, "flops": tot["flops"] + extra_f}
     classes = {}
     for cls in ("chunk", "direct", "fft", "tc", "token"):
         n, ms = prof[cls]
@@ -530,7 +553,7 @@ def gpu_arm(args, world, rank, local):
 
     launches_per_step = sum(prof[k][0] for k in prof) / args.steps
     res = {
-        "metric": metric_name(w, args.api), "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "metric": metric_name(w, args.api, args.block), "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32" if w.dtype == "f32" else "bf16", "data": "synthetic",
         "config": {"workload": w.name, "layers": w.layers, "channels": w.channels, "seq_len": w.length,
@@ -543,6 +566,7 @@ def gpu_arm(args, world, rank, local):
                    "step": ("fi_reset + one fi_step per position over all L given tokens (host loop)" if step_api
                             else "fi_reset + fi_generate over all L positions, closed loop"),
                    "api": args.api,
+                   "block": (f"MLP + GELU, hidden {mlp_hidden}, random weights" if mlp_hidden else "tanh"),
                    "init_s": t_init},
         "roofline": roof,
         "step_roofline": step_roof,
@@ -573,6 +597,9 @@ def main():
                     help="largest block side on the tensor cores (0 = automatic, -1 = none)")
     ap.add_argument("--api", default="generate", choices=["generate", "step"],
                     help="generate: closed-loop fi_generate per step; step: one fi_step call per position")
+    ap.add_argument("--block", default="tanh", choices=["tanh", "mlp"],
+                    help="block after every layer: elementwise tanh, or the channel-mixing MLP + GELU")
+    ap.add_argument("--hidden", type=int, default=0, help="MLP hidden width (0 = channels)")
     ap.add_argument("--e2e-steps", dest="e2e_steps", type=int, default=3)
     ap.add_argument("--lazy-prefix", dest="lazy_prefix", type=int, default=4096)
     ap.add_argument("--oracle-positions", dest="oracle_positions", type=int, default=6144)
@@ -616,7 +643,7 @@ def main():
             import torch.distributed as dist
             dist.destroy_process_group()
     if rank == 0:
-        if args.cpu_baseline and world == 1:
+        if args.cpu_baseline and world == 1 and args.block == "tanh":
             res["cpu_baseline"] = oracle_baseline(w, args.seed, args.oracle_positions, args.oracle_streams)
         else:
             res["cpu_baseline"] = None

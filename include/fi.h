@@ -161,6 +161,25 @@ FI_API fi_status fi_sync(fi_ctx* ctx);
  * their precomputed spectra ("Precomputazione FFT") are kept. */
 FI_API fi_status fi_reset(fi_ctx* ctx);
 
+/* Channel-mixing block (summary page, "Architettura del Modello": block^l maps
+ * R^D to R^D and includes an MLP; "Configurazione Sperimentale": in the
+ * synthetic setting the blocks are MLP + GELU and the sampler adds noise).
+ * Replaces the elementwise tanh after every layer by
+ *   a^l_t = R(W2^l GELU(W1^l y^l_t + b1^l) + b2^l)   per sequence, across channels,
+ * GELU(u) = u Phi(u) (exact, erf form), R = bf16 rounding in bf16 contexts; the
+ * sampler becomes x_{t+1} = R(a^M_t + eps_scale eps_t). fi_step and fi_generate
+ * then run position by position (every layer's block needs all channels of the
+ * layer below), blocks of the schedule as before.
+ * hidden: Dh >= 1, or 0 to return to the tanh block (weights may be NULL).
+ * w1 [M][Dh][D], b1 [M][Dh], w2 [M][D][Dh], b2 [M][D]: fp32, device pointers,
+ * copied (the caller may free them after the call's stream work completes).
+ * Errors: FI_E_INVALID (NULL weight, hidden < 0), FI_E_STATE (position != 0:
+ * call fi_reset first), FI_E_UNSUPPORTED (D or Dh beyond one CTA's shared
+ * memory), FI_E_CUDA (allocation, copy). fi_prefill and fi_generate_lazy return
+ * FI_E_UNSUPPORTED while the block is set. */
+FI_API fi_status fi_set_mlp_block(fi_ctx* ctx, int32_t hidden, const float* w1, const float* b1, const float* w2,
+                                  const float* b2);
+
 /* Current position (number of positions already produced). */
 FI_API fi_status fi_position(const fi_ctx* ctx, int32_t* pos);
 

@@ -63,6 +63,7 @@ struct fi_ctx {
   float2* part_xs = nullptr;       // forward spectra of source sub-blocks (blocks wider than one transform)
   float2* pf_spec = nullptr;       // prompt prefill: padded filter spectra (allocated on first use)
   size_t pf_spec_n = 0;
+  MlpBlock mlp;                    // channel-mixing block (hidden = 0: elementwise tanh)
   // staging for fi_generate_host
   void* d_x0 = nullptr;
   float* d_eps = nullptr;
@@ -84,6 +85,11 @@ void free_ctx(fi_ctx* c) {
   cudaFree(c->spectra);
   cudaFree(c->part_xs);
   cudaFree(c->pf_spec);
+  cudaFree(c->mlp.w1);
+  cudaFree(c->mlp.b1);
+  cudaFree(c->mlp.w2);
+  cudaFree(c->mlp.b2);
+  cudaFree(c->mlp.z);
   cudaFree(c->twiddle);
   cudaFree(c->err);
   cudaFree(c->d_x0);
@@ -333,6 +339,38 @@ fi_status fi_reset(fi_ctx* c) {
   return FI_OK;
 }
 
+fi_status fi_set_mlp_block(fi_ctx* c, int32_t hidden, const float* w1, const float* b1, const float* w2,
+                           const float* b2) {
+  if (!c) return fail(FI_E_INVALID, "ctx is NULL");
+  if (c->pos != 0 || c->lazy_mode) return fail(FI_E_STATE, "the block can change at position 0 only (call fi_reset)");
+  if (hidden < 0) return fail(FI_E_INVALID, "hidden < 0");
+  if (hidden > 0 && (!w1 || !b1 || !w2 || !b2)) return fail(FI_E_INVALID, "NULL weight");
+  if ((size_t)c->g.D * sizeof(float) > c->max_smem || (size_t)hidden * sizeof(float) > c->max_smem)
+    return fail(FI_E_UNSUPPORTED, "channels or hidden width beyond one CTA's shared memory");
+  MlpBlock& m = c->mlp;
+  cudaFree(m.w1);
+  cudaFree(m.b1);
+  cudaFree(m.w2);
+  cudaFree(m.b2);
+  cudaFree(m.z);
+  m = MlpBlock{};
+  if (hidden == 0) return FI_OK;
+  const size_t M = c->g.M, D = c->g.D, H = hidden;
+  fi_status s;
+  if ((s = dev_alloc((void**)&m.w1, M * H * D * sizeof(float), "block weights")) != FI_OK ||
+      (s = dev_alloc((void**)&m.b1, M * H * sizeof(float), "block biases")) != FI_OK ||
+      (s = dev_alloc((void**)&m.w2, M * D * H * sizeof(float), "block weights")) != FI_OK ||
+      (s = dev_alloc((void**)&m.b2, M * D * sizeof(float), "block biases")) != FI_OK ||
+      (s = dev_alloc((void**)&m.z, (size_t)c->g.B * H * sizeof(float), "block scratch")) != FI_OK)
+    return s;
+  FI_CUDA(cudaMemcpyAsync(m.w1, w1, M * H * D * sizeof(float), cudaMemcpyDeviceToDevice, c->st), "copy block weights");
+  FI_CUDA(cudaMemcpyAsync(m.b1, b1, M * H * sizeof(float), cudaMemcpyDeviceToDevice, c->st), "copy block biases");
+  FI_CUDA(cudaMemcpyAsync(m.w2, w2, M * D * H * sizeof(float), cudaMemcpyDeviceToDevice, c->st), "copy block weights");
+  FI_CUDA(cudaMemcpyAsync(m.b2, b2, M * D * sizeof(float), cudaMemcpyDeviceToDevice, c->st), "copy block biases");
+  m.hidden = hidden;
+  return FI_OK;
+}
+
 fi_status fi_position(const fi_ctx* c, int32_t* pos) {
   if (!c || !pos) return fail(FI_E_INVALID, "NULL argument");
   *pos = c->pos;
@@ -353,12 +391,39 @@ fi_status fi_get_plan(const fi_ctx* c, int32_t* chunk, int32_t* fft_from, int32_
   return FI_OK;
 }
 
+// One position with the channel-mixing block: the block of step t from HBM,
+// then per layer the red cells, the block and (after the last layer, with noise)
+// the sampler. x_t (may be NULL: the token is already in the state) goes to
+// layer 0 first.
+fi_status mlp_position(fi_ctx* c, int t, const void* x_t, const float* eps_t, float eps_scale, float* y_out,
+                       float* rec, int n_gen, int gen_base) {
+  fi_status s;
+  if (x_t && (s = timed(c, KC_TOKEN, [&] { return launch_mlp_token(c->g, c->state, x_t, t, c->st); },
+                        "token store")) != FI_OK)
+    return s;
+  if (t >= 1 && (s = run_block(c, t)) != FI_OK) return s;
+  for (int l = 1; l <= c->g.M; ++l)
+    if ((s = timed(c, KC_TOKEN,
+                   [&] {
+                     return launch_mlp_layer(c->g, c->state, c->taps, c->mlp, l, t, eps_t, eps_scale, y_out, rec,
+                                             n_gen, gen_base, c->st);
+                   },
+                   "channel-mixing block launch")) != FI_OK)
+      return s;
+  return FI_OK;
+}
+
 fi_status fi_step(fi_ctx* c, const void* x_t, float* y_t) {
   if (!c || !x_t || !y_t) return fail(FI_E_INVALID, "NULL argument");
   if (c->pos >= c->g.L) return fail(FI_E_STATE, "position == max_len");
   if (c->lazy_mode) return fail(FI_E_STATE, "context holds a lazy generation; call fi_reset");
   fi_status s;
   const int t = c->pos;
+  if (c->mlp.hidden > 0) {
+    if ((s = mlp_position(c, t, x_t, nullptr, 0.f, y_t, nullptr, 1, t)) != FI_OK) return s;
+    c->pos++;
+    return FI_OK;
+  }
   // small blocks (direct, side <= kTokenBlockMax) run inside the red-cell launch
   const int fused_u = (t >= 1 && token_block_fused(c->g, lowbit(t))) ? lowbit(t) : 0;
   if (t >= 1 && !fused_u && (s = run_block(c, t)) != FI_OK) return s;
@@ -383,6 +448,14 @@ fi_status fi_generate(fi_ctx* c, int32_t n, const void* x0, const float* eps, fl
   const int base = c->pos, end = c->pos + n;
   int p = base;
   fi_status s;
+  if (c->mlp.hidden > 0) {
+    for (int t = base; t < end; ++t)
+      if ((s = mlp_position(c, t, t == base ? x0 : nullptr, eps + (size_t)(t - base) * c->g.S, eps_scale, y_out, rec,
+                            n, base)) != FI_OK)
+        return s;
+    c->pos = end;
+    return FI_OK;
+  }
   while (p < end) {
     const int cst = (p / CH) * CH;
     const int p1 = (cst + CH < end) ? cst + CH : end;
@@ -418,6 +491,7 @@ fi_status fi_generate(fi_ctx* c, int32_t n, const void* x0, const float* eps, fl
 
 fi_status fi_prefill(fi_ctx* c, int32_t p, const void* x, float* y_out, float* rec) {
   if (!c || !x) return fail(FI_E_INVALID, "NULL argument");
+  if (c->mlp.hidden > 0) return fail(FI_E_UNSUPPORTED, "prefill with the channel-mixing block is not supported");
   if (p < 1 || p > c->g.L) return fail(FI_E_INVALID, "p must be in [1, max_len]");
   if (p > (1 << kMaxFftLog2))
     return fail(FI_E_UNSUPPORTED, "prompts longer than " + std::to_string(1 << kMaxFftLog2) + " positions");
@@ -429,6 +503,11 @@ fi_status fi_prefill(fi_ctx* c, int32_t p, const void* x, float* y_out, float* r
   if (need > c->pf_spec_n) {
     FI_CUDA(cudaStreamSynchronize(c->st), "synchronize");
     cudaFree(c->pf_spec);
+  cudaFree(c->mlp.w1);
+  cudaFree(c->mlp.b1);
+  cudaFree(c->mlp.w2);
+  cudaFree(c->mlp.b2);
+  cudaFree(c->mlp.z);
     c->pf_spec = nullptr;
     c->pf_spec_n = 0;
     fi_status s = dev_alloc((void**)&c->pf_spec, need * sizeof(float2), "prefill spectra");
@@ -490,6 +569,7 @@ fi_status fi_generate_lazy(fi_ctx* c, int32_t n, const void* x0, const float* ep
   if (n == 0) return FI_OK;
   if (!x0 || !eps || !y_out) return fail(FI_E_INVALID, "NULL buffer");
   if ((int64_t)c->pos + n > c->g.L) return fail(FI_E_STATE, "position + n > max_len");
+  if (c->mlp.hidden > 0) return fail(FI_E_UNSUPPORTED, "the lazy baseline runs the elementwise block only");
   if (c->pos > 0 && !c->lazy_mode) return fail(FI_E_STATE, "context holds a relaxed generation; call fi_reset");
   c->lazy_mode = 1;
   const size_t row = (size_t)c->g.S;

@@ -179,6 +179,25 @@ cudaError_t launch_prefix(const Dims& g, float* state, const float* taps, float2
 cudaError_t launch_debug_fft(int log2n, int count, const float2* in, float2* out, int inverse,
                              const float2* twiddle, cudaStream_t st);
 
+// Channel-mixing block (MLP + GELU) state: weights copied from the caller and
+// the hidden activations of one position.
+struct MlpBlock {
+  int hidden = 0;            // Dh; 0 = the elementwise tanh block
+  float* w1 = nullptr;       // [M][Dh][D]
+  float* b1 = nullptr;       // [M][Dh]
+  float* w2 = nullptr;       // [M][D][Dh]
+  float* b2 = nullptr;       // [M][D]
+  float* z = nullptr;        // [B][Dh] scratch
+};
+// Token x [B][D] into layer 0 at position t.
+cudaError_t launch_mlp_token(const Dims& g, float* state, const void* x, int t, cudaStream_t st);
+// Layer l at position t: red cells and block for every (sequence, channel);
+// the block's output goes to the state (l < M) or, with eps_t, to the next
+// token; y^l_t to rec [M][n_gen][B][D] and (l = M) y_out [n_gen][B][D] if given.
+cudaError_t launch_mlp_layer(const Dims& g, float* state, const float* taps, const MlpBlock& m, int l, int t,
+                             const float* eps_t, float eps_scale, float* y_out, float* rec, int n_gen, int gen_base,
+                             cudaStream_t st);
+
 // Message returned by fi_last_error() for the calling thread.
 void set_last_error(const std::string& msg);
 

@@ -22,7 +22,8 @@ KERNEL_CLASSES = ("chunk", "direct", "fft", "token", "lazy", "tc")
 EXPORTED = ("fi_init", "fi_step", "fi_generate", "fi_generate_host", "fi_generate_lazy", "fi_sync", "fi_reset",
             "fi_position", "fi_read_activations", "fi_set_stream", "fi_get_plan", "fi_profile",
             "fi_profile_read", "fi_destroy", "fi_status_str", "fi_last_error", "fi_debug_fft",
-            "fi_generate_noalloc", "fi_debug_set_wait_limit", "fi_debug_chunk_schedule", "fi_prefill", "fi_profile_read_sides")
+            "fi_generate_noalloc", "fi_debug_set_wait_limit", "fi_debug_chunk_schedule", "fi_prefill", "fi_profile_read_sides",
+            "fi_set_mlp_block")
 
 
 class FiError(RuntimeError):
@@ -63,6 +64,7 @@ def _load():
         "fi_debug_set_wait_limit": [vp, i32],
         "fi_debug_chunk_schedule": [i32, i32, vp, i32, ctypes.POINTER(i32), ctypes.POINTER(i32)],
         "fi_prefill": [vp, i32, vp, vp, vp],
+        "fi_set_mlp_block": [vp, i32, vp, vp, vp, vp],
         "fi_profile_read_sides": [vp, ctypes.POINTER(i32), ctypes.POINTER(ctypes.c_double), ctypes.POINTER(i32),
                                   ctypes.POINTER(ctypes.c_double)],
     }
@@ -157,6 +159,13 @@ class Context:
 
     def prefill(self, p: int, x, y_out=None, rec=None):
         _check(lib.fi_prefill(self._h, p, _ptr(x), _ptr(y_out), _ptr(rec)), "fi_prefill")
+
+    def set_mlp_block(self, w1=None, b1=None, w2=None, b2=None):
+        """Channel-mixing block W2 GELU(W1 y + b1) + b2 after every layer (fp32 CUDA
+        tensors w1 [M][Dh][D], b1 [M][Dh], w2 [M][D][Dh], b2 [M][D]); no arguments
+        return to the elementwise tanh block."""
+        hidden = 0 if w1 is None else int(w1.shape[1])
+        _check(lib.fi_set_mlp_block(self._h, hidden, _ptr(w1), _ptr(b1), _ptr(w2), _ptr(b2)), "fi_set_mlp_block")
 
     def generate_host(self, n: int, x0: np.ndarray, eps: np.ndarray, y_out: np.ndarray, eps_scale: float = 0.1):
         for a in (x0, eps, y_out):
