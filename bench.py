@@ -528,8 +528,9 @@ def gpu_arm(args, world, rank, local):
                  "roofline_ms_onchip_small_blocks": 1e3 * t_onchip, "frac_onchip_small_blocks": t_onchip / run_s}
 
     # --- quadratic Lazy baseline on the GPU: measured on two prefixes, extrapolated a*n + b*n^2/2
+    # (it runs the elementwise block only)
     lazy = None
-    if args.lazy_prefix > 0 and rank == 0 and not step_api:
+    if args.lazy_prefix > 0 and rank == 0 and not step_api and not mlp_hidden:
         n2 = min(args.lazy_prefix, w.length)
         n1 = n2 // 4
         times = []

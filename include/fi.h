@@ -169,13 +169,15 @@ FI_API fi_status fi_reset(fi_ctx* ctx);
  * GELU(u) = u Phi(u) (exact, erf form), R = bf16 rounding in bf16 contexts; the
  * sampler becomes x_{t+1} = R(a^M_t + eps_scale eps_t). fi_step and fi_generate
  * then run position by position (every layer's block needs all channels of the
- * layer below), blocks of the schedule as before.
+ * layer below), blocks of the schedule as before; fi_generate replays the
+ * layers of a position as one CUDA graph, captured on the first call of more
+ * than one position after this one. Synchronises the context's stream.
  * hidden: Dh >= 1, or 0 to return to the tanh block (weights may be NULL).
  * w1 [M][Dh][D], b1 [M][Dh], w2 [M][D][Dh], b2 [M][D]: fp32, device pointers,
  * copied (the caller may free them after the call's stream work completes).
  * Errors: FI_E_INVALID (NULL weight, hidden < 0), FI_E_STATE (position != 0:
- * call fi_reset first), FI_E_UNSUPPORTED (D or Dh beyond one CTA's shared
- * memory), FI_E_CUDA (allocation, copy). fi_prefill and fi_generate_lazy return
+ * call fi_reset first), FI_E_UNSUPPORTED (min(B, 8) x D or min(B, 8) x Dh
+ * floats beyond one CTA's shared memory), FI_E_OOM, FI_E_CUDA. fi_prefill and fi_generate_lazy return
  * FI_E_UNSUPPORTED while the block is set. */
 FI_API fi_status fi_set_mlp_block(fi_ctx* ctx, int32_t hidden, const float* w1, const float* b1, const float* w2,
                                   const float* b2);
@@ -201,8 +203,9 @@ FI_API fi_status fi_get_plan(const fi_ctx* ctx, int32_t* chunk, int32_t* fft_fro
 
 /* Kernel timing. With profiling on, every kernel launch of fi_generate is
  * bracketed by CUDA events on the context's stream; fi_profile_read
- * synchronises and returns, per kernel class, the launch count and the summed
- * device time in milliseconds since the last read. Classes: 0 = on-chip chunk
+ * synchronises and returns, per kernel class, the count of kernels launched
+ * and the summed device time in milliseconds since the last read (a replayed
+ * graph is one bracket and counts its kernels). Classes: 0 = on-chip chunk
  * (small blocks + red cells), 1 = direct blocks from HBM, 2 = FFT blocks,
  * 3 = per-position red cells (fi_step / lazy), 4 = lazy sums, 5 = tensor-core
  * blocks. */

@@ -35,6 +35,7 @@ struct EventPair {
   cudaEvent_t a, b;
   int cls;
   int side_q;   // log2 of the block side for block launches, else -1
+  int kernels;  // kernels the bracketed launch runs (a graph: its kernel nodes)
 };
 
 }  // namespace
@@ -64,6 +65,8 @@ struct fi_ctx {
   float2* pf_spec = nullptr;       // prompt prefill: padded filter spectra (allocated on first use)
   size_t pf_spec_n = 0;
   MlpBlock mlp;                    // channel-mixing block (hidden = 0: elementwise tanh)
+  cudaGraphExec_t mlp_graph = nullptr;   // the block's layers at *mlp.pos, then the position advanced
+  cudaStream_t cap_st = nullptr;         // capture stream for mlp_graph
   // staging for fi_generate_host
   void* d_x0 = nullptr;
   float* d_eps = nullptr;
@@ -78,18 +81,29 @@ namespace {
 
 bool pow2(int64_t v) { return v > 0 && (v & (v - 1)) == 0; }
 
+void free_mlp(fi_ctx* c) {
+  if (c->mlp_graph) cudaGraphExecDestroy(c->mlp_graph);
+  c->mlp_graph = nullptr;
+  MlpBlock& m = c->mlp;
+  cudaFree(m.w1);
+  cudaFree(m.b1);
+  cudaFree(m.w2);
+  cudaFree(m.b2);
+  cudaFree(m.z);
+  cudaFree(m.y);
+  cudaFree(m.pos);
+  m = MlpBlock{};
+}
+
 void free_ctx(fi_ctx* c) {
   if (!c) return;
+  free_mlp(c);
+  if (c->cap_st) cudaStreamDestroy(c->cap_st);
   cudaFree(c->state);
   cudaFree(c->taps);
   cudaFree(c->spectra);
   cudaFree(c->part_xs);
   cudaFree(c->pf_spec);
-  cudaFree(c->mlp.w1);
-  cudaFree(c->mlp.b1);
-  cudaFree(c->mlp.w2);
-  cudaFree(c->mlp.b2);
-  cudaFree(c->mlp.z);
   cudaFree(c->twiddle);
   cudaFree(c->err);
   cudaFree(c->d_x0);
@@ -113,7 +127,7 @@ fi_status dev_alloc(void** p, size_t bytes, const char* what) {
 
 // Kernel launch wrapped in profiling events when enabled.
 template <class F>
-fi_status timed(fi_ctx* c, int cls, F&& launch, const char* what, int side_q = -1) {
+fi_status timed(fi_ctx* c, int cls, F&& launch, const char* what, int side_q = -1, int kernels = 1) {
   EventPair ep{};
   if (c->prof) {
     if (!c->ev_free.empty()) {
@@ -125,6 +139,7 @@ fi_status timed(fi_ctx* c, int cls, F&& launch, const char* what, int side_q = -
     }
     ep.cls = cls;
     ep.side_q = side_q;
+    ep.kernels = kernels;
     FI_CUDA(cudaEventRecord(ep.a, c->st), "cudaEventRecord");
   }
   cudaError_t e = launch();
@@ -345,29 +360,31 @@ fi_status fi_set_mlp_block(fi_ctx* c, int32_t hidden, const float* w1, const flo
   if (c->pos != 0 || c->lazy_mode) return fail(FI_E_STATE, "the block can change at position 0 only (call fi_reset)");
   if (hidden < 0) return fail(FI_E_INVALID, "hidden < 0");
   if (hidden > 0 && (!w1 || !b1 || !w2 || !b2)) return fail(FI_E_INVALID, "NULL weight");
-  if ((size_t)c->g.D * sizeof(float) > c->max_smem || (size_t)hidden * sizeof(float) > c->max_smem)
+  if (hidden > 0 && mlp_smem_bytes(c->g, hidden) > c->max_smem)
     return fail(FI_E_UNSUPPORTED, "channels or hidden width beyond one CTA's shared memory");
-  MlpBlock& m = c->mlp;
-  cudaFree(m.w1);
-  cudaFree(m.b1);
-  cudaFree(m.w2);
-  cudaFree(m.b2);
-  cudaFree(m.z);
-  m = MlpBlock{};
+  // a captured position of an earlier fi_generate may still be in flight
+  FI_CUDA(cudaStreamSynchronize(c->st), "synchronize");
+  free_mlp(c);
   if (hidden == 0) return FI_OK;
-  const size_t M = c->g.M, D = c->g.D, H = hidden;
+  MlpBlock& m = c->mlp;
+  const size_t M = c->g.M, D = c->g.D, H = hidden, B = c->g.B;
   fi_status s;
   if ((s = dev_alloc((void**)&m.w1, M * H * D * sizeof(float), "block weights")) != FI_OK ||
       (s = dev_alloc((void**)&m.b1, M * H * sizeof(float), "block biases")) != FI_OK ||
       (s = dev_alloc((void**)&m.w2, M * D * H * sizeof(float), "block weights")) != FI_OK ||
       (s = dev_alloc((void**)&m.b2, M * D * sizeof(float), "block biases")) != FI_OK ||
-      (s = dev_alloc((void**)&m.z, (size_t)c->g.B * H * sizeof(float), "block scratch")) != FI_OK)
+      (s = dev_alloc((void**)&m.z, B * H * sizeof(float), "block scratch")) != FI_OK ||
+      (s = dev_alloc((void**)&m.y, B * D * sizeof(float), "block scratch")) != FI_OK ||
+      (s = dev_alloc((void**)&m.pos, sizeof(MlpPos), "block position")) != FI_OK) {
+    free_mlp(c);
     return s;
+  }
+  m.hidden = hidden;
+  FI_CUDA(prepare_mlp(c->g, m), "block shared memory limit");
   FI_CUDA(cudaMemcpyAsync(m.w1, w1, M * H * D * sizeof(float), cudaMemcpyDeviceToDevice, c->st), "copy block weights");
   FI_CUDA(cudaMemcpyAsync(m.b1, b1, M * H * sizeof(float), cudaMemcpyDeviceToDevice, c->st), "copy block biases");
   FI_CUDA(cudaMemcpyAsync(m.w2, w2, M * D * H * sizeof(float), cudaMemcpyDeviceToDevice, c->st), "copy block weights");
   FI_CUDA(cudaMemcpyAsync(m.b2, b2, M * D * sizeof(float), cudaMemcpyDeviceToDevice, c->st), "copy block biases");
-  m.hidden = hidden;
   return FI_OK;
 }
 
@@ -391,24 +408,51 @@ fi_status fi_get_plan(const fi_ctx* c, int32_t* chunk, int32_t* fft_from, int32_
   return FI_OK;
 }
 
-// One position with the channel-mixing block: the block of step t from HBM,
-// then per layer the red cells, the block and (after the last layer, with noise)
-// the sampler. x_t (may be NULL: the token is already in the state) goes to
-// layer 0 first.
-fi_status mlp_position(fi_ctx* c, int t, const void* x_t, const float* eps_t, float eps_scale, float* y_out,
-                       float* rec, int n_gen, int gen_base) {
+// The channel-mixing block's layers of one position as a graph: every layer's
+// two launches read the position record *mlp.pos, and a last node advances it,
+// so one instantiation serves every position of every fi_generate call (the
+// per-call record is written by a launch before the first position). Captured
+// once per fi_set_mlp_block, on a stream of the context's own.
+fi_status mlp_layers_graph(fi_ctx* c) {
+  if (c->mlp_graph) return FI_OK;
+  if (!c->cap_st) FI_CUDA(cudaStreamCreateWithFlags(&c->cap_st, cudaStreamNonBlocking), "capture stream");
+  FI_CUDA(cudaStreamBeginCapture(c->cap_st, cudaStreamCaptureModeThreadLocal), "begin capture");
+  cudaError_t e = cudaSuccess;
+  const MlpPos unused{};
+  for (int l = 1; l <= c->g.M && e == cudaSuccess; ++l)
+    e = launch_mlp_layer(c->g, c->state, c->taps, c->mlp, l, unused, c->mlp.pos, c->cap_st);
+  if (e == cudaSuccess) e = launch_mlp_next(c->mlp.pos, c->cap_st);
+  cudaGraph_t graph = nullptr;
+  const cudaError_t e_end = cudaStreamEndCapture(c->cap_st, &graph);
+  if (e == cudaSuccess) e = e_end;
+  if (e == cudaSuccess) e = cudaGraphInstantiate(&c->mlp_graph, graph, 0);
+  if (graph) cudaGraphDestroy(graph);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    c->mlp_graph = nullptr;
+    return fail(FI_E_CUDA, std::string("capturing the block's layers: ") + cudaGetErrorString(e));
+  }
+  return FI_OK;
+}
+
+// One position with the channel-mixing block: the token (x_t may be NULL: it
+// is already in the state), the block of step t from HBM, then per layer the
+// block's products (after the last layer, with noise, the sampler). graph:
+// the layers run as one launch of the captured graph, at the position *mlp.pos
+// holds (set to p before the first position).
+fi_status mlp_position(fi_ctx* c, const MlpPos& p, const void* x_t, bool graph) {
   fi_status s;
+  const int t = p.t;
   if (x_t && (s = timed(c, KC_TOKEN, [&] { return launch_mlp_token(c->g, c->state, x_t, t, c->st); },
                         "token store")) != FI_OK)
     return s;
   if (t >= 1 && (s = run_block(c, t)) != FI_OK) return s;
+  if (graph)
+    return timed(c, KC_TOKEN, [&] { return cudaGraphLaunch(c->mlp_graph, c->st); }, "block graph launch", -1,
+                 2 * c->g.M + 1);
   for (int l = 1; l <= c->g.M; ++l)
-    if ((s = timed(c, KC_TOKEN,
-                   [&] {
-                     return launch_mlp_layer(c->g, c->state, c->taps, c->mlp, l, t, eps_t, eps_scale, y_out, rec,
-                                             n_gen, gen_base, c->st);
-                   },
-                   "channel-mixing block launch")) != FI_OK)
+    if ((s = timed(c, KC_TOKEN, [&] { return launch_mlp_layer(c->g, c->state, c->taps, c->mlp, l, p, nullptr, c->st); },
+                   "channel-mixing block launch", -1, 2)) != FI_OK)
       return s;
   return FI_OK;
 }
@@ -420,7 +464,8 @@ fi_status fi_step(fi_ctx* c, const void* x_t, float* y_t) {
   fi_status s;
   const int t = c->pos;
   if (c->mlp.hidden > 0) {
-    if ((s = mlp_position(c, t, x_t, nullptr, 0.f, y_t, nullptr, 1, t)) != FI_OK) return s;
+    const MlpPos p{t, t, 1, 0.f, nullptr, y_t, nullptr};
+    if ((s = mlp_position(c, p, x_t, false)) != FI_OK) return s;
     c->pos++;
     return FI_OK;
   }
@@ -449,10 +494,19 @@ fi_status fi_generate(fi_ctx* c, int32_t n, const void* x0, const float* eps, fl
   int p = base;
   fi_status s;
   if (c->mlp.hidden > 0) {
-    for (int t = base; t < end; ++t)
-      if ((s = mlp_position(c, t, t == base ? x0 : nullptr, eps + (size_t)(t - base) * c->g.S, eps_scale, y_out, rec,
-                            n, base)) != FI_OK)
+    // one position alone runs its launches directly; more replay the captured layers
+    const bool graph = n >= 2;
+    const MlpPos p0{base, base, n, eps_scale, eps, y_out, rec};
+    if (graph) {
+      if ((s = mlp_layers_graph(c)) != FI_OK) return s;
+      if ((s = timed(c, KC_TOKEN, [&] { return launch_mlp_set(c->mlp.pos, p0, c->st); }, "block position")) != FI_OK)
         return s;
+    }
+    for (int t = base; t < end; ++t) {
+      MlpPos p = p0;
+      p.t = t;
+      if ((s = mlp_position(c, p, t == base ? x0 : nullptr, graph)) != FI_OK) return s;
+    }
     c->pos = end;
     return FI_OK;
   }
@@ -503,11 +557,6 @@ fi_status fi_prefill(fi_ctx* c, int32_t p, const void* x, float* y_out, float* r
   if (need > c->pf_spec_n) {
     FI_CUDA(cudaStreamSynchronize(c->st), "synchronize");
     cudaFree(c->pf_spec);
-  cudaFree(c->mlp.w1);
-  cudaFree(c->mlp.b1);
-  cudaFree(c->mlp.w2);
-  cudaFree(c->mlp.b2);
-  cudaFree(c->mlp.z);
     c->pf_spec = nullptr;
     c->pf_spec_n = 0;
     fi_status s = dev_alloc((void**)&c->pf_spec, need * sizeof(float2), "prefill spectra");
@@ -622,7 +671,7 @@ fi_status fi_profile_read_sides(fi_ctx* c, int32_t counts[FI_NUM_KERNEL_CLASSES]
   for (auto& e : c->ev_live) {
     float t = 0.f;
     FI_CUDA(cudaEventElapsedTime(&t, e.a, e.b), "cudaEventElapsedTime");
-    counts[e.cls] += 1;
+    counts[e.cls] += e.kernels;
     ms[e.cls] += t;
     if (e.side_q >= 0 && e.side_q < 32) {
       if (side_counts) side_counts[e.side_q] += 1;

@@ -179,8 +179,20 @@ cudaError_t launch_prefix(const Dims& g, float* state, const float* taps, float2
 cudaError_t launch_debug_fft(int log2n, int count, const float2* in, float2* out, int inverse,
                              const float2* twiddle, cudaStream_t st);
 
-// Channel-mixing block (MLP + GELU) state: weights copied from the caller and
-// the hidden activations of one position.
+// Channel-mixing block (MLP + GELU) state: weights copied from the caller, the
+// hidden activations and red cells of one position, and the position record a
+// captured position reads.
+constexpr int kMlpGroup = 8;  // sequences one CTA applies each weight row to
+// One position of the block: t, and where its outputs go (y^l_t to
+// rec [M][n_gen][B][D] and, l = M, y_out [n_gen][B][D], rows t - gen_base; eps
+// [n_gen][B][D] noise of the sampler, NULL: no next token is written).
+struct MlpPos {
+  int t, gen_base, n_gen;
+  float eps_scale;
+  const float* eps;
+  float* y_out;
+  float* rec;
+};
 struct MlpBlock {
   int hidden = 0;            // Dh; 0 = the elementwise tanh block
   float* w1 = nullptr;       // [M][Dh][D]
@@ -188,15 +200,24 @@ struct MlpBlock {
   float* w2 = nullptr;       // [M][D][Dh]
   float* b2 = nullptr;       // [M][D]
   float* z = nullptr;        // [B][Dh] scratch
+  float* y = nullptr;        // [B][D] scratch: the next layer's red cells
+  MlpPos* pos = nullptr;     // the position a captured position reads (advanced by the capture)
 };
+// Dynamic shared memory the block's kernels need (must fit one CTA).
+size_t mlp_smem_bytes(const Dims& g, int hidden);
 // Token x [B][D] into layer 0 at position t.
 cudaError_t launch_mlp_token(const Dims& g, float* state, const void* x, int t, cudaStream_t st);
-// Layer l at position t: red cells and block for every (sequence, channel);
-// the block's output goes to the state (l < M) or, with eps_t, to the next
-// token; y^l_t to rec [M][n_gen][B][D] and (l = M) y_out [n_gen][B][D] if given.
-cudaError_t launch_mlp_layer(const Dims& g, float* state, const float* taps, const MlpBlock& m, int l, int t,
-                             const float* eps_t, float eps_scale, float* y_out, float* rec, int n_gen, int gen_base,
-                             cudaStream_t st);
+// Shared-memory limits of the block's kernels (call before launching or capturing).
+cudaError_t prepare_mlp(const Dims& g, const MlpBlock& m);
+// Layer l at position p.t (or at *p_dev, when p_dev is given: a captured
+// position): the block's two products for every (sequence, channel). The
+// block's output goes to the state (l < M) or, with noise, to the next token.
+// The block of step t must have run before layer 1.
+cudaError_t launch_mlp_layer(const Dims& g, float* state, const float* taps, const MlpBlock& m, int l,
+                             const MlpPos& p, const MlpPos* p_dev, cudaStream_t st);
+// p_dev->t += 1 (the last node of a captured position); *p_dev = v.
+cudaError_t launch_mlp_next(MlpPos* p_dev, cudaStream_t st);
+cudaError_t launch_mlp_set(MlpPos* p_dev, const MlpPos& v, cudaStream_t st);
 
 // Message returned by fi_last_error() for the calling thread.
 void set_last_error(const std::string& msg);

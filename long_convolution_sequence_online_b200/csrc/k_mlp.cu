@@ -6,89 +6,205 @@
 // with y^l_t = acc^l_t + h^l_0 a^{l-1}_t (the red cell) and GELU(u) = u Phi(u)
 // (the exact form, from erff). Unlike tanh the block mixes channels, so layer
 // l+1 at position t needs every channel of layer l at t: each position runs,
-// per layer, one launch for the red cells and the first product (every CTA
-// forms the y it needs in shared memory) and one for the second product, which
-// writes the activations back into the state slots (or, after the last layer,
-// the sampler's next token).
+// per layer, one launch for the first product and one for the second.
+//
+// Both products are matrix-vector work on weights that stay in L2 (a few MB
+// per layer), so they are latency-bound: one warp owns one weight row, its
+// lanes load the row as independent float4s, and every row is applied to up to
+// kMlpGroup sequences at once (the row is read once per group, not once per
+// sequence). The second product also forms the next layer's red cell y^{l+1}_t
+// for its channel (one strided read of acc^{l+1}_t) into a dense [B][D]
+// buffer, so only layer 1 gathers its inputs from the strided state.
 #include "fi_internal.cuh"
 
 namespace fi {
 
 namespace {
 
-constexpr int kMlpThreads = 256;               // 8 warps, one output row per warp at a time
-constexpr int kMlpRowsPerCta = 32;
+constexpr int kMlpThreads = 256;   // 8 warps, one weight row each
+constexpr int kMlpRows = kMlpThreads / 32;
 
 __device__ __forceinline__ float gelu_exact(float u) { return 0.5f * u * (1.0f + erff(u * 0.70710678118654752f)); }
 
-// Dot product of a weight row (length n, contiguous) with the vector in shared
-// memory, by one warp: lanes stride the row, then a shuffle reduction.
-__device__ __forceinline__ float warp_dot(const float* __restrict__ w, const float* v, int n, int lane) {
-  float sum = 0.f;
-  for (int k = lane; k < n; k += 32) sum = fmaf(__ldg(w + k), v[k], sum);
+// A weight row held by one warp: the first kMlpPre float4s per lane are
+// loaded before the kernel waits for the launch before it (they do not depend
+// on it), the rest of a longer row is streamed in dots().
+constexpr int kMlpPre = 8;
+struct WarpRow {
+  float4 w[kMlpPre];
+
+  __device__ __forceinline__ void preload(const float* __restrict__ row, int n, int lane) {
+    const float4* w4 = reinterpret_cast<const float4*>(row);
+    const int n4 = (n & 3) == 0 ? n >> 2 : 0;
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-  return sum;
+    for (int u = 0; u < kMlpPre; ++u) {
+      const int c = lane + 32 * u;
+      w[u] = c < n4 ? __ldg(w4 + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  }
+
+  // acc[b] = row . v[b] over n for b < nb (all lanes get the sums); v: nb
+  // vectors of length n in shared memory, stride n.
+  __device__ __forceinline__ void dots(const float* __restrict__ row, const float* v, int n, int nb, int lane,
+                                       float (&acc)[kMlpGroup]) const {
+#pragma unroll
+    for (int b = 0; b < kMlpGroup; ++b) acc[b] = 0.f;
+    if ((n & 3) == 0) {
+      const int n4 = n >> 2;
+#pragma unroll
+      for (int u = 0; u < kMlpPre; ++u) {
+        const int c = lane + 32 * u;
+        if (c >= n4) break;
+        add4(w[u], v, n, c, nb, acc);
+      }
+      const float4* w4 = reinterpret_cast<const float4*>(row);
+      for (int c0 = lane + 32 * kMlpPre; c0 < n4; c0 += 4 * 32) {
+        float4 wv[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int c = c0 + 32 * u;
+          wv[u] = c < n4 ? __ldg(w4 + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int c = c0 + 32 * u;
+          if (c >= n4) break;
+          add4(wv[u], v, n, c, nb, acc);
+        }
+      }
+    } else {
+      for (int k = lane; k < n; k += 32) {
+        const float wk = __ldg(row + k);
+#pragma unroll
+        for (int b = 0; b < kMlpGroup; ++b) {
+          if (b >= nb) break;
+          acc[b] = fmaf(wk, v[(size_t)b * n + k], acc[b]);
+        }
+      }
+    }
+#pragma unroll
+    for (int b = 0; b < kMlpGroup; ++b) {
+      if (b >= nb) break;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) acc[b] += __shfl_xor_sync(0xffffffffu, acc[b], o);
+    }
+  }
+
+  static __device__ __forceinline__ void add4(const float4& wv, const float* v, int n, int c, int nb,
+                                              float (&acc)[kMlpGroup]) {
+#pragma unroll
+    for (int b = 0; b < kMlpGroup; ++b) {
+      if (b >= nb) break;
+      const float4 x = *reinterpret_cast<const float4*>(v + (size_t)b * n + 4 * c);
+      acc[b] = fmaf(wv.x, x.x, acc[b]);
+      acc[b] = fmaf(wv.y, x.y, acc[b]);
+      acc[b] = fmaf(wv.z, x.z, acc[b]);
+      acc[b] = fmaf(wv.w, x.w, acc[b]);
+    }
+  }
+};
+
+// Where y^l_t goes besides the block's input: rec [M][n_gen][B][D] and, for
+// the last layer, y_out [n_gen][B][D].
+__device__ __forceinline__ void record_y(const Dims& g, int l, const MlpPos& p, int b, int d, float y) {
+  const size_t io = (size_t)b * g.D + d;
+  if (p.rec) p.rec[((size_t)(l - 1) * p.n_gen + (p.t - p.gen_base)) * g.S + io] = y;
+  if (p.y_out && l == g.M) p.y_out[(size_t)(p.t - p.gen_base) * g.S + io] = y;
 }
 
-// Red cells of layer l at position t for sequence b (all D channels, into
-// shared memory), then z[b][k] = GELU(W1[k] . y + b1[k]) for this CTA's rows k.
-// The first CTA of each sequence also writes y^l_t to rec (and to y_out for the
-// last layer). grid = (ceil(Dh / kMlpRowsPerCta), B).
+// z[b][k] = GELU(W1[k] . y_b + b1[k]) for the CTA's rows k and its group of
+// sequences. y_b is the dense ybuf [B][D] (layers 2..M), or, for layer 1, the
+// red cells gathered from the state (the first CTA of the group records them).
+// grid = (ceil(Dh / kMlpRows), ceil(B / kMlpGroup)).
 __global__ void __launch_bounds__(kMlpThreads) k_mlp_in(Dims g, const float* __restrict__ state,
-                                                       const float* __restrict__ taps, int l, int t, int hidden,
+                                                       const float* __restrict__ taps, int l, MlpPos p_host,
+                                                       const MlpPos* __restrict__ p_dev, int hidden,
                                                        const float* __restrict__ w1, const float* __restrict__ b1,
-                                                       float* __restrict__ z, float* __restrict__ y_out,
-                                                       float* __restrict__ rec, int n_gen, int gen_base) {
-  extern __shared__ float ysm[];   // [D]
-  const int b = blockIdx.y;
-  for (int d = threadIdx.x; d < g.D; d += blockDim.x) {
-    const int s = d * g.B + b;
-    const float acc = t == 0 ? 0.f : state[slot_index(g, l, s, t)];
-    const float a_in = state[slot_index(g, l - 1, s, t)];
-    const float y = fmaf(taps[((size_t)(l - 1) * g.D + d) * g.L], a_in, acc);
-    ysm[d] = y;
-    if (blockIdx.x == 0) {
-      const size_t io = (size_t)b * g.D + d;
-      if (rec) rec[((size_t)(l - 1) * n_gen + (t - gen_base)) * g.S + io] = y;
-      if (y_out && l == g.M) y_out[(size_t)(t - gen_base) * g.S + io] = y;
+                                                       const float* __restrict__ ybuf, float* __restrict__ z) {
+  extern __shared__ __align__(16) float ysm[];   // [nb][D]
+  pdl_launch_dependents();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int k = blockIdx.x * kMlpRows + warp;
+  const float* row = w1 + ((size_t)(l - 1) * hidden + (k < hidden ? k : 0)) * g.D;
+  WarpRow wr;
+  wr.preload(row, k < hidden ? g.D : 0, lane);
+  const float bias = k < hidden ? __ldg(b1 + (size_t)(l - 1) * hidden + k) : 0.f;
+  pdl_wait_primary();   // the position record, the state and ybuf come from earlier launches
+  const MlpPos p = p_dev ? *p_dev : p_host;
+  const int t = p.t;
+  const int b0 = blockIdx.y * kMlpGroup, nb = min(kMlpGroup, g.B - b0);
+  const int n_in = nb * g.D;
+  if (l == 1) {
+    for (int i = threadIdx.x; i < n_in; i += blockDim.x) {
+      const int b = b0 + i / g.D, d = i - (i / g.D) * g.D;
+      const int s = d * g.B + b;
+      const float acc = t == 0 ? 0.f : state[slot_index(g, 1, s, t)];
+      const float y = fmaf(taps[(size_t)d * g.L], state[slot_index(g, 0, s, t)], acc);
+      ysm[i] = y;
+      if (blockIdx.x == 0) record_y(g, 1, p, b, d, y);
     }
+  } else {
+    for (int i = threadIdx.x; i < n_in; i += blockDim.x) ysm[i] = ybuf[(size_t)b0 * g.D + i];
   }
   __syncthreads();
+  if (k >= hidden) return;
+  float acc[kMlpGroup];
+  wr.dots(row, ysm, g.D, nb, lane, acc);
+#pragma unroll
+  for (int b = 0; b < kMlpGroup; ++b)
+    if (b < nb && lane == b) z[(size_t)(b0 + b) * hidden + k] = gelu_exact(acc[b] + bias);
+}
+
+// a[b][d] = W2[d] . z_b + b2[d] for the CTA's channels d. Layers l < M store
+// R(a) as the activation a^l_t and form the next red cell
+// y^{l+1}_t = acc^{l+1}_t + h^{l+1}_0 R(a) into ybuf; the last layer, with
+// noise given, stores the next token x_{t+1} = R(a + eps_scale eps_t).
+// grid = (ceil(D / kMlpRows), ceil(B / kMlpGroup)).
+__global__ void __launch_bounds__(kMlpThreads) k_mlp_out(Dims g, float* __restrict__ state,
+                                                        const float* __restrict__ taps, int l, MlpPos p_host,
+                                                        const MlpPos* __restrict__ p_dev, int hidden,
+                                                        const float* __restrict__ w2, const float* __restrict__ b2,
+                                                        const float* __restrict__ z, float* __restrict__ ybuf) {
+  extern __shared__ __align__(16) float zsm[];   // [nb][hidden]
+  pdl_launch_dependents();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const float* W1 = w1 + (size_t)(l - 1) * hidden * g.D;
-  const int k_hi = min(hidden, (int)(blockIdx.x + 1) * kMlpRowsPerCta);
-  for (int k = blockIdx.x * kMlpRowsPerCta + warp; k < k_hi; k += kMlpThreads / 32) {
-    const float u = warp_dot(W1 + (size_t)k * g.D, ysm, g.D, lane) + b1[(size_t)(l - 1) * hidden + k];
-    if (lane == 0) z[(size_t)b * hidden + k] = gelu_exact(u);
+  const int d = blockIdx.x * kMlpRows + warp;
+  const float* row = w2 + ((size_t)(l - 1) * g.D + (d < g.D ? d : 0)) * hidden;
+  WarpRow wr;
+  wr.preload(row, d < g.D ? hidden : 0, lane);
+  const float bias = d < g.D ? __ldg(b2 + (size_t)(l - 1) * g.D + d) : 0.f;
+  const float h0 = l < g.M && d < g.D ? __ldg(taps + ((size_t)l * g.D + d) * g.L) : 0.f;
+  pdl_wait_primary();   // z, the position record and the state come from earlier launches
+  const MlpPos p = p_dev ? *p_dev : p_host;
+  const int t = p.t;
+  const int b0 = blockIdx.y * kMlpGroup, nb = min(kMlpGroup, g.B - b0);
+  for (int i = threadIdx.x; i < nb * hidden; i += blockDim.x) zsm[i] = z[(size_t)b0 * hidden + i];
+  __syncthreads();
+  if (d >= g.D) return;
+  float acc[kMlpGroup];
+  wr.dots(row, zsm, hidden, nb, lane, acc);
+  float a = 0.f;
+#pragma unroll
+  for (int b = 0; b < kMlpGroup; ++b)
+    if (lane == b) a = acc[b] + bias;
+  if (lane >= nb) return;
+  const int b = b0 + lane, s = d * g.B + b;
+  if (l < g.M) {
+    const float a_r = round_act(a, g.bf16);
+    state[slot_index(g, l, s, t)] = a_r;
+    const float acc_next = t == 0 ? 0.f : state[slot_index(g, l + 1, s, t)];
+    const float y = fmaf(h0, a_r, acc_next);
+    ybuf[(size_t)b * g.D + d] = y;
+    record_y(g, l + 1, p, b, d, y);
+  } else if (p.eps && t + 1 < g.L) {
+    const float e = p.eps[(size_t)(t - p.gen_base) * g.S + (size_t)b * g.D + d];
+    state[slot_index(g, 0, s, t + 1)] = round_act(a + p.eps_scale * e, g.bf16);
   }
 }
 
-// a[d] = W2[d] . z_b + b2[d] for this CTA's channels d; stored as the
-// activation a^l_t (l < M), or, after the last layer and with noise given, as
-// the next token x_{t+1} = R(a + eps_scale eps_t). grid = (ceil(D / kMlpRowsPerCta), B).
-__global__ void __launch_bounds__(kMlpThreads) k_mlp_out(Dims g, float* __restrict__ state, int l, int t, int hidden,
-                                                        const float* __restrict__ w2, const float* __restrict__ b2,
-                                                        const float* __restrict__ z, const float* __restrict__ eps_t,
-                                                        float eps_scale) {
-  extern __shared__ float zsm[];   // [hidden]
-  const int b = blockIdx.y;
-  for (int k = threadIdx.x; k < hidden; k += blockDim.x) zsm[k] = z[(size_t)b * hidden + k];
-  __syncthreads();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const float* W2 = w2 + (size_t)(l - 1) * g.D * hidden;
-  const int d_hi = min(g.D, (int)(blockIdx.x + 1) * kMlpRowsPerCta);
-  for (int d = blockIdx.x * kMlpRowsPerCta + warp; d < d_hi; d += kMlpThreads / 32) {
-    const float a = warp_dot(W2 + (size_t)d * hidden, zsm, hidden, lane) + b2[(size_t)(l - 1) * g.D + d];
-    if (lane != 0) continue;
-    const int s = d * g.B + b;
-    if (l < g.M) {
-      state[slot_index(g, l, s, t)] = round_act(a, g.bf16);
-    } else if (eps_t && t + 1 < g.L) {
-      state[slot_index(g, 0, s, t + 1)] = round_act(a + eps_scale * eps_t[(size_t)b * g.D + d], g.bf16);
-    }
-  }
-}
+// The position counter of a captured position: advanced once all its layers ran.
+__global__ void k_mlp_next(MlpPos* p_dev) { p_dev->t += 1; }
+__global__ void k_mlp_set(MlpPos* p_dev, MlpPos v) { *p_dev = v; }
 
 // Token x_t [B][D] (context dtype) into slot (0, s, t), rounded as the state holds it.
 __global__ void k_mlp_token(Dims g, float* __restrict__ state, const void* __restrict__ x, int t) {
@@ -98,17 +214,25 @@ __global__ void k_mlp_token(Dims g, float* __restrict__ state, const void* __res
   state[slot_index(g, 0, d * g.B + b, t)] = round_act(load_token(x, (size_t)i, g.bf16), g.bf16);
 }
 
+size_t smem_in_bytes(const Dims& g) { return (size_t)(g.B < kMlpGroup ? g.B : kMlpGroup) * g.D * sizeof(float); }
+size_t smem_out_bytes(const Dims& g, int hidden) {
+  return (size_t)(g.B < kMlpGroup ? g.B : kMlpGroup) * hidden * sizeof(float);
+}
+
 }  // namespace
+
+size_t mlp_smem_bytes(const Dims& g, int hidden) {
+  const size_t a = smem_in_bytes(g), b = smem_out_bytes(g, hidden);
+  return a > b ? a : b;
+}
 
 cudaError_t launch_mlp_token(const Dims& g, float* state, const void* x, int t, cudaStream_t st) {
   k_mlp_token<<<(g.S + 255) / 256, 256, 0, st>>>(g, state, x, t);
   return cudaGetLastError();
 }
 
-cudaError_t launch_mlp_layer(const Dims& g, float* state, const float* taps, const MlpBlock& m, int l, int t,
-                             const float* eps_t, float eps_scale, float* y_out, float* rec, int n_gen, int gen_base,
-                             cudaStream_t st) {
-  const size_t smem_in = (size_t)g.D * sizeof(float), smem_out = (size_t)m.hidden * sizeof(float);
+cudaError_t prepare_mlp(const Dims& g, const MlpBlock& m) {
+  const size_t smem_in = smem_in_bytes(g), smem_out = smem_out_bytes(g, m.hidden);
   if (smem_in > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(k_mlp_in, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_in);
     if (e != cudaSuccess) return e;
@@ -117,13 +241,40 @@ cudaError_t launch_mlp_layer(const Dims& g, float* state, const float* taps, con
     cudaError_t e = cudaFuncSetAttribute(k_mlp_out, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_out);
     if (e != cudaSuccess) return e;
   }
-  const dim3 grid_in((unsigned)((m.hidden + kMlpRowsPerCta - 1) / kMlpRowsPerCta), (unsigned)g.B);
-  k_mlp_in<<<grid_in, kMlpThreads, smem_in, st>>>(g, state, taps, l, t, m.hidden, m.w1, m.b1, m.z, y_out, rec, n_gen,
-                                                  gen_base);
-  cudaError_t e = cudaGetLastError();
+  return cudaSuccess;
+}
+
+// Both launches allow programmatic stream serialization: each kernel may start
+// while the launch before it drains, loads its weight rows, then waits for it.
+cudaError_t launch_mlp_layer(const Dims& g, float* state, const float* taps, const MlpBlock& m, int l,
+                             const MlpPos& p, const MlpPos* p_dev, cudaStream_t st) {
+  const unsigned groups = (unsigned)((g.B + kMlpGroup - 1) / kMlpGroup);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(kMlpThreads);
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cfg.gridDim = dim3((unsigned)((m.hidden + kMlpRows - 1) / kMlpRows), groups);
+  cfg.dynamicSmemBytes = smem_in_bytes(g);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, k_mlp_in, g, (const float*)state, taps, l, p, p_dev, m.hidden,
+                                     (const float*)m.w1, (const float*)m.b1, (const float*)m.y, m.z);
   if (e != cudaSuccess) return e;
-  const dim3 grid_out((unsigned)((g.D + kMlpRowsPerCta - 1) / kMlpRowsPerCta), (unsigned)g.B);
-  k_mlp_out<<<grid_out, kMlpThreads, smem_out, st>>>(g, state, l, t, m.hidden, m.w2, m.b2, m.z, eps_t, eps_scale);
+  cfg.gridDim = dim3((unsigned)((g.D + kMlpRows - 1) / kMlpRows), groups);
+  cfg.dynamicSmemBytes = smem_out_bytes(g, m.hidden);
+  return cudaLaunchKernelEx(&cfg, k_mlp_out, g, state, taps, l, p, p_dev, m.hidden, (const float*)m.w2,
+                            (const float*)m.b2, (const float*)m.z, m.y);
+}
+
+cudaError_t launch_mlp_next(MlpPos* p_dev, cudaStream_t st) {
+  k_mlp_next<<<1, 1, 0, st>>>(p_dev);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_mlp_set(MlpPos* p_dev, const MlpPos& v, cudaStream_t st) {
+  k_mlp_set<<<1, 1, 0, st>>>(p_dev, v);
   return cudaGetLastError();
 }
 

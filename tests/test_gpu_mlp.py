@@ -167,3 +167,52 @@ def test_mlp_block_state_rules(fi):
     assert torch.equal(y, y2)
     ctx.close()
     ref.close()
+
+
+def test_mlp_block_groups_and_scalar_rows(fi):
+    # B = 10 sequences: two CTA groups (8 + 2); D = 6 and Dh = 10 are not
+    # multiples of 4, so both products take the scalar row path.
+    w = synth.Workload("mlp-2x6-L128-B10", 2, 6, 128, 10, "f32", 1e-1, 5e-1)
+    inp = gpu_inputs(w, 71)
+    ws = _weights(w.layers, w.channels, 10, 72)
+    ctx = fi.Context(inp["h"], w.batch, w.dtype)
+    _set(ctx, ws)
+    n = 96                                   # a ragged stop inside the sequence
+    y = torch.empty((n, w.batch, w.channels), dtype=torch.float32, device="cuda")
+    rec = torch.empty((w.layers, n, w.batch, w.channels), dtype=torch.float32, device="cuda")
+    ctx.generate(n, inp["x0"], inp["eps"][:n].contiguous(), y, 0.1, rec)
+    ctx.sync()
+    acts = [a.cpu().numpy() for a in read_all_activations(ctx, n)]
+    ctx.close()
+    rec = rec.cpu().numpy()
+    assert np.array_equal(y.cpu().numpy(), rec[-1])
+    _check_teacher_forced(w, oracle_filters(inp["h_np"], "f32"), ws, acts, rec, inp["eps_np"])
+
+
+def test_captured_positions_equal_direct_launches(fi):
+    # fi_generate replays the captured layers (position read on the device);
+    # fi_step launches them directly. Fed the tokens fi_generate produced,
+    # fi_step must give the same outputs bit for bit. The generation runs in
+    # two calls, so the second call's record (new base, buffers) is used too.
+    w = synth.Workload("mlp-3x12-L256", 3, 12, 256, 3, "f32", 1e-1, 5e-1)
+    inp = gpu_inputs(w, 81)
+    ws = _weights(w.layers, w.channels, 20, 82)
+    gen = fi.Context(inp["h"], w.batch, w.dtype)
+    _set(gen, ws)
+    n1, n = 57, 160
+    y = torch.empty((n, w.batch, w.channels), dtype=torch.float32, device="cuda")
+    eps = inp["eps"][:n].contiguous()
+    gen.generate(n1, inp["x0"], eps[:n1].contiguous(), y[:n1], 0.1)
+    y2 = torch.empty((n - n1, w.batch, w.channels), dtype=torch.float32, device="cuda")
+    gen.generate(n - n1, None, eps[n1:].contiguous(), y2, 0.1)
+    gen.sync()
+    toks = read_all_activations(gen, n)[0]     # [n][B][D] tokens x_t
+    gen.close()
+    step = fi.Context(inp["h"], w.batch, w.dtype)
+    _set(step, ws)
+    ys = torch.empty_like(y)
+    for t in range(n):
+        step.step(toks[t].contiguous().cuda(), ys[t])
+    step.sync()
+    step.close()
+    assert torch.equal(torch.cat([y[:n1], y2]), ys)
