@@ -408,8 +408,9 @@ fi_status fi_get_plan(const fi_ctx* c, int32_t* chunk, int32_t* fft_from, int32_
   return FI_OK;
 }
 
-// The channel-mixing block's layers of one position as a graph: every layer's
-// two launches read the position record *mlp.pos, and a last node advances it,
+// The channel-mixing block's launches of one position as a graph: the small
+// block of step t, then every layer's two launches, all reading the position
+// record *mlp.pos, and a last node that advances it,
 // so one instantiation serves every position of every fi_generate call (the
 // per-call record is written by a launch before the first position). Captured
 // once per fi_set_mlp_block, on a stream of the context's own.
@@ -419,6 +420,7 @@ fi_status mlp_layers_graph(fi_ctx* c) {
   FI_CUDA(cudaStreamBeginCapture(c->cap_st, cudaStreamCaptureModeThreadLocal), "begin capture");
   cudaError_t e = cudaSuccess;
   const MlpPos unused{};
+  e = launch_mlp_block(c->g, c->state, c->taps, unused, c->mlp.pos, c->cap_st);
   for (int l = 1; l <= c->g.M && e == cudaSuccess; ++l)
     e = launch_mlp_layer(c->g, c->state, c->taps, c->mlp, l, unused, c->mlp.pos, c->cap_st);
   if (e == cudaSuccess) e = launch_mlp_next(c->mlp.pos, c->cap_st);
@@ -436,20 +438,25 @@ fi_status mlp_layers_graph(fi_ctx* c) {
 }
 
 // One position with the channel-mixing block: the token (x_t may be NULL: it
-// is already in the state), the block of step t from HBM, then per layer the
+// is already in the state), the block of step t (from HBM when wider than
+// kMlpBlockMax, else in the position's own launches), then per layer the
 // block's products (after the last layer, with noise, the sampler). graph:
-// the layers run as one launch of the captured graph, at the position *mlp.pos
-// holds (set to p before the first position).
+// those launches run as one launch of the captured graph, at the position
+// *mlp.pos holds (set to p before the first position).
 fi_status mlp_position(fi_ctx* c, const MlpPos& p, const void* x_t, bool graph) {
   fi_status s;
   const int t = p.t;
   if (x_t && (s = timed(c, KC_TOKEN, [&] { return launch_mlp_token(c->g, c->state, x_t, t, c->st); },
                         "token store")) != FI_OK)
     return s;
-  if (t >= 1 && (s = run_block(c, t)) != FI_OK) return s;
+  // blocks wider than kMlpBlockMax from HBM first; narrower ones run in the position's launches
+  if (t >= 1 && lowbit(t) > kMlpBlockMax && (s = run_block(c, t)) != FI_OK) return s;
   if (graph)
     return timed(c, KC_TOKEN, [&] { return cudaGraphLaunch(c->mlp_graph, c->st); }, "block graph launch", -1,
-                 2 * c->g.M + 1);
+                 2 * c->g.M + 2);
+  if ((s = timed(c, KC_TOKEN, [&] { return launch_mlp_block(c->g, c->state, c->taps, p, nullptr, c->st); },
+                 "small block launch")) != FI_OK)
+    return s;
   for (int l = 1; l <= c->g.M; ++l)
     if ((s = timed(c, KC_TOKEN, [&] { return launch_mlp_layer(c->g, c->state, c->taps, c->mlp, l, p, nullptr, c->st); },
                    "channel-mixing block launch", -1, 2)) != FI_OK)

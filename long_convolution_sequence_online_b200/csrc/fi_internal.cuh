@@ -182,7 +182,8 @@ cudaError_t launch_debug_fft(int log2n, int count, const float2* in, float2* out
 // Channel-mixing block (MLP + GELU) state: weights copied from the caller, the
 // hidden activations and red cells of one position, and the position record a
 // captured position reads.
-constexpr int kMlpGroup = 8;  // sequences one CTA applies each weight row to
+constexpr int kMlpGroup = 8;      // sequences one CTA applies each weight row to
+constexpr int kMlpBlockMax = 8;   // blocks of side <= this run in the position's own launches
 // One position of the block: t, and where its outputs go (y^l_t to
 // rec [M][n_gen][B][D] and, l = M, y_out [n_gen][B][D], rows t - gen_base; eps
 // [n_gen][B][D] noise of the sampler, NULL: no next token is written).
@@ -215,6 +216,11 @@ cudaError_t prepare_mlp(const Dims& g, const MlpBlock& m);
 // The block of step t must have run before layer 1.
 cudaError_t launch_mlp_layer(const Dims& g, float* state, const float* taps, const MlpBlock& m, int l,
                              const MlpPos& p, const MlpPos* p_dev, cudaStream_t st);
+// The small block of step p.t (or *p_dev's), side lowbit(t) <= kMlpBlockMax,
+// for every layer and stream; nothing for t = 0 or a wider block (run from HBM
+// before). Launched before layer 1's launches.
+cudaError_t launch_mlp_block(const Dims& g, float* state, const float* taps, const MlpPos& p, const MlpPos* p_dev,
+                             cudaStream_t st);
 // p_dev->t += 1 (the last node of a captured position); *p_dev = v.
 cudaError_t launch_mlp_next(MlpPos* p_dev, cudaStream_t st);
 cudaError_t launch_mlp_set(MlpPos* p_dev, const MlpPos& v, cudaStream_t st);

@@ -15,6 +15,8 @@
 // sequence). The second product also forms the next layer's red cell y^{l+1}_t
 // for its channel (one strided read of acc^{l+1}_t) into a dense [B][D]
 // buffer, so only layer 1 gathers its inputs from the strided state.
+#include <type_traits>
+
 #include "fi_internal.cuh"
 
 namespace fi {
@@ -122,15 +124,15 @@ __global__ void __launch_bounds__(kMlpThreads) k_mlp_in(Dims g, const float* __r
                                                        const float* __restrict__ w1, const float* __restrict__ b1,
                                                        const float* __restrict__ ybuf, float* __restrict__ z) {
   extern __shared__ __align__(16) float ysm[];   // [nb][D]
-  pdl_launch_dependents();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int k = blockIdx.x * kMlpRows + warp;
   const float* row = w1 + ((size_t)(l - 1) * hidden + (k < hidden ? k : 0)) * g.D;
   WarpRow wr;
   wr.preload(row, k < hidden ? g.D : 0, lane);
   const float bias = k < hidden ? __ldg(b1 + (size_t)(l - 1) * hidden + k) : 0.f;
-  pdl_wait_primary();   // the position record, the state and ybuf come from earlier launches
-  const MlpPos p = p_dev ? *p_dev : p_host;
+  const MlpPos p = p_dev ? *p_dev : p_host;   // written before the position's first launch
+  pdl_wait_primary();   // the state (small block) and ybuf come from the launch before
+  pdl_launch_dependents();
   const int t = p.t;
   const int b0 = blockIdx.y * kMlpGroup, nb = min(kMlpGroup, g.B - b0);
   const int n_in = nb * g.D;
@@ -166,7 +168,6 @@ __global__ void __launch_bounds__(kMlpThreads) k_mlp_out(Dims g, float* __restri
                                                         const float* __restrict__ w2, const float* __restrict__ b2,
                                                         const float* __restrict__ z, float* __restrict__ ybuf) {
   extern __shared__ __align__(16) float zsm[];   // [nb][hidden]
-  pdl_launch_dependents();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int d = blockIdx.x * kMlpRows + warp;
   const float* row = w2 + ((size_t)(l - 1) * g.D + (d < g.D ? d : 0)) * hidden;
@@ -174,10 +175,21 @@ __global__ void __launch_bounds__(kMlpThreads) k_mlp_out(Dims g, float* __restri
   wr.preload(row, d < g.D ? hidden : 0, lane);
   const float bias = d < g.D ? __ldg(b2 + (size_t)(l - 1) * g.D + d) : 0.f;
   const float h0 = l < g.M && d < g.D ? __ldg(taps + ((size_t)l * g.D + d) * g.L) : 0.f;
-  pdl_wait_primary();   // z, the position record and the state come from earlier launches
   const MlpPos p = p_dev ? *p_dev : p_host;
   const int t = p.t;
   const int b0 = blockIdx.y * kMlpGroup, nb = min(kMlpGroup, g.B - b0);
+  // Launches trigger their dependents only after their own wait, so every
+  // launch before the previous one has completed here: the next layer's
+  // accumulator at t (final once the small block ran) and the noise can be read
+  // before waiting.
+  float acc_next = 0.f, e = 0.f;
+  if (d < g.D && lane < nb) {
+    const int s = d * g.B + b0 + lane;
+    if (l < g.M && t > 0) acc_next = state[slot_index(g, l + 1, s, t)];
+    if (l == g.M && p.eps && t + 1 < g.L) e = p.eps[(size_t)(t - p.gen_base) * g.S + (size_t)(b0 + lane) * g.D + d];
+  }
+  pdl_wait_primary();   // z comes from the launch before
+  pdl_launch_dependents();
   for (int i = threadIdx.x; i < nb * hidden; i += blockDim.x) zsm[i] = z[(size_t)b0 * hidden + i];
   __syncthreads();
   if (d >= g.D) return;
@@ -192,13 +204,68 @@ __global__ void __launch_bounds__(kMlpThreads) k_mlp_out(Dims g, float* __restri
   if (l < g.M) {
     const float a_r = round_act(a, g.bf16);
     state[slot_index(g, l, s, t)] = a_r;
-    const float acc_next = t == 0 ? 0.f : state[slot_index(g, l + 1, s, t)];
     const float y = fmaf(h0, a_r, acc_next);
     ybuf[(size_t)b * g.D + d] = y;
     record_y(g, l + 1, p, b, d, y);
   } else if (p.eps && t + 1 < g.L) {
-    const float e = p.eps[(size_t)(t - p.gen_base) * g.S + (size_t)b * g.D + d];
     state[slot_index(g, 0, s, t + 1)] = round_act(a + p.eps_scale * e, g.bf16);
+  }
+}
+
+// The block of step t, side UB = lowbit(t) <= kMlpBlockMax, for layer l and
+// stream s (channel d): slot(l, s, t+u') (+)= sum_{u<UB} h^l[UB+u'-u]
+// a^{l-1}_{t-UB+u}, stored when t is a power of two (the first block to reach
+// these targets). Sources, targets and taps are read as vectors: t is a
+// multiple of UB and every row of the state and taps starts 16-byte aligned.
+template <int UB>
+__device__ __forceinline__ void small_block(const Dims& g, float* __restrict__ state, const float* __restrict__ taps,
+                                            int t, int l, int s, int d) {
+  constexpr int V = UB >= 4 ? 4 : UB;   // floats per vector access
+  using vec = typename std::conditional<V == 4, float4, typename std::conditional<V == 2, float2, float>::type>::type;
+  float x[UB], h[2 * UB], cur[UB];
+  const float* xp = state + slot_index(g, l - 1, s, t - UB);
+  float* dp = state + slot_index(g, l, s, t);
+  const float* hp = taps + ((size_t)(l - 1) * g.D + d) * g.L;
+#pragma unroll
+  for (int u = 0; u < UB; u += V) *reinterpret_cast<vec*>(x + u) = *reinterpret_cast<const vec*>(xp + u);
+  if constexpr (V == 1) {
+    *reinterpret_cast<float2*>(h) = __ldg(reinterpret_cast<const float2*>(hp));
+  } else {
+#pragma unroll
+    for (int k = 0; k < 2 * UB; k += V) *reinterpret_cast<vec*>(h + k) = __ldg(reinterpret_cast<const vec*>(hp + k));
+  }
+  if (t == UB) {
+#pragma unroll
+    for (int up = 0; up < UB; ++up) cur[up] = 0.f;
+  } else {
+#pragma unroll
+    for (int up = 0; up < UB; up += V) *reinterpret_cast<vec*>(cur + up) = *reinterpret_cast<const vec*>(dp + up);
+  }
+#pragma unroll
+  for (int up = 0; up < UB; ++up) {
+#pragma unroll
+    for (int u = 0; u < UB; ++u) cur[up] = fmaf(h[UB + up - u], x[u], cur[up]);
+  }
+#pragma unroll
+  for (int up = 0; up < UB; up += V) *reinterpret_cast<vec*>(dp + up) = *reinterpret_cast<const vec*>(cur + up);
+}
+
+// The position's small block for every (layer, stream), one thread each; a
+// no-op at t = 0 and where lowbit(t) > kMlpBlockMax (that block ran before,
+// from HBM).
+__global__ void k_mlp_block(Dims g, float* __restrict__ state, const float* __restrict__ taps, MlpPos p_host,
+                            const MlpPos* __restrict__ p_dev) {
+  pdl_launch_dependents();   // the first layer's launch loads its weights meanwhile
+  const int t = p_dev ? p_dev->t : p_host.t;
+  const int U = t & -t;
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (t == 0 || U > kMlpBlockMax || i >= g.M * g.S) return;
+  const int l = i / g.S + 1, s = i - (l - 1) * g.S, d = s / g.B;
+  switch (U) {
+    case 1: small_block<1>(g, state, taps, t, l, s, d); break;
+    case 2: small_block<2>(g, state, taps, t, l, s, d); break;
+    case 4: small_block<4>(g, state, taps, t, l, s, d); break;
+    default: small_block<kMlpBlockMax>(g, state, taps, t, l, s, d); break;
   }
 }
 
@@ -266,6 +333,13 @@ cudaError_t launch_mlp_layer(const Dims& g, float* state, const float* taps, con
   cfg.dynamicSmemBytes = smem_out_bytes(g, m.hidden);
   return cudaLaunchKernelEx(&cfg, k_mlp_out, g, state, taps, l, p, p_dev, m.hidden, (const float*)m.w2,
                             (const float*)m.b2, (const float*)m.z, m.y);
+}
+
+cudaError_t launch_mlp_block(const Dims& g, float* state, const float* taps, const MlpPos& p, const MlpPos* p_dev,
+                             cudaStream_t st) {
+  const int n = g.M * g.S;
+  k_mlp_block<<<(n + 255) / 256, 256, 0, st>>>(g, state, taps, p, p_dev);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_mlp_next(MlpPos* p_dev, cudaStream_t st) {
