@@ -420,7 +420,7 @@ fi_status mlp_layers_graph(fi_ctx* c) {
   FI_CUDA(cudaStreamBeginCapture(c->cap_st, cudaStreamCaptureModeThreadLocal), "begin capture");
   cudaError_t e = cudaSuccess;
   const MlpPos unused{};
-  e = launch_mlp_block(c->g, c->state, c->taps, unused, c->mlp.pos, c->cap_st);
+  e = launch_mlp_block(c->g, c->state, c->taps, unused, c->mlp.pos, c->mlp.y, c->cap_st);
   for (int l = 1; l <= c->g.M && e == cudaSuccess; ++l)
     e = launch_mlp_layer(c->g, c->state, c->taps, c->mlp, l, unused, c->mlp.pos, c->cap_st);
   if (e == cudaSuccess) e = launch_mlp_next(c->mlp.pos, c->cap_st);
@@ -454,7 +454,7 @@ fi_status mlp_position(fi_ctx* c, const MlpPos& p, const void* x_t, bool graph) 
   if (graph)
     return timed(c, KC_TOKEN, [&] { return cudaGraphLaunch(c->mlp_graph, c->st); }, "block graph launch", -1,
                  2 * c->g.M + 2);
-  if ((s = timed(c, KC_TOKEN, [&] { return launch_mlp_block(c->g, c->state, c->taps, p, nullptr, c->st); },
+  if ((s = timed(c, KC_TOKEN, [&] { return launch_mlp_block(c->g, c->state, c->taps, p, nullptr, c->mlp.y, c->st); },
                  "small block launch")) != FI_OK)
     return s;
   for (int l = 1; l <= c->g.M; ++l)

@@ -217,10 +217,11 @@ cudaError_t prepare_mlp(const Dims& g, const MlpBlock& m);
 cudaError_t launch_mlp_layer(const Dims& g, float* state, const float* taps, const MlpBlock& m, int l,
                              const MlpPos& p, const MlpPos* p_dev, cudaStream_t st);
 // The small block of step p.t (or *p_dev's), side lowbit(t) <= kMlpBlockMax,
-// for every layer and stream; nothing for t = 0 or a wider block (run from HBM
-// before). Launched before layer 1's launches.
+// for every layer and stream (nothing for t = 0 or a wider block, run from HBM
+// before), then layer 1's red cells into m.y and the records. Launched before
+// layer 1's launches.
 cudaError_t launch_mlp_block(const Dims& g, float* state, const float* taps, const MlpPos& p, const MlpPos* p_dev,
-                             cudaStream_t st);
+                             float* ybuf, cudaStream_t st);
 // p_dev->t += 1 (the last node of a captured position); *p_dev = v.
 cudaError_t launch_mlp_next(MlpPos* p_dev, cudaStream_t st);
 cudaError_t launch_mlp_set(MlpPos* p_dev, const MlpPos& v, cudaStream_t st);

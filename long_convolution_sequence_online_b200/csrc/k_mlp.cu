@@ -115,14 +115,11 @@ __device__ __forceinline__ void record_y(const Dims& g, int l, const MlpPos& p, 
 }
 
 // z[b][k] = GELU(W1[k] . y_b + b1[k]) for the CTA's rows k and its group of
-// sequences. y_b is the dense ybuf [B][D] (layers 2..M), or, for layer 1, the
-// red cells gathered from the state (the first CTA of the group records them).
-// grid = (ceil(Dh / kMlpRows), ceil(B / kMlpGroup)).
-__global__ void __launch_bounds__(kMlpThreads) k_mlp_in(Dims g, const float* __restrict__ state,
-                                                       const float* __restrict__ taps, int l, MlpPos p_host,
-                                                       const MlpPos* __restrict__ p_dev, int hidden,
-                                                       const float* __restrict__ w1, const float* __restrict__ b1,
-                                                       const float* __restrict__ ybuf, float* __restrict__ z) {
+// sequences, y_b the layer's red cells in the dense ybuf [B][D] (written by the
+// launch before). grid = (ceil(Dh / kMlpRows), ceil(B / kMlpGroup)).
+__global__ void __launch_bounds__(kMlpThreads) k_mlp_in(Dims g, int l, int hidden, const float* __restrict__ w1,
+                                                       const float* __restrict__ b1, const float* __restrict__ ybuf,
+                                                       float* __restrict__ z) {
   extern __shared__ __align__(16) float ysm[];   // [nb][D]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int k = blockIdx.x * kMlpRows + warp;
@@ -130,24 +127,11 @@ __global__ void __launch_bounds__(kMlpThreads) k_mlp_in(Dims g, const float* __r
   WarpRow wr;
   wr.preload(row, k < hidden ? g.D : 0, lane);
   const float bias = k < hidden ? __ldg(b1 + (size_t)(l - 1) * hidden + k) : 0.f;
-  const MlpPos p = p_dev ? *p_dev : p_host;   // written before the position's first launch
-  pdl_wait_primary();   // the state (small block) and ybuf come from the launch before
+  pdl_wait_primary();   // ybuf comes from the launch before
   pdl_launch_dependents();
-  const int t = p.t;
   const int b0 = blockIdx.y * kMlpGroup, nb = min(kMlpGroup, g.B - b0);
   const int n_in = nb * g.D;
-  if (l == 1) {
-    for (int i = threadIdx.x; i < n_in; i += blockDim.x) {
-      const int b = b0 + i / g.D, d = i - (i / g.D) * g.D;
-      const int s = d * g.B + b;
-      const float acc = t == 0 ? 0.f : state[slot_index(g, 1, s, t)];
-      const float y = fmaf(taps[(size_t)d * g.L], state[slot_index(g, 0, s, t)], acc);
-      ysm[i] = y;
-      if (blockIdx.x == 0) record_y(g, 1, p, b, d, y);
-    }
-  } else {
-    for (int i = threadIdx.x; i < n_in; i += blockDim.x) ysm[i] = ybuf[(size_t)b0 * g.D + i];
-  }
+  for (int i = threadIdx.x; i < n_in; i += blockDim.x) ysm[i] = ybuf[(size_t)b0 * g.D + i];
   __syncthreads();
   if (k >= hidden) return;
   float acc[kMlpGroup];
@@ -218,7 +202,7 @@ __global__ void __launch_bounds__(kMlpThreads) k_mlp_out(Dims g, float* __restri
 // these targets). Sources, targets and taps are read as vectors: t is a
 // multiple of UB and every row of the state and taps starts 16-byte aligned.
 template <int UB>
-__device__ __forceinline__ void small_block(const Dims& g, float* __restrict__ state, const float* __restrict__ taps,
+__device__ __forceinline__ float small_block(const Dims& g, float* __restrict__ state, const float* __restrict__ taps,
                                             int t, int l, int s, int d) {
   constexpr int V = UB >= 4 ? 4 : UB;   // floats per vector access
   using vec = typename std::conditional<V == 4, float4, typename std::conditional<V == 2, float2, float>::type>::type;
@@ -248,25 +232,43 @@ __device__ __forceinline__ void small_block(const Dims& g, float* __restrict__ s
   }
 #pragma unroll
   for (int up = 0; up < UB; up += V) *reinterpret_cast<vec*>(dp + up) = *reinterpret_cast<const vec*>(cur + up);
+  return cur[0];
 }
 
-// The position's small block for every (layer, stream), one thread each; a
-// no-op at t = 0 and where lowbit(t) > kMlpBlockMax (that block ran before,
-// from HBM).
+// The position's small block for every (layer, stream), one thread each (a
+// no-op at t = 0 and where lowbit(t) > kMlpBlockMax: that block ran before,
+// from HBM); the layer-1 threads then form the red cell
+// y^1_t = acc^1_t + h^1_0 x_t into ybuf [B][D] (and the records), the first
+// layer's input.
 __global__ void k_mlp_block(Dims g, float* __restrict__ state, const float* __restrict__ taps, MlpPos p_host,
-                            const MlpPos* __restrict__ p_dev) {
+                            const MlpPos* __restrict__ p_dev, float* __restrict__ ybuf) {
   pdl_launch_dependents();   // the first layer's launch loads its weights meanwhile
-  const int t = p_dev ? p_dev->t : p_host.t;
+  const MlpPos p = p_dev ? *p_dev : p_host;
+  const int t = p.t;
   const int U = t & -t;
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (t == 0 || U > kMlpBlockMax || i >= g.M * g.S) return;
+  if (i >= g.M * g.S) return;
   const int l = i / g.S + 1, s = i - (l - 1) * g.S, d = s / g.B;
-  switch (U) {
-    case 1: small_block<1>(g, state, taps, t, l, s, d); break;
-    case 2: small_block<2>(g, state, taps, t, l, s, d); break;
-    case 4: small_block<4>(g, state, taps, t, l, s, d); break;
-    default: small_block<kMlpBlockMax>(g, state, taps, t, l, s, d); break;
+  float acc;
+  if (t == 0) {
+    acc = 0.f;
+  } else {
+    switch (U) {
+      case 1: acc = small_block<1>(g, state, taps, t, l, s, d); break;
+      case 2: acc = small_block<2>(g, state, taps, t, l, s, d); break;
+      case 4: acc = small_block<4>(g, state, taps, t, l, s, d); break;
+      case kMlpBlockMax: acc = small_block<kMlpBlockMax>(g, state, taps, t, l, s, d); break;
+      default:   // the block ran before: only layer 1's accumulator is read here
+        if (l != 1) return;
+        acc = state[slot_index(g, 1, s, t)];
+        break;
+    }
   }
+  if (l != 1) return;
+  const int b = s - d * g.B;
+  const float y = fmaf(__ldg(taps + (size_t)d * g.L), state[slot_index(g, 0, s, t)], acc);
+  ybuf[(size_t)b * g.D + d] = y;
+  record_y(g, 1, p, b, d, y);
 }
 
 // The position counter of a captured position: advanced once all its layers ran.
@@ -326,8 +328,8 @@ cudaError_t launch_mlp_layer(const Dims& g, float* state, const float* taps, con
   cfg.numAttrs = 1;
   cfg.gridDim = dim3((unsigned)((m.hidden + kMlpRows - 1) / kMlpRows), groups);
   cfg.dynamicSmemBytes = smem_in_bytes(g);
-  cudaError_t e = cudaLaunchKernelEx(&cfg, k_mlp_in, g, (const float*)state, taps, l, p, p_dev, m.hidden,
-                                     (const float*)m.w1, (const float*)m.b1, (const float*)m.y, m.z);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, k_mlp_in, g, l, m.hidden, (const float*)m.w1, (const float*)m.b1,
+                                     (const float*)m.y, m.z);
   if (e != cudaSuccess) return e;
   cfg.gridDim = dim3((unsigned)((g.D + kMlpRows - 1) / kMlpRows), groups);
   cfg.dynamicSmemBytes = smem_out_bytes(g, m.hidden);
@@ -336,9 +338,9 @@ cudaError_t launch_mlp_layer(const Dims& g, float* state, const float* taps, con
 }
 
 cudaError_t launch_mlp_block(const Dims& g, float* state, const float* taps, const MlpPos& p, const MlpPos* p_dev,
-                             cudaStream_t st) {
+                             float* ybuf, cudaStream_t st) {
   const int n = g.M * g.S;
-  k_mlp_block<<<(n + 255) / 256, 256, 0, st>>>(g, state, taps, p, p_dev);
+  k_mlp_block<<<(n + 255) / 256, 256, 0, st>>>(g, state, taps, p, p_dev, ybuf);
   return cudaGetLastError();
 }
 
