@@ -136,8 +136,13 @@ FI_API fi_status fi_prefill(fi_ctx* ctx, int32_t p, const void* x, float* y_out,
 
 /* fi_generate with HOST buffers: copies x0_host and eps_host to the device,
  * generates, copies y^M back to y_out_host, and returns when the copy is done.
- * Host buffers may be pageable or pinned (pinned is faster). Staging device
- * buffers are allocated on first use and kept by the context. */
+ * The work runs in segments of whole chunks (about 16 per call, none shorter
+ * than 1024 positions): the noise of later segments uploads and the outputs of
+ * earlier ones download on two streams of the context's own while a segment
+ * generates, so with pinned host buffers the copies overlap the generation.
+ * The results equal those of one fi_generate call. Host buffers may be
+ * pageable (no overlap) or pinned. Staging device buffers are allocated on
+ * first use and kept by the context. */
 FI_API fi_status fi_generate_host(fi_ctx* ctx, int32_t n, const void* x0_host, const float* eps_host,
                            float eps_scale, float* y_out_host);
 

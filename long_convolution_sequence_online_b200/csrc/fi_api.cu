@@ -1,6 +1,7 @@
 // C-ABI of the library (declared in include/fi.h): argument checks, device
 // memory, and the host side of the relaxed schedule (which block runs at
 // which step, and on which kernel).
+#include <algorithm>
 #include <cmath>
 #include <cstdio>
 #include <cstring>
@@ -30,6 +31,12 @@ fi_status cuda_fail(cudaError_t e, const char* what) {
     cudaError_t e_ = (call);                        \
     if (e_ != cudaSuccess) return cuda_fail(e_, what); \
   } while (0)
+
+// fi_generate_host splits a generation into about kHostSegments segments of
+// whole chunks (none shorter than kHostSegmentMin positions) so that copies
+// overlap work.
+constexpr int kHostSegments = 16;
+constexpr int kHostSegmentMin = 1024;
 
 struct EventPair {
   cudaEvent_t a, b;
@@ -72,6 +79,8 @@ struct fi_ctx {
   float* d_eps = nullptr;
   float* d_y = nullptr;
   size_t stage_n = 0;
+  cudaStream_t up_st = nullptr, dn_st = nullptr;   // host copies of fi_generate_host, beside the work
+  std::vector<cudaEvent_t> seg_ev;                 // per segment: uploaded, generated
   // profiling
   int prof = 0;
   std::vector<EventPair> ev_live, ev_free;
@@ -109,6 +118,9 @@ void free_ctx(fi_ctx* c) {
   cudaFree(c->d_x0);
   cudaFree(c->d_eps);
   cudaFree(c->d_y);
+  for (cudaEvent_t e : c->seg_ev) cudaEventDestroy(e);
+  if (c->up_st) cudaStreamDestroy(c->up_st);
+  if (c->dn_st) cudaStreamDestroy(c->dn_st);
   for (auto& e : c->ev_live) { cudaEventDestroy(e.a); cudaEventDestroy(e.b); }
   for (auto& e : c->ev_free) { cudaEventDestroy(e.a); cudaEventDestroy(e.b); }
   delete c;
@@ -606,11 +618,49 @@ fi_status fi_generate_host(fi_ctx* c, int32_t n, const void* x0_host, const floa
     if ((s = dev_alloc((void**)&c->d_y, row * n * sizeof(float), "staging y")) != FI_OK) return s;
     c->stage_n = (size_t)n;
   }
-  FI_CUDA(cudaMemcpyAsync(c->d_x0, x0_host, row * esz, cudaMemcpyHostToDevice, c->st), "x0 upload");
-  FI_CUDA(cudaMemcpyAsync(c->d_eps, eps_host, row * n * sizeof(float), cudaMemcpyHostToDevice, c->st), "eps upload");
-  fi_status s = fi_generate(c, n, c->d_x0, c->d_eps, eps_scale, c->d_y, nullptr);
-  if (s != FI_OK) return s;
-  FI_CUDA(cudaMemcpyAsync(y_out_host, c->d_y, row * n * sizeof(float), cudaMemcpyDeviceToHost, c->st), "y download");
+  // Segments of whole chunks: segment k's noise is uploaded on up_st, generated
+  // on the context's stream once it has arrived, and its outputs are read back
+  // on dn_st once generated, so the copies of one segment overlap the
+  // generation of others (with pinned host buffers). The generation itself is
+  // the same as one fi_generate call: each segment continues from the state
+  // the previous one left.
+  const int per = (n + kHostSegments - 1) / kHostSegments;
+  const int seg = per <= kHostSegmentMin ? n : ((per + kChunkMaxSteps - 1) / kChunkMaxSteps) * kChunkMaxSteps;
+  const int nseg = (n + seg - 1) / seg;
+  if (!c->up_st) FI_CUDA(cudaStreamCreateWithFlags(&c->up_st, cudaStreamNonBlocking), "copy stream");
+  if (!c->dn_st) FI_CUDA(cudaStreamCreateWithFlags(&c->dn_st, cudaStreamNonBlocking), "copy stream");
+  while (c->seg_ev.size() < 2 * (size_t)nseg + 1) {
+    cudaEvent_t e;
+    FI_CUDA(cudaEventCreateWithFlags(&e, cudaEventDisableTiming), "cudaEventCreate");
+    c->seg_ev.push_back(e);
+  }
+  // the staging buffers may still be read or written by an earlier call's work
+  FI_CUDA(cudaEventRecord(c->seg_ev[2 * nseg], c->st), "cudaEventRecord");
+  FI_CUDA(cudaStreamWaitEvent(c->up_st, c->seg_ev[2 * nseg], 0), "cudaStreamWaitEvent");
+  FI_CUDA(cudaMemcpyAsync(c->d_x0, x0_host, row * esz, cudaMemcpyHostToDevice, c->up_st), "x0 upload");
+  for (int k = 0; k < nseg; ++k) {
+    const size_t off = (size_t)k * seg * row, cnt = (size_t)std::min(seg, n - k * seg) * row;
+    FI_CUDA(cudaMemcpyAsync(c->d_eps + off, eps_host + off, cnt * sizeof(float), cudaMemcpyHostToDevice, c->up_st),
+            "eps upload");
+    FI_CUDA(cudaEventRecord(c->seg_ev[2 * k], c->up_st), "cudaEventRecord");
+  }
+  for (int k = 0; k < nseg; ++k) {
+    const int nk = std::min(seg, n - k * seg);
+    const size_t off = (size_t)k * seg * row;
+    FI_CUDA(cudaStreamWaitEvent(c->st, c->seg_ev[2 * k], 0), "cudaStreamWaitEvent");
+    fi_status s = fi_generate(c, nk, k == 0 ? c->d_x0 : nullptr, c->d_eps + off, eps_scale, c->d_y + off, nullptr);
+    if (s != FI_OK) {
+      cudaStreamSynchronize(c->up_st);
+      cudaStreamSynchronize(c->dn_st);
+      return s;
+    }
+    FI_CUDA(cudaEventRecord(c->seg_ev[2 * k + 1], c->st), "cudaEventRecord");
+    FI_CUDA(cudaStreamWaitEvent(c->dn_st, c->seg_ev[2 * k + 1], 0), "cudaStreamWaitEvent");
+    FI_CUDA(cudaMemcpyAsync(y_out_host + off, c->d_y + off, (size_t)nk * row * sizeof(float), cudaMemcpyDeviceToHost,
+                            c->dn_st),
+            "y download");
+  }
+  FI_CUDA(cudaStreamSynchronize(c->dn_st), "synchronize");
   return sync_and_check(c);
 }
 

@@ -242,6 +242,25 @@ def test_generate_host_matches_device(fi):
     assert np.array_equal(yh, y.cpu().numpy())
 
 
+def test_generate_host_in_segments_matches_device(fi):
+    # 20000 positions: 16 segments of 1280 (the last one 800), copies on their
+    # own streams from pinned buffers; the outputs equal one device call's.
+    w = _workload(2, 4, 32768, 2)
+    inp = gpu_inputs(w, 6)
+    n = 20000
+    ctx = fi.Context(inp["h"], w.batch, w.dtype)
+    eps = inp["eps"][:n].contiguous()
+    y = torch.empty((n, w.batch, w.channels), dtype=torch.float32, device="cuda")
+    ctx.generate(n, inp["x0"], eps, y, 0.1)
+    ctx.reset()
+    x0_h = inp["x0"].cpu().pin_memory()
+    eps_h = eps.cpu().pin_memory()
+    y_h = torch.empty((n, w.batch, w.channels), dtype=torch.float32).pin_memory()
+    ctx.generate_host_ptr(n, x0_h.data_ptr(), eps_h.data_ptr(), y_h.data_ptr(), 0.1)
+    assert torch.equal(y_h, y.cpu())
+    ctx.close()
+
+
 def test_reset_replays_identically(fi):
     w = _workload(2, 5, 512, 1)
     inp = gpu_inputs(w, 8)
