@@ -137,7 +137,7 @@ FI_API fi_status fi_prefill(fi_ctx* ctx, int32_t p, const void* x, float* y_out,
 /* fi_generate with HOST buffers: copies x0_host and eps_host to the device,
  * generates, copies y^M back to y_out_host, and returns when the copy is done.
  * The work runs in segments of whole chunks (about 16 per call, none shorter
- * than 1024 positions): the noise of later segments uploads and the outputs of
+ * than 256 positions): the noise of later segments uploads and the outputs of
  * earlier ones download on two streams of the context's own while a segment
  * generates, so with pinned host buffers the copies overlap the generation.
  * The results equal those of one fi_generate call. Host buffers may be

@@ -36,7 +36,7 @@ fi_status cuda_fail(cudaError_t e, const char* what) {
 // whole chunks (none shorter than kHostSegmentMin positions) so that copies
 // overlap work.
 constexpr int kHostSegments = 16;
-constexpr int kHostSegmentMin = 1024;
+constexpr int kHostSegmentMin = 256;
 
 struct EventPair {
   cudaEvent_t a, b;

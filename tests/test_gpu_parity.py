@@ -245,6 +245,7 @@ def test_generate_host_matches_device(fi):
 def test_generate_host_in_segments_matches_device(fi):
     # 20000 positions: 16 segments of 1280 (the last one 800), copies on their
     # own streams from pinned buffers; the outputs equal one device call's.
+    # (Segments are at least 256 positions: a call of 4096 or fewer is one.)
     w = _workload(2, 4, 32768, 2)
     inp = gpu_inputs(w, 6)
     n = 20000
