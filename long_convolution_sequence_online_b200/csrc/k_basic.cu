@@ -1,5 +1,7 @@
 // Per-position red cells, direct blocks read from HBM, the Lazy method's sums
 // and the layout conversions.
+#include <type_traits>
+
 #include "fi_internal.cuh"
 
 namespace fi {
@@ -77,46 +79,63 @@ __global__ void k_token_par(Dims g, float* __restrict__ state, const float* __re
   const int s = blockIdx.x * 32 + lane;
   const bool ok = s < g.S;
   const int d = ok ? s / g.B : 0;
+  const int b = s - d * g.B;
+  const size_t io = (size_t)b * g.D + d;
+  // The chain's token and noise depend on no layer's sum: read them first.
+  float a_tok = 0.f, e = 0.f;
+  if (li == 0 && ok) {
+    a_tok = x_t ? round_act(load_token(x_t, io, g.bf16), g.bf16) : state[slot_index(g, 0, s, t)];
+    if (eps_t && t + 1 < g.L) e = eps_t[io];
+  }
   if (ok) {
     const int l = li + 1;
     const float* hp = taps + ((size_t)(l - 1) * g.D + d) * g.L;
-    h0s[li * 32 + lane] = __ldg(hp);
     float* dp = state + slot_index(g, l, s, t);
     float acc;
     if constexpr (U == 0) {
+      h0s[li * 32 + lane] = __ldg(hp);
       acc = (t == 0) ? 0.f : dp[0];
     } else {
+      // Vector accesses: t is a multiple of U, and rows of the state and the
+      // taps start 16-byte aligned (L >= 2U).
+      constexpr int V = U >= 4 ? 4 : U;
+      using vec = typename std::conditional<V == 4, float4, typename std::conditional<V == 2, float2, float>::type>::type;
       const bool overwrite = (t == U);   // lowbit(t) == t: t is a power of two
       const float* xp = state + slot_index(g, l - 1, s, t - U);
-      float x[U], hw[2 * U - 1], cur[U];
+      float x[U], h[2 * U], cur[U];
 #pragma unroll
-      for (int u = 0; u < U; ++u) x[u] = xp[u];
+      for (int u = 0; u < U; u += V) *reinterpret_cast<vec*>(x + u) = *reinterpret_cast<const vec*>(xp + u);
+      if constexpr (V == 1) {
+        *reinterpret_cast<float2*>(h) = __ldg(reinterpret_cast<const float2*>(hp));
+      } else {
 #pragma unroll
-      for (int k = 0; k < 2 * U - 1; ++k) hw[k] = __ldg(hp + 1 + k);   // h[1 .. 2U-1]
+        for (int k = 0; k < 2 * U; k += V) *reinterpret_cast<vec*>(h + k) = __ldg(reinterpret_cast<const vec*>(hp + k));
+      }
+      if (overwrite) {
 #pragma unroll
-      for (int up = 0; up < U; ++up) cur[up] = overwrite ? 0.f : dp[up];
+        for (int up = 0; up < U; ++up) cur[up] = 0.f;
+      } else {
+#pragma unroll
+        for (int up = 0; up < U; up += V) *reinterpret_cast<vec*>(cur + up) = *reinterpret_cast<const vec*>(dp + up);
+      }
 #pragma unroll
       for (int up = 0; up < U; ++up) {
 #pragma unroll
-        for (int u = 0; u < U; ++u) cur[up] = fmaf(hw[U + up - u - 1], x[u], cur[up]);
+        for (int u = 0; u < U; ++u) cur[up] = fmaf(h[U + up - u], x[u], cur[up]);
       }
+      h0s[li * 32 + lane] = h[0];
       acc = cur[0];
+      // targets t+1 .. t+U-1 back to the state (slot t receives the red cell's
+      // activation below, or for the last layer is not read again)
 #pragma unroll
-      for (int up = 1; up < U; ++up) dp[up] = cur[up];
+      for (int up = 0; up < U; up += V) *reinterpret_cast<vec*>(dp + up) = *reinterpret_cast<const vec*>(cur + up);
     }
     accs[li * 32 + lane] = acc;
   }
   __syncthreads();
   if (li != 0 || !ok) return;
-  const int b = s - d * g.B;
-  const size_t io = (size_t)b * g.D + d;
-  float a;
-  if (x_t) {
-    a = round_act(load_token(x_t, io, g.bf16), g.bf16);
-    state[slot_index(g, 0, s, t)] = a;
-  } else {
-    a = state[slot_index(g, 0, s, t)];
-  }
+  float a = a_tok;
+  if (x_t) state[slot_index(g, 0, s, t)] = a;
   float y = 0.f;
   for (int l = 1; l <= g.M; ++l) {
     y = fmaf(h0s[(l - 1) * 32 + lane], a, accs[(l - 1) * 32 + lane]);
@@ -126,7 +145,7 @@ __global__ void k_token_par(Dims g, float* __restrict__ state, const float* __re
     }
   }
   y_t[io] = y;
-  if (eps_t && t + 1 < g.L) state[slot_index(g, 0, s, t + 1)] = round_act(tanhf(y) + eps_scale * eps_t[io], g.bf16);
+  if (eps_t && t + 1 < g.L) state[slot_index(g, 0, s, t + 1)] = round_act(tanhf(y) + eps_scale * e, g.bf16);
 }
 
 cudaError_t launch_token(const Dims& g, float* state, const float* taps, int t, const void* x_t,
@@ -191,10 +210,13 @@ __global__ void k_tile_direct(Dims g, float* __restrict__ state, const float* __
 // most positions): one thread per (row, target), U threads per row, so a launch
 // is a few waves of short threads instead of one CTA per row. Taps h[U+u'-u] are
 // contiguous across a row's threads; its sources are the same for all of them.
+// U is a template argument so that the whole sum unrolls and a thread issues
+// all its loads before the first product.
+template <int U>
 __global__ void k_tile_direct_small(Dims g, float* __restrict__ state, const float* __restrict__ taps, int i,
-                                    int log2u, int overwrite, int t_min) {
+                                    int overwrite, int t_min) {
   pdl_launch_dependents();
-  const int U = 1 << log2u;
+  constexpr int log2u = U >= 32 ? 5 : U >= 16 ? 4 : U >= 8 ? 3 : U >= 4 ? 2 : U >= 2 ? 1 : 0;
   const long gid = (long)blockIdx.x * blockDim.x + threadIdx.x;
   const long row = gid >> log2u;        // ((l-1)*D + d)*B + b
   if (row >= (long)g.M * g.S) return;
@@ -207,8 +229,15 @@ __global__ void k_tile_direct_small(Dims g, float* __restrict__ state, const flo
   const int s = d * g.B + b;
   const float* hp = taps + ((size_t)(l - 1) * g.D + d) * g.L + U + up;
   const float* xp = state + slot_index(g, l - 1, s, i - U);
+  float hv[U], xv[U];
+#pragma unroll
+  for (int u = 0; u < U; ++u) {
+    hv[u] = __ldg(hp - u);
+    xv[u] = __ldg(xp + u);
+  }
   float sum = 0.f;
-  for (int u = 0; u < U; ++u) sum = fmaf(__ldg(hp - u), __ldg(xp + u), sum);
+#pragma unroll
+  for (int u = 0; u < U; ++u) sum = fmaf(hv[u], xv[u], sum);
   float* dp = state + slot_index(g, l, s, i + up);
   *dp = overwrite ? sum : *dp + sum;
 }
@@ -246,8 +275,16 @@ cudaError_t launch_tile_direct(const Dims& g, float* state, const float* taps, i
   if (U <= 32) {
     const long threads_total = (long)g.M * g.S * U;
     const int threads = 256;
-    k_tile_direct_small<<<(unsigned)((threads_total + threads - 1) / threads), threads, 0, st>>>(
-        g, state, taps, i, ilog2(U), is_pow2(i) ? 1 : 0, t_min);
+    const unsigned blocks = (unsigned)((threads_total + threads - 1) / threads);
+    const int ow = is_pow2(i) ? 1 : 0;
+    switch (U) {
+      case 1: k_tile_direct_small<1><<<blocks, threads, 0, st>>>(g, state, taps, i, ow, t_min); break;
+      case 2: k_tile_direct_small<2><<<blocks, threads, 0, st>>>(g, state, taps, i, ow, t_min); break;
+      case 4: k_tile_direct_small<4><<<blocks, threads, 0, st>>>(g, state, taps, i, ow, t_min); break;
+      case 8: k_tile_direct_small<8><<<blocks, threads, 0, st>>>(g, state, taps, i, ow, t_min); break;
+      case 16: k_tile_direct_small<16><<<blocks, threads, 0, st>>>(g, state, taps, i, ow, t_min); break;
+      default: k_tile_direct_small<32><<<blocks, threads, 0, st>>>(g, state, taps, i, ow, t_min); break;
+    }
     return cudaGetLastError();
   }
   const size_t smem = (size_t)3 * U * sizeof(float);
