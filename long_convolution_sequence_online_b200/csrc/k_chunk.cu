@@ -571,6 +571,9 @@ __global__ void __launch_bounds__(kChunkMaxThreads) k_chunk(Dims g, ChunkArgs a,
   cp_async_wait_all();
   __syncthreads();
 
+  // Every CTA has its window: the next launch (the block at the next chunk
+  // boundary) may be launched now; it waits for this grid before reading.
+  pdl_launch_dependents();
   const int warp = tid >> 5, lane = tid & 31;
   // Hand-off. In the re-timed table the chain adds the terms of lags
   // 1..nlag (h^l[k] a^{l-1}_{t-k}) itself and the pieces of step i (sources

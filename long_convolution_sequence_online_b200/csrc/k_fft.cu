@@ -250,6 +250,7 @@ __global__ void __launch_bounds__(T >= 128 ? T : 128)
 k_tile_fft(Dims g, float* __restrict__ state, const float2* __restrict__ spec,
            const float2* __restrict__ tw, int i, int overwrite, int t_min) {
   pdl_launch_dependents();
+  pdl_wait_primary();   // sources and accumulators come from the launch before
   constexpr int F = T >= 128 ? 1 : 128 / T;
   extern __shared__ float2 fsm[];
   const int sub = threadIdx.x / T, tid = threadIdx.x - sub * T;
@@ -391,6 +392,7 @@ __global__ void __launch_bounds__(T >= 128 ? T : 128, fft2_min_blocks(N2))
 k_tile_fft2(Dims g, float* __restrict__ state, const float2* __restrict__ spec, int i,
             int overwrite, int t_min) {
   pdl_launch_dependents();
+  pdl_wait_primary();   // sources and accumulators come from the launch before
   constexpr int U = N2 / 2;
   constexpr int F = T >= 128 ? 1 : 128 / T;
   extern __shared__ float2 fsm[];
@@ -565,6 +567,23 @@ k_debug_fft(int count, const float2* __restrict__ in, float2* __restrict__ out, 
 }
 
 // ------------------------------------------------------------------ dispatch
+// Block launches allow programmatic stream serialization: the grid may be
+// launched while the chunk kernel before it finishes (its CTAs wait for it
+// with pdl_wait_primary before reading the state).
+static cudaLaunchConfig_t pdl_config(cudaLaunchAttribute (&attr)[1], unsigned blocks, int threads, size_t smem,
+                                     cudaStream_t st) {
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(blocks);
+  cfg.blockDim = dim3((unsigned)threads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cfg;
+}
+
 template <int N>
 static size_t fft_smem_bytes() { return (size_t)fft_per_cta(N) * fft_smem_elems(N) * sizeof(float2); }
 
@@ -584,8 +603,9 @@ static cudaError_t tile_fft_n(const Dims& g, float* state, const float2* spec, c
   const long items = (long)g.M * g.S;
   const long blocks = (items + F - 1) / F;
   const int overwrite = is_pow2(i) ? 1 : 0;
-  k_tile_fft<N, T><<<(unsigned)blocks, T * F, smem, st>>>(g, state, spec, tw, i, overwrite, t_min);
-  return cudaGetLastError();
+  cudaLaunchAttribute attr[1];
+  cudaLaunchConfig_t cfg = pdl_config(attr, (unsigned)blocks, T * F, smem, st);
+  return cudaLaunchKernelEx(&cfg, k_tile_fft<N, T>, g, state, spec, tw, i, overwrite, t_min);
 }
 
 // Points per thread of the paired blocks (N2 = 2U points per pair): the choice
@@ -608,8 +628,9 @@ static cudaError_t tile_fft2_n(const Dims& g, float* state, const float2* spec, 
   const long items = (long)g.M * (g.S / 2);
   const long blocks = (items + F - 1) / F;
   const int overwrite = is_pow2(i) ? 1 : 0;
-  k_tile_fft2<N2, T, PL><<<(unsigned)blocks, T * F, smem, st>>>(g, state, spec, i, overwrite, t_min);
-  return cudaGetLastError();
+  cudaLaunchAttribute attr[1];
+  cudaLaunchConfig_t cfg = pdl_config(attr, (unsigned)blocks, T * F, smem, st);
+  return cudaLaunchKernelEx(&cfg, k_tile_fft2<N2, T, PL>, g, state, spec, i, overwrite, t_min);
 }
 
 template <int N>
