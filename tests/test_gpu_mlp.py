@@ -169,6 +169,29 @@ def test_mlp_block_state_rules(fi):
     ref.close()
 
 
+@pytest.mark.parametrize("M,D,Dh,B,dtype", [
+    (1, 8, 10, 3, "f32"),      # one layer: the small-block launch records y^M itself
+    (2, 12, 16, 9, "bf16"),    # two CTA groups (8 + 1) in a bf16 context
+    (3, 8, 10, 2, "f32"),      # W1 rows float4 (D = 8), W2 rows scalar (Dh = 10)
+])
+def test_mlp_block_shapes_teacher_forced(fi, M, D, Dh, B, dtype):
+    w = synth.Workload(f"mlp-{M}x{D}-L256-B{B}-{dtype}", M, D, 256, B, dtype, 1e-1, 5e-1)
+    inp = gpu_inputs(w, 100 + M + D)
+    ws = _weights(M, D, Dh, 200 + Dh)
+    ctx = fi.Context(inp["h"], B, dtype)
+    _set(ctx, ws)
+    n = 200                                   # a ragged stop inside the sequence
+    y = torch.empty((n, B, D), dtype=torch.float32, device="cuda")
+    rec = torch.empty((M, n, B, D), dtype=torch.float32, device="cuda")
+    ctx.generate(n, inp["x0"], inp["eps"][:n].contiguous(), y, 0.1, rec)
+    ctx.sync()
+    acts = [a.cpu().numpy() for a in read_all_activations(ctx, n)]
+    ctx.close()
+    rec = rec.cpu().numpy()
+    assert np.array_equal(y.cpu().numpy(), rec[-1])
+    _check_teacher_forced(w, oracle_filters(inp["h_np"], dtype), ws, acts, rec, inp["eps_np"])
+
+
 def test_mlp_block_groups_and_scalar_rows(fi):
     # B = 10 sequences: two CTA groups (8 + 2); D = 6 and Dh = 10 are not
     # multiples of 4, so both products take the scalar row path.
