@@ -5,16 +5,19 @@
 //   a^l_t = R(W2^l GELU(W1^l y^l_t + b1^l) + b2^l)   (per sequence b, across channels),
 // with y^l_t = acc^l_t + h^l_0 a^{l-1}_t (the red cell) and GELU(u) = u Phi(u)
 // (the exact form, from erff). Unlike tanh the block mixes channels, so layer
-// l+1 at position t needs every channel of layer l at t: each position runs,
-// per layer, one launch for the first product and one for the second.
+// l+1 at position t needs every channel of layer l at t. Each position runs one
+// launch for the schedule's small block of step t and layer 1's red cells,
+// then per layer one launch for the first product and one for the second.
 //
 // Both products are matrix-vector work on weights that stay in L2 (a few MB
 // per layer), so they are latency-bound: one warp owns one weight row, its
 // lanes load the row as independent float4s, and every row is applied to up to
 // kMlpGroup sequences at once (the row is read once per group, not once per
 // sequence). The second product also forms the next layer's red cell y^{l+1}_t
-// for its channel (one strided read of acc^{l+1}_t) into a dense [B][D]
-// buffer, so only layer 1 gathers its inputs from the strided state.
+// for its channel into a dense [B][D] buffer, so no launch gathers a layer's
+// inputs from the strided state. Launches are programmatic: each loads what
+// does not depend on the launch before it (weights, biases, taps, and for the
+// second product the next accumulator and the noise) before it waits.
 #include <type_traits>
 
 #include "fi_internal.cuh"
