@@ -61,6 +61,7 @@ struct fi_ctx {
   int tc_q_hi = -1;                // block sides 2^6 .. 2^tc_q_hi run on the tensor cores
   TcPlan tc[32] = {};
   int chunk_G = 0;
+  bool pdl_blocks = false;         // FFT blocks launched programmatically (the chunk grid fills the SMs)
   float* state = nullptr;
   float* taps = nullptr;
   float2* spectra = nullptr;
@@ -184,7 +185,10 @@ fi_status run_block(fi_ctx* c, int i, int t_min = 0) {
   }
   if (q >= c->q_lo && q <= c->q_hi) {
     return timed(c, KC_FFT,
-                 [&] { return launch_tile_fft(c->g, c->state, c->spectra + c->spec_off[q], c->twiddle, i, t_min, c->st); },
+                 [&] {
+                   return launch_tile_fft(c->g, c->state, c->spectra + c->spec_off[q], c->twiddle, i, t_min, c->st,
+                                          c->pdl_blocks);
+                 },
                  "FFT block launch", q);
   }
   return timed(c, KC_DIRECT, [&] { return launch_tile_direct(c->g, c->state, c->taps, i, t_min, c->st); },
@@ -301,6 +305,13 @@ fi_status fi_init(fi_ctx** out, const fi_config* cfg, const void* h, void* strea
   }
   c->chunk_G = chunk_streams_per_cta(g, c->chunk, c->num_sms, c->max_smem);
   if (c->chunk_G == 0) return bail(fail(FI_E_UNSUPPORTED, "too many layers for the on-chip chunk window"));
+  // Measured: an FFT grid launched early settles wherever it finds room and
+  // runs slower there, on SMs a small chunk grid leaves idle (B = 1 stacks)
+  // or beside chunk CTAs that leave registers free (short stacks). So only
+  // chunk grids of whole-SM CTAs that leave at most a sixteenth of the SMs
+  // idle take it.
+  c->pdl_blocks = chunk_cta_fills_sm(g, c->chunk_G) &&
+                  (g.S + c->chunk_G - 1) / c->chunk_G >= c->num_sms - c->num_sms / 16;
   if ((e = configure_chunk(chunk_smem_bytes(g, c->chunk, c->chunk_G))) != cudaSuccess)
     return bail(cuda_fail(e, "configure chunk kernel"));
 
@@ -554,6 +565,7 @@ fi_status fi_generate(fi_ctx* c, int32_t n, const void* x0, const float* eps, fl
     a.last_done = last_done;
     a.err = c->err;
     a.wait_limit = c->wait_limit;
+    a.trigger = c->pdl_blocks ? 1 : 0;
     if ((s = timed(c, KC_CHUNK, [&] { return launch_chunk(c->g, a, c->chunk_G, c->st); }, "chunk launch")) != FI_OK)
       return s;
     p = p1;

@@ -84,8 +84,11 @@ cudaError_t launch_tile_direct(const Dims& g, float* state, const float* taps, i
                                int t_min, cudaStream_t st);
 
 // FFT block of step i (side U = lowbit(i), 2^kMinFftLog2 <= U <= 2^kMaxFftLog2).
+// pdl: launched with programmatic stream serialization (worth it after a chunk
+// kernel that fills nearly every SM; with many idle SMs the early grid would
+// settle there and run on fewer SMs).
 cudaError_t launch_tile_fft(const Dims& g, float* state, const float2* spectrum_q,
-                            const float2* twiddle, int i, int t_min, cudaStream_t st);
+                            const float2* twiddle, int i, int t_min, cudaStream_t st, bool pdl = false);
 
 // Spectra of one level q for all (layer, channel).
 cudaError_t launch_spectra(const Dims& g, const float* taps, float2* spectrum_q,
@@ -152,6 +155,7 @@ struct ChunkArgs {
   int last_done;         // last step whose blocks have reached HBM before this launch
   int* err;              // device flag set to 1 when a bounded wait gives up
   int wait_limit;        // barrier checks before a wait gives up
+  int trigger;           // let the next block launch (programmatic) start early
   ChunkTable tab;        // filled by launch_chunk
 };
 
@@ -161,6 +165,9 @@ constexpr int kDefaultWaitLimit = 1 << 20;
 cudaError_t launch_chunk(const Dims& g, const ChunkArgs& a, int streams_per_cta, cudaStream_t st);
 cudaError_t configure_chunk(size_t smem);   // allow `smem` bytes of dynamic shared memory
 int chunk_streams_per_cta(const Dims& g, int chunk, int num_sms, size_t max_smem);
+// A chunk CTA of this shape takes a whole SM (every register), so no other
+// grid's CTA can share its SM while it runs.
+bool chunk_cta_fills_sm(const Dims& g, int streams_per_cta);
 size_t chunk_smem_bytes(const Dims& g, int chunk, int streams_per_cta);
 
 // Lazy sums of position t for all layers: slot(l, s, t) = sum_{s' < t} h^l[t-s'] a^{l-1}_{s'}.

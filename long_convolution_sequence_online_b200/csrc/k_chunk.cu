@@ -429,7 +429,10 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, int parity, int* err, b
 // layer of the group has arrived); the chain waits on tile_done before reading a
 // group's accumulators. Each barrier thus advances at most one phase ahead of
 // its waiters, parity waits are exact, and every wait is bounded.
-template <bool BF16, bool REC>
+// TRIG: the variant that lets the next block launch (programmatic) start once
+// every CTA holds its window; launches followed by a plain block launch use the
+// variant without the instruction.
+template <bool BF16, bool REC, bool TRIG>
 __global__ void __launch_bounds__(kChunkMaxThreads) k_chunk(Dims g, ChunkArgs a, int G) {
   extern __shared__ float csm[];
   const ChunkShape cs = chunk_shape(g, a.chunk, G);
@@ -572,8 +575,9 @@ __global__ void __launch_bounds__(kChunkMaxThreads) k_chunk(Dims g, ChunkArgs a,
   __syncthreads();
 
   // Every CTA has its window: the next launch (the block at the next chunk
-  // boundary) may be launched now; it waits for this grid before reading.
-  pdl_launch_dependents();
+  // boundary, when launched programmatically) may start now; it waits for
+  // this grid before reading.
+  if constexpr (TRIG) pdl_launch_dependents();
   const int warp = tid >> 5, lane = tid & 31;
   // Hand-off. In the re-timed table the chain adds the terms of lags
   // 1..nlag (h^l[k] a^{l-1}_{t-k}) itself and the pieces of step i (sources
@@ -821,6 +825,10 @@ static int chunk_threads(const Dims& g, int G) {
   return 32 * (cw + (want < max_w - cw ? want : max_w - cw));
 }
 
+bool chunk_cta_fills_sm(const Dims& g, int streams_per_cta) {
+  return chunk_threads(g, streams_per_cta) >= kChunkMaxThreads;
+}
+
 int chunk_streams_per_cta(const Dims& g, int chunk, int num_sms, size_t max_smem) {
   int G = (g.S + num_sms - 1) / num_sms;
   if (G > kChunkMaxStreams) G = kChunkMaxStreams;
@@ -846,13 +854,21 @@ static cudaError_t raise_smem_cap(K kernel, size_t smem) {
   return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
 }
 
+using ChunkKernel = void (*)(Dims, ChunkArgs, int);
+static ChunkKernel chunk_variant(bool bf16, bool rec, bool trig) {
+  if (bf16) {
+    if (rec) return trig ? k_chunk<true, true, true> : k_chunk<true, true, false>;
+    return trig ? k_chunk<true, false, true> : k_chunk<true, false, false>;
+  }
+  if (rec) return trig ? k_chunk<false, true, true> : k_chunk<false, true, false>;
+  return trig ? k_chunk<false, false, true> : k_chunk<false, false, false>;
+}
+
 cudaError_t configure_chunk(size_t smem) {
   static std::mutex mu;
   std::lock_guard<std::mutex> lock(mu);
-  cudaError_t e = raise_smem_cap(k_chunk<false, false>, smem);
-  if (e == cudaSuccess) e = raise_smem_cap(k_chunk<false, true>, smem);
-  if (e == cudaSuccess) e = raise_smem_cap(k_chunk<true, false>, smem);
-  if (e == cudaSuccess) e = raise_smem_cap(k_chunk<true, true>, smem);
+  cudaError_t e = cudaSuccess;
+  for (int v = 0; v < 8 && e == cudaSuccess; ++v) e = raise_smem_cap(chunk_variant(v & 1, v & 2, v & 4), smem);
   return e;
 }
 
@@ -879,11 +895,9 @@ cudaError_t launch_chunk(const Dims& g, const ChunkArgs& a_in, int G, cudaStream
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   if (g.bf16) {
-    if (a.rec) return cudaLaunchKernelEx(&cfg, k_chunk<true, true>, g, a, G);
-    return cudaLaunchKernelEx(&cfg, k_chunk<true, false>, g, a, G);
+    return cudaLaunchKernelEx(&cfg, chunk_variant(true, a.rec != nullptr, a.trigger != 0), g, a, G);
   }
-  if (a.rec) return cudaLaunchKernelEx(&cfg, k_chunk<false, true>, g, a, G);
-  return cudaLaunchKernelEx(&cfg, k_chunk<false, false>, g, a, G);
+  return cudaLaunchKernelEx(&cfg, chunk_variant(false, a.rec != nullptr, a.trigger != 0), g, a, G);
 }
 
 }  // namespace fi

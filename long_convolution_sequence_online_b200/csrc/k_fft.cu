@@ -245,12 +245,14 @@ k_part_inv(Dims g, float* __restrict__ state, const float2* __restrict__ xs, con
 
 // One FFT block for every (layer, stream): item = (l-1)*S + s. T threads per
 // transform, F = cta_threads / T transforms per CTA.
-template <int N, int T = fft_threads(N)>
+// PDLW: the variant launched programmatically, which waits for the launch
+// before it; plain launches use the variant without the instruction.
+template <int N, int T = fft_threads(N), bool PDLW = false>
 __global__ void __launch_bounds__(T >= 128 ? T : 128)
 k_tile_fft(Dims g, float* __restrict__ state, const float2* __restrict__ spec,
            const float2* __restrict__ tw, int i, int overwrite, int t_min) {
   pdl_launch_dependents();
-  pdl_wait_primary();   // sources and accumulators come from the launch before
+  if constexpr (PDLW) pdl_wait_primary();   // sources and accumulators come from the launch before
   constexpr int F = T >= 128 ? 1 : 128 / T;
   extern __shared__ float2 fsm[];
   const int sub = threadIdx.x / T, tid = threadIdx.x - sub * T;
@@ -387,12 +389,12 @@ __device__ __forceinline__ void tile_fft2_body(float2* sm, float* ds, int tid, b
 // sides that hold 32 points per thread (8192: 4.1 -> 6.5 ms).
 __host__ __device__ constexpr int fft2_min_blocks(int n2) { return n2 == 512 ? 3 : n2 == 4096 ? 2 : 1; }
 
-template <int N2, int T, int PL = 0>
+template <int N2, int T, int PL = 0, bool PDLW = false>
 __global__ void __launch_bounds__(T >= 128 ? T : 128, fft2_min_blocks(N2))
 k_tile_fft2(Dims g, float* __restrict__ state, const float2* __restrict__ spec, int i,
             int overwrite, int t_min) {
   pdl_launch_dependents();
-  pdl_wait_primary();   // sources and accumulators come from the launch before
+  if constexpr (PDLW) pdl_wait_primary();   // sources and accumulators come from the launch before
   constexpr int U = N2 / 2;
   constexpr int F = T >= 128 ? 1 : 128 / T;
   extern __shared__ float2 fsm[];
@@ -567,9 +569,9 @@ k_debug_fft(int count, const float2* __restrict__ in, float2* __restrict__ out, 
 }
 
 // ------------------------------------------------------------------ dispatch
-// Block launches allow programmatic stream serialization: the grid may be
-// launched while the chunk kernel before it finishes (its CTAs wait for it
-// with pdl_wait_primary before reading the state).
+// Block launches with pdl allow programmatic stream serialization: the grid
+// may be launched while the chunk kernel before it finishes (its CTAs wait for
+// it with pdl_wait_primary before reading the state).
 static cudaLaunchConfig_t pdl_config(cudaLaunchAttribute (&attr)[1], unsigned blocks, int threads, size_t smem,
                                      cudaStream_t st) {
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -595,17 +597,21 @@ static cudaError_t prepare(K kernel, size_t smem) {
 
 template <int N, int T = fft_threads(N)>
 static cudaError_t tile_fft_n(const Dims& g, float* state, const float2* spec, const float2* tw, int i,
-                              int t_min, cudaStream_t st) {
+                              int t_min, cudaStream_t st, bool pdl) {
   constexpr int F = T >= 128 ? 1 : 128 / T;
   const size_t smem = (size_t)F * (fft_smem_elems(N) + N / 2) * sizeof(float2);
-  cudaError_t e = prepare(k_tile_fft<N, T>, smem);
+  cudaError_t e = pdl ? prepare(k_tile_fft<N, T, true>, smem) : prepare(k_tile_fft<N, T, false>, smem);
   if (e != cudaSuccess) return e;
   const long items = (long)g.M * g.S;
   const long blocks = (items + F - 1) / F;
   const int overwrite = is_pow2(i) ? 1 : 0;
+  if (!pdl) {   // the plain launch costs the host less (launch-bound stacks)
+    k_tile_fft<N, T, false><<<(unsigned)blocks, T * F, smem, st>>>(g, state, spec, tw, i, overwrite, t_min);
+    return cudaGetLastError();
+  }
   cudaLaunchAttribute attr[1];
   cudaLaunchConfig_t cfg = pdl_config(attr, (unsigned)blocks, T * F, smem, st);
-  return cudaLaunchKernelEx(&cfg, k_tile_fft<N, T>, g, state, spec, tw, i, overwrite, t_min);
+  return cudaLaunchKernelEx(&cfg, k_tile_fft<N, T, true>, g, state, spec, tw, i, overwrite, t_min);
 }
 
 // Points per thread of the paired blocks (N2 = 2U points per pair): the choice
@@ -619,18 +625,22 @@ __host__ __device__ constexpr int fft2_plan(int /*n2*/) { return 0; }
 
 template <int N2, int P = fft2_points(N2), int PL = fft2_plan(N2)>
 static cudaError_t tile_fft2_n(const Dims& g, float* state, const float2* spec, const float2* tw, int i,
-                               int t_min, cudaStream_t st) {
+                               int t_min, cudaStream_t st, bool pdl) {
   constexpr int T = N2 / P;
   constexpr int F = T >= 128 ? 1 : 128 / T;
   const size_t smem = (size_t)F * (fft_smem_elems(N2) * sizeof(float2) + (size_t)N2 * sizeof(float));
-  cudaError_t e = prepare(k_tile_fft2<N2, T, PL>, smem);
+  cudaError_t e = pdl ? prepare(k_tile_fft2<N2, T, PL, true>, smem) : prepare(k_tile_fft2<N2, T, PL, false>, smem);
   if (e != cudaSuccess) return e;
   const long items = (long)g.M * (g.S / 2);
   const long blocks = (items + F - 1) / F;
   const int overwrite = is_pow2(i) ? 1 : 0;
+  if (!pdl) {   // the plain launch costs the host less (launch-bound stacks)
+    k_tile_fft2<N2, T, PL, false><<<(unsigned)blocks, T * F, smem, st>>>(g, state, spec, i, overwrite, t_min);
+    return cudaGetLastError();
+  }
   cudaLaunchAttribute attr[1];
   cudaLaunchConfig_t cfg = pdl_config(attr, (unsigned)blocks, T * F, smem, st);
-  return cudaLaunchKernelEx(&cfg, k_tile_fft2<N2, T, PL>, g, state, spec, i, overwrite, t_min);
+  return cudaLaunchKernelEx(&cfg, k_tile_fft2<N2, T, PL, true>, g, state, spec, i, overwrite, t_min);
 }
 
 template <int N>
@@ -671,12 +681,12 @@ static cudaError_t debug_fft_n(int count, const float2* in, float2* out, int inv
   }
 
 cudaError_t launch_tile_fft(const Dims& g, float* state, const float2* spectrum_q, const float2* twiddle, int i,
-                            int t_min, cudaStream_t st) {
+                            int t_min, cudaStream_t st, bool pdl) {
   const int U = i & -i;
   const int q = ilog2((uint32_t)U);
   if (g.B % 2 == 0 && q <= kMaxFftLog2 - 1) {
     // two sequences of a channel per complex transform of 2U points
-#define CALL(n) tile_fft2_n<2 * (n)>(g, state, spectrum_q, twiddle, i, t_min, st)
+#define CALL(n) tile_fft2_n<2 * (n)>(g, state, spectrum_q, twiddle, i, t_min, st, pdl)
     switch (q) {
       case 6: return CALL(64);
       case 7: return CALL(128);
@@ -690,7 +700,7 @@ cudaError_t launch_tile_fft(const Dims& g, float* state, const float2* spectrum_
     }
 #undef CALL
   }
-#define CALL(n) tile_fft_n<n>(g, state, spectrum_q, twiddle, i, t_min, st)
+#define CALL(n) tile_fft_n<n>(g, state, spectrum_q, twiddle, i, t_min, st, pdl)
   FI_FFT_SWITCH(q, CALL)
 #undef CALL
 }
