@@ -18,6 +18,7 @@
 // inputs from the strided state. Launches are programmatic: each loads what
 // does not depend on the launch before it (weights, biases, taps, and for the
 // second product the next accumulator and the noise) before it waits.
+#include <mutex>
 #include <type_traits>
 
 #include "fi_internal.cuh"
@@ -303,17 +304,25 @@ cudaError_t launch_mlp_token(const Dims& g, float* state, const void* x, int t, 
   return cudaGetLastError();
 }
 
+// The dynamic shared-memory cap is one value per kernel for the whole process:
+// raise it when this shape needs more, never lower it (another context may
+// need more).
+template <class K>
+static cudaError_t raise_cap(K kernel, size_t smem) {
+  if (smem <= 48 * 1024) return cudaSuccess;
+  static std::mutex mu;
+  std::lock_guard<std::mutex> lock(mu);
+  cudaFuncAttributes fa{};
+  cudaError_t e = cudaFuncGetAttributes(&fa, kernel);
+  if (e != cudaSuccess) return e;
+  if ((size_t)fa.maxDynamicSharedSizeBytes >= smem) return cudaSuccess;
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+}
+
 cudaError_t prepare_mlp(const Dims& g, const MlpBlock& m) {
-  const size_t smem_in = smem_in_bytes(g), smem_out = smem_out_bytes(g, m.hidden);
-  if (smem_in > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(k_mlp_in, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_in);
-    if (e != cudaSuccess) return e;
-  }
-  if (smem_out > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(k_mlp_out, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_out);
-    if (e != cudaSuccess) return e;
-  }
-  return cudaSuccess;
+  cudaError_t e = raise_cap(k_mlp_in, smem_in_bytes(g));
+  if (e == cudaSuccess) e = raise_cap(k_mlp_out, smem_out_bytes(g, m.hidden));
+  return e;
 }
 
 // Both launches allow programmatic stream serialization: each kernel may start

@@ -239,3 +239,30 @@ def test_captured_positions_equal_direct_launches(fi):
     step.sync()
     step.close()
     assert torch.equal(torch.cat([y[:n1], y2]), ys)
+
+
+def test_second_context_does_not_lower_the_shared_memory_cap(fi):
+    # The block's kernels take min(B, 8) x D floats of shared memory (128 KB at
+    # D = 4096). A second context that needs less (64 KB at D = 2048) must not
+    # lower the per-kernel cap under the first, whose next positions still run
+    # and repeat its first generation bit for bit.
+    def make(D, seed):
+        w = synth.Workload(f"mlp-1x{D}-L64-B8", 1, D, 64, 8, "f32", 1e-1, 5e-1)
+        inp = gpu_inputs(w, seed)
+        ctx = fi.Context(inp["h"], 8, "f32")
+        _set(ctx, _weights(1, D, 256, seed + 1, scale=0.2))
+        return w, inp, ctx
+
+    w1, inp1, big = make(4096, 111)
+    n = 16
+    y = torch.empty((n, 8, 4096), dtype=torch.float32, device="cuda")
+    big.generate(n, inp1["x0"], inp1["eps"][:n].contiguous(), y, 0.1)
+    big.sync()
+    _, _, small = make(2048, 121)
+    big.reset()
+    y2 = torch.empty_like(y)
+    big.generate(n, inp1["x0"], inp1["eps"][:n].contiguous(), y2, 0.1)
+    big.sync()
+    assert torch.equal(y, y2)
+    small.close()
+    big.close()
