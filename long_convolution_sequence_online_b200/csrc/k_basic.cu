@@ -1,5 +1,6 @@
 // Per-position red cells, direct blocks read from HBM, the Lazy method's sums
 // and the layout conversions.
+#include <mutex>
 #include <type_traits>
 
 #include "fi_internal.cuh"
@@ -289,7 +290,14 @@ cudaError_t launch_tile_direct(const Dims& g, float* state, const float* taps, i
   }
   const size_t smem = (size_t)3 * U * sizeof(float);
   if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(k_tile_direct, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    // one cap per kernel for the whole process: raise it, never lower it
+    // (another context's launch may need more)
+    static std::mutex mu;
+    std::lock_guard<std::mutex> lock(mu);
+    cudaFuncAttributes fa{};
+    cudaError_t e = cudaFuncGetAttributes(&fa, k_tile_direct);
+    if (e == cudaSuccess && (size_t)fa.maxDynamicSharedSizeBytes < smem)
+      e = cudaFuncSetAttribute(k_tile_direct, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
   }
   const long blocks = (long)g.M * g.D * g.B;
