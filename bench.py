@@ -115,6 +115,31 @@ def cost_model(w: synth.Workload, chunk: int, fft_from: int, fft_max: int = 1 <<
     return out, tot
 
 
+# Widest block the per-position launches add themselves (fi_step's red-cell
+# kernel for stacks of up to 32 layers, the channel-mixing block's small-block
+# launch always); wider ones are launches of their own.
+TOKEN_BLOCK_MAX, TOKEN_MAX_LAYERS, MLP_BLOCK_MAX = 8, 32, 8
+
+
+def per_position_model(w: synth.Workload, fft_from: int, tc_max: int, mlp_hidden: int = 0):
+    """cost_model for the position-by-position paths (fi_step, the channel-mixing
+    block): the per-position bytes and flops, and the blocks the per-position
+    launches add themselves, belong to "token"; wider blocks keep their classes
+    (direct, FFT, tensor cores). The channel-mixing block adds its weights (read
+    once per position) and 2 * 2 * D * Dh flops per (layer, sequence)."""
+    fused = MLP_BLOCK_MAX if mlp_hidden else (TOKEN_BLOCK_MAX if w.layers <= TOKEN_MAX_LAYERS else 0)
+    model, tot = cost_model(w, 2 * fused if fused else 1, fft_from, tc_max=tc_max)
+    model["token"] = dict(model["chunk"])
+    model["chunk"] = {"bytes": 0.0, "flops": 0.0, "blocks": 0}
+    if mlp_hidden:
+        extra_b = w.length * w.layers * (2.0 * w.channels * mlp_hidden + mlp_hidden + w.channels) * 4
+        extra_f = w.length * w.layers * w.batch * 4.0 * w.channels * mlp_hidden
+        model["token"]["bytes"] += extra_b
+        model["token"]["flops"] += extra_f
+        tot = {"bytes": tot["bytes"] + extra_b, "flops": tot["flops"] + extra_f}
+    return model, tot
+
+
 def closed_form_block_bytes(w: synth.Workload) -> float:
     """The schedule's block bytes in closed form, M*D*(L/2)*log2(L)*(8 + B(s_x+8))."""
     s = 2 if w.dtype == "bf16" else 4
@@ -471,20 +496,15 @@ def gpu_arm(args, world, rank, local):
     # --- roofline: dominant kernel class during the timed steps
     peaks = measured_peaks()
     clk = clocks.summary()
-    # fi_step (and any generation with the channel-mixing block) computes every block
-    # from HBM (no on-chip chunk) and each position's red cells in the per-position
-    # kernels, so the per-position bytes and flops belong to "token" there; the block's
-    # two products add their weights (read once per position) and 2 * 2 * D * Dh flops
-    # per (layer, sequence)
+    # fi_step and the channel-mixing block run position by position: no on-chip
+    # chunk; the per-position launches take the red cells and the narrowest blocks
+    # ("token", per_position_model), wider blocks their own launches
     per_pos = step_api or mlp_hidden > 0
-    model, tot = cost_model(w, 1 if per_pos else chunk, fft_from, tc_max=tc_max)
-    model["token"] = dict(model["chunk"]) if per_pos else {"bytes": 0.0, "flops": 0.0}
-    if mlp_hidden:
-        extra_b = w.length * w.layers * (2.0 * w.channels * mlp_hidden + mlp_hidden + w.channels) * 4
-        extra_f = w.length * w.layers * w.batch * 4.0 * w.channels * mlp_hidden
-        model["token"]["bytes"] += extra_b
-        model["token"]["flops"] += extra_f
-        tot = {"bytes": tot["bytes"] + extra_b, "flops": tot["flops"] + extra_f}
+    if per_pos:
+        model, tot = per_position_model(w, fft_from, tc_max, mlp_hidden)
+    else:
+        model, tot = cost_model(w, chunk, fft_from, tc_max=tc_max)
+        model["token"] = {"bytes": 0.0, "flops": 0.0}
     classes = {}
     for cls in ("chunk", "direct", "fft", "tc", "token"):
         n, ms = prof[cls]

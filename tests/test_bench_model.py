@@ -44,3 +44,28 @@ def test_fft_flop_model():
     assert bench.fft_flops(64) == pytest.approx(2 * 2.5 * 128 * 7 + 7 * 64)
     assert bench.fft_flops(1 << 14) == pytest.approx(5 * (1 << 15) * 15 + 7 * (1 << 14))
     assert math.isclose(bench.fft_flops(1024) / bench.fft_flops(512), 2 * 11 / 10, rel_tol=0.02)
+
+
+@pytest.mark.parametrize("mlp_hidden", [0, 768])
+def test_per_position_classes(mlp_hidden):
+    # fi_step and the channel-mixing path add blocks of side <= 8 inside their
+    # per-position launches ("token"); sides 16 and 32 are direct launches and
+    # sides from fft_from FFT launches; every block is counted once.
+    w = synth.WORKLOADS["hyena-18x864-L32K-B4"]
+    model, tot = bench.per_position_model(w, fft_from=64, tc_max=0, mlp_hidden=mlp_hidden)
+    levels = dict(bench.schedule_levels(w.length))
+    assert model["token"]["blocks"] == sum(n for U, n in levels.items() if U <= 8)
+    assert model["direct"]["blocks"] == levels[16] + levels[32]
+    assert model["fft"]["blocks"] == sum(n for U, n in levels.items() if U >= 64)
+    assert model["chunk"]["bytes"] == 0
+    assert sum(v["blocks"] for v in model.values()) == w.length - 1
+    assert tot["bytes"] == pytest.approx(sum(v["bytes"] for v in model.values()))
+
+
+def test_per_token_path_of_a_deep_stack_fuses_no_block():
+    # fi_step fuses blocks only for stacks of up to 32 layers
+    w = synth.Workload("deep", 40, 8, 1024, 1, "f32", 1e-3, 1e-1)
+    model, _ = bench.per_position_model(w, fft_from=64, tc_max=0)
+    assert model["token"]["blocks"] == 0
+    mlp, _ = bench.per_position_model(w, fft_from=64, tc_max=0, mlp_hidden=16)
+    assert mlp["token"]["blocks"] == sum(n for U, n in bench.schedule_levels(w.length) if U <= 8)
