@@ -646,31 +646,41 @@ fi_status fi_generate_host(fi_ctx* c, int32_t n, const void* x0_host, const floa
     FI_CUDA(cudaEventCreateWithFlags(&e, cudaEventDisableTiming), "cudaEventCreate");
     c->seg_ev.push_back(e);
   }
+  // Once a copy is queued, no return may leave one in flight on the caller's
+  // host buffers: every failure below waits for both copy streams first.
+  auto quiesce = [&](fi_status s) {
+    cudaStreamSynchronize(c->up_st);
+    cudaStreamSynchronize(c->dn_st);
+    return s;
+  };
+  auto check = [&](cudaError_t e, const char* what) { return e == cudaSuccess ? FI_OK : quiesce(cuda_fail(e, what)); };
+  fi_status s;
   // the staging buffers may still be read or written by an earlier call's work
-  FI_CUDA(cudaEventRecord(c->seg_ev[2 * nseg], c->st), "cudaEventRecord");
-  FI_CUDA(cudaStreamWaitEvent(c->up_st, c->seg_ev[2 * nseg], 0), "cudaStreamWaitEvent");
-  FI_CUDA(cudaMemcpyAsync(c->d_x0, x0_host, row * esz, cudaMemcpyHostToDevice, c->up_st), "x0 upload");
+  if ((s = check(cudaEventRecord(c->seg_ev[2 * nseg], c->st), "cudaEventRecord")) != FI_OK ||
+      (s = check(cudaStreamWaitEvent(c->up_st, c->seg_ev[2 * nseg], 0), "cudaStreamWaitEvent")) != FI_OK ||
+      (s = check(cudaMemcpyAsync(c->d_x0, x0_host, row * esz, cudaMemcpyHostToDevice, c->up_st), "x0 upload")) != FI_OK)
+    return s;
   for (int k = 0; k < nseg; ++k) {
     const size_t off = (size_t)k * seg * row, cnt = (size_t)std::min(seg, n - k * seg) * row;
-    FI_CUDA(cudaMemcpyAsync(c->d_eps + off, eps_host + off, cnt * sizeof(float), cudaMemcpyHostToDevice, c->up_st),
-            "eps upload");
-    FI_CUDA(cudaEventRecord(c->seg_ev[2 * k], c->up_st), "cudaEventRecord");
+    if ((s = check(cudaMemcpyAsync(c->d_eps + off, eps_host + off, cnt * sizeof(float), cudaMemcpyHostToDevice,
+                                   c->up_st),
+                   "eps upload")) != FI_OK ||
+        (s = check(cudaEventRecord(c->seg_ev[2 * k], c->up_st), "cudaEventRecord")) != FI_OK)
+      return s;
   }
   for (int k = 0; k < nseg; ++k) {
     const int nk = std::min(seg, n - k * seg);
     const size_t off = (size_t)k * seg * row;
-    FI_CUDA(cudaStreamWaitEvent(c->st, c->seg_ev[2 * k], 0), "cudaStreamWaitEvent");
-    fi_status s = fi_generate(c, nk, k == 0 ? c->d_x0 : nullptr, c->d_eps + off, eps_scale, c->d_y + off, nullptr);
-    if (s != FI_OK) {
-      cudaStreamSynchronize(c->up_st);
-      cudaStreamSynchronize(c->dn_st);
+    if ((s = check(cudaStreamWaitEvent(c->st, c->seg_ev[2 * k], 0), "cudaStreamWaitEvent")) != FI_OK) return s;
+    if ((s = fi_generate(c, nk, k == 0 ? c->d_x0 : nullptr, c->d_eps + off, eps_scale, c->d_y + off, nullptr)) !=
+        FI_OK)
+      return quiesce(s);
+    if ((s = check(cudaEventRecord(c->seg_ev[2 * k + 1], c->st), "cudaEventRecord")) != FI_OK ||
+        (s = check(cudaStreamWaitEvent(c->dn_st, c->seg_ev[2 * k + 1], 0), "cudaStreamWaitEvent")) != FI_OK ||
+        (s = check(cudaMemcpyAsync(y_out_host + off, c->d_y + off, (size_t)nk * row * sizeof(float),
+                                   cudaMemcpyDeviceToHost, c->dn_st),
+                   "y download")) != FI_OK)
       return s;
-    }
-    FI_CUDA(cudaEventRecord(c->seg_ev[2 * k + 1], c->st), "cudaEventRecord");
-    FI_CUDA(cudaStreamWaitEvent(c->dn_st, c->seg_ev[2 * k + 1], 0), "cudaStreamWaitEvent");
-    FI_CUDA(cudaMemcpyAsync(y_out_host + off, c->d_y + off, (size_t)nk * row * sizeof(float), cudaMemcpyDeviceToHost,
-                            c->dn_st),
-            "y download");
   }
   FI_CUDA(cudaStreamSynchronize(c->dn_st), "synchronize");
   return sync_and_check(c);
